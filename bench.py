@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark: single-token decode attention with ART on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--mode art|full|q8|q8_art]
+
+A step is one decode call over the whole batch of the workload (default: GQA
+bf16, B=4, Hq=32, Hkv=8, d=128, L=32768, tile 64 -- the long-context decode
+shape the pages' results are quoted on): Q load, K/V tile stream, scores,
+online softmax, PV, the ART probe and rule, the early-exit vote and the
+epilogue, all in one kernel launch.  The KV cache (512 MiB) is larger than L2,
+so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  `value` is decoded query-heads per second over
+all ranks, device-timed with CUDA events; `e2e` times the same call with the
+step's query copied from pinned host memory and its result copied back; the
+`roofline` object rates the decode kernel on the KV bytes it actually read
+(device counters) against the measured HBM copy bandwidth.  With N > 1 every
+rank decodes its own batch of the same shape (weak scaling, no collective in
+the data path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_early_split_b200 import inputs as I  # noqa: E402
+
+METRIC = "decode attention query-heads/s and KV GB/s (fraction of HBM peak), full vs ART"
+UNIT = "query-heads/s"
+DEFAULT_WORKLOAD = "gqa_b4_h32x8_d128_L32k"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOADS)
+    ap.add_argument("--mode", default=None, choices=("art", "full", "q8", "q8_art"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.mode is None:
+        a.mode = "q8_art" if a.workload.startswith("q8") else "art"
+    return a
+
+
+# ----------------------------------------------------------------------------- ranks
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def init_dist(world, backend):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def aggregate(elapsed_ms: float, units: float):
+    """Max elapsed and summed units over ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return elapsed_ms, units
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    u = torch.tensor([units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def hbm_peak():
+    try:
+        v = json.load(open(PEAKS_FILE))["hbm_gbs"]
+        return float(v), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "kv_cache_early_split_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload, mode):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    try:
+        kv = dict(l.split(":", 1) for l in open(TRAFFIC_FILE).read().splitlines() if ":" in l)
+        kv = {k.strip(): v.strip() for k, v in kv.items()}
+        key = f"{workload}/{mode}"
+        if kv.get("source_sha256_16") != kernel_source_hash():
+            return None
+        return float(kv[f"dram_bytes_per_launch[{key}]"])
+    except Exception:
+        return None
+
+
+def kv_row_bytes(w):
+    return w.d * {"f32": 4, "bf16": 2, "q8": 1}[w.kind] + (2 * (w.d // 32) if w.kind == "q8" else 0)
+
+
+def bytes_read(w, tiles_read):
+    """KV bytes fetched: per (b, kvh, split) `tiles_read` tiles of the split, K and V (+ q8 scales)."""
+    rowb = kv_row_bytes(w)
+    total = 0
+    S = tiles_read.shape[2]
+    for b in range(w.B):
+        L = int(w.seq_lens[b])
+        n = -(-L // w.tile)
+        for s in range(S):
+            ta = (s * n) // S
+            tb = ((s + 1) * n) // S
+            split_rows = min(tb * w.tile, L) - ta * w.tile
+            for h in range(w.Hkv):
+                rows = min(int(tiles_read[b, h, s]) * w.tile, split_rows)
+                total += 2 * rows * rowb
+    return total
+
+
+def bytes_consumed(w, used):
+    """KV bytes the rule needed: per (b, kvh, split) the slowest head's tiles."""
+    rowb = kv_row_bytes(w)
+    G = w.G
+    total = 0
+    S = used.shape[2]
+    for b in range(w.B):
+        L = int(w.seq_lens[b])
+        n = -(-L // w.tile)
+        for s in range(S):
+            ta = (s * n) // S
+            tb = ((s + 1) * n) // S
+            split_rows = min(tb * w.tile, L) - ta * w.tile
+            for h in range(w.Hkv):
+                t = int(used[b, h * G:(h + 1) * G, s].max())
+                total += 2 * min(t * w.tile, split_rows) * rowb
+    return total
+
+
+def oracle_sample(w, mode, heads_slabs, n_threads):
+    """Run the oracle on a list of (b, kvh) slabs; returns (#query heads, seconds)."""
+    import oracle
+
+    kind = {"f32": oracle.KV_F32, "bf16": oracle.KV_BF16, "q8": oracle.KV_Q8}[w.kind]
+    G = w.G
+    heads = 0
+    t0 = time.perf_counter()
+    for (b, h) in heads_slabs:
+        oracle.decode(
+            kind=kind, q=w.q[b:b + 1, h * G:(h + 1) * G], k=w.k[b:b + 1, h:h + 1], v=w.v[b:b + 1, h:h + 1],
+            k_scale=None if w.k_scale is None else w.k_scale[b:b + 1, h:h + 1],
+            v_scale=None if w.v_scale is None else w.v_scale[b:b + 1, h:h + 1],
+            seq_lens=w.seq_lens[b:b + 1], tile=w.tile, num_splits=w.num_splits,
+            art=w.art if mode in ("art", "q8_art") else None, tau=w.tau if mode in ("q8", "q8_art") else 0.0,
+            n_threads=n_threads)
+        heads += G
+    return heads, time.perf_counter() - t0
+
+
+def config_obj(w, mode, args, world):
+    return {
+        "workload": w.name, "mode": mode, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "L_max": w.L_max,
+        "tile": w.tile, "num_splits": w.num_splits, "kv_storage": w.kind,
+        "art": {k: w.art[k] for k in ("eps_scale", "eps_dir", "patience")} | {"n_probe": len(w.art["lanes"])},
+        "tau": w.tau if mode.startswith("q8") else None,
+        "l2": "no flush: KV inputs larger than the 126 MB L2",
+        "parallelism": f"replicas x{world} (weak scaling)" if world > 1 else "single GPU",
+    }
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = I.workload(args.workload)
+    cores = os.cpu_count() or 1
+    slabs = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:2]
+    for _ in range(args.warmup):
+        oracle_sample(w, args.mode, slabs, cores)
+    tot_h = 0
+    tot_s = 0.0
+    for _ in range(args.steps):
+        h, s = oracle_sample(w, args.mode, slabs, cores)
+        tot_h += h
+        tot_s += s
+    val = tot_h / tot_s
+    sample = f"{len(slabs)} (batch, kv head) slabs = {len(slabs) * w.G} query heads of the workload per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_obj(w, args.mode, args, 1),
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def time_mode(K, dp, mode, steps, warmup, stream):
+    """Device time of `steps` calls: (total ms, mean per-launch ms from per-launch events)."""
+    import torch
+
+    for _ in range(warmup):
+        K.decode(dp, mode, stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        K.decode(dp, mode, stream=stream.cuda_stream)
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    per = [a.elapsed_time(b) for a, b in ev]
+    return total, sum(per) / len(per)
+
+
+def run_ours(args):
+    import torch
+
+    import kv_cache_early_split_b200 as K
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        init_dist(world, "nccl")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = I.workload(args.workload)
+    dp = K.upload(w, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    heads = w.B * w.Hq
+
+    # main timed region (the method's mode), clocks sampled meanwhile
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(torch.cuda.current_device()))
+    for _ in range(args.warmup):
+        K.decode(dp, args.mode, stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    sampler.start()
+    total_ms, launch_ms = time_mode(K, dp, args.mode, args.steps, 0, stream)
+    clocks = sampler.stop()
+    if K.device_status(dp) != 0:
+        raise RuntimeError("device status not OK after the timed region")
+    tiles_read = dp.tiles_read().cpu().numpy()
+    used = dp.split_tiles().cpu().numpy()
+    tiles = dp.tiles.cpu().numpy()
+    gpu_launches = args.steps * (1 + (1 if w.num_splits > 1 else 0))
+
+    max_ms, all_heads = aggregate(total_ms, heads * args.steps)
+    value = all_heads / (max_ms / 1e3)
+    peak, peak_kind = hbm_peak()
+    rb = bytes_read(w, tiles_read)
+    cb = bytes_consumed(w, used)
+    achieved = rb / (launch_ms / 1e3) / 1e9
+    n_full = -(-w.seq_lens.astype(np.int64) // w.tile)
+
+    # the other mode (full vs ART) on the same buffers
+    other = {"art": "full", "full": "art", "q8": "q8_art", "q8_art": "q8"}[args.mode]
+    o_total, o_launch = time_mode(K, dp, other, args.steps, args.warmup, stream)
+    o_read = bytes_read(w, dp.tiles_read().cpu().numpy())
+    o_max, _ = aggregate(o_total, 0)
+    modes = {
+        args.mode: {"query_heads_per_s": value, "ms_per_step": max_ms / args.steps,
+                    "kv_gbs_read": achieved, "frac_of_hbm": achieved / peak,
+                    "kv_bytes_read": rb, "kv_bytes_consumed": cb,
+                    "mean_tiles_frac": float(tiles.mean() / n_full.mean())},
+        other: {"query_heads_per_s": heads * world * args.steps / (o_max / 1e3), "ms_per_step": o_max / args.steps,
+                "kv_gbs_read": o_read / (o_launch / 1e3) / 1e9, "frac_of_hbm": o_read / (o_launch / 1e3) / 1e9 / peak,
+                "kv_bytes_read": o_read},
+    }
+
+    # end to end through the public call: the step's query in from pinned host memory, O and tiles back out
+    q_host = dp.q.cpu().pin_memory()
+    o_host = torch.empty_like(dp.o, device="cpu").pin_memory()
+    t_host = torch.empty_like(dp.tiles, device="cpu").pin_memory()
+    for _ in range(args.warmup):
+        dp.q.copy_(q_host, non_blocking=True)
+        K.decode(dp, args.mode)
+        o_host.copy_(dp.o, non_blocking=True)
+        t_host.copy_(dp.tiles, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream()
+    e0.record(cur)
+    for _ in range(args.steps):
+        dp.q.copy_(q_host, non_blocking=True)
+        K.decode(dp, args.mode)
+        o_host.copy_(dp.o, non_blocking=True)
+        t_host.copy_(dp.tiles, non_blocking=True)
+    e1.record(cur)
+    torch.cuda.synchronize()
+    e2e_ms, e2e_heads = aggregate(e0.elapsed_time(e1), heads * args.steps)
+    e2e = {"value": e2e_heads / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size()),
+           "d2h_bytes_per_step": int(o_host.numel() * 4 + t_host.numel() * 4),
+           "note": "KV cache resident in HBM as in serving; per step the query goes in and O + tiles come out"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        slabs = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+        h_done, secs = oracle_sample(w, args.mode, slabs, cores)
+        cpu = {"value": h_done / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"all {h_done} query heads of the workload once ({secs:.1f} s)"}
+
+    traffic = measured_traffic(w.name, args.mode)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "storage": w.kind, "data": "synthetic",
+        "config": config_obj(w, args.mode, args, world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} hbm_gbs (copy)", "traffic": traffic,
+                     "kernel": "art_decode_kernel", "bytes_per_launch": rb, "launch_ms": launch_ms},
+        "modes": modes,
+        "e2e": e2e,
+        "gpu_launches": gpu_launches,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,155 @@
+/*
+ * art_decode.h -- C ABI of the B200 (sm_100a) decode-attention library with
+ * ART (runtime attention termination) and the q8 V-dequantisation skip.
+ *
+ * What it computes (web pages, cited by title and section):
+ *   "Resumen Tecnico: ART (Terminacion de la Atencion en Tiempo de Ejecucion)",
+ *   gist.science summary of arXiv 2606.00024:
+ *     S1   one decode query per head attends to the whole cached K/V;
+ *     S2.1 attention is accumulated tile by tile (online softmax), which
+ *          exposes the partial output O^(t) after every KV tile;
+ *     S2.2 ART watches a probe x^(t) (fixed lanes of O^(t)) and stops reading
+ *          KV tiles once both its magnitude change d_scale and its direction
+ *          change d_direction fall below the thresholds;
+ *     S2.3 the criterion must hold on `patience` consecutive tiles;
+ *     S2.4 tile 0 is always processed before any termination.
+ *   "La paradoja de la eficiencia: como omitir redefine la velocidad de los
+ *   LLM", puntofijo.es, section "La Elegancia de la Omision": with an int8
+ *   (q8_0) cache the V rows whose softmax weight is negligible are not
+ *   dequantised.
+ *
+ * Readings this library implements (the pages leave them open):
+ *   d_scale   = | ||x^(t)|| - ||x^(t-1)|| |
+ *   d_dir     = 1 - cos(x^(t), x^(t-1)), >= 0; 0 if both probes are zero,
+ *               1 if exactly one is; the probe before a split's first tile is
+ *               the zero vector (so +inf thresholds stop after one tile);
+ *   hold      = d_scale < eps_scale && d_dir < eps_dir (strict; NaN never holds);
+ *   the rule runs per (batch, query head) and independently per KV split;
+ *   a head whose rule fires keeps the state of its stop tile; the KV head's
+ *   reads stop when all of its query heads have stopped;
+ *   split s covers tiles [floor(s*n/S), floor((s+1)*n/S)), n = ceil(L_b/T);
+ *   V skip: a row is left out of the numerator when exp(s_j - m') < tau, m'
+ *   the running maximum of the split after the row's tile; its weight stays
+ *   in the denominator.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are caller-owned DEVICE pointers, contiguous, row-major:
+ *       q      [B, Hq, d]          fp32 (ART_F32) or bf16 (ART_BF16, q8 mode)
+ *       k, v   [B, Hkv, L_max, d]  fp32 / bf16 / int8 codes
+ *       k_scale_f16, v_scale_f16   [B, Hkv, L_max, d/32] IEEE fp16 bits (q8)
+ *       seq_lens [B] int32, each in [1, L_max] (checked on the device)
+ *       o      [B, Hq, d] fp32 output
+ *       tiles  [B, Hq] int32 output: KV tiles consumed per query head (summed
+ *              over splits); may be NULL
+ *     Query head hq reads KV head hq / (Hq/Hkv).  Device pointers must be
+ *     16-byte aligned.
+ *   - ws is a caller-owned DEVICE workspace of at least
+ *     art_workspace_bytes(shape) bytes, zero-filled once before its first use
+ *     (it holds a sticky device status word, per-split partial results and
+ *     the per-(batch, kv head, split) count of KV tiles actually read).
+ *     One workspace must not be used by two calls that overlap in time.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work and return; nothing is synchronised.  The library
+ *     allocates no memory and keeps no global state besides cached kernel
+ *     attributes.
+ *   - Argument errors are returned synchronously and enqueue nothing.  Errors
+ *     found on the device (a seq_len outside [1, L_max], a wait that timed
+ *     out) set the status word in ws; art_read_device_status() reports and
+ *     clears it.  A head whose seq_len is invalid gets NaN outputs and 0 tiles.
+ *   - Constraints (else ART_ERR_UNSUPPORTED or ART_ERR_INVALID_ARG):
+ *       d in {64, 128}; tile in {16, 32, 64, 128, 256} and small enough that
+ *       two K+V tiles fit in shared memory; 1 <= Hq/Hkv <= 8 with Hq % Hkv == 0;
+ *       num_splits >= 1; for q8, L_max*(d/32)*2 bytes a multiple of 16;
+ *       1 <= n_probe <= 32 distinct lanes in [0, d); patience >= 1.
+ */
+#ifndef ART_DECODE_H
+#define ART_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ART_OK = 0,
+  ART_ERR_INVALID_ARG = -1, /* a NULL pointer, a negative size, bad lanes ... */
+  ART_ERR_UNSUPPORTED = -2, /* valid but outside what the kernels implement */
+  ART_ERR_WORKSPACE = -3,   /* ws NULL or smaller than art_workspace_bytes() */
+  ART_ERR_CUDA = -4,        /* a CUDA runtime call failed (launch, attribute) */
+  ART_ERR_TIMEOUT = -5,     /* device: a bounded wait gave up (status word) */
+  ART_ERR_SEQLEN = -6       /* device: a seq_len outside [1, L_max] (status word) */
+} art_status;
+
+typedef enum { ART_F32 = 0, ART_BF16 = 1 } art_dtype;
+
+/* Problem shape.  tile = KV positions per tile (T); num_splits = KV splits per
+ * sequence (S): each split runs its own online softmax (and its own ART rule)
+ * and a combine step merges them. */
+typedef struct {
+  int32_t B, Hq, Hkv, d, L_max, tile, num_splits;
+} art_shape;
+
+/* ART settings (page S2.2, S2.3).  eps_scale is the page's tau (magnitude),
+ * eps_dir its phi (direction).  probe_lanes is a HOST array of n_probe lane
+ * indices of O; it is copied during the call. */
+typedef struct {
+  float eps_scale;
+  float eps_dir;
+  int32_t patience;
+  const int32_t* probe_lanes;
+  int32_t n_probe;
+} art_params;
+
+/* Bytes of workspace a call with this shape needs (0 on an invalid shape). */
+size_t art_workspace_bytes(const art_shape* shape);
+
+/* Byte offset inside ws of the int32 array tiles_read[B, Hkv, num_splits]:
+ * KV tiles actually fetched from HBM for each (batch, kv head, split) by the
+ * last call, speculative prefetch included.  Written by every call. */
+size_t art_workspace_tiles_read_offset(const art_shape* shape);
+
+/* Byte offset inside ws of the int32 array split_tiles[B, Hq, num_splits]:
+ * KV tiles consumed by each (batch, query head, split) in the last call (the
+ * per-split terms of `tiles`).  Written by every call. */
+size_t art_workspace_split_tiles_offset(const art_shape* shape);
+
+/* Plain tile-wise decode attention over every KV position (page S1, S2.1):
+ * o = softmax(q K^T / sqrt(d)) V per query head; tiles = ceil(L_b / tile). */
+art_status art_decode_attn_full(const art_shape* shape, art_dtype dtype, const void* q,
+                                const void* k, const void* v, const int32_t* seq_lens, float* o,
+                                int32_t* tiles, void* ws, size_t ws_bytes, void* stream);
+
+/* Decode attention with ART (page S2.2-S2.4): each (query head, split) stops
+ * consuming KV tiles once the probe has been stable for `patience` tiles; o is
+ * the normalised partial output at the stop tile, tiles the tiles consumed. */
+art_status art_decode_attn_terminate(const art_shape* shape, art_dtype dtype, const void* q,
+                                     const void* k, const void* v, const int32_t* seq_lens,
+                                     const art_params* params, float* o, int32_t* tiles, void* ws,
+                                     size_t ws_bytes, void* stream);
+
+/* Decode attention over an int8 KV cache in 32-element blocks with one fp16
+ * scale each (q8_0 style; value = code * scale), bf16 query.  V rows whose
+ * weight exp(s_j - m') is below tau are neither dequantised nor accumulated
+ * (puntofijo.es, "La Elegancia de la Omision").  params == NULL runs without
+ * ART; otherwise ART as in art_decode_attn_terminate. */
+art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
+                                    const uint16_t* k_scale_f16, const int8_t* v_q,
+                                    const uint16_t* v_scale_f16, const int32_t* seq_lens,
+                                    float tau, const art_params* params, float* o, int32_t* tiles,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the sticky status word of ws, clear it, and
+ * return ART_OK, ART_ERR_SEQLEN or ART_ERR_TIMEOUT (ART_ERR_CUDA if the
+ * synchronisation or copy failed). */
+art_status art_read_device_status(void* ws, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* art_status_string(art_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ART_DECODE_H */

@@ -1,0 +1,143 @@
+"""B200 (sm_100a) single-token decode attention with ART (runtime attention
+termination) and the q8 V-dequantisation skip.
+
+The computation lives in CUDA kernels behind the C ABI of
+``include/art_decode.h`` (``libart_decode.so``).  ``capi`` is the ctypes
+binding with the C names; this module adds tensor-level helpers that only
+allocate outputs / workspace with PyTorch and marshal pointers.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+from . import capi
+from .capi import ArtError
+
+__all__ = ["capi", "ArtError", "DeviceProblem", "upload", "decode"]
+
+
+@dataclass
+class DeviceProblem:
+    """A workload resident on the GPU (torch tensors), plus its output buffers."""
+
+    kind: str
+    shape: "capi.art_shape"
+    q: object
+    k: object
+    v: object
+    k_scale: object
+    v_scale: object
+    seq_lens: object
+    o: object
+    tiles: object
+    ws: object
+    art: dict
+    tau: float
+
+    @property
+    def ws_bytes(self) -> int:
+        return int(self.ws.numel())
+
+    def tiles_read(self):
+        """int32 [B, Hkv, S]: KV tiles fetched by the last call (device tensor view)."""
+        import torch
+
+        off = capi.art_workspace_tiles_read_offset(self.shape)
+        s = self.shape
+        n = s.B * s.Hkv * s.num_splits
+        return self.ws[off:off + 4 * n].view(torch.int32).view(s.B, s.Hkv, s.num_splits)
+
+
+    def split_tiles(self):
+        """int32 [B, Hq, S]: KV tiles consumed per split by the last call (device tensor view)."""
+        import torch
+
+        off = capi.art_workspace_split_tiles_offset(self.shape)
+        s = self.shape
+        n = s.B * s.Hq * s.num_splits
+        return self.ws[off:off + 4 * n].view(torch.int32).view(s.B, s.Hq, s.num_splits)
+
+
+def _t(torch, arr, device, dtype=None):
+    import numpy as np
+
+    if arr is None:
+        return None
+    a = np.ascontiguousarray(arr)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    t = torch.from_numpy(a)
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.to(device)
+
+
+def upload(w, device="cuda", num_splits=None, tile=None):
+    """Copy a kv_cache_early_split_b200.inputs.Workload to the GPU and allocate o / tiles / workspace."""
+    import torch
+
+    S = w.num_splits if num_splits is None else int(num_splits)
+    T = w.tile if tile is None else int(tile)
+    shape = capi.art_shape(w.B, w.Hq, w.Hkv, w.d, w.L_max, T, S)
+    wsb = capi.art_workspace_bytes(shape)
+    if wsb == 0:
+        raise ArtError(capi.ART_ERR_INVALID_ARG, "art_workspace_bytes")
+    return DeviceProblem(
+        kind=w.kind, shape=shape,
+        q=_t(torch, w.q, device), k=_t(torch, w.k, device), v=_t(torch, w.v, device),
+        k_scale=_t(torch, w.k_scale, device), v_scale=_t(torch, w.v_scale, device),
+        seq_lens=_t(torch, w.seq_lens, device, torch.int32),
+        o=torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=device),
+        tiles=torch.empty((w.B, w.Hq), dtype=torch.int32, device=device),
+        ws=torch.zeros(wsb, dtype=torch.uint8, device=device),
+        art=dict(w.art), tau=float(w.tau),
+    )
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float | None = None, stream=None,
+           check: bool = True) -> int:
+    """Launch one decode call on dp's buffers.
+
+    mode: "full" | "art" (art_decode_attn_terminate) | "q8" (q8_skipv without ART) |
+          "q8_art" (q8_skipv with ART).  Returns the C status code; raises
+    ArtError on a non-zero code when check is True.
+    """
+    import torch
+
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    a = dp.art if art is None else art
+    dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
+    if mode == "full":
+        rc = capi.art_decode_attn_full(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens),
+                                       _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
+        name = "art_decode_attn_full"
+    elif mode == "art":
+        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+        rc = capi.art_decode_attn_terminate(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens),
+                                            params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
+        name = "art_decode_attn_terminate"
+    elif mode in ("q8", "q8_art"):
+        params = None
+        if mode == "q8_art":
+            params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+        rc = capi.art_decode_attn_q8_skipv(
+            dp.shape, _ptr(dp.q), _ptr(dp.k), _ptr(dp.k_scale), _ptr(dp.v), _ptr(dp.v_scale), _ptr(dp.seq_lens),
+            dp.tau if tau is None else tau, params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
+        name = "art_decode_attn_q8_skipv"
+    else:
+        raise ValueError(mode)
+    if check and rc != capi.ART_OK:
+        raise ArtError(rc, name)
+    return rc
+
+
+def device_status(dp: DeviceProblem, stream=None) -> int:
+    """Synchronise and return (and clear) the sticky device status of dp's workspace."""
+    import torch
+
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    return capi.art_read_device_status(_ptr(dp.ws), st)

@@ -1,0 +1,146 @@
+"""ctypes binding of the C ABI in include/art_decode.h (argument marshalling only).
+
+Every function here has the name of the C entry point it forwards to and takes
+raw pointers (ints) and sizes, exactly like the C signature.  There is no
+fallback: if libart_decode.so cannot be loaded, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libart_decode.so")
+
+ART_OK = 0
+ART_ERR_INVALID_ARG = -1
+ART_ERR_UNSUPPORTED = -2
+ART_ERR_WORKSPACE = -3
+ART_ERR_CUDA = -4
+ART_ERR_TIMEOUT = -5
+ART_ERR_SEQLEN = -6
+ART_F32 = 0
+ART_BF16 = 1
+
+# every symbol the header declares
+EXPORTS = (
+    "art_workspace_bytes",
+    "art_workspace_tiles_read_offset",
+    "art_workspace_split_tiles_offset",
+    "art_decode_attn_full",
+    "art_decode_attn_terminate",
+    "art_decode_attn_q8_skipv",
+    "art_read_device_status",
+    "art_status_string",
+)
+
+
+class art_shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "d", "L_max", "tile", "num_splits")]
+
+
+class art_params(ctypes.Structure):
+    _fields_ = [
+        ("eps_scale", ctypes.c_float),
+        ("eps_dir", ctypes.c_float),
+        ("patience", ctypes.c_int32),
+        ("probe_lanes", ctypes.POINTER(ctypes.c_int32)),
+        ("n_probe", ctypes.c_int32),
+    ]
+
+
+class ArtError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {art_status_string(code)} ({code})")
+        self.code = code
+
+
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.c_void_p
+_SH = ctypes.POINTER(art_shape)
+_PA = ctypes.POINTER(art_params)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libart_decode.so (built in-tree by kv_cache_early_split_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise OSError(
+                    f"{LIB_PATH} is missing: build it with `python -m kv_cache_early_split_b200.build` "
+                    "(there is no fallback implementation)"
+                )
+            L = ctypes.CDLL(LIB_PATH)
+            L.art_workspace_bytes.restype = ctypes.c_size_t
+            L.art_workspace_bytes.argtypes = [_SH]
+            L.art_workspace_tiles_read_offset.restype = ctypes.c_size_t
+            L.art_workspace_tiles_read_offset.argtypes = [_SH]
+            L.art_workspace_split_tiles_offset.restype = ctypes.c_size_t
+            L.art_workspace_split_tiles_offset.argtypes = [_SH]
+            L.art_decode_attn_full.restype = ctypes.c_int
+            L.art_decode_attn_full.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+            L.art_decode_attn_terminate.restype = ctypes.c_int
+            L.art_decode_attn_terminate.argtypes = [
+                _SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, ctypes.c_size_t, _P]
+            L.art_decode_attn_q8_skipv.restype = ctypes.c_int
+            L.art_decode_attn_q8_skipv.argtypes = [
+                _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, _P]
+            L.art_read_device_status.restype = ctypes.c_int
+            L.art_read_device_status.argtypes = [_P, _P]
+            L.art_status_string.restype = ctypes.c_char_p
+            L.art_status_string.argtypes = [ctypes.c_int]
+            _lib = L
+    return _lib
+
+
+def _ref(x):
+    return None if x is None else ctypes.byref(x)
+
+
+def art_workspace_bytes(shape: art_shape) -> int:
+    return int(lib().art_workspace_bytes(ctypes.byref(shape)))
+
+
+def art_workspace_tiles_read_offset(shape: art_shape) -> int:
+    return int(lib().art_workspace_tiles_read_offset(ctypes.byref(shape)))
+
+
+def art_workspace_split_tiles_offset(shape: art_shape) -> int:
+    return int(lib().art_workspace_split_tiles_offset(ctypes.byref(shape)))
+
+
+def art_decode_attn_full(shape, dtype, q, k, v, seq_lens, o, tiles, ws, ws_bytes, stream) -> int:
+    return int(lib().art_decode_attn_full(ctypes.byref(shape), dtype, q, k, v, seq_lens, o, tiles, ws, ws_bytes, stream))
+
+
+def art_decode_attn_terminate(shape, dtype, q, k, v, seq_lens, params, o, tiles, ws, ws_bytes, stream) -> int:
+    return int(lib().art_decode_attn_terminate(
+        ctypes.byref(shape), dtype, q, k, v, seq_lens, _ref(params), o, tiles, ws, ws_bytes, stream))
+
+
+def art_decode_attn_q8_skipv(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, params, o, tiles,
+                             ws, ws_bytes, stream) -> int:
+    return int(lib().art_decode_attn_q8_skipv(
+        ctypes.byref(shape), q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, float(tau), _ref(params), o,
+        tiles, ws, ws_bytes, stream))
+
+
+def art_read_device_status(ws, stream) -> int:
+    return int(lib().art_read_device_status(ws, stream))
+
+
+def art_status_string(code: int) -> str:
+    return lib().art_status_string(int(code)).decode()
+
+
+def make_params(eps_scale: float, eps_dir: float, patience: int, lanes) -> art_params:
+    """art_params with its own HOST copy of the lane list (kept alive on the object)."""
+    arr = (ctypes.c_int32 * len(lanes))(*[int(x) for x in lanes])
+    p = art_params(float(eps_scale), float(eps_dir), int(patience),
+                   ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)), len(lanes))
+    p._lanes_keepalive = arr
+    return p

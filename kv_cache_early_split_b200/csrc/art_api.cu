@@ -1,0 +1,408 @@
+// art_api.cu -- host side of the C ABI declared in include/art_decode.h:
+// argument validation, workspace layout, launch configuration (cluster size,
+// pipeline depth) and kernel dispatch.  No memory is allocated here.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "art_decode.h"
+#include "art_kernels.cuh"
+
+namespace {
+
+using artk::Layout;
+using artk::Params;
+
+constexpr size_t kWsHeader = 256;  // status word lives at offset 0
+constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+constexpr int kSmemPerSm = 233472;   // 228 KB per SM
+constexpr int kSmemReservedPerBlock = 1024;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t tiles_read, used, partial, total;
+};
+
+bool shape_ok(const art_shape* s) {
+  return s && s->B >= 1 && s->Hq >= 1 && s->Hkv >= 1 && s->d >= 1 && s->L_max >= 1 && s->tile >= 1 &&
+         s->num_splits >= 1;
+}
+
+WsLayout ws_layout(const art_shape* s) {
+  WsLayout w;
+  const size_t units = size_t(s->B) * s->Hkv * s->num_splits;
+  const size_t heads = size_t(s->B) * s->Hq * s->num_splits;
+  w.tiles_read = kWsHeader;
+  w.used = align256(w.tiles_read + 4 * units);
+  w.partial = align256(w.used + 4 * heads);
+  w.total = align256(w.partial + 4 * heads * (size_t(s->d) + 2));
+  return w;
+}
+
+using KernelFn = void (*)(Params);
+
+struct KernelInfo {
+  KernelFn fn;
+  Layout (*layout)(int T, int nstage, int C);
+  int epc;
+};
+
+template <int KIND, int D, int GP, int MODE>
+Layout layout_thunk(int T, int nstage, int C) {
+  return artk::make_layout<KIND, D, GP>(T, nstage, C);
+}
+
+template <int KIND, int D, int GP, int MODE>
+KernelInfo info() {
+  return KernelInfo{&artk::art_decode_kernel<KIND, D, GP, MODE>, &layout_thunk<KIND, D, GP, MODE>,
+                    artk::KvGeom<KIND, D>::EPC};
+}
+
+template <int KIND, int D, int MODE>
+bool pick_gp(int G, KernelInfo* out) {
+  if (G == 1) *out = info<KIND, D, 1, MODE>();
+  else if (G == 2) *out = info<KIND, D, 2, MODE>();
+  else if (G <= 4) *out = info<KIND, D, 4, MODE>();
+  else if (G <= 8) *out = info<KIND, D, 8, MODE>();
+  else return false;
+  return true;
+}
+
+template <int KIND, int MODE>
+bool pick_d(int d, int G, KernelInfo* out) {
+  if (d == 64) return pick_gp<KIND, 64, MODE>(G, out);
+  if (d == 128) return pick_gp<KIND, 128, MODE>(G, out);
+  return false;
+}
+
+bool pick_kernel(int kind, int mode, int d, int G, KernelInfo* out) {
+  using namespace artk;
+  if (kind == KV_F32 && mode == MODE_FULL) return pick_d<KV_F32, MODE_FULL>(d, G, out);
+  if (kind == KV_F32 && mode == MODE_ART) return pick_d<KV_F32, MODE_ART>(d, G, out);
+  if (kind == KV_BF16 && mode == MODE_FULL) return pick_d<KV_BF16, MODE_FULL>(d, G, out);
+  if (kind == KV_BF16 && mode == MODE_ART) return pick_d<KV_BF16, MODE_ART>(d, G, out);
+  if (kind == KV_Q8 && mode == MODE_SKIP) return pick_d<KV_Q8, MODE_SKIP>(d, G, out);
+  if (kind == KV_Q8 && mode == MODE_SKIP_ART) return pick_d<KV_Q8, MODE_SKIP_ART>(d, G, out);
+  return false;
+}
+
+// Per-device facts and per-kernel attributes, set once.
+std::mutex g_mu;
+struct DevInfo {
+  int sms = 0;
+};
+DevInfo g_dev[64];
+struct AttrEntry {
+  KernelFn fn;
+  int device;
+};
+AttrEntry g_attr[512];
+int g_attr_n = 0;
+
+art_status prepare(KernelFn fn, int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ART_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_dev[dev].sms == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ART_ERR_CUDA;
+    g_dev[dev].sms = v;
+  }
+  *sms = g_dev[dev].sms;
+  for (int i = 0; i < g_attr_n; ++i)
+    if (g_attr[i].fn == fn && g_attr[i].device == dev) return ART_OK;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kMaxDynSmem) != cudaSuccess)
+    return ART_ERR_CUDA;
+  if (cudaFuncSetAttribute(reinterpret_cast<const void*>(fn), cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+      cudaSuccess)
+    return ART_ERR_CUDA;
+  if (g_attr_n < 512) g_attr[g_attr_n++] = AttrEntry{fn, dev};
+  return ART_OK;
+}
+
+struct LaunchCfg {
+  int C, nstage;
+  uint32_t smem;
+};
+
+struct OccEntry {
+  KernelFn fn;
+  int device, tile, nstage, per_sm;
+};
+OccEntry g_occ[1024];
+int g_occ_n = 0;
+
+// Pipeline depth and resident CTAs per SM for a kernel and tile size: prefer
+// two resident CTAs per SM with an (at least) three-deep ring, else one CTA
+// with the deepest ring that fits.  Occupancy comes from the runtime, so the
+// register count of the compiled kernel is taken into account.
+bool pick_depth(const KernelInfo& ki, int tile, int* nstage, int* per_sm) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_occ_n; ++i)
+      if (g_occ[i].fn == ki.fn && g_occ[i].device == dev && g_occ[i].tile == tile) {
+        *nstage = g_occ[i].nstage;
+        *per_sm = g_occ[i].per_sm;
+        return *nstage > 0;
+      }
+  }
+  int best_ns = 0, best_occ = 0;
+  for (int ns = 4; ns >= 2; --ns) {
+    const Layout L = ki.layout(tile, ns, artk::CMAX);
+    if (L.total > static_cast<uint32_t>(kMaxDynSmem)) continue;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, ki.fn, artk::NT, L.total) != cudaSuccess) return false;
+    if (occ < 1) continue;
+    const bool better = (best_ns == 0) || (occ >= 2 && best_occ < 2 && ns >= 3);
+    if (better) {
+      best_ns = ns;
+      best_occ = occ;
+    }
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_occ_n < 1024) g_occ[g_occ_n++] = OccEntry{ki.fn, dev, tile, best_ns, best_occ};
+  *nstage = best_ns;
+  *per_sm = best_occ;
+  return best_ns > 0;
+}
+
+// Cluster size: fill the GPU in one wave -- the largest power-of-two C with
+// units*C no more than the resident-CTA count (and no more CTAs than tiles).
+bool choose_config(const KernelInfo& ki, const art_shape* s, int sms, int max_tiles_per_split, LaunchCfg* out) {
+  const int units = s->B * s->Hkv * s->num_splits;
+  int nstage = 0, per_sm = 0;
+  if (!pick_depth(ki, s->tile, &nstage, &per_sm)) return false;
+  const int target = sms * (per_sm > 2 ? 2 : per_sm);
+  int C = 1;
+  while (C < artk::CMAX && units * (2 * C) <= target && 2 * C <= max_tiles_per_split) C *= 2;
+  // shrink the cluster until the runtime can co-schedule one of that size
+  while (C > 1) {
+    cudaLaunchConfig_t lc;
+    memset(&lc, 0, sizeof lc);
+    cudaLaunchAttribute attr[1];
+    lc.gridDim = dim3(static_cast<unsigned>(units * C), 1, 1);
+    lc.blockDim = dim3(artk::NT, 1, 1);
+    lc.dynamicSmemBytes = ki.layout(s->tile, nstage, C).total;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, ki.fn, &lc) == cudaSuccess && nclusters > 0) break;
+    cudaGetLastError();  // clear a sticky-free query error
+    C /= 2;
+  }
+  out->C = C;
+  out->nstage = nstage;
+  out->smem = ki.layout(s->tile, nstage, C).total;
+  return true;
+}
+
+art_status validate_common(const art_shape* s, const void* q, const void* k, const void* v,
+                           const int32_t* seq_lens, const float* o, void* ws, size_t ws_bytes) {
+  if (!shape_ok(s)) return ART_ERR_INVALID_ARG;
+  if (!q || !k || !v || !seq_lens || !o) return ART_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return ART_ERR_INVALID_ARG;
+  const int G = s->Hq / s->Hkv;
+  if (G > artk::GMAX) return ART_ERR_UNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return ART_ERR_UNSUPPORTED;
+  if (s->tile != 16 && s->tile != 32 && s->tile != 64 && s->tile != 128 && s->tile != 256) return ART_ERR_UNSUPPORTED;
+  auto mis = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+  if (mis(q) || mis(k) || mis(v) || mis(o)) return ART_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < art_workspace_bytes(s) || mis(ws)) return ART_ERR_WORKSPACE;
+  // index arithmetic stays in 64-bit on the device; keep the grid within limits
+  const long long units = 1LL * s->B * s->Hkv * s->num_splits;
+  if (units * artk::CMAX > 0x7fffffffLL) return ART_ERR_UNSUPPORTED;
+  return ART_OK;
+}
+
+art_status validate_params(const art_params* a, int d, int epc, int* emask) {
+  if (!a || !a->probe_lanes) return ART_ERR_INVALID_ARG;
+  if (a->n_probe < 1 || a->n_probe > artk::PMAX || a->patience < 1) return ART_ERR_INVALID_ARG;
+  uint64_t seen[2] = {0, 0};
+  *emask = 0;
+  for (int i = 0; i < a->n_probe; ++i) {
+    const int l = a->probe_lanes[i];
+    if (l < 0 || l >= d) return ART_ERR_INVALID_ARG;
+    if (seen[l >> 6] & (1ull << (l & 63))) return ART_ERR_INVALID_ARG;
+    seen[l >> 6] |= 1ull << (l & 63);
+    *emask |= 1 << (l % epc);
+  }
+  return ART_OK;
+}
+
+art_status launch(int kind, int mode, const art_shape* s, const void* q, const void* k, const void* v,
+                  const uint16_t* ks, const uint16_t* vs, const int32_t* seq_lens, const art_params* a,
+                  float tau, float* o, int32_t* tiles, void* ws, void* stream) {
+  const int G = s->Hq / s->Hkv;
+  KernelInfo ki;
+  if (!pick_kernel(kind, mode, s->d, G, &ki)) return ART_ERR_UNSUPPORTED;
+  Params p;
+  memset(&p, 0, sizeof p);
+  p.emask = 0;
+  if (a) {
+    const art_status st = validate_params(a, s->d, ki.epc, &p.emask);
+    if (st != ART_OK) return st;
+    p.eps_scale = a->eps_scale;
+    p.eps_dir = a->eps_dir;
+    p.patience = a->patience;
+    p.n_probe = a->n_probe;
+    for (int i = 0; i < a->n_probe; ++i) p.lanes[i] = static_cast<int8_t>(a->probe_lanes[i]);
+  }
+  int sms = 0;
+  art_status st = prepare(ki.fn, &sms);
+  if (st != ART_OK) return st;
+  const int max_tiles = (s->L_max + s->tile - 1) / s->tile;
+  const int max_tiles_per_split = (max_tiles + s->num_splits - 1) / s->num_splits;
+  LaunchCfg cfg;
+  if (!choose_config(ki, s, sms, max_tiles_per_split, &cfg)) return ART_ERR_UNSUPPORTED;
+
+  const WsLayout w = ws_layout(s);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.ks = ks;
+  p.vs = vs;
+  p.seq_lens = seq_lens;
+  p.o = o;
+  p.tiles = tiles;
+  p.ws_status = reinterpret_cast<int32_t*>(wsb);
+  p.ws_tiles_read = reinterpret_cast<int32_t*>(wsb + w.tiles_read);
+  p.ws_used = reinterpret_cast<int32_t*>(wsb + w.used);
+  p.ws_partial = reinterpret_cast<float*>(wsb + w.partial);
+  p.B = s->B;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.L_max = s->L_max;
+  p.T = s->tile;
+  p.S = s->num_splits;
+  p.G = G;
+  p.C = cfg.C;
+  p.nstage = cfg.nstage;
+  p.qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(s->d)));
+  p.tau = tau;
+
+  cudaLaunchConfig_t lc;
+  memset(&lc, 0, sizeof lc);
+  cudaLaunchAttribute attr[1];
+  lc.gridDim = dim3(static_cast<unsigned>(s->B * s->Hkv * s->num_splits * cfg.C), 1, 1);
+  lc.blockDim = dim3(artk::NT, 1, 1);
+  lc.dynamicSmemBytes = cfg.smem;
+  lc.stream = static_cast<cudaStream_t>(stream);
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cfg.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, ki.fn, p) != cudaSuccess) return ART_ERR_CUDA;
+  if (s->num_splits > 1) {
+    const int heads = s->B * s->Hq;
+    const dim3 grid((heads + 7) / 8);
+    if (s->d == 64)
+      artk::art_combine_kernel<64><<<grid, 256, 0, lc.stream>>>(p.ws_partial, p.ws_used, o, tiles, heads,
+                                                                 s->num_splits);
+    else
+      artk::art_combine_kernel<128><<<grid, 256, 0, lc.stream>>>(p.ws_partial, p.ws_used, o, tiles, heads,
+                                                                  s->num_splits);
+    if (cudaGetLastError() != cudaSuccess) return ART_ERR_CUDA;
+  }
+  return ART_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t art_workspace_bytes(const art_shape* shape) {
+  if (!shape_ok(shape)) return 0;
+  return ws_layout(shape).total;
+}
+
+size_t art_workspace_tiles_read_offset(const art_shape* shape) {
+  if (!shape_ok(shape)) return 0;
+  return ws_layout(shape).tiles_read;
+}
+
+size_t art_workspace_split_tiles_offset(const art_shape* shape) {
+  if (!shape_ok(shape)) return 0;
+  return ws_layout(shape).used;
+}
+
+art_status art_decode_attn_full(const art_shape* shape, art_dtype dtype, const void* q, const void* k,
+                                const void* v, const int32_t* seq_lens, float* o, int32_t* tiles, void* ws,
+                                size_t ws_bytes, void* stream) {
+  art_status st = validate_common(shape, q, k, v, seq_lens, o, ws, ws_bytes);
+  if (st != ART_OK) return st;
+  if (dtype != ART_F32 && dtype != ART_BF16) return ART_ERR_INVALID_ARG;
+  const int kind = dtype == ART_F32 ? artk::KV_F32 : artk::KV_BF16;
+  return launch(kind, artk::MODE_FULL, shape, q, k, v, nullptr, nullptr, seq_lens, nullptr, 0.f, o, tiles, ws,
+                stream);
+}
+
+art_status art_decode_attn_terminate(const art_shape* shape, art_dtype dtype, const void* q, const void* k,
+                                     const void* v, const int32_t* seq_lens, const art_params* params, float* o,
+                                     int32_t* tiles, void* ws, size_t ws_bytes, void* stream) {
+  art_status st = validate_common(shape, q, k, v, seq_lens, o, ws, ws_bytes);
+  if (st != ART_OK) return st;
+  if (dtype != ART_F32 && dtype != ART_BF16) return ART_ERR_INVALID_ARG;
+  if (!params) return ART_ERR_INVALID_ARG;
+  const int kind = dtype == ART_F32 ? artk::KV_F32 : artk::KV_BF16;
+  return launch(kind, artk::MODE_ART, shape, q, k, v, nullptr, nullptr, seq_lens, params, 0.f, o, tiles, ws,
+                stream);
+}
+
+art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
+                                    const uint16_t* k_scale_f16, const int8_t* v_q, const uint16_t* v_scale_f16,
+                                    const int32_t* seq_lens, float tau, const art_params* params, float* o,
+                                    int32_t* tiles, void* ws, size_t ws_bytes, void* stream) {
+  art_status st = validate_common(shape, q_bf16, k_q, v_q, seq_lens, o, ws, ws_bytes);
+  if (st != ART_OK) return st;
+  if (!k_scale_f16 || !v_scale_f16) return ART_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_scale_f16) & 15u) || (reinterpret_cast<uintptr_t>(v_scale_f16) & 15u))
+    return ART_ERR_INVALID_ARG;
+  if (isnan(tau)) return ART_ERR_INVALID_ARG;
+  const long long scale_row_bytes = (shape->d / 32) * 2;
+  if ((1LL * shape->L_max * scale_row_bytes) % 16 != 0) return ART_ERR_UNSUPPORTED;
+  const int mode = params ? artk::MODE_SKIP_ART : artk::MODE_SKIP;
+  return launch(artk::KV_Q8, mode, shape, q_bf16, k_q, v_q, k_scale_f16, v_scale_f16, seq_lens, params, tau, o,
+                tiles, ws, stream);
+}
+
+art_status art_read_device_status(void* ws, void* stream) {
+  if (!ws) return ART_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ART_ERR_CUDA;
+  if (cudaMemcpyAsync(&h, ws, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return ART_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof h, s) != cudaSuccess) return ART_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ART_ERR_CUDA;
+  if (h & artk::kStatusSeqLen) return ART_ERR_SEQLEN;
+  if (h & artk::kStatusTimeout) return ART_ERR_TIMEOUT;
+  return ART_OK;
+}
+
+const char* art_status_string(art_status status) {
+  switch (status) {
+    case ART_OK: return "ART_OK";
+    case ART_ERR_INVALID_ARG: return "ART_ERR_INVALID_ARG";
+    case ART_ERR_UNSUPPORTED: return "ART_ERR_UNSUPPORTED";
+    case ART_ERR_WORKSPACE: return "ART_ERR_WORKSPACE";
+    case ART_ERR_CUDA: return "ART_ERR_CUDA";
+    case ART_ERR_TIMEOUT: return "ART_ERR_TIMEOUT";
+    case ART_ERR_SEQLEN: return "ART_ERR_SEQLEN";
+  }
+  return "ART_ERR_UNKNOWN";
+}
+
+}  // extern "C"

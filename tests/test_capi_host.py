@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+symbol include/art_decode.h declares, sizes its workspace, and rejects invalid
+arguments synchronously without touching the device (fake, never-dereferenced
+pointer values are passed)."""
+import ctypes
+import re
+import os
+
+import pytest
+
+from kv_cache_early_split_b200 import build, capi
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "art_decode.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return capi.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(art_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 8
+    assert sorted(capi.EXPORTS) == names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(0, -7, -1):
+        assert capi.art_status_string(code).startswith("ART_")
+    assert capi.art_status_string(-99) == "ART_ERR_UNKNOWN"
+
+
+def shape(**kw):
+    d = dict(B=4, Hq=32, Hkv=8, d=128, L_max=32768, tile=64, num_splits=1)
+    d.update(kw)
+    return capi.art_shape(**d)
+
+
+def test_workspace_sizes(L):
+    s = shape()
+    ws = capi.art_workspace_bytes(s)
+    off_r = capi.art_workspace_tiles_read_offset(s)
+    off_u = capi.art_workspace_split_tiles_offset(s)
+    assert off_r >= 4 and off_r % 16 == 0
+    assert off_u >= off_r + 4 * 4 * 8
+    assert ws >= off_u + 4 * 4 * 32 + 4 * 4 * 32 * 130
+    s8 = shape(num_splits=8)
+    assert capi.art_workspace_bytes(s8) > ws
+    assert capi.art_workspace_bytes(shape(B=0)) == 0
+    assert capi.art_workspace_bytes(shape(num_splits=0)) == 0
+
+
+A = 0x100000  # fake 16-byte aligned device addresses (never dereferenced)
+
+
+def full(s, **kw):
+    args = dict(dtype=capi.ART_BF16, q=A, k=A * 2, v=A * 3, seq=A * 4, o=A * 5, tiles=A * 6, ws=A * 7,
+                ws_bytes=capi.art_workspace_bytes(s) if capi.art_workspace_bytes(s) else 1 << 20)
+    args.update(kw)
+    return capi.art_decode_attn_full(s, args["dtype"], args["q"], args["k"], args["v"], args["seq"], args["o"],
+                                     args["tiles"], args["ws"], args["ws_bytes"], None)
+
+
+def term(s, params, **kw):
+    wsb = capi.art_workspace_bytes(s) or (1 << 20)
+    return capi.art_decode_attn_terminate(s, kw.get("dtype", capi.ART_BF16), A, A * 2, A * 3, A * 4, params, A * 5,
+                                          A * 6, A * 7, kw.get("ws_bytes", wsb), None)
+
+
+def q8(s, params=None, tau=1e-6, **kw):
+    wsb = capi.art_workspace_bytes(s) or (1 << 20)
+    return capi.art_decode_attn_q8_skipv(s, A, A * 2, kw.get("ks", A * 8), A * 3, kw.get("vs", A * 9), A * 4, tau,
+                                         params, A * 5, A * 6, A * 7, wsb, None)
+
+
+def test_invalid_arguments_full(L):
+    s = shape()
+    assert full(s, q=None) == capi.ART_ERR_INVALID_ARG
+    assert full(s, o=None) == capi.ART_ERR_INVALID_ARG
+    assert full(s, seq=None) == capi.ART_ERR_INVALID_ARG
+    assert full(s, q=A + 4) == capi.ART_ERR_INVALID_ARG  # misaligned
+    assert full(s, dtype=7) == capi.ART_ERR_INVALID_ARG
+    assert full(s, ws=None) == capi.ART_ERR_WORKSPACE
+    assert full(s, ws_bytes=capi.art_workspace_bytes(s) - 1) == capi.ART_ERR_WORKSPACE
+    assert full(shape(Hq=30)) == capi.ART_ERR_INVALID_ARG  # Hq % Hkv
+    assert full(shape(B=0)) == capi.ART_ERR_INVALID_ARG
+    assert full(shape(d=96)) == capi.ART_ERR_UNSUPPORTED
+    assert full(shape(tile=48)) == capi.ART_ERR_UNSUPPORTED
+    assert full(shape(Hq=128, Hkv=8)) == capi.ART_ERR_UNSUPPORTED  # 16 query heads per kv head
+
+
+def test_invalid_arguments_terminate(L):
+    s = shape()
+    ok = capi.make_params(1e-3, 1e-4, 1, list(range(0, 128, 8)))
+    assert term(s, None) == capi.ART_ERR_INVALID_ARG
+    assert term(s, capi.make_params(1e-3, 1e-4, 0, [0])) == capi.ART_ERR_INVALID_ARG  # patience 0
+    assert term(s, capi.make_params(1e-3, 1e-4, 1, [])) == capi.ART_ERR_INVALID_ARG  # no lanes
+    assert term(s, capi.make_params(1e-3, 1e-4, 1, list(range(33)))) == capi.ART_ERR_INVALID_ARG
+    assert term(s, capi.make_params(1e-3, 1e-4, 1, [0, 128])) == capi.ART_ERR_INVALID_ARG  # lane >= d
+    assert term(s, capi.make_params(1e-3, 1e-4, 1, [-1])) == capi.ART_ERR_INVALID_ARG
+    assert term(s, capi.make_params(1e-3, 1e-4, 1, [3, 3])) == capi.ART_ERR_INVALID_ARG  # duplicate
+    assert term(shape(d=64), capi.make_params(1e-3, 1e-4, 1, [64])) == capi.ART_ERR_INVALID_ARG
+    assert term(s, ok, ws_bytes=16) == capi.ART_ERR_WORKSPACE
+
+
+def test_invalid_arguments_q8(L):
+    s = shape()
+    assert q8(s, ks=None) == capi.ART_ERR_INVALID_ARG
+    assert q8(s, vs=A + 2) == capi.ART_ERR_INVALID_ARG
+    assert q8(s, tau=float("nan")) == capi.ART_ERR_INVALID_ARG
+    assert q8(shape(L_max=32767)) == capi.ART_ERR_UNSUPPORTED  # scale rows not 16-byte granular
+    assert q8(s, params=capi.make_params(1e-3, 1e-4, 1, [200])) == capi.ART_ERR_INVALID_ARG
+
+
+def test_read_status_rejects_null(L):
+    assert capi.art_read_device_status(None, None) == capi.ART_ERR_INVALID_ARG

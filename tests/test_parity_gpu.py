@@ -1,0 +1,194 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, element
+by element, on seeded synthetic inputs that span several tiles and a ragged
+tail, for every entry point and mode, plus edge cases.
+
+Bars: outputs within 1e-5 (fp32 inputs) or 2e-3 (bf16 / q8 inputs) max-abs of
+the oracle run to the GPU's own per-split stop tiles; tiles consumed equal to
+the oracle's unless an oracle metric lies within 1e-4 of its threshold (see
+tests/helpers.py).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import kv_cache_early_split_b200 as K  # noqa: E402
+from kv_cache_early_split_b200 import capi  # noqa: E402
+from kv_cache_early_split_b200 import inputs as I  # noqa: E402
+from helpers import TOL, check_tiles, oracle_run  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu(w, mode, *, tile=None, S=None, art=None, tau=None, stream=None):
+    dp = K.upload(w, num_splits=S, tile=tile)
+    K.decode(dp, mode, art=art, tau=tau, stream=stream)
+    st = K.device_status(dp, stream=stream)
+    return dict(
+        o=dp.o.cpu().numpy(), tiles=dp.tiles.cpu().numpy(), used=dp.split_tiles().cpu().numpy(),
+        read=dp.tiles_read().cpu().numpy(), status=st, dp=dp,
+    )
+
+
+def n_tiles(w, tile):
+    return -(-w.seq_lens.astype(np.int64) // tile)
+
+
+def check_full(w, mode="full", tile=None, S=None, tau=None):
+    tile = tile or w.tile
+    S = S or w.num_splits
+    g = gpu(w, mode, tile=tile, S=S, tau=tau)
+    assert g["status"] == capi.ART_OK
+    r = oracle_run(w, mode, tile=tile, num_splits=S, tau=tau)
+    err = np.max(np.abs(g["o"] - r.o))
+    assert err <= TOL[w.kind], f"max abs err {err}"
+    n = n_tiles(w, tile)
+    assert np.array_equal(g["tiles"], np.repeat(n[:, None], w.Hq, axis=1))
+    assert np.array_equal(g["used"], r.used)
+    assert np.array_equal(g["read"].sum(axis=2), np.repeat(n[:, None], w.Hkv, axis=1))
+    return g
+
+
+def check_art(w, mode="art", tile=None, S=None, art=None, tau=None):
+    tile = tile or w.tile
+    S = S or w.num_splits
+    a = art or w.art
+    g = gpu(w, mode, tile=tile, S=S, art=a, tau=tau)
+    assert g["status"] == capi.ART_OK
+    ref = oracle_run(w, mode, tile=tile, num_splits=S, art=a, tau=tau, metrics=True)
+    exact, amb = check_tiles(w, ref.metrics, g["used"], a, tile, S)
+    assert np.array_equal(g["used"].sum(axis=2), g["tiles"])
+    forced = oracle_run(w, "q8" if mode == "q8_art" else "full", tile=tile, num_splits=S, tau=tau,
+                        forced_used=g["used"])
+    err = np.max(np.abs(g["o"] - forced.o))
+    assert err <= TOL[w.kind], f"max abs err {err}"
+    # KV tiles read per (b, kvh, split): at least what the slowest head consumed, at most the split
+    n = n_tiles(w, tile)
+    G = w.G
+    for b in range(w.B):
+        for s in range(S):
+            ln = ((s + 1) * n[b]) // S - (s * n[b]) // S
+            for h in range(w.Hkv):
+                need = g["used"][b, h * G:(h + 1) * G, s].max()
+                assert need <= g["read"][b, h, s] <= ln
+    return g, exact, amb
+
+
+SMALL = [
+    # kind, d, Hq, Hkv, B, L_max, lens, tile, S
+    ("f32", 64, 1, 1, 1, 1000, [1000], 64, 1),
+    ("f32", 128, 8, 2, 2, 700, [700, 333], 32, 2),
+    ("bf16", 128, 8, 2, 2, 2000, [2000, 777], 64, 1),
+    ("bf16", 64, 8, 1, 3, 500, [500, 17, 250], 16, 1),
+    ("bf16", 128, 4, 2, 2, 3000, [2999, 1290], 128, 3),
+    ("bf16", 128, 6, 2, 2, 900, [900, 45], 32, 1),
+    ("bf16", 128, 2, 1, 1, 5000, [4999], 64, 1),
+    ("bf16", 64, 16, 2, 2, 1200, [1200, 1], 64, 2),
+    ("bf16", 64, 4, 4, 1, 2048, [2048], 256, 1),
+    ("q8", 128, 8, 2, 2, 2048, [2048, 1001], 64, 1),
+    ("q8", 64, 4, 1, 1, 1500, [1499], 32, 2),
+]
+
+
+def make_small(kind, d, Hq, Hkv, B, L_max, lens, tile, S, seed=0, **kw):
+    return I.make_workload(kind=kind, B=B, Hq=Hq, Hkv=Hkv, d=d, L_max=L_max, tile=tile, num_splits=S,
+                           seq_lens=lens, seed=1000 + seed, **kw)
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}-d{c[1]}-g{c[2] // c[3]}-T{c[7]}-S{c[8]}")
+def test_full_small(case):
+    w = make_small(*case)
+    if w.kind == "q8":
+        check_full(w, "q8", tau=0.0)
+        check_full(w, "q8", tau=1e-6)
+    else:
+        check_full(w)
+
+
+ART_SETTINGS = [
+    dict(eps_scale=2e-2, eps_dir=5e-3, patience=1),
+    dict(eps_scale=5e-2, eps_dir=2e-2, patience=3),
+    dict(eps_scale=float("inf"), eps_dir=float("inf"), patience=2),
+    dict(eps_scale=0.0, eps_dir=0.0, patience=1),
+]
+
+
+@pytest.mark.parametrize("setting", range(len(ART_SETTINGS)))
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"{c[0]}-d{c[1]}-g{c[2] // c[3]}-T{c[7]}-S{c[8]}")
+def test_art_small(case, setting):
+    w = make_small(*case, seed=setting, sink=6.0)
+    a = dict(ART_SETTINGS[setting], lanes=I.probe_lanes_strided(w.d, 16 if w.d == 128 else 8))
+    mode = "q8_art" if w.kind == "q8" else "art"
+    g, exact, amb = check_art(w, mode, art=a, tau=(1e-6 if w.kind == "q8" else None))
+    n = n_tiles(w, w.tile)
+    S = w.num_splits
+    if a["eps_scale"] == float("inf"):
+        for b in range(w.B):
+            lens = [((s + 1) * n[b]) // S - (s * n[b]) // S for s in range(S)]
+            assert np.array_equal(g["used"][b], np.tile([min(a["patience"], x) for x in lens], (w.Hq, 1)))
+    if a["eps_scale"] == 0.0:
+        assert np.array_equal(g["tiles"], np.repeat(n[:, None], w.Hq, axis=1))
+
+
+def test_art_stops_somewhere_midway():
+    """A case where the rule fires inside the sequence for most heads (not at the ends)."""
+    w = make_small("bf16", 128, 8, 2, 2, 4096, [4096, 3000], 64, 1, sink=8.0)
+    a = dict(eps_scale=1e-2, eps_dir=2e-3, patience=2, lanes=I.probe_lanes_strided(128, 16))
+    g, exact, amb = check_art(w, art=a)
+    n = n_tiles(w, 64)
+    mid = (g["tiles"] > 2) & (g["tiles"] < n[:, None])
+    assert mid.mean() > 0.5, g["tiles"]
+
+
+def test_vskip_actually_skips_and_matches():
+    """Skewed logits so that many rows fall below tau; GPU matches the oracle's skip rule."""
+    w = I.make_workload(kind="q8", B=1, Hq=4, Hkv=1, d=128, L_max=2048, tile=64, seed=5, gumbel_scale=6.0,
+                        q_scale=2.0)
+    for tau in (1e-3, 1e-6, 0.0, 2.0):
+        check_full(w, "q8", tau=tau)
+    full = oracle_run(w, "q8", tau=0.0)
+    skip = oracle_run(w, "q8", tau=1e-3)
+    assert np.max(np.abs(full.o - skip.o)) > 1e-6  # the skip changed something measurable
+
+
+def test_empty_splits_and_tiny_lengths():
+    w = make_small("bf16", 128, 8, 2, 3, 300, [1, 63, 300], 64, 8)
+    check_full(w)
+    check_art(w, art=dict(eps_scale=1e-2, eps_dir=1e-3, patience=1, lanes=[0, 5, 77]))
+
+
+def test_invalid_seq_len_sets_status_and_nan():
+    w = make_small("bf16", 128, 8, 2, 2, 256, [256, 100], 64, 1)
+    w.seq_lens[1] = 300  # > L_max
+    dp = K.upload(w)
+    K.decode(dp, "full")
+    assert K.device_status(dp) == capi.ART_ERR_SEQLEN
+    assert K.device_status(dp) == capi.ART_OK  # cleared on read
+    o = dp.o.cpu().numpy()
+    assert np.all(np.isnan(o[1])) and not np.any(np.isnan(o[0]))
+    assert np.all(dp.tiles.cpu().numpy()[1] == 0)
+    w.seq_lens[1] = 0
+    dp = K.upload(w)
+    K.decode(dp, "art")
+    assert K.device_status(dp) == capi.ART_ERR_SEQLEN
+
+
+def test_deterministic_and_stream():
+    w = make_small("bf16", 128, 8, 2, 2, 3000, [3000, 1234], 64, 2, sink=6.0)
+    dp = K.upload(w)
+    s = torch.cuda.Stream()
+    outs = []
+    for mode in ("full", "art", "full", "art"):
+        with torch.cuda.stream(s):
+            K.decode(dp, mode, stream=s.cuda_stream)
+        s.synchronize()
+        outs.append((dp.o.cpu().numpy().copy(), dp.tiles.cpu().numpy().copy()))
+    assert np.array_equal(outs[0][0], outs[2][0]) and np.array_equal(outs[1][0], outs[3][0])
+    assert np.array_equal(outs[1][1], outs[3][1])
+
+
+def test_unsupported_tile_returns_error():
+    w = make_small("bf16", 128, 4, 1, 1, 1024, [1024], 256, 1)
+    dp = K.upload(w)
+    rc = K.decode(dp, "full", check=False)
+    assert rc == capi.ART_ERR_UNSUPPORTED
