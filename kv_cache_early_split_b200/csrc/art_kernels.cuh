@@ -716,6 +716,7 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
   }
 
   // ---- reduce the owned numerators over the position subsets of this CTA
+  // (warp shuffles, then warps add in a fixed order: the result is deterministic)
 #pragma unroll
   for (int g = 0; g < GP; ++g) {
 #pragma unroll
@@ -723,8 +724,18 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
       float x = acc_o[g][e];
 #pragma unroll
       for (int off = CH; off < 32; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-      if (lane < CH && g < G) atomicAdd(&s_red[g * D + pv_c * EPC + e], x);
+      acc_o[g][e] = x;
     }
+  }
+  for (int w = 0; w < NW; ++w) {
+    if (warp == w && lane < CH) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g)
+#pragma unroll
+        for (int e = 0; e < EPC; ++e)
+          if (g < G) s_red[g * D + pv_c * EPC + e] += acc_o[g][e];
+    }
+    __syncthreads();
   }
   if (tid == 0) {
 #pragma unroll
