@@ -129,6 +129,33 @@ art_status art_decode_attn_terminate(const art_shape* shape, art_dtype dtype, co
                                      const art_params* params, float* o, int32_t* tiles, void* ws,
                                      size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of art_decode_attn_terminate, for callers that
+ * cannot allocate device memory: a host framework that hands a plugin or
+ * custom op only its input and output buffers (no workspace argument, no
+ * allocator), or code that must not call cudaMalloc on the hot path.  The
+ * pages have no counterpart to this entry point; it exists only for those
+ * callers.  Same arguments and results as art_decode_attn_terminate, minus
+ * ws / ws_bytes: the workspace is a 4 MiB array inside the library
+ * (a file-scope __device__ variable, held on every GPU that loads the
+ * library until the process exits).
+ *   - Shapes whose art_workspace_bytes() exceeds 4 MiB (4194304 bytes) are
+ *     rejected with ART_ERR_WORKSPACE before anything is enqueued.
+ *   - Calls no cudaMalloc / cudaFree and no allocating library routine.  The
+ *     first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture on that device.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind.  No word of it has to start at zero (the kernels write all they
+ *     read), so nothing is cleared between calls.  Calls whose executions
+ *     overlap on the GPU (different streams, or concurrent host threads) race
+ *     on the array: serialise them.
+ *   - Device-side errors (a seq_len outside [1, L_max]) show as NaN outputs
+ *     and 0 tiles for that sequence; there is no status to read back. */
+art_status art_decode_attn_terminate_noalloc(const art_shape* shape, art_dtype dtype, const void* q,
+                                             const void* k, const void* v, const int32_t* seq_lens,
+                                             const art_params* params, float* o, int32_t* tiles,
+                                             void* stream);
+
 /* Decode attention over an int8 KV cache in 32-element blocks with one fp16
  * scale each (q8_0 style; value = code * scale), bf16 query.  V rows whose
  * weight exp(s_j - m') is below tau are neither dequantised nor accumulated

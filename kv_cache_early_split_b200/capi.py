@@ -30,6 +30,7 @@ EXPORTS = (
     "art_workspace_split_tiles_offset",
     "art_decode_attn_full",
     "art_decode_attn_terminate",
+    "art_decode_attn_terminate_noalloc",
     "art_decode_attn_q8_skipv",
     "art_read_device_status",
     "art_status_string",
@@ -86,6 +87,9 @@ def lib() -> ctypes.CDLL:
             L.art_decode_attn_terminate.restype = ctypes.c_int
             L.art_decode_attn_terminate.argtypes = [
                 _SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, ctypes.c_size_t, _P]
+            L.art_decode_attn_terminate_noalloc.restype = ctypes.c_int
+            L.art_decode_attn_terminate_noalloc.argtypes = [
+                _SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P]
             L.art_decode_attn_q8_skipv.restype = ctypes.c_int
             L.art_decode_attn_q8_skipv.argtypes = [
                 _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, _P]
@@ -120,6 +124,12 @@ def art_decode_attn_full(shape, dtype, q, k, v, seq_lens, o, tiles, ws, ws_bytes
 def art_decode_attn_terminate(shape, dtype, q, k, v, seq_lens, params, o, tiles, ws, ws_bytes, stream) -> int:
     return int(lib().art_decode_attn_terminate(
         ctypes.byref(shape), dtype, q, k, v, seq_lens, _ref(params), o, tiles, ws, ws_bytes, stream))
+
+
+def art_decode_attn_terminate_noalloc(shape, dtype, q, k, v, seq_lens, params, o, tiles, stream) -> int:
+    """Allocation-free art_decode_attn_terminate (library-held 4 MiB device scratch; see the header)."""
+    return int(lib().art_decode_attn_terminate_noalloc(
+        ctypes.byref(shape), dtype, q, k, v, seq_lens, _ref(params), o, tiles, stream))
 
 
 def art_decode_attn_q8_skipv(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, params, o, tiles,

@@ -320,6 +320,32 @@ art_status launch(int kind, int mode, const art_shape* s, const void* q, const v
   return ART_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch memory for art_decode_attn_terminate_noalloc.  The array is a
+// file-scope device variable: every GPU that loads this library holds it until
+// the process exits.  Host code may not pass the symbol itself to a kernel (on
+// the host it only names a stand-in); its device address is looked up once per
+// device with cudaGetSymbolAddress while that device is current.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device (set up on first use).
+art_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ART_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ART_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ART_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -360,6 +386,24 @@ art_status art_decode_attn_terminate(const art_shape* shape, art_dtype dtype, co
   const int kind = dtype == ART_F32 ? artk::KV_F32 : artk::KV_BF16;
   return launch(kind, artk::MODE_ART, shape, q, k, v, nullptr, nullptr, seq_lens, params, 0.f, o, tiles, ws,
                 stream);
+}
+
+// Allocation-free variant of art_decode_attn_terminate: the workspace is the
+// library's own device array (g_noalloc_scratch) instead of caller memory.
+// Nothing in that array has to start at zero: the kernels write every word
+// they later read (the status word is only ever OR-ed into, and this entry
+// point has no way to read it back), so no clearing is enqueued.
+art_status art_decode_attn_terminate_noalloc(const art_shape* shape, art_dtype dtype, const void* q,
+                                             const void* k, const void* v, const int32_t* seq_lens,
+                                             const art_params* params, float* o, int32_t* tiles,
+                                             void* stream) {
+  if (!shape_ok(shape)) return ART_ERR_INVALID_ARG;
+  if (art_workspace_bytes(shape) > kNoAllocScratchBytes) return ART_ERR_WORKSPACE;
+  void* scratch = nullptr;  // looking the address up enqueues no work
+  const art_status sst = noalloc_scratch(&scratch);
+  if (sst != ART_OK) return sst;
+  return art_decode_attn_terminate(shape, dtype, q, k, v, seq_lens, params, o, tiles, scratch,
+                                   kNoAllocScratchBytes, stream);
 }
 
 art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
