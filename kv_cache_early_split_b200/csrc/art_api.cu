@@ -10,6 +10,7 @@
 
 #include "art_decode.h"
 #include "art_kernels.cuh"
+#include "art_tc.cuh"
 
 namespace {
 
@@ -207,6 +208,148 @@ bool choose_config(const KernelInfo& ki, const art_shape* s, int sms, int max_ti
   return true;
 }
 
+art_status validate_params(const art_params* a, int d, int epc, int* emask);
+
+// ---------------------------------------------------------------------------
+// Tensor-core path: bf16 K/V, d = 128, tile 64 or 128, up to 8 heads per kv head.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::mutex g_enc_mu;
+EncodeTiledFn g_encode = nullptr;
+
+EncodeTiledFn encode_fn() {
+  std::lock_guard<std::mutex> lock(g_enc_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess || !fn)
+      return nullptr;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+bool tc_eligible(int kind, int mode, const art_shape* s) {
+  const int G = s->Hq / s->Hkv;
+  return kind == artk::KV_BF16 && (mode == artk::MODE_FULL || mode == artk::MODE_ART) && s->d == 128 &&
+         (s->tile == 64 || s->tile == 128) && G >= 1 && G <= 8;
+}
+
+// K/V [B*Hkv][L_max][128] bf16 as a 3-D tensor map; box = 64 d x 128 positions, 128-byte swizzle.
+bool make_kv_map(CUtensorMap* m, const void* base, const art_shape* s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(s->L_max), static_cast<cuuint64_t>(s->B) * s->Hkv};
+  const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(s->L_max) * 256};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+using TcFn = void (*)(artk::tc::TcParams);
+
+template <int MODE>
+TcFn tc_pick(int G) {
+  if (G == 1) return &artk::tc::art_decode_tc_kernel<1, MODE>;
+  if (G == 2) return &artk::tc::art_decode_tc_kernel<2, MODE>;
+  if (G <= 4) return &artk::tc::art_decode_tc_kernel<4, MODE>;
+  return &artk::tc::art_decode_tc_kernel<8, MODE>;
+}
+
+art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k, const void* v,
+                     const int32_t* seq_lens, const art_params* a, float* o, int32_t* tiles, void* ws,
+                     void* stream) {
+  const int G = s->Hq / s->Hkv;
+  const TcFn fn = (mode == artk::MODE_ART) ? tc_pick<artk::MODE_ART>(G) : tc_pick<artk::MODE_FULL>(G);
+  artk::tc::TcParams p;
+  memset(&p, 0, sizeof p);
+  if (a) {
+    int emask = 0;
+    const art_status st = validate_params(a, s->d, 8, &emask);
+    if (st != ART_OK) return st;
+    p.eps_scale = a->eps_scale;
+    p.eps_dir = a->eps_dir;
+    p.patience = a->patience;
+    p.n_probe = a->n_probe;
+    for (int i = 0; i < a->n_probe; ++i) p.lanes[i] = static_cast<int8_t>(a->probe_lanes[i]);
+  }
+  if (!make_kv_map(&p.tmK, k, s) || !make_kv_map(&p.tmV, v, s)) return ART_ERR_CUDA;
+  int sms = 0;
+  art_status st = prepare(reinterpret_cast<KernelFn>(fn), &sms);
+  if (st != ART_OK) return st;
+  // one CTA per SM; cluster size C: power of two, units*C <= SMs, C*tiles_per_block <= 32 (one rule lane
+  // per tile of a round), and no more CTAs than 128-position blocks in a split.
+  const int units = s->B * s->Hkv * s->num_splits;
+  const int kt = 128 / s->tile;
+  const long long max_tiles = (s->L_max + s->tile - 1) / s->tile;
+  const long long max_blocks = ((max_tiles + s->num_splits - 1) / s->num_splits * s->tile + 127) / 128;
+  int C = 1;
+  while (C < artk::CMAX && 1LL * units * (2 * C) <= sms && 2 * C * kt <= 32 && 2 * C <= max_blocks) C *= 2;
+  while (C > 1) {
+    cudaLaunchConfig_t lc;
+    memset(&lc, 0, sizeof lc);
+    cudaLaunchAttribute attr[1];
+    lc.gridDim = dim3(static_cast<unsigned>(units * C), 1, 1);
+    lc.blockDim = dim3(artk::tc::NTHR, 1, 1);
+    lc.dynamicSmemBytes = artk::tc::SMEM_BYTES;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int nclusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, fn, &lc) == cudaSuccess && nclusters > 0) break;
+    cudaGetLastError();
+    C /= 2;
+  }
+  const WsLayout w = ws_layout(s);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  p.q = static_cast<const uint16_t*>(q);
+  p.seq_lens = seq_lens;
+  p.o = o;
+  p.tiles = tiles;
+  p.ws_status = reinterpret_cast<int32_t*>(wsb);
+  p.ws_tiles_read = reinterpret_cast<int32_t*>(wsb + w.tiles_read);
+  p.ws_used = reinterpret_cast<int32_t*>(wsb + w.used);
+  p.ws_partial = reinterpret_cast<float*>(wsb + w.partial);
+  p.B = s->B;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.L_max = s->L_max;
+  p.T = s->tile;
+  p.S = s->num_splits;
+  p.G = G;
+  p.C = C;
+  p.qscale = static_cast<float>(1.4426950408889634 / sqrt(128.0));
+
+  cudaLaunchConfig_t lc;
+  memset(&lc, 0, sizeof lc);
+  cudaLaunchAttribute attr[1];
+  lc.gridDim = dim3(static_cast<unsigned>(units * C), 1, 1);
+  lc.blockDim = dim3(artk::tc::NTHR, 1, 1);
+  lc.dynamicSmemBytes = artk::tc::SMEM_BYTES;
+  lc.stream = static_cast<cudaStream_t>(stream);
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, fn, p) != cudaSuccess) return ART_ERR_CUDA;
+  if (s->num_splits > 1) {
+    const int heads = s->B * s->Hq;
+    artk::art_combine_kernel<128><<<(heads + 7) / 8, 256, 0, lc.stream>>>(p.ws_partial, p.ws_used, o, tiles, heads,
+                                                                           s->num_splits);
+    if (cudaGetLastError() != cudaSuccess) return ART_ERR_CUDA;
+  }
+  return ART_OK;
+}
+
 art_status validate_common(const art_shape* s, const void* q, const void* k, const void* v,
                            const int32_t* seq_lens, const float* o, void* ws, size_t ws_bytes) {
   if (!shape_ok(s)) return ART_ERR_INVALID_ARG;
@@ -244,6 +387,7 @@ art_status launch(int kind, int mode, const art_shape* s, const void* q, const v
                   const uint16_t* ks, const uint16_t* vs, const int32_t* seq_lens, const art_params* a,
                   float tau, float* o, int32_t* tiles, void* ws, void* stream) {
   const int G = s->Hq / s->Hkv;
+  if (tc_eligible(kind, mode, s)) return launch_tc(mode, s, q, k, v, seq_lens, a, o, tiles, ws, stream);
   KernelInfo ki;
   if (!pick_kernel(kind, mode, s->d, G, &ki)) return ART_ERR_UNSUPPORTED;
   Params p;

@@ -1,0 +1,752 @@
+// art_tc.cuh -- tensor-core (tcgen05 + TMA) decode kernel for bf16 K/V, d = 128,
+// tile 64 or 128, up to 8 query heads per kv head; full attention and ART.
+//
+// Same computation as art_decode_kernel (web pages, cited by title and section):
+//   "Resumen Tecnico: ART" (gist.science, arXiv 2606.00024) S2.1 tile-wise online
+//   softmax; S2.2 probe of the normalised partial output, d_scale / d_direction,
+//   both below threshold; S2.3 patience; S2.4 tile 0 first.
+//
+// The GQA group's G query heads against a K/V block of 128 positions are two
+// real dense contractions, so they run on the 5th-generation tensor cores:
+//   S^T[128 pos x 16]  = K_blk[128 x 128 d] . Q^T      (A: K, K-major, 128-byte swizzle)
+//   O_t^T[128 d x 16]  = V_t^T[128 d x T]  . P_t^T      (A: V, MN-major, 128-byte swizzle)
+// with accumulators in tensor memory.  P is split into bf16 hi + lo parts
+// (columns 0..7 and 8..15) so that the weights keep ~16 bits of precision.
+//
+// Warp roles (224 threads, one CTA per SM):
+//   warp 0      TMA producer: K/V blocks (4 tiled 3-D TMA loads, 64 KiB) into a 3-deep ring
+//   warp 1      MMA issuer (one lane) and tensor-memory owner
+//   warps 2..5  epilogue: scores -> per-tile max / weights -> P^T in smem; O readback
+//               (thread = d row) -> online merge in registers; ART publication
+//   warp 6      ART controller: per round, reads all CTAs' publications through
+//               distributed shared memory and replays the rule in tile order
+// Blocks are dealt round-robin over the cluster exactly as in art_decode_kernel,
+// and the ART exchange runs one round behind the streaming pipeline.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "art_device.cuh"
+#include "art_kernels.cuh"
+
+namespace artk {
+namespace tc {
+
+constexpr int BLK = 128;  // positions per block (= MMA M for the scores)
+constexpr int D = 128;
+constexpr int NSTG = 3;
+constexpr int NWARP = 7;
+constexpr int NTHR = NWARP * 32;
+constexpr int KT_MAX = 2;  // tiles per block (tile 64)
+constexpr int STAGE_BYTES = 4 * 16384;
+constexpr uint32_t TMEM_COLS = 128;
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_CTL = 6;
+constexpr int BAR_EPI = 1;  // named barrier of the 128 epilogue threads
+
+struct TcParams {
+  CUtensorMap tmK;  // 64-byte aligned (first members)
+  CUtensorMap tmV;
+  const uint16_t* q;
+  const int32_t* seq_lens;
+  float* o;
+  int32_t* tiles;
+  float* ws_partial;
+  int32_t* ws_used;
+  int32_t* ws_tiles_read;
+  int32_t* ws_status;
+  int B, Hq, Hkv, L_max, T, S, G, C, n_probe, patience;
+  float qscale, eps_scale, eps_dir;
+  int8_t lanes[PMAX];
+};
+
+// ---- shared-memory map (byte offsets from a 1024-aligned base)
+constexpr uint32_t OFF_STAGE = 0;
+constexpr uint32_t OFF_Q = NSTG * STAGE_BYTES;        // 2 halves x 2 KiB
+constexpr uint32_t OFF_P = OFF_Q + 4096;              // 2 buffers x 4 KiB
+constexpr uint32_t OFF_BAR = OFF_P + 8192;            // mbarriers
+enum : int {
+  B_FULL = 0, B_EMPTY = B_FULL + NSTG, B_SFULL = B_EMPTY + NSTG, B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2,
+  B_OFULL = B_PFULL + 2, B_OFREE = B_OFULL + 2, B_XFULL = B_OFREE + 2, B_XFREE = B_XFULL + 2, B_DEC = B_XFREE + 2,
+  B_DRAIN = B_DEC + 2, B_COUNT = B_DRAIN + 1
+};
+constexpr uint32_t OFF_WRED = OFF_BAR + 256;                          // [2][4][GMAX] per-warp maxima
+constexpr uint32_t OFF_WSUM = OFF_WRED + 4 * 2 * 4 * GMAX;            // [2][4][GMAX] per-warp sums
+constexpr uint32_t OFF_TST = OFF_WSUM + 4 * 2 * 4 * GMAX;             // [2][KT][GMAX][2] tile (m, l)
+constexpr uint32_t OFF_PUB = OFF_TST + 4 * 2 * KT_MAX * GMAX * 2;     // [2][KT][GMAX][2+PMAX]
+constexpr uint32_t PUB_SLOT = 4 * KT_MAX * GMAX * (2 + PMAX);
+constexpr uint32_t OFF_DEC = OFF_PUB + 2 * PUB_SLOT;                  // [2][GMAX] int
+constexpr uint32_t OFF_CTL = OFF_DEC + 4 * 2 * GMAX;                  // [16] int
+constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;                         // [GMAX][RF_SIZE] float
+constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;              // [GMAX][RI_SIZE] int
+constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;             // [D] int8
+constexpr uint32_t SMEM_USED = OFF_L2P + D;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+// final reduction (aliases stage 0 after the pipeline has drained)
+constexpr uint32_t OFF_RED = 0;  // [GMAX][D] numerators, then [GMAX] m, [GMAX] l, [4] ints
+enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, CTL_TREAD, CTL_TMEM };
+
+__device__ __forceinline__ uint32_t s_col(int b) { return 16u * b; }
+__device__ __forceinline__ uint32_t o_col(int b, int i) { return 32u + 32u * b + 16u * i; }
+
+// Bounded wait that also gives up when the CTA aborted (a timeout elsewhere) or,
+// with watch_exit, when the ART controller ended the run.  Returns true when the
+// phase completed.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* ctl, bool watch_exit,
+                                           int32_t* status, bool cluster_scope = false) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 32; ++i) {
+      const bool ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+      if (ok) return true;
+    }
+    if (ctl[CTL_ABORT]) return false;
+    if (watch_exit && ctl[CTL_EXIT]) {
+      __threadfence_block();
+      return cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    }
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(status, kStatusTimeout);
+      ctl[CTL_ABORT] = 1;
+      return false;
+    }
+  }
+}
+
+template <int GP, int MODE>
+__global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
+  constexpr bool ART = (MODE == MODE_ART);
+  static_assert(GP >= 1 && GP <= 8, "up to 8 query heads per kv head");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int C = p.C, T = p.T, G = p.G, P = p.n_probe;
+  const int KT = BLK / T;  // 1 or 2 tiles per block
+  const int rank = (C > 1) ? static_cast<int>(cluster_ctarank()) : 0;
+  const int unit = blockIdx.x / C;
+  const int split = unit % p.S;
+  const int bk = unit / p.S;
+  const int kvh = bk % p.Hkv;
+  const int b = bk / p.Hkv;
+
+  int L = p.seq_lens[b];
+  const bool bad_len = (L < 1 || L > p.L_max);
+  if (bad_len) L = 0;
+  const int n_tiles = (L + T - 1) / T;
+  const int t0 = static_cast<int>((static_cast<long long>(split) * n_tiles) / p.S);
+  const int t1 = static_cast<int>((static_cast<long long>(split + 1) * n_tiles) / p.S);
+  const int ns = t1 - t0;
+  const int pbeg = t0 * T;
+  const int pend = min(t1 * T, L);
+  const int nblk = pend > pbeg ? (pend - pbeg + BLK - 1) / BLK : 0;
+  const int my_blocks = nblk > rank ? (nblk - rank + C - 1) / C : 0;
+  const int R = (nblk + C - 1) / C;
+  const int zc = b * p.Hkv + kvh;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  volatile int* ctl = reinterpret_cast<volatile int*>(sm + OFF_CTL);
+  float* wred = reinterpret_cast<float*>(sm + OFF_WRED);
+  float* wsum = reinterpret_cast<float*>(sm + OFF_WSUM);
+  float* tst = reinterpret_cast<float*>(sm + OFF_TST);
+  float* pub = reinterpret_cast<float*>(sm + OFF_PUB);
+  int* dec = reinterpret_cast<int*>(sm + OFF_DEC);
+  float* rf = reinterpret_cast<float*>(sm + OFF_RF);
+  int* ri = reinterpret_cast<int*>(sm + OFF_RI);
+  int8_t* l2p = reinterpret_cast<int8_t*>(sm + OFF_L2P);
+
+  // ---------------------------------------------------------------- setup
+  if (tid == 0) {
+    for (int s = 0; s < NSTG; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_SFULL + s), 1);
+      mbar_init(bar(B_SFREE + s), 128);
+      mbar_init(bar(B_PFULL + s), 128);
+      mbar_init(bar(B_OFULL + s), 1);
+      mbar_init(bar(B_OFREE + s), 128);
+      mbar_init(bar(B_XFULL + s), C);
+      mbar_init(bar(B_XFREE + s), C);
+      mbar_init(bar(B_DEC + s), 1);
+    }
+    mbar_init(bar(B_DRAIN), 1);
+    fence_mbar_init();
+    if (bad_len && rank == 0) atomicOr(p.ws_status, kStatusSeqLen);
+  }
+  if (tid < 16) ctl[tid] = 0;
+  for (int i = tid; i < D; i += NTHR) l2p[i] = -1;
+  for (int i = tid; i < 8192 / 16; i += NTHR) reinterpret_cast<uint4*>(sm + OFF_P)[i] = make_uint4(0, 0, 0, 0);
+  if (tid < GMAX) {
+    float* r = rf + tid * RF_SIZE;
+    r[RF_M] = -INFINITY;
+    r[RF_L] = 0.f;
+    r[RF_NRM] = 0.f;
+    for (int k = 0; k < PMAX; ++k) r[RF_A + k] = r[RF_XP + k] = 0.f;
+    int* q = ri + tid * RI_SIZE;
+    q[RI_RUN] = 0;
+    q[RI_STOPPED] = (tid < G) ? 0 : 1;
+    q[RI_USED] = ns;
+    q[RI_STOPREL] = -1;
+  }
+  // Q^T as the scores' B operand: K-major, 128-byte swizzle, 16 rows (heads) x 2 halves of 64 d
+  for (int i = tid; i < 16 * 16; i += NTHR) {
+    const int n = i >> 4, c = i & 15, h = c >> 3, cc = c & 7;
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (n < G) w = *reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(b) * p.Hq + kvh * G + n) * D + c * 8);
+    *reinterpret_cast<uint4*>(sm + OFF_Q + h * 2048 + n * 128 + ((cc ^ (n & 7)) * 16)) = w;
+  }
+  if (warp == WARP_MMA) tmem_alloc(smem_u32(sm + OFF_CTL + 4 * CTL_TMEM), TMEM_COLS);
+  __syncthreads();
+  if (tid < P) l2p[p.lanes[tid]] = static_cast<int8_t>(tid);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (C > 1) cluster_sync_all();  // every CTA's barriers exist before any remote arrive
+  const uint32_t tmem = static_cast<uint32_t>(ctl[CTL_TMEM]);
+
+  // owned online-softmax state of the epilogue threads (thread = d row)
+  float acc[GP], m_own[GP], l_own[GP];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    acc[g] = 0.f;
+    m_own[g] = -INFINITY;
+    l_own[g] = 0.f;
+  }
+
+  // ---------------------------------------------------------------- roles
+  if (warp == WARP_TMA) {
+    if (lane == 0) {
+      int issued = 0, tiles_read = 0;
+      for (int jl = 0; jl < my_blocks; ++jl) {
+        if (ART && ctl[CTL_EXIT]) break;
+        const int stage = jl % NSTG;
+        if (jl >= NSTG && !wait_phase(bar(B_EMPTY + stage), ((jl / NSTG) - 1) & 1, ctl, ART, p.ws_status)) break;
+        const int j = jl * C + rank;
+        const int p0 = pbeg + j * BLK;
+        const uint32_t fb = bar(B_FULL + stage);
+        const uint32_t st = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES);
+        mbar_arrive_expect_tx(fb, STAGE_BYTES);
+        tma_load_3d(st, &p.tmK, fb, 0, p0, zc);
+        tma_load_3d(st + 16384, &p.tmK, fb, 64, p0, zc);
+        tma_load_3d(st + 32768, &p.tmV, fb, 0, p0, zc);
+        tma_load_3d(st + 49152, &p.tmV, fb, 64, p0, zc);
+        ++issued;
+        tiles_read += min(KT, t1 - (t0 + j * KT));
+      }
+      ctl[CTL_ISSUED] = issued;
+      ctl[CTL_TREAD] = tiles_read;
+    }
+  } else if (warp == WARP_MMA) {
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, 16, false, false);
+      constexpr uint32_t idO = idesc_bf16(128, 16, true, true);
+      const uint32_t q_addr = smem_u32(sm + OFF_Q);
+      int consumed = 0;
+      auto issue_scores = [&](int jl) -> bool {
+        const int stage = jl % NSTG, bb = jl & 1;
+        if (!wait_phase(bar(B_FULL + stage), (jl / NSTG) & 1, ctl, ART, p.ws_status)) return false;
+        consumed = jl + 1;
+        if (jl >= 2 && !wait_phase(bar(B_SFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t h = kk >> 2, off = (kk & 3) * 32;
+          umma_bf16(tmem + s_col(bb), smem_desc(k_addr + h * 16384 + off, 16, 1024, 2),
+                    smem_desc(q_addr + h * 2048 + off, 16, 1024, 2), idS, kk > 0);
+        }
+        umma_commit(bar(B_SFULL + bb));
+        return true;
+      };
+      bool ok = (my_blocks == 0) || issue_scores(0);
+      for (int jl = 0; ok && jl < my_blocks; ++jl) {
+        if (jl + 1 < my_blocks && !issue_scores(jl + 1)) break;
+        const int stage = jl % NSTG, bb = jl & 1;
+        if (!wait_phase(bar(B_PFULL + bb), (jl >> 1) & 1, ctl, ART, p.ws_status)) break;
+        if (jl >= 2 && !wait_phase(bar(B_OFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status)) break;
+        tc_fence_after();
+        const int j = jl * C + rank;
+        const int ntl = min(KT, t1 - (t0 + j * KT));
+        const uint32_t v_addr = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES + 32768);
+        const uint32_t p_addr = smem_u32(sm + OFF_P + bb * 4096);
+        for (int i = 0; i < ntl; ++i) {
+          for (int s = 0; s < T / 16; ++s) {
+            const int pos0 = i * T + s * 16;
+            umma_bf16(tmem + o_col(bb, i), smem_desc(v_addr + pos0 * 128, 16384, 1024, 2),
+                      smem_desc(p_addr + (pos0 / 8) * 256, 256, 128, 0), idO, s > 0);
+          }
+        }
+        umma_commit(bar(B_OFULL + bb));
+        umma_commit(bar(B_EMPTY + stage));
+      }
+      ctl[CTL_CONSUMED] = consumed;
+      // every issued tensor-core op has completed before the drain barrier fires
+      umma_commit(bar(B_DRAIN));
+      wait_phase(bar(B_DRAIN), 0, ctl, false, p.ws_status);
+    }
+    __syncwarp();
+  } else if (warp < WARP_CTL) {
+    // ------------------------------------------------------------ epilogue warpgroup
+    // All 128 threads take every branch together: mbarrier waits are done by one
+    // leader thread and their outcome is shared with a reducing named barrier.
+    const int wq = warp & 3;
+    const int er = 32 * wq + lane;  // TMEM lane: position row of S, d row of O
+    const bool leader = (er == 0);
+    const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
+    const int tile_of_row = er / T;
+    const int w_n = (T == 64) ? 2 : 4;
+    const int w_lo = (T == 64) ? 2 * tile_of_row : 0;
+    auto epi_wait = [&](uint32_t bb_, uint32_t parity, bool watch_exit, bool cluster) -> bool {
+      bool ok = true;
+      if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status, cluster);
+      return named_barrier_and(BAR_EPI, 128, ok);
+    };
+    float ot[KT_MAX][GP], ot_prev[KT_MAX][GP];
+#pragma unroll
+    for (int i = 0; i < KT_MAX; ++i)
+#pragma unroll
+      for (int g = 0; g < GP; ++g) ot[i][g] = ot_prev[i][g] = 0.f;
+    int ntl_prev = 0;
+    auto merge_tile = [&](int g, float mt, float lt, float o) {
+      const float M = fmaxf(m_own[g], mt);
+      const float a = rescale(m_own[g], M), bt = rescale(mt, M);
+      acc[g] = a * acc[g] + bt * o;
+      l_own[g] = a * l_own[g] + bt * lt;
+      m_own[g] = M;
+    };
+    auto merge_decided = [&](int rp) {
+      const int sp = rp & 1;
+#pragma unroll
+      for (int i = 0; i < KT_MAX; ++i) {
+        if (i < ntl_prev) {
+          const int q = rank * KT + i;
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            const int d = dec[sp * GMAX + g];
+            if (g < G && (d == -1 || (d >= 0 && q <= d)))
+              merge_tile(g, tst[(sp * KT_MAX + i) * GMAX * 2 + g * 2], tst[(sp * KT_MAX + i) * GMAX * 2 + g * 2 + 1],
+                         ot_prev[i][g]);
+          }
+        }
+      }
+      ntl_prev = 0;
+    };
+    const int iters = ART ? R : my_blocks;
+    for (int it = 0; it < iters; ++it) {
+      const int jl = it;  // own block index (== round index in ART mode)
+      const int j = jl * C + rank;
+      bool have = j < nblk;  // uniform
+      int ntl = 0;
+      if (have) {
+        const int bb = jl & 1, stage = jl % NSTG;
+        have = epi_wait(bar(B_SFULL + bb), (jl >> 1) & 1, ART, false);
+        if (have) {
+          tc_fence_after();
+          float sv[8];
+          tmem_ld8(tmem + lane_base + s_col(bb), sv);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(bar(B_SFREE + bb));
+          const int pos = pbeg + j * BLK + er;
+          const bool valid = pos < pend;
+          float s2[GP], pw[GP];
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            s2[g] = (valid && g < G) ? sv[g] * p.qscale : -INFINITY;
+            const float wm = warp_max(s2[g]);
+            if (lane == 0) wred[(bb * 4 + wq) * GMAX + g] = wm;
+          }
+          named_barrier(BAR_EPI, 128);
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            float mt = -INFINITY;
+            for (int w = w_lo; w < w_lo + w_n; ++w) mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
+            pw[g] = (s2[g] == -INFINITY) ? 0.f : exp2f(s2[g] - mt);
+            const float ws = warp_sum(pw[g]);
+            if (lane == 0) wsum[(bb * 4 + wq) * GMAX + g] = ws;
+          }
+          // P^T (hi, lo) of this position; V rows of positions past the end are zeroed
+          {
+            uint8_t* prow = sm + OFF_P + bb * 4096 + (er >> 3) * 256 + (er & 7) * 16;
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+              const __nv_bfloat16 h = __float2bfloat16_rn(pw[g]);
+              const __nv_bfloat16 l = __float2bfloat16_rn(pw[g] - __bfloat162float(h));
+              reinterpret_cast<uint16_t*>(prow)[g] = __bfloat16_as_ushort(h);
+              reinterpret_cast<uint16_t*>(prow + 128)[g] = __bfloat16_as_ushort(l);
+            }
+            if (!valid) {
+              uint8_t* vrow = sm + OFF_STAGE + stage * STAGE_BYTES + 32768 + er * 128;
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                reinterpret_cast<uint4*>(vrow)[c] = make_uint4(0, 0, 0, 0);
+                reinterpret_cast<uint4*>(vrow + 16384)[c] = make_uint4(0, 0, 0, 0);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(bar(B_PFULL + bb));
+          ntl = min(KT, t1 - (t0 + j * KT));
+          have = epi_wait(bar(B_OFULL + bb), (jl >> 1) & 1, ART, false);
+          if (have) {
+            // O_t^T rows: this thread's d row; hi columns 0..7, lo columns 8..15
+            tc_fence_after();
+#pragma unroll
+            for (int i = 0; i < KT_MAX; ++i) {
+              if (i < ntl) {
+                float ov[16];
+                tmem_ld16(tmem + lane_base + o_col(bb, i), ov);
+                tmem_ld_wait();
+#pragma unroll
+                for (int g = 0; g < GP; ++g) ot[i][g] = ov[g] + ov[8 + g];
+              }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_OFREE + bb));
+#pragma unroll
+            for (int i = 0; i < KT_MAX; ++i) {
+              if (i >= ntl) continue;
+              const int lo_w = (T == 64) ? 2 * i : 0;
+#pragma unroll
+              for (int g = 0; g < GP; ++g) {
+                float mt = -INFINITY, lt = 0.f;
+                for (int w = lo_w; w < lo_w + w_n; ++w) {
+                  mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
+                  lt += wsum[(bb * 4 + w) * GMAX + g];
+                }
+                if (!ART) {
+                  if (g < G) merge_tile(g, mt, lt, ot[i][g]);
+                } else if (leader) {
+                  tst[((jl & 1) * KT_MAX + i) * GMAX * 2 + g * 2 + 0] = mt;
+                  tst[((jl & 1) * KT_MAX + i) * GMAX * 2 + g * 2 + 1] = lt;
+                }
+              }
+            }
+          } else {
+            ntl = 0;
+          }
+        }
+        // uniform: the run ended (exit or abort).  ART still merges the decided rounds below.
+        if (!have) {
+          ntl = 0;
+          if (!ART) break;
+        }
+      }
+      if constexpr (ART) {
+        const int r = it;
+        // merge the previous round by its decision
+        if (r >= 1) {
+          bool got = true;
+          if (leader) {
+            const int rp = r - 1;
+            got = false;
+            const unsigned long long t0w = globaltimer_ns();
+            while (true) {
+              if (mbar_try_wait(bar(B_DEC + (rp & 1)), (rp >> 1) & 1)) {
+                got = true;
+                break;
+              }
+              if (ctl[CTL_ABORT]) break;
+              if (ctl[CTL_EXIT]) {
+                __threadfence_block();
+                if (rp > ctl[CTL_EXIT_ROUND]) break;
+              }
+              if (globaltimer_ns() - t0w > kWaitLimitNs) {
+                atomicOr(p.ws_status, kStatusTimeout);
+                ctl[CTL_ABORT] = 1;
+                break;
+              }
+            }
+          }
+          got = named_barrier_and(BAR_EPI, 128, got);
+          if (!got) break;
+          merge_decided(r - 1);
+        }
+        // everything decided is merged; stop once the controller ended the run
+        const bool stop_now = named_barrier_or(BAR_EPI, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]));
+        if (stop_now) break;
+        // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
+        const int sl = r & 1;
+        if (r >= 2 && !epi_wait(bar(B_XFREE + sl), ((r >> 1) - 1) & 1, true, true)) break;
+        float* ps = pub + sl * (PUB_SLOT / 4);
+        const int pi = l2p[er];
+#pragma unroll
+        for (int i = 0; i < KT_MAX; ++i) {
+          if (i >= ntl) continue;
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            if (g < G) {
+              float* e = ps + (i * GMAX + g) * (2 + PMAX);
+              if (leader) {
+                e[0] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2];
+                e[1] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2 + 1];
+              }
+              if (pi >= 0) e[2 + pi] = ot[i][g];
+            }
+          }
+        }
+        named_barrier(BAR_EPI, 128);
+        if (leader) {
+          fence_acq_rel_cluster();
+          const uint32_t xb = bar(B_XFULL + sl);
+          for (int c = 0; c < C; ++c) mbar_arrive_cluster(map_to_rank(xb, c));
+        }
+#pragma unroll
+        for (int i = 0; i < KT_MAX; ++i)
+#pragma unroll
+          for (int g = 0; g < GP; ++g) ot_prev[i][g] = ot[i][g];
+        ntl_prev = ntl;
+        if (r == R - 1) {
+          // the last round waits for its own decision
+          bool got = true;
+          if (leader) got = wait_phase(bar(B_DEC + (r & 1)), (r >> 1) & 1, ctl, false, p.ws_status);
+          if (named_barrier_and(BAR_EPI, 128, got)) merge_decided(r);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ ART controller
+    if constexpr (ART) {
+      const int TQ = C * KT;          // tiles per round (power of two <= 32)
+      const int HPP = 32 / TQ;        // heads per pass
+      const int hh = lane / TQ, q = lane % TQ;
+      const int c = q / KT, i = q % KT;
+      const unsigned segmask = (TQ == 32) ? 0xffffffffu : ((1u << TQ) - 1u);
+      for (int r = 0; r < R; ++r) {
+        const int sl = r & 1;
+        int okw = 1;
+        if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r >> 1) & 1, ctl, false, p.ws_status, true);
+        if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+        const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
+        const uint32_t slot_base = smem_u32(pub) + sl * PUB_SLOT;
+        for (int g0 = 0; g0 < G; g0 += HPP) {
+          const int g = g0 + hh;
+          const bool active = g < G;
+          const int gs = active ? g : 0;
+          float* R_f = rf + gs * RF_SIZE;
+          int* R_i = ri + gs * RI_SIZE;
+          const bool stopped_before = !active || R_i[RI_STOPPED] != 0;
+          const bool valid = !stopped_before && q < nv;
+          float m = -INFINITY, l = 0.f, a[PMAX];
+#pragma unroll
+          for (int k = 0; k < PMAX; ++k) a[k] = 0.f;
+          if (valid) {
+            const uint32_t src = map_to_rank(slot_base + ((i * GMAX + g) * (2 + PMAX)) * 4, c);
+            ld_dsmem_v2(src, m, l);
+#pragma unroll
+            for (int k = 0; k < PMAX; k += 2)
+              if (k < P) ld_dsmem_v2(src + 8 + 4 * k, a[k], a[k + 1]);
+          }
+          // inclusive scan of the merge over the round's tiles (segments of TQ lanes)
+          float cs[5], co[5];
+#pragma unroll
+          for (int lv = 0; lv < 5; ++lv) {
+            const int off = 1 << lv;
+            cs[lv] = 1.f;
+            co[lv] = 0.f;
+            if (off < TQ) {
+              const float mo = __shfl_up_sync(0xffffffffu, m, off, TQ);
+              const float lo = __shfl_up_sync(0xffffffffu, l, off, TQ);
+              if (q >= off) {
+                const float M = fmaxf(m, mo);
+                cs[lv] = rescale(m, M);
+                co[lv] = rescale(mo, M);
+                l = cs[lv] * l + co[lv] * lo;
+                m = M;
+              }
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < PMAX; ++k) {
+            if (k < P) {
+#pragma unroll
+              for (int lv = 0; lv < 5; ++lv) {
+                const int off = 1 << lv;
+                if (off < TQ) {
+                  const float ao = __shfl_up_sync(0xffffffffu, a[k], off, TQ);
+                  a[k] = cs[lv] * a[k] + co[lv] * ao;
+                }
+              }
+            }
+          }
+          // prepend the state carried over from earlier rounds
+          const float mR = R_f[RF_M], lR = R_f[RF_L];
+          const float Mf = fmaxf(mR, m);
+          const float aR = rescale(mR, Mf), aS = rescale(m, Mf);
+          l = aR * lR + aS * l;
+          m = Mf;
+          const float inv_l = 1.f / l;
+          float nrm2 = 0.f;
+#pragma unroll
+          for (int k = 0; k < PMAX; ++k) {
+            if (k < P) {
+              a[k] = aR * R_f[RF_A + k] + aS * a[k];
+              const float x = a[k] * inv_l;
+              nrm2 = fmaf(x, x, nrm2);
+            }
+          }
+          const float nrm = sqrtf(nrm2);
+          float nrmp = __shfl_up_sync(0xffffffffu, nrm, 1, TQ);
+          if (q == 0) nrmp = R_f[RF_NRM];
+          float dd2 = 0.f;
+          const bool both = nrm > 0.f && nrmp > 0.f;
+          const float in = both ? 1.f / nrm : 0.f, ip = both ? 1.f / nrmp : 0.f;
+#pragma unroll
+          for (int k = 0; k < PMAX; ++k) {
+            if (k < P) {
+              const float x = a[k] * inv_l;
+              float xp = __shfl_up_sync(0xffffffffu, x, 1, TQ);
+              if (q == 0) xp = R_f[RF_XP + k];
+              const float dl = x * in - xp * ip;
+              dd2 = fmaf(dl, dl, dd2);
+            }
+          }
+          const float d_scale = fabsf(nrm - nrmp);
+          const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd2);
+          const bool hold = valid && (d_scale < p.eps_scale) && (d_dir < p.eps_dir);
+          const unsigned seg = (__ballot_sync(0xffffffffu, hold) >> (hh * TQ)) & segmask;
+          int run = stopped_before ? 0 : R_i[RI_RUN];
+          int stop = -1;
+          if (!stopped_before) {
+            for (int qq = 0; qq < nv; ++qq) {
+              run = ((seg >> qq) & 1u) ? run + 1 : 0;
+              if (run >= p.patience) {
+                stop = qq;
+                break;
+              }
+            }
+          }
+          __syncwarp();
+          const int srcq = (stop >= 0) ? stop : nv - 1;
+          if (active && !stopped_before && nv > 0 && q == srcq) {
+            R_f[RF_M] = m;
+            R_f[RF_L] = l;
+            R_f[RF_NRM] = nrm;
+#pragma unroll
+            for (int k = 0; k < PMAX; ++k)
+              if (k < P) {
+                R_f[RF_A + k] = a[k];
+                R_f[RF_XP + k] = a[k] * inv_l;
+              }
+            R_i[RI_RUN] = run;
+            if (stop >= 0) {
+              R_i[RI_STOPPED] = 1;
+              R_i[RI_USED] = r * TQ + stop + 1;
+            }
+          }
+          if (active && q == 0) dec[sl * GMAX + g] = stopped_before ? -2 : stop;
+          __syncwarp();
+        }
+        __syncwarp();
+        if (lane == 0) {
+          // the peers' publications of this slot have been read: free the slot everywhere
+          const uint32_t fb = bar(B_XFREE + sl);
+          for (int cc = 0; cc < C; ++cc) mbar_arrive_cluster(map_to_rank(fb, cc));
+          bool all = true;
+          for (int g = 0; g < G; ++g) all &= (ri[g * RI_SIZE + RI_STOPPED] != 0);
+          __threadfence_block();
+          mbar_arrive(bar(B_DEC + sl));
+          if (all) {
+            ctl[CTL_EXIT_ROUND] = r;
+            __threadfence_block();
+            ctl[CTL_EXIT] = 1;
+          }
+        }
+        __syncwarp();
+        if (ctl[CTL_EXIT]) break;
+      }
+    }
+  }
+
+  __syncthreads();  // (1) every role has left its loop
+  // drain: copies that were issued but never consumed still land in shared memory
+  if (warp == WARP_TMA && lane == 0) {
+    for (int ord = ctl[CTL_CONSUMED]; ord < ctl[CTL_ISSUED]; ++ord)
+      wait_phase(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, ctl, false, p.ws_status);
+  }
+  __syncthreads();  // (2) the ring is quiet: stage 0 can hold the final reduction
+  if (warp >= 2 && warp < WARP_CTL) {
+    float* red = reinterpret_cast<float*>(sm + OFF_RED);
+    const int er = 32 * (warp & 3) + lane;
+#pragma unroll
+    for (int g = 0; g < GP; ++g)
+      if (g < G) red[g * D + er] = acc[g];
+    if (er == 0) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        red[GMAX * D + g] = m_own[g];
+        red[GMAX * D + GMAX + g] = l_own[g];
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- cluster merge and output
+  float* red = reinterpret_cast<float*>(sm + OFF_RED);
+  int* redi = reinterpret_cast<int*>(sm + OFF_RED + 4 * (GMAX * D + 2 * GMAX));
+  if (tid == 0) redi[0] = ctl[CTL_TREAD];
+  if (C > 1) cluster_sync_all(); else __syncthreads();
+  if (rank == 0) {
+    const uint32_t rb = smem_u32(red);
+    for (int idx = tid; idx < G * D; idx += NTHR) {
+      const int g = idx / D, dd = idx % D;
+      float M = -INFINITY;
+      for (int cc = 0; cc < C; ++cc) {
+        const float mc = (C > 1) ? ld_dsmem_f32(map_to_rank(rb + 4 * (GMAX * D + g), cc)) : red[GMAX * D + g];
+        M = fmaxf(M, mc);
+      }
+      float den = 0.f, num = 0.f;
+      for (int cc = 0; cc < C; ++cc) {
+        float mc, lc, ac;
+        if (C > 1) {
+          mc = ld_dsmem_f32(map_to_rank(rb + 4 * (GMAX * D + g), cc));
+          lc = ld_dsmem_f32(map_to_rank(rb + 4 * (GMAX * D + GMAX + g), cc));
+          ac = ld_dsmem_f32(map_to_rank(rb + 4 * (g * D + dd), cc));
+        } else {
+          mc = red[GMAX * D + g];
+          lc = red[GMAX * D + GMAX + g];
+          ac = red[g * D + dd];
+        }
+        if (mc == -INFINITY) continue;
+        const float w = exp2f(mc - M);
+        den += w * lc;
+        num += w * ac;
+      }
+      const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + g;
+      if (p.S == 1) {
+        p.o[hq * D + dd] = bad_len ? __int_as_float(0x7fc00000) : num / den;
+      } else {
+        float* part = p.ws_partial + (hq * p.S + split) * (D + 2);
+        if (dd == 0) {
+          part[0] = M;
+          part[1] = den;
+        }
+        part[2 + dd] = num;
+      }
+    }
+    if (tid < G) {
+      const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + tid;
+      const int used = bad_len ? 0 : (ART ? ri[tid * RI_SIZE + RI_USED] : ns);
+      p.ws_used[hq * p.S + split] = used;
+      if (p.S == 1 && p.tiles) p.tiles[hq] = used;
+    }
+    if (tid == 0) {
+      int total = 0;
+      const uint32_t a = smem_u32(redi);
+      for (int cc = 0; cc < C; ++cc) total += (C > 1) ? ld_dsmem_s32(map_to_rank(a, cc)) : redi[0];
+      p.ws_tiles_read[(static_cast<long long>(b) * p.Hkv + kvh) * p.S + split] = total;
+    }
+  }
+  if (C > 1) cluster_sync_all();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace tc
+}  // namespace artk
