@@ -67,18 +67,24 @@ constexpr uint32_t OFF_STAGE = 0;
 constexpr uint32_t OFF_Q = NSTG * STAGE_BYTES;        // 2 halves x 2 KiB
 constexpr uint32_t OFF_P = OFF_Q + 4096;              // 2 buffers x 4 KiB
 constexpr uint32_t OFF_BAR = OFF_P + 8192;            // mbarriers
+// ART exchange: rounds cycle through NSLOT publication slots; a round's tiles are
+// merged LAG rounds after they were published, so the streaming epilogue does
+// not wait for the controller's decision of the round it has just finished.
+constexpr int NSLOT = 4;
+constexpr int LAG = 2;
 enum : int {
   B_FULL = 0, B_EMPTY = B_FULL + NSTG, B_SFULL = B_EMPTY + NSTG, B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2,
-  B_OFULL = B_PFULL + 2, B_OFREE = B_OFULL + 2, B_XFULL = B_OFREE + 2, B_XFREE = B_XFULL + 2, B_DEC = B_XFREE + 2,
-  B_DRAIN = B_DEC + 2, B_COUNT = B_DRAIN + 1
+  B_OFULL = B_PFULL + 2, B_OFREE = B_OFULL + 2, B_XFULL = B_OFREE + 2, B_XFREE = B_XFULL + NSLOT,
+  B_DEC = B_XFREE + NSLOT, B_DRAIN = B_DEC + NSLOT, B_COUNT = B_DRAIN + 1
 };
+static_assert(B_COUNT * 8 <= 256, "barrier area");
 constexpr uint32_t OFF_WRED = OFF_BAR + 256;                          // [2][4][GMAX] per-warp maxima
 constexpr uint32_t OFF_WSUM = OFF_WRED + 4 * 2 * 4 * GMAX;            // [2][4][GMAX] per-warp sums
-constexpr uint32_t OFF_TST = OFF_WSUM + 4 * 2 * 4 * GMAX;             // [2][KT][GMAX][2] tile (m, l)
-constexpr uint32_t OFF_PUB = OFF_TST + 4 * 2 * KT_MAX * GMAX * 2;     // [2][KT][GMAX][2+PMAX]
+constexpr uint32_t OFF_TST = OFF_WSUM + 4 * 2 * 4 * GMAX;             // [NSLOT][KT][GMAX][2] tile (m, l)
+constexpr uint32_t OFF_PUB = OFF_TST + 4 * NSLOT * KT_MAX * GMAX * 2; // [NSLOT][KT][GMAX][2+PMAX]
 constexpr uint32_t PUB_SLOT = 4 * KT_MAX * GMAX * (2 + PMAX);
-constexpr uint32_t OFF_DEC = OFF_PUB + 2 * PUB_SLOT;                  // [2][GMAX] int
-constexpr uint32_t OFF_CTL = OFF_DEC + 4 * 2 * GMAX;                  // [16] int
+constexpr uint32_t OFF_DEC = OFF_PUB + NSLOT * PUB_SLOT;              // [NSLOT][GMAX] int
+constexpr uint32_t OFF_CTL = OFF_DEC + 4 * NSLOT * GMAX;              // [16] int
 constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;                         // [GMAX][RF_SIZE] float
 constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;              // [GMAX][RI_SIZE] int
 constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;             // [D] int8
@@ -169,6 +175,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       mbar_init(bar(B_PFULL + s), 128);
       mbar_init(bar(B_OFULL + s), 1);
       mbar_init(bar(B_OFREE + s), 128);
+    }
+    for (int s = 0; s < NSLOT; ++s) {
       mbar_init(bar(B_XFULL + s), C);
       mbar_init(bar(B_XFREE + s), C);
       mbar_init(bar(B_DEC + s), 1);
@@ -306,12 +314,14 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status, cluster);
       return named_barrier_and(BAR_EPI, 128, ok);
     };
-    float ot[KT_MAX][GP], ot_prev[KT_MAX][GP];
+    // The scores step of block j+1 runs before the readback of block j, so the
+    // PV MMAs of block j overlap the softmax of the next block.
+    float ot[KT_MAX][GP], pend1[KT_MAX][GP], pend2[KT_MAX][GP];
 #pragma unroll
     for (int i = 0; i < KT_MAX; ++i)
 #pragma unroll
-      for (int g = 0; g < GP; ++g) ot[i][g] = ot_prev[i][g] = 0.f;
-    int ntl_prev = 0;
+      for (int g = 0; g < GP; ++g) ot[i][g] = pend1[i][g] = pend2[i][g] = 0.f;
+    int ntl1 = 0, ntl2 = 0;
     auto merge_tile = [&](int g, float mt, float lt, float o) {
       const float M = fmaxf(m_own[g], mt);
       const float a = rescale(m_own[g], M), bt = rescale(mt, M);
@@ -319,160 +329,173 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       l_own[g] = a * l_own[g] + bt * lt;
       m_own[g] = M;
     };
-    auto merge_decided = [&](int rp) {
-      const int sp = rp & 1;
+    // merge the pending tiles `pt` (ntlp of them) of round rp by that round's decision
+    auto merge_round = [&](int rp, const float (&pt)[KT_MAX][GP], int ntlp) {
+      const int sp = rp % NSLOT;
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i) {
-        if (i < ntl_prev) {
+        if (i < ntlp) {
           const int q = rank * KT + i;
 #pragma unroll
           for (int g = 0; g < GP; ++g) {
             const int d = dec[sp * GMAX + g];
             if (g < G && (d == -1 || (d >= 0 && q <= d)))
               merge_tile(g, tst[(sp * KT_MAX + i) * GMAX * 2 + g * 2], tst[(sp * KT_MAX + i) * GMAX * 2 + g * 2 + 1],
-                         ot_prev[i][g]);
+                         pt[i][g]);
           }
         }
       }
-      ntl_prev = 0;
     };
-    const int iters = ART ? R : my_blocks;
-    for (int it = 0; it < iters; ++it) {
-      const int jl = it;  // own block index (== round index in ART mode)
-      const int j = jl * C + rank;
-      bool have = j < nblk;  // uniform
-      int ntl = 0;
-      if (have) {
-        const int bb = jl & 1, stage = jl % NSTG;
-        have = epi_wait(bar(B_SFULL + bb), (jl >> 1) & 1, ART, false);
-        if (have) {
-          tc_fence_after();
-          float sv[8];
-          tmem_ld8(tmem + lane_base + s_col(bb), sv);
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(bar(B_SFREE + bb));
-          const int pos = pbeg + j * BLK + er;
-          const bool valid = pos < pend;
-          float s2[GP], pw[GP];
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            s2[g] = (valid && g < G) ? sv[g] * p.qscale : -INFINITY;
-            const float wm = warp_max(s2[g]);
-            if (lane == 0) wred[(bb * 4 + wq) * GMAX + g] = wm;
+    // wait (leader) for the controller's decision of round rp; false if it will never come
+    auto wait_decision = [&](int rp) -> bool {
+      bool got = true;
+      if (leader) {
+        got = false;
+        const unsigned long long t0w = globaltimer_ns();
+        while (true) {
+          if (mbar_try_wait(bar(B_DEC + rp % NSLOT), (rp / NSLOT) & 1)) {
+            got = true;
+            break;
           }
-          named_barrier(BAR_EPI, 128);
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            float mt = -INFINITY;
-            for (int w = w_lo; w < w_lo + w_n; ++w) mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
-            pw[g] = (s2[g] == -INFINITY) ? 0.f : exp2f(s2[g] - mt);
-            const float ws = warp_sum(pw[g]);
-            if (lane == 0) wsum[(bb * 4 + wq) * GMAX + g] = ws;
+          if (ctl[CTL_ABORT]) break;
+          if (ctl[CTL_EXIT]) {
+            __threadfence_block();
+            if (rp > ctl[CTL_EXIT_ROUND]) break;
           }
-          // P^T (hi, lo) of this position; V rows of positions past the end are zeroed
-          {
-            uint8_t* prow = sm + OFF_P + bb * 4096 + (er >> 3) * 256 + (er & 7) * 16;
-#pragma unroll
-            for (int g = 0; g < GP; ++g) {
-              const __nv_bfloat16 h = __float2bfloat16_rn(pw[g]);
-              const __nv_bfloat16 l = __float2bfloat16_rn(pw[g] - __bfloat162float(h));
-              reinterpret_cast<uint16_t*>(prow)[g] = __bfloat16_as_ushort(h);
-              reinterpret_cast<uint16_t*>(prow + 128)[g] = __bfloat16_as_ushort(l);
-            }
-            if (!valid) {
-              uint8_t* vrow = sm + OFF_STAGE + stage * STAGE_BYTES + 32768 + er * 128;
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                reinterpret_cast<uint4*>(vrow)[c] = make_uint4(0, 0, 0, 0);
-                reinterpret_cast<uint4*>(vrow + 16384)[c] = make_uint4(0, 0, 0, 0);
-              }
-            }
+          if (globaltimer_ns() - t0w > kWaitLimitNs) {
+            atomicOr(p.ws_status, kStatusTimeout);
+            ctl[CTL_ABORT] = 1;
+            break;
           }
-          fence_proxy_async_smem();
-          mbar_arrive(bar(B_PFULL + bb));
-          ntl = min(KT, t1 - (t0 + j * KT));
-          have = epi_wait(bar(B_OFULL + bb), (jl >> 1) & 1, ART, false);
-          if (have) {
-            // O_t^T rows: this thread's d row; hi columns 0..7, lo columns 8..15
-            tc_fence_after();
-#pragma unroll
-            for (int i = 0; i < KT_MAX; ++i) {
-              if (i < ntl) {
-                float ov[16];
-                tmem_ld16(tmem + lane_base + o_col(bb, i), ov);
-                tmem_ld_wait();
-#pragma unroll
-                for (int g = 0; g < GP; ++g) ot[i][g] = ov[g] + ov[8 + g];
-              }
-            }
-            tc_fence_before();
-            mbar_arrive(bar(B_OFREE + bb));
-#pragma unroll
-            for (int i = 0; i < KT_MAX; ++i) {
-              if (i >= ntl) continue;
-              const int lo_w = (T == 64) ? 2 * i : 0;
-#pragma unroll
-              for (int g = 0; g < GP; ++g) {
-                float mt = -INFINITY, lt = 0.f;
-                for (int w = lo_w; w < lo_w + w_n; ++w) {
-                  mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
-                  lt += wsum[(bb * 4 + w) * GMAX + g];
-                }
-                if (!ART) {
-                  if (g < G) merge_tile(g, mt, lt, ot[i][g]);
-                } else if (leader) {
-                  tst[((jl & 1) * KT_MAX + i) * GMAX * 2 + g * 2 + 0] = mt;
-                  tst[((jl & 1) * KT_MAX + i) * GMAX * 2 + g * 2 + 1] = lt;
-                }
-              }
-            }
-          } else {
-            ntl = 0;
-          }
-        }
-        // uniform: the run ended (exit or abort).  ART still merges the decided rounds below.
-        if (!have) {
-          ntl = 0;
-          if (!ART) break;
         }
       }
-      if constexpr (ART) {
-        const int r = it;
-        // merge the previous round by its decision
-        if (r >= 1) {
-          bool got = true;
-          if (leader) {
-            const int rp = r - 1;
-            got = false;
-            const unsigned long long t0w = globaltimer_ns();
-            while (true) {
-              if (mbar_try_wait(bar(B_DEC + (rp & 1)), (rp >> 1) & 1)) {
-                got = true;
-                break;
-              }
-              if (ctl[CTL_ABORT]) break;
-              if (ctl[CTL_EXIT]) {
-                __threadfence_block();
-                if (rp > ctl[CTL_EXIT_ROUND]) break;
-              }
-              if (globaltimer_ns() - t0w > kWaitLimitNs) {
-                atomicOr(p.ws_status, kStatusTimeout);
-                ctl[CTL_ABORT] = 1;
-                break;
-              }
-            }
-          }
-          got = named_barrier_and(BAR_EPI, 128, got);
-          if (!got) break;
-          merge_decided(r - 1);
+      return named_barrier_and(BAR_EPI, 128, got);
+    };
+
+    // scores -> weights -> P^T (hi, lo) in smem for own block jl; false if the run ended
+    auto s_phase = [&](int jl) -> bool {
+      const int bb = jl & 1, stage = jl % NSTG;
+      const int j = jl * C + rank;
+      if (!epi_wait(bar(B_SFULL + bb), (jl >> 1) & 1, ART, false)) return false;
+      tc_fence_after();
+      float sv[8];
+      tmem_ld8(tmem + lane_base + s_col(bb), sv);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(B_SFREE + bb));
+      const int pos = pbeg + j * BLK + er;
+      const bool valid = pos < pend;
+      float s2[GP], pw[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        s2[g] = (valid && g < G) ? sv[g] * p.qscale : -INFINITY;
+        const float wm = warp_max(s2[g]);
+        if (lane == 0) wred[(bb * 4 + wq) * GMAX + g] = wm;
+      }
+      named_barrier(BAR_EPI, 128);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float mt = -INFINITY;
+        for (int w = w_lo; w < w_lo + w_n; ++w) mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
+        pw[g] = (s2[g] == -INFINITY) ? 0.f : exp2f(s2[g] - mt);
+        const float ws = warp_sum(pw[g]);
+        if (lane == 0) wsum[(bb * 4 + wq) * GMAX + g] = ws;
+      }
+      uint8_t* prow = sm + OFF_P + bb * 4096 + (er >> 3) * 256 + (er & 7) * 16;
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(pw[g]);
+        const __nv_bfloat16 l = __float2bfloat16_rn(pw[g] - __bfloat162float(h));
+        reinterpret_cast<uint16_t*>(prow)[g] = __bfloat16_as_ushort(h);
+        reinterpret_cast<uint16_t*>(prow + 128)[g] = __bfloat16_as_ushort(l);
+      }
+      if (!valid) {  // V rows of positions past the end must not reach the MMA
+        uint8_t* vrow = sm + OFF_STAGE + stage * STAGE_BYTES + 32768 + er * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          reinterpret_cast<uint4*>(vrow)[c] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(vrow + 16384)[c] = make_uint4(0, 0, 0, 0);
         }
-        // everything decided is merged; stop once the controller ended the run
-        const bool stop_now = named_barrier_or(BAR_EPI, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]));
-        if (stop_now) break;
-        // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
-        const int sl = r & 1;
-        if (r >= 2 && !epi_wait(bar(B_XFREE + sl), ((r >> 1) - 1) & 1, true, true)) break;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_PFULL + bb));
+      return true;
+    };
+    // O_t readback (thread = d row) for own block jl into ot; tile stats to tst; false if the run ended
+    auto o_phase = [&](int jl, int& ntl) -> bool {
+      const int bb = jl & 1;
+      const int j = jl * C + rank;
+      ntl = min(KT, t1 - (t0 + j * KT));
+      if (!epi_wait(bar(B_OFULL + bb), (jl >> 1) & 1, ART, false)) {
+        ntl = 0;
+        return false;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int i = 0; i < KT_MAX; ++i) {
+        if (i < ntl) {
+          float ov[16];
+          tmem_ld16(tmem + lane_base + o_col(bb, i), ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int g = 0; g < GP; ++g) ot[i][g] = ov[g] + ov[8 + g];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(B_OFREE + bb));
+#pragma unroll
+      for (int i = 0; i < KT_MAX; ++i) {
+        if (i >= ntl) continue;
+        const int lo_w = (T == 64) ? 2 * i : 0;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          float mt = -INFINITY, lt = 0.f;
+          for (int w = lo_w; w < lo_w + w_n; ++w) {
+            mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
+            lt += wsum[(bb * 4 + w) * GMAX + g];
+          }
+          if (!ART) {
+            if (g < G) merge_tile(g, mt, lt, ot[i][g]);
+          } else if (leader) {
+            tst[((jl % NSLOT) * KT_MAX + i) * GMAX * 2 + g * 2 + 0] = mt;
+            tst[((jl % NSLOT) * KT_MAX + i) * GMAX * 2 + g * 2 + 1] = lt;
+          }
+        }
+      }
+      return true;
+    };
+
+    const int iters = ART ? R : my_blocks;
+    bool streaming = my_blocks > 0 && s_phase(0);
+    for (int it = 0; it < iters; ++it) {
+      int ntl = 0;
+      if (it < my_blocks && streaming) {
+        const bool next_ok = (it + 1 < my_blocks) ? s_phase(it + 1) : true;
+        streaming = o_phase(it, ntl) && next_ok;
+      }
+      if (!ART) {
+        if (!streaming && it + 1 < iters) break;  // aborted
+        continue;
+      }
+      const int r = it;
+      // stop once the controller has ended the run: merge every round it decided, then leave
+      if (named_barrier_or(BAR_EPI, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]))) {
+        const bool aborted = named_barrier_or(BAR_EPI, 128, leader && ctl[CTL_ABORT] != 0);
+        const int er_round = ctl[CTL_EXIT_ROUND];  // written before the exit flag, never changed after
+        if (!aborted) {
+          if (r - 2 >= 0 && r - 2 <= er_round && wait_decision(r - 2)) merge_round(r - 2, pend2, ntl2);
+          if (r - 1 >= 0 && r - 1 <= er_round && wait_decision(r - 1)) merge_round(r - 1, pend1, ntl1);
+          if (r <= er_round && wait_decision(r)) merge_round(r, ot, ntl);
+        }
+        ntl1 = ntl2 = 0;
+        break;
+      }
+      // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
+      const int sl = r % NSLOT;
+      if (r >= NSLOT && !epi_wait(bar(B_XFREE + sl), ((r / NSLOT) - 1) & 1, true, true)) {
+        // the run ended while waiting for the slot: fall back to the exit path next round
+        ntl = 0;
+      } else {
         float* ps = pub + sl * (PUB_SLOT / 4);
         const int pi = l2p[er];
 #pragma unroll
@@ -496,17 +519,30 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           const uint32_t xb = bar(B_XFULL + sl);
           for (int c = 0; c < C; ++c) mbar_arrive_cluster(map_to_rank(xb, c));
         }
-#pragma unroll
-        for (int i = 0; i < KT_MAX; ++i)
-#pragma unroll
-          for (int g = 0; g < GP; ++g) ot_prev[i][g] = ot[i][g];
-        ntl_prev = ntl;
-        if (r == R - 1) {
-          // the last round waits for its own decision
-          bool got = true;
-          if (leader) got = wait_phase(bar(B_DEC + (r & 1)), (r >> 1) & 1, ctl, false, p.ws_status);
-          if (named_barrier_and(BAR_EPI, 128, got)) merge_decided(r);
+      }
+      // merge round r - LAG by its decision
+      if (r >= LAG) {
+        if (!wait_decision(r - LAG)) {
+          // no decision: the run ended (exit beyond this round or abort); the exit path above merges
+          // what was decided on the next pass
+        } else {
+          merge_round(r - LAG, pend2, ntl2);
+          ntl2 = 0;
         }
+      }
+#pragma unroll
+      for (int i = 0; i < KT_MAX; ++i)
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          pend2[i][g] = pend1[i][g];
+          pend1[i][g] = ot[i][g];
+        }
+      ntl2 = ntl1;
+      ntl1 = ntl;
+      if (r == iters - 1) {
+        // end of the rounds: the last LAG rounds still wait for their decisions
+        if (r - 1 >= 0 && wait_decision(r - 1)) merge_round(r - 1, pend2, ntl2);
+        if (wait_decision(r)) merge_round(r, pend1, ntl1);
       }
     }
   } else {
@@ -518,9 +554,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       const int c = q / KT, i = q % KT;
       const unsigned segmask = (TQ == 32) ? 0xffffffffu : ((1u << TQ) - 1u);
       for (int r = 0; r < R; ++r) {
-        const int sl = r & 1;
+        const int sl = r % NSLOT;
         int okw = 1;
-        if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r >> 1) & 1, ctl, false, p.ws_status, true);
+        if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r / NSLOT) & 1, ctl, false, p.ws_status, true);
         if (!__shfl_sync(0xffffffffu, okw, 0)) break;
         const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
         const uint32_t slot_base = smem_u32(pub) + sl * PUB_SLOT;
