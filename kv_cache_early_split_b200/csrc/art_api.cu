@@ -252,19 +252,24 @@ bool make_kv_map(CUtensorMap* m, const void* base, const art_shape* s) {
 
 using TcFn = void (*)(artk::tc::TcParams);
 
-template <int MODE>
-TcFn tc_pick(int G) {
-  if (G == 1) return &artk::tc::art_decode_tc_kernel<1, MODE>;
-  if (G == 2) return &artk::tc::art_decode_tc_kernel<2, MODE>;
-  if (G <= 4) return &artk::tc::art_decode_tc_kernel<4, MODE>;
-  return &artk::tc::art_decode_tc_kernel<8, MODE>;
+template <int MODE, int PC>
+TcFn tc_pick_gp(int G) {
+  if (G == 1) return &artk::tc::art_decode_tc_kernel<1, MODE, PC>;
+  if (G == 2) return &artk::tc::art_decode_tc_kernel<2, MODE, PC>;
+  if (G <= 4) return &artk::tc::art_decode_tc_kernel<4, MODE, PC>;
+  return &artk::tc::art_decode_tc_kernel<8, MODE, PC>;
+}
+
+TcFn tc_pick(int mode, int G, int n_probe) {
+  if (mode != artk::MODE_ART) return tc_pick_gp<artk::MODE_FULL, 16>(G);
+  return n_probe <= 16 ? tc_pick_gp<artk::MODE_ART, 16>(G) : tc_pick_gp<artk::MODE_ART, 32>(G);
 }
 
 art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k, const void* v,
                      const int32_t* seq_lens, const art_params* a, float* o, int32_t* tiles, void* ws,
                      void* stream) {
   const int G = s->Hq / s->Hkv;
-  const TcFn fn = (mode == artk::MODE_ART) ? tc_pick<artk::MODE_ART>(G) : tc_pick<artk::MODE_FULL>(G);
+  const TcFn fn = tc_pick(mode, G, a ? a->n_probe : 0);
   artk::tc::TcParams p;
   memset(&p, 0, sizeof p);
   if (a) {

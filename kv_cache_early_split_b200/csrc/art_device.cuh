@@ -264,3 +264,41 @@ __device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool v) {
   return r != 0;
 }
 }  // namespace artk
+
+namespace artk {
+// 2^x with the hardware ex2 instruction (PTX ex2.approx.ftz.f32, max rel. error ~2^-22).
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^(m_old - m_new) for an online-softmax rescale; 0 for an empty state (m_old = -inf).
+__device__ __forceinline__ float rescale_fast(float m_old, float m_new) {
+  return (m_old == -INFINITY) ? 0.f : ex2_fast(m_old - m_new);
+}
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+// Max / sum of GP per-lane values over the 32 lanes of a warp with the
+// head-splitting butterfly: afterwards lanes [h*32/GP, (h+1)*32/GP) hold head h.
+template <int GP, bool MAX>
+__device__ __forceinline__ float warp_reduce_heads(float (&v)[GP], int lane) {
+#pragma unroll
+  for (int h = GP / 2, off = 16; h >= 1; h >>= 1, off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < h; ++i) {
+      const float send = upper ? v[i] : v[i + h];
+      const float keep = upper ? v[i + h] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, off);
+      v[i] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+#pragma unroll
+  for (int off = 16 / GP; off >= 1; off >>= 1) {
+    const float got = __shfl_xor_sync(0xffffffffu, v[0], off);
+    v[0] = MAX ? fmaxf(v[0], got) : v[0] + got;
+  }
+  return v[0];
+}
+}  // namespace artk

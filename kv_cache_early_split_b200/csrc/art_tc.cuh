@@ -12,16 +12,25 @@
 //   O_t^T[128 d x 16]  = V_t^T[128 d x T]  . P_t^T      (A: V, MN-major, 128-byte swizzle)
 // with accumulators in tensor memory.  P is split into bf16 hi + lo parts
 // (columns 0..7 and 8..15) so that the weights keep ~16 bits of precision.
+// Full attention treats a whole 128-position block as one tile (the tile size
+// has no effect on its result); ART keeps the caller's tiles.
 //
 // Warp roles (224 threads, one CTA per SM):
 //   warp 0      TMA producer: K/V blocks (4 tiled 3-D TMA loads, 64 KiB) into a 3-deep ring
 //   warp 1      MMA issuer (one lane) and tensor-memory owner
 //   warps 2..5  epilogue: scores -> per-tile max / weights -> P^T in smem; O readback
-//               (thread = d row) -> online merge in registers; ART publication
+//               (thread = d row) -> online merge in registers; ART publication.
+//               The scores step of block j+1 runs before the readback of block j.
 //   warp 6      ART controller: per round, reads all CTAs' publications through
-//               distributed shared memory and replays the rule in tile order
-// Blocks are dealt round-robin over the cluster exactly as in art_decode_kernel,
-// and the ART exchange runs one round behind the streaming pipeline.
+//               distributed shared memory and replays the rule in tile order.
+// Blocks are dealt round-robin over the cluster exactly as in art_decode_kernel.
+//
+// ART exchange without back-pressure barriers: rounds cycle through NSLOT = 6
+// publication slots and the epilogue merges round r - LAG (LAG = 2) after
+// publishing round r.  Before a CTA publishes round x it has merged round
+// x-1-LAG, so its controller has decided that round, so every CTA had published
+// it, so every CTA had merged round x-2-2*LAG, so every controller had decided
+// -- and finished reading -- round x-2-2*LAG = x-NSLOT: the slot is free.
 #pragma once
 
 #include <cuda.h>
@@ -40,11 +49,13 @@ constexpr int D = 128;
 constexpr int NSTG = 3;
 constexpr int NWARP = 7;
 constexpr int NTHR = NWARP * 32;
-constexpr int KT_MAX = 2;  // tiles per block (tile 64)
+constexpr int KT_MAX = 2;  // ART tiles per block (tile 64)
 constexpr int STAGE_BYTES = 4 * 16384;
 constexpr uint32_t TMEM_COLS = 128;
 constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_CTL = 6;
 constexpr int BAR_EPI = 1;  // named barrier of the 128 epilogue threads
+constexpr int LAG = 2;
+constexpr int NSLOT = 2 + 2 * LAG;
 
 struct TcParams {
   CUtensorMap tmK;  // 64-byte aligned (first members)
@@ -64,32 +75,29 @@ struct TcParams {
 
 // ---- shared-memory map (byte offsets from a 1024-aligned base)
 constexpr uint32_t OFF_STAGE = 0;
-constexpr uint32_t OFF_Q = NSTG * STAGE_BYTES;        // 2 halves x 2 KiB
-constexpr uint32_t OFF_P = OFF_Q + 4096;              // 2 buffers x 4 KiB
-constexpr uint32_t OFF_BAR = OFF_P + 8192;            // mbarriers
-// ART exchange: rounds cycle through NSLOT publication slots; a round's tiles are
-// merged LAG rounds after they were published, so the streaming epilogue does
-// not wait for the controller's decision of the round it has just finished.
-constexpr int NSLOT = 4;
-constexpr int LAG = 2;
+constexpr uint32_t OFF_Q = NSTG * STAGE_BYTES;  // 2 halves x 2 KiB
+constexpr uint32_t OFF_P = OFF_Q + 4096;        // 2 buffers x 4 KiB
+constexpr uint32_t OFF_BAR = OFF_P + 8192;      // mbarriers
 enum : int {
   B_FULL = 0, B_EMPTY = B_FULL + NSTG, B_SFULL = B_EMPTY + NSTG, B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2,
-  B_OFULL = B_PFULL + 2, B_OFREE = B_OFULL + 2, B_XFULL = B_OFREE + 2, B_XFREE = B_XFULL + NSLOT,
-  B_DEC = B_XFREE + NSLOT, B_DRAIN = B_DEC + NSLOT, B_COUNT = B_DRAIN + 1
+  B_OFULL = B_PFULL + 2, B_OFREE = B_OFULL + 2, B_XFULL = B_OFREE + 2, B_DEC = B_XFULL + NSLOT,
+  B_DRAIN = B_DEC + NSLOT, B_COUNT = B_DRAIN + 1
 };
 static_assert(B_COUNT * 8 <= 256, "barrier area");
-constexpr uint32_t OFF_WRED = OFF_BAR + 256;                          // [2][4][GMAX] per-warp maxima
-constexpr uint32_t OFF_WSUM = OFF_WRED + 4 * 2 * 4 * GMAX;            // [2][4][GMAX] per-warp sums
-constexpr uint32_t OFF_TST = OFF_WSUM + 4 * 2 * 4 * GMAX;             // [NSLOT][KT][GMAX][2] tile (m, l)
-constexpr uint32_t OFF_PUB = OFF_TST + 4 * NSLOT * KT_MAX * GMAX * 2; // [NSLOT][KT][GMAX][2+PMAX]
-constexpr uint32_t PUB_SLOT = 4 * KT_MAX * GMAX * (2 + PMAX);
-constexpr uint32_t OFF_DEC = OFF_PUB + NSLOT * PUB_SLOT;              // [NSLOT][GMAX] int
-constexpr uint32_t OFF_CTL = OFF_DEC + 4 * NSLOT * GMAX;              // [16] int
-constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;                         // [GMAX][RF_SIZE] float
-constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;              // [GMAX][RI_SIZE] int
-constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;             // [D] int8
+constexpr uint32_t OFF_WRED = OFF_BAR + 256;                           // [2][4][GMAX] per-warp maxima
+constexpr uint32_t OFF_WSUM = OFF_WRED + 4 * 2 * 4 * GMAX;             // [2][4][GMAX] per-warp sums
+constexpr uint32_t OFF_TST = OFF_WSUM + 4 * 2 * 4 * GMAX;              // [NSLOT][KT][GMAX][2] tile (m, l)
+constexpr uint32_t OFF_PUB = OFF_TST + 4 * NSLOT * KT_MAX * GMAX * 2;  // [NSLOT][KT][GMAX][2+PMAX]
+constexpr uint32_t PUB_ENTRY = 2 + PMAX;
+constexpr uint32_t PUB_SLOT = 4 * KT_MAX * GMAX * PUB_ENTRY;
+constexpr uint32_t OFF_DEC = OFF_PUB + NSLOT * PUB_SLOT;  // [NSLOT][GMAX] int
+constexpr uint32_t OFF_CTL = OFF_DEC + 4 * NSLOT * GMAX;  // [16] int
+constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;             // [GMAX][RF_SIZE] float
+constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;  // [GMAX][RI_SIZE] int
+constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;  // [D] int8
 constexpr uint32_t SMEM_USED = OFF_L2P + D;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 // final reduction (aliases stage 0 after the pipeline has drained)
 constexpr uint32_t OFF_RED = 0;  // [GMAX][D] numerators, then [GMAX] m, [GMAX] l, [4] ints
 enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, CTL_TREAD, CTL_TMEM };
@@ -121,15 +129,20 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
   }
 }
 
-template <int GP, int MODE>
+// GP: query heads per kv head (padded to 1, 2, 4 or 8); MODE: full or ART;
+// PC: probe-lane capacity of the rule replay (16 or 32, lanes beyond n_probe are zero).
+template <int GP, int MODE, int PC>
 __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
   static_assert(GP >= 1 && GP <= 8, "up to 8 query heads per kv head");
+  static_assert(PC == 16 || PC == 32, "probe capacity");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int C = p.C, T = p.T, G = p.G, P = p.n_probe;
-  const int KT = BLK / T;  // 1 or 2 tiles per block
+  const int C = p.C, G = p.G, P = p.n_probe;
+  const int T = p.T;
+  const int KT = ART ? BLK / T : 1;  // tiles per block (full attention: the block is one tile)
+  const int TE = ART ? T : BLK;      // positions per tile inside the kernel
   const int rank = (C > 1) ? static_cast<int>(cluster_ctarank()) : 0;
   const int unit = blockIdx.x / C;
   const int split = unit % p.S;
@@ -150,6 +163,12 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   const int my_blocks = nblk > rank ? (nblk - rank + C - 1) / C : 0;
   const int R = (nblk + C - 1) / C;
   const int zc = b * p.Hkv + kvh;
+  // tiles of own block jl that lie inside the split
+  auto block_tiles = [&](int jl) -> int {
+    if (!ART) return 1;
+    const int j = jl * C + rank;
+    return min(KT, t1 - (t0 + j * KT));
+  };
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -178,7 +197,6 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     }
     for (int s = 0; s < NSLOT; ++s) {
       mbar_init(bar(B_XFULL + s), C);
-      mbar_init(bar(B_XFREE + s), C);
       mbar_init(bar(B_DEC + s), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
@@ -188,6 +206,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   if (tid < 16) ctl[tid] = 0;
   for (int i = tid; i < D; i += NTHR) l2p[i] = -1;
   for (int i = tid; i < 8192 / 16; i += NTHR) reinterpret_cast<uint4*>(sm + OFF_P)[i] = make_uint4(0, 0, 0, 0);
+  if (ART)
+    for (int i = tid; i < static_cast<int>(NSLOT * PUB_SLOT / 16); i += NTHR)
+      reinterpret_cast<uint4*>(sm + OFF_PUB)[i] = make_uint4(0, 0, 0, 0);
   if (tid < GMAX) {
     float* r = rf + tid * RF_SIZE;
     r[RF_M] = -INFINITY;
@@ -244,7 +265,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         tma_load_3d(st + 32768, &p.tmV, fb, 0, p0, zc);
         tma_load_3d(st + 49152, &p.tmV, fb, 64, p0, zc);
         ++issued;
-        tiles_read += min(KT, t1 - (t0 + j * KT));
+        tiles_read += min(BLK / T, t1 - (t0 + j * (BLK / T)));
       }
       ctl[CTL_ISSUED] = issued;
       ctl[CTL_TREAD] = tiles_read;
@@ -278,13 +299,12 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         if (!wait_phase(bar(B_PFULL + bb), (jl >> 1) & 1, ctl, ART, p.ws_status)) break;
         if (jl >= 2 && !wait_phase(bar(B_OFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status)) break;
         tc_fence_after();
-        const int j = jl * C + rank;
-        const int ntl = min(KT, t1 - (t0 + j * KT));
+        const int ntl = block_tiles(jl);
         const uint32_t v_addr = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES + 32768);
         const uint32_t p_addr = smem_u32(sm + OFF_P + bb * 4096);
         for (int i = 0; i < ntl; ++i) {
-          for (int s = 0; s < T / 16; ++s) {
-            const int pos0 = i * T + s * 16;
+          for (int s = 0; s < TE / 16; ++s) {
+            const int pos0 = i * TE + s * 16;
             umma_bf16(tmem + o_col(bb, i), smem_desc(v_addr + pos0 * 128, 16384, 1024, 2),
                       smem_desc(p_addr + (pos0 / 8) * 256, 256, 128, 0), idO, s > 0);
           }
@@ -306,16 +326,13 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     const int er = 32 * wq + lane;  // TMEM lane: position row of S, d row of O
     const bool leader = (er == 0);
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
-    const int tile_of_row = er / T;
-    const int w_n = (T == 64) ? 2 : 4;
-    const int w_lo = (T == 64) ? 2 * tile_of_row : 0;
-    auto epi_wait = [&](uint32_t bb_, uint32_t parity, bool watch_exit, bool cluster) -> bool {
+    const int w_n = TE / 32;           // warps per tile
+    const int w_lo = (er / TE) * w_n;  // first warp of this row's tile
+    auto epi_wait = [&](uint32_t bb_, uint32_t parity, bool watch_exit) -> bool {
       bool ok = true;
-      if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status, cluster);
+      if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status);
       return named_barrier_and(BAR_EPI, 128, ok);
     };
-    // The scores step of block j+1 runs before the readback of block j, so the
-    // PV MMAs of block j overlap the softmax of the next block.
     float ot[KT_MAX][GP], pend1[KT_MAX][GP], pend2[KT_MAX][GP];
 #pragma unroll
     for (int i = 0; i < KT_MAX; ++i)
@@ -324,7 +341,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     int ntl1 = 0, ntl2 = 0;
     auto merge_tile = [&](int g, float mt, float lt, float o) {
       const float M = fmaxf(m_own[g], mt);
-      const float a = rescale(m_own[g], M), bt = rescale(mt, M);
+      const float a = rescale_fast(m_own[g], M), bt = rescale_fast(mt, M);
       acc[g] = a * acc[g] + bt * o;
       l_own[g] = a * l_own[g] + bt * lt;
       m_own[g] = M;
@@ -376,7 +393,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     auto s_phase = [&](int jl) -> bool {
       const int bb = jl & 1, stage = jl % NSTG;
       const int j = jl * C + rank;
-      if (!epi_wait(bar(B_SFULL + bb), (jl >> 1) & 1, ART, false)) return false;
+      if (!epi_wait(bar(B_SFULL + bb), (jl >> 1) & 1, ART)) return false;
       tc_fence_after();
       float sv[8];
       tmem_ld8(tmem + lane_base + s_col(bb), sv);
@@ -385,21 +402,23 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       mbar_arrive(bar(B_SFREE + bb));
       const int pos = pbeg + j * BLK + er;
       const bool valid = pos < pend;
-      float s2[GP], pw[GP];
+      float s2[GP], red[GP], pw[GP];
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        s2[g] = (valid && g < G) ? sv[g] * p.qscale : -INFINITY;
-        const float wm = warp_max(s2[g]);
-        if (lane == 0) wred[(bb * 4 + wq) * GMAX + g] = wm;
+      for (int g = 0; g < GP; ++g) red[g] = s2[g] = (valid && g < G) ? sv[g] * p.qscale : -INFINITY;
+      {
+        const float wm = warp_reduce_heads<GP, true>(red, lane);
+        if ((lane & (32 / GP - 1)) == 0) wred[(bb * 4 + wq) * GMAX + lane / (32 / GP)] = wm;
       }
       named_barrier(BAR_EPI, 128);
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float mt = -INFINITY;
         for (int w = w_lo; w < w_lo + w_n; ++w) mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
-        pw[g] = (s2[g] == -INFINITY) ? 0.f : exp2f(s2[g] - mt);
-        const float ws = warp_sum(pw[g]);
-        if (lane == 0) wsum[(bb * 4 + wq) * GMAX + g] = ws;
+        red[g] = pw[g] = (s2[g] == -INFINITY) ? 0.f : ex2_fast(s2[g] - mt);
+      }
+      {
+        const float ws = warp_reduce_heads<GP, false>(red, lane);
+        if ((lane & (32 / GP - 1)) == 0) wsum[(bb * 4 + wq) * GMAX + lane / (32 / GP)] = ws;
       }
       uint8_t* prow = sm + OFF_P + bb * 4096 + (er >> 3) * 256 + (er & 7) * 16;
 #pragma unroll
@@ -424,9 +443,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     // O_t readback (thread = d row) for own block jl into ot; tile stats to tst; false if the run ended
     auto o_phase = [&](int jl, int& ntl) -> bool {
       const int bb = jl & 1;
-      const int j = jl * C + rank;
-      ntl = min(KT, t1 - (t0 + j * KT));
-      if (!epi_wait(bar(B_OFULL + bb), (jl >> 1) & 1, ART, false)) {
+      ntl = block_tiles(jl);
+      if (!epi_wait(bar(B_OFULL + bb), (jl >> 1) & 1, ART)) {
         ntl = 0;
         return false;
       }
@@ -446,7 +464,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i) {
         if (i >= ntl) continue;
-        const int lo_w = (T == 64) ? 2 * i : 0;
+        const int lo_w = i * w_n;
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
           float mt = -INFINITY, lt = 0.f;
@@ -492,10 +510,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       }
       // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
       const int sl = r % NSLOT;
-      if (r >= NSLOT && !epi_wait(bar(B_XFREE + sl), ((r / NSLOT) - 1) & 1, true, true)) {
-        // the run ended while waiting for the slot: fall back to the exit path next round
-        ntl = 0;
-      } else {
+      {
         float* ps = pub + sl * (PUB_SLOT / 4);
         const int pi = l2p[er];
 #pragma unroll
@@ -504,7 +519,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
           for (int g = 0; g < GP; ++g) {
             if (g < G) {
-              float* e = ps + (i * GMAX + g) * (2 + PMAX);
+              float* e = ps + (i * GMAX + g) * PUB_ENTRY;
               if (leader) {
                 e[0] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2];
                 e[1] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2 + 1];
@@ -514,22 +529,13 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           }
         }
         named_barrier(BAR_EPI, 128);
-        if (leader) {
+        if (er < C) {  // one thread per peer: make the slot visible, then signal that CTA
           fence_acq_rel_cluster();
-          const uint32_t xb = bar(B_XFULL + sl);
-          for (int c = 0; c < C; ++c) mbar_arrive_cluster(map_to_rank(xb, c));
+          mbar_arrive_cluster_relaxed(map_to_rank(bar(B_XFULL + sl), er));
         }
       }
-      // merge round r - LAG by its decision
-      if (r >= LAG) {
-        if (!wait_decision(r - LAG)) {
-          // no decision: the run ended (exit beyond this round or abort); the exit path above merges
-          // what was decided on the next pass
-        } else {
-          merge_round(r - LAG, pend2, ntl2);
-          ntl2 = 0;
-        }
-      }
+      // merge round r - LAG by its decision (no decision: the run ended; the exit path covers it)
+      if (r >= LAG && wait_decision(r - LAG)) merge_round(r - LAG, pend2, ntl2);
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i)
 #pragma unroll
@@ -548,8 +554,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   } else {
     // ------------------------------------------------------------ ART controller
     if constexpr (ART) {
-      const int TQ = C * KT;          // tiles per round (power of two <= 32)
-      const int HPP = 32 / TQ;        // heads per pass
+      const int TQ = C * KT;    // tiles per round (power of two <= 32)
+      const int HPP = 32 / TQ;  // heads per pass
       const int hh = lane / TQ, q = lane % TQ;
       const int c = q / KT, i = q % KT;
       const unsigned segmask = (TQ == 32) ? 0xffffffffu : ((1u << TQ) - 1u);
@@ -568,15 +574,14 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           int* R_i = ri + gs * RI_SIZE;
           const bool stopped_before = !active || R_i[RI_STOPPED] != 0;
           const bool valid = !stopped_before && q < nv;
-          float m = -INFINITY, l = 0.f, a[PMAX];
+          float m = -INFINITY, l = 0.f, a[PC];
 #pragma unroll
-          for (int k = 0; k < PMAX; ++k) a[k] = 0.f;
-          if (valid) {
-            const uint32_t src = map_to_rank(slot_base + ((i * GMAX + g) * (2 + PMAX)) * 4, c);
+          for (int k = 0; k < PC; ++k) a[k] = 0.f;
+          if (valid) {  // this tile's (m, l, probe) from the CTA that computed it
+            const uint32_t src = map_to_rank(slot_base + ((i * GMAX + g) * PUB_ENTRY) * 4, c);
             ld_dsmem_v2(src, m, l);
 #pragma unroll
-            for (int k = 0; k < PMAX; k += 2)
-              if (k < P) ld_dsmem_v2(src + 8 + 4 * k, a[k], a[k + 1]);
+            for (int k = 0; k < PC; k += 2) ld_dsmem_v2(src + 8 + 4 * k, a[k], a[k + 1]);
           }
           // inclusive scan of the merge over the round's tiles (segments of TQ lanes)
           float cs[5], co[5];
@@ -590,57 +595,50 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
               const float lo = __shfl_up_sync(0xffffffffu, l, off, TQ);
               if (q >= off) {
                 const float M = fmaxf(m, mo);
-                cs[lv] = rescale(m, M);
-                co[lv] = rescale(mo, M);
+                cs[lv] = rescale_fast(m, M);
+                co[lv] = rescale_fast(mo, M);
                 l = cs[lv] * l + co[lv] * lo;
                 m = M;
               }
             }
           }
 #pragma unroll
-          for (int k = 0; k < PMAX; ++k) {
-            if (k < P) {
+          for (int lv = 0; lv < 5; ++lv) {
+            const int off = 1 << lv;
+            if (off < TQ) {
 #pragma unroll
-              for (int lv = 0; lv < 5; ++lv) {
-                const int off = 1 << lv;
-                if (off < TQ) {
-                  const float ao = __shfl_up_sync(0xffffffffu, a[k], off, TQ);
-                  a[k] = cs[lv] * a[k] + co[lv] * ao;
-                }
+              for (int k = 0; k < PC; ++k) {
+                const float ao = __shfl_up_sync(0xffffffffu, a[k], off, TQ);
+                a[k] = cs[lv] * a[k] + co[lv] * ao;
               }
             }
           }
           // prepend the state carried over from earlier rounds
           const float mR = R_f[RF_M], lR = R_f[RF_L];
           const float Mf = fmaxf(mR, m);
-          const float aR = rescale(mR, Mf), aS = rescale(m, Mf);
+          const float aR = rescale_fast(mR, Mf), aS = rescale_fast(m, Mf);
           l = aR * lR + aS * l;
           m = Mf;
-          const float inv_l = 1.f / l;
-          float nrm2 = 0.f;
+          const float inv_l = __fdividef(1.f, l);
+          float x[PC], nrm2 = 0.f;
 #pragma unroll
-          for (int k = 0; k < PMAX; ++k) {
-            if (k < P) {
-              a[k] = aR * R_f[RF_A + k] + aS * a[k];
-              const float x = a[k] * inv_l;
-              nrm2 = fmaf(x, x, nrm2);
-            }
+          for (int k = 0; k < PC; ++k) {
+            a[k] = aR * R_f[RF_A + k] + aS * a[k];
+            x[k] = a[k] * inv_l;
+            nrm2 = fmaf(x[k], x[k], nrm2);
           }
-          const float nrm = sqrtf(nrm2);
+          const float nrm = __fsqrt_rn(nrm2);
           float nrmp = __shfl_up_sync(0xffffffffu, nrm, 1, TQ);
           if (q == 0) nrmp = R_f[RF_NRM];
-          float dd2 = 0.f;
           const bool both = nrm > 0.f && nrmp > 0.f;
-          const float in = both ? 1.f / nrm : 0.f, ip = both ? 1.f / nrmp : 0.f;
+          const float in = both ? __fdividef(1.f, nrm) : 0.f, ip = both ? __fdividef(1.f, nrmp) : 0.f;
+          float dd2 = 0.f;
 #pragma unroll
-          for (int k = 0; k < PMAX; ++k) {
-            if (k < P) {
-              const float x = a[k] * inv_l;
-              float xp = __shfl_up_sync(0xffffffffu, x, 1, TQ);
-              if (q == 0) xp = R_f[RF_XP + k];
-              const float dl = x * in - xp * ip;
-              dd2 = fmaf(dl, dl, dd2);
-            }
+          for (int k = 0; k < PC; ++k) {
+            float xp = __shfl_up_sync(0xffffffffu, x[k], 1, TQ);
+            if (q == 0) xp = R_f[RF_XP + k];
+            const float dl = x[k] * in - xp * ip;
+            dd2 = fmaf(dl, dl, dd2);
           }
           const float d_scale = fabsf(nrm - nrmp);
           const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd2);
@@ -664,11 +662,10 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
             R_f[RF_L] = l;
             R_f[RF_NRM] = nrm;
 #pragma unroll
-            for (int k = 0; k < PMAX; ++k)
-              if (k < P) {
-                R_f[RF_A + k] = a[k];
-                R_f[RF_XP + k] = a[k] * inv_l;
-              }
+            for (int k = 0; k < PC; ++k) {
+              R_f[RF_A + k] = a[k];
+              R_f[RF_XP + k] = x[k];
+            }
             R_i[RI_RUN] = run;
             if (stop >= 0) {
               R_i[RI_STOPPED] = 1;
@@ -678,11 +675,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           if (active && q == 0) dec[sl * GMAX + g] = stopped_before ? -2 : stop;
           __syncwarp();
         }
-        __syncwarp();
         if (lane == 0) {
-          // the peers' publications of this slot have been read: free the slot everywhere
-          const uint32_t fb = bar(B_XFREE + sl);
-          for (int cc = 0; cc < C; ++cc) mbar_arrive_cluster(map_to_rank(fb, cc));
           bool all = true;
           for (int g = 0; g < G; ++g) all &= (ri[g * RI_SIZE + RI_STOPPED] != 0);
           __threadfence_block();
@@ -706,8 +699,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       wait_phase(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, ctl, false, p.ws_status);
   }
   __syncthreads();  // (2) the ring is quiet: stage 0 can hold the final reduction
+  float* red = reinterpret_cast<float*>(sm + OFF_RED);
+  int* redi = reinterpret_cast<int*>(sm + OFF_RED + 4 * (GMAX * D + 2 * GMAX));
   if (warp >= 2 && warp < WARP_CTL) {
-    float* red = reinterpret_cast<float*>(sm + OFF_RED);
     const int er = 32 * (warp & 3) + lane;
 #pragma unroll
     for (int g = 0; g < GP; ++g)
@@ -720,11 +714,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       }
     }
   }
+  if (tid == 0) redi[0] = ctl[CTL_TREAD];
 
   // ---------------------------------------------------------------- cluster merge and output
-  float* red = reinterpret_cast<float*>(sm + OFF_RED);
-  int* redi = reinterpret_cast<int*>(sm + OFF_RED + 4 * (GMAX * D + 2 * GMAX));
-  if (tid == 0) redi[0] = ctl[CTL_TREAD];
   if (C > 1) cluster_sync_all(); else __syncthreads();
   if (rank == 0) {
     const uint32_t rb = smem_u32(red);
