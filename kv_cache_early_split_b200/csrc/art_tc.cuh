@@ -105,23 +105,49 @@ enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, 
 __device__ __forceinline__ uint32_t s_col(int b) { return 16u * b; }
 __device__ __forceinline__ uint32_t o_col(int b, int i) { return 32u + 32u * b + 16u * i; }
 
+// A wait gives up after this many SM clock cycles (about one second at B200 clocks).
+constexpr long long kWaitLimitCycles = 2000000000LL;
+// Longest single sleep of a waiting thread between checks of the exit / abort flags.
+constexpr uint32_t kSuspendNs = 2000;
+
 // Bounded wait that also gives up when the CTA aborted (a timeout elsewhere) or,
 // with watch_exit, when the ART controller ended the run.  Returns true when the
-// phase completed.
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* ctl, bool watch_exit,
-                                           int32_t* status, bool cluster_scope = false) {
-  const unsigned long long t0 = globaltimer_ns();
+// phase completed.  The barrier is polled before any clock is read, and the
+// limit uses the SM cycle counter (cheap) rather than the global timer.
+__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* ctl, bool watch_exit,
+                                        int32_t* status, bool cluster_scope) {
+  if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
   while (true) {
-    for (int i = 0; i < 32; ++i) {
-      const bool ok = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
-      if (ok) return true;
-    }
+    if (cluster_scope ? mbar_try_wait_cluster_sleep(bar, parity, kSuspendNs) : mbar_try_wait_sleep(bar, parity, kSuspendNs))
+      return true;
     if (ctl[CTL_ABORT]) return false;
     if (watch_exit && ctl[CTL_EXIT]) {
       __threadfence_block();
       return cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
     }
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(status, kStatusTimeout);
+      ctl[CTL_ABORT] = 1;
+      return false;
+    }
+  }
+}
+
+// Wait for the controller's decision of round rp; false when it will never come
+// (the run ended before that round, or the CTA aborted).
+__device__ __noinline__ bool wait_decision_phase(uint32_t bar, uint32_t parity, int rp, volatile int* ctl,
+                                                 int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (ctl[CTL_ABORT]) return false;
+    if (ctl[CTL_EXIT]) {
+      __threadfence_block();
+      if (rp > ctl[CTL_EXIT_ROUND]) return false;
+    }
+    if (clock64() - t0 > kWaitLimitCycles) {
       atomicOr(status, kStatusTimeout);
       ctl[CTL_ABORT] = 1;
       return false;
@@ -254,7 +280,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       for (int jl = 0; jl < my_blocks; ++jl) {
         if (ART && ctl[CTL_EXIT]) break;
         const int stage = jl % NSTG;
-        if (jl >= NSTG && !wait_phase(bar(B_EMPTY + stage), ((jl / NSTG) - 1) & 1, ctl, ART, p.ws_status)) break;
+        if (jl >= NSTG && !wait_phase(bar(B_EMPTY + stage), ((jl / NSTG) - 1) & 1, ctl, ART, p.ws_status, false)) break;
         const int j = jl * C + rank;
         const int p0 = pbeg + j * BLK;
         const uint32_t fb = bar(B_FULL + stage);
@@ -278,9 +304,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       int consumed = 0;
       auto issue_scores = [&](int jl) -> bool {
         const int stage = jl % NSTG, bb = jl & 1;
-        if (!wait_phase(bar(B_FULL + stage), (jl / NSTG) & 1, ctl, ART, p.ws_status)) return false;
+        if (!wait_phase(bar(B_FULL + stage), (jl / NSTG) & 1, ctl, ART, p.ws_status, false)) return false;
         consumed = jl + 1;
-        if (jl >= 2 && !wait_phase(bar(B_SFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status)) return false;
+        if (jl >= 2 && !wait_phase(bar(B_SFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status, false)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES);
 #pragma unroll
@@ -296,8 +322,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       for (int jl = 0; ok && jl < my_blocks; ++jl) {
         if (jl + 1 < my_blocks && !issue_scores(jl + 1)) break;
         const int stage = jl % NSTG, bb = jl & 1;
-        if (!wait_phase(bar(B_PFULL + bb), (jl >> 1) & 1, ctl, ART, p.ws_status)) break;
-        if (jl >= 2 && !wait_phase(bar(B_OFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status)) break;
+        if (!wait_phase(bar(B_PFULL + bb), (jl >> 1) & 1, ctl, ART, p.ws_status, false)) break;
+        if (jl >= 2 && !wait_phase(bar(B_OFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status, false)) break;
         tc_fence_after();
         const int ntl = block_tiles(jl);
         const uint32_t v_addr = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES + 32768);
@@ -315,7 +341,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       ctl[CTL_CONSUMED] = consumed;
       // every issued tensor-core op has completed before the drain barrier fires
       umma_commit(bar(B_DRAIN));
-      wait_phase(bar(B_DRAIN), 0, ctl, false, p.ws_status);
+      wait_phase(bar(B_DRAIN), 0, ctl, false, p.ws_status, false);
     }
     __syncwarp();
   } else if (warp < WARP_CTL) {
@@ -330,7 +356,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     const int w_lo = (er / TE) * w_n;  // first warp of this row's tile
     auto epi_wait = [&](uint32_t bb_, uint32_t parity, bool watch_exit) -> bool {
       bool ok = true;
-      if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status);
+      if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status, false);
       return named_barrier_and(BAR_EPI, 128, ok);
     };
     float ot[KT_MAX][GP], pend1[KT_MAX][GP], pend2[KT_MAX][GP];
@@ -366,26 +392,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     // wait (leader) for the controller's decision of round rp; false if it will never come
     auto wait_decision = [&](int rp) -> bool {
       bool got = true;
-      if (leader) {
-        got = false;
-        const unsigned long long t0w = globaltimer_ns();
-        while (true) {
-          if (mbar_try_wait(bar(B_DEC + rp % NSLOT), (rp / NSLOT) & 1)) {
-            got = true;
-            break;
-          }
-          if (ctl[CTL_ABORT]) break;
-          if (ctl[CTL_EXIT]) {
-            __threadfence_block();
-            if (rp > ctl[CTL_EXIT_ROUND]) break;
-          }
-          if (globaltimer_ns() - t0w > kWaitLimitNs) {
-            atomicOr(p.ws_status, kStatusTimeout);
-            ctl[CTL_ABORT] = 1;
-            break;
-          }
-        }
-      }
+      if (leader) got = wait_decision_phase(bar(B_DEC + rp % NSLOT), (rp / NSLOT) & 1, rp, ctl, p.ws_status);
       return named_barrier_and(BAR_EPI, 128, got);
     };
 
@@ -484,28 +491,39 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     };
 
     const int iters = ART ? R : my_blocks;
-    bool streaming = my_blocks > 0 && s_phase(0);
-    for (int it = 0; it < iters; ++it) {
+    bool streaming = true;
+    for (int it = -1; it < iters; ++it) {
+      // scores of the next own block first, then the readback of this one
+      if (it + 1 < my_blocks && streaming) streaming = s_phase(it + 1);
+      if (it < 0) continue;
       int ntl = 0;
-      if (it < my_blocks && streaming) {
-        const bool next_ok = (it + 1 < my_blocks) ? s_phase(it + 1) : true;
-        streaming = o_phase(it, ntl) && next_ok;
-      }
+      if (it < my_blocks && streaming) streaming = o_phase(it, ntl);
       if (!ART) {
         if (!streaming && it + 1 < iters) break;  // aborted
         continue;
       }
       const int r = it;
+      // Merge, in order, the pending rounds lo..hi (a subset of r-2, r-1, r held in pend2,
+      // pend1, ot) by their decisions.  A single call site keeps the loop body small.
+      auto merge_span = [&](int lo, int hi) -> bool {
+#pragma unroll 1
+        for (int rk = lo; rk <= hi; ++rk) {
+          if (!wait_decision(rk)) return false;
+          const int k = rk - (r - 2);
+          float tmp[KT_MAX][GP];
+#pragma unroll
+          for (int i = 0; i < KT_MAX; ++i)
+#pragma unroll
+            for (int g = 0; g < GP; ++g) tmp[i][g] = (k == 0) ? pend2[i][g] : ((k == 1) ? pend1[i][g] : ot[i][g]);
+          merge_round(rk, tmp, (k == 0) ? ntl2 : ((k == 1) ? ntl1 : ntl));
+        }
+        return true;
+      };
       // stop once the controller has ended the run: merge every round it decided, then leave
       if (named_barrier_or(BAR_EPI, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]))) {
         const bool aborted = named_barrier_or(BAR_EPI, 128, leader && ctl[CTL_ABORT] != 0);
         const int er_round = ctl[CTL_EXIT_ROUND];  // written before the exit flag, never changed after
-        if (!aborted) {
-          if (r - 2 >= 0 && r - 2 <= er_round && wait_decision(r - 2)) merge_round(r - 2, pend2, ntl2);
-          if (r - 1 >= 0 && r - 1 <= er_round && wait_decision(r - 1)) merge_round(r - 1, pend1, ntl1);
-          if (r <= er_round && wait_decision(r)) merge_round(r, ot, ntl);
-        }
-        ntl1 = ntl2 = 0;
+        if (!aborted) merge_span(max(0, r - LAG), min(r, er_round));
         break;
       }
       // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
@@ -534,8 +552,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           mbar_arrive_cluster_relaxed(map_to_rank(bar(B_XFULL + sl), er));
         }
       }
-      // merge round r - LAG by its decision (no decision: the run ended; the exit path covers it)
-      if (r >= LAG && wait_decision(r - LAG)) merge_round(r - LAG, pend2, ntl2);
+      // merge round r - LAG by its decision; after the last round, everything still pending
+      // (no decision: the run ended, and the exit path above merges what was decided)
+      merge_span(max(0, r - LAG), (r == iters - 1) ? r : r - LAG);
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i)
 #pragma unroll
@@ -545,11 +564,6 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         }
       ntl2 = ntl1;
       ntl1 = ntl;
-      if (r == iters - 1) {
-        // end of the rounds: the last LAG rounds still wait for their decisions
-        if (r - 1 >= 0 && wait_decision(r - 1)) merge_round(r - 1, pend2, ntl2);
-        if (wait_decision(r)) merge_round(r, pend1, ntl1);
-      }
     }
   } else {
     // ------------------------------------------------------------ ART controller
@@ -696,7 +710,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   // drain: copies that were issued but never consumed still land in shared memory
   if (warp == WARP_TMA && lane == 0) {
     for (int ord = ctl[CTL_CONSUMED]; ord < ctl[CTL_ISSUED]; ++ord)
-      wait_phase(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, ctl, false, p.ws_status);
+      wait_phase(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, ctl, false, p.ws_status, false);
   }
   __syncthreads();  // (2) the ring is quiet: stage 0 can hold the final reduction
   float* red = reinterpret_cast<float*>(sm + OFF_RED);
