@@ -114,7 +114,7 @@ constexpr uint32_t kSuspendNs = 2000;
 // with watch_exit, when the ART controller ended the run.  Returns true when the
 // phase completed.  The barrier is polled before any clock is read, and the
 // limit uses the SM cycle counter (cheap) rather than the global timer.
-__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* ctl, bool watch_exit,
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* ctl, bool watch_exit,
                                         int32_t* status, bool cluster_scope) {
   if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -136,7 +136,7 @@ __device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile 
 
 // Wait for the controller's decision of round rp; false when it will never come
 // (the run ended before that round, or the CTA aborted).
-__device__ __noinline__ bool wait_decision_phase(uint32_t bar, uint32_t parity, int rp, volatile int* ctl,
+__device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parity, int rp, volatile int* ctl,
                                                  int32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
