@@ -172,6 +172,16 @@ art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, 
  * synchronisation or copy failed). */
 art_status art_read_device_status(void* ws, void* stream);
 
+/* Base name of the CUDA kernel a call with this shape would launch for its
+ * main pass: "art_decode_tc_kernel" (tcgen05 tensor-core path: bf16, d = 128,
+ * tile 64 or 128, Hq/Hkv <= 8, full or ART) or "art_decode_kernel" (CUDA-core
+ * path, everything else); NULL for an invalid or unsupported shape.  kv_q8 != 0
+ * asks about art_decode_attn_q8_skipv (dtype is then ignored); with_art != 0
+ * about the ART variant.  A query only: no CUDA call, nothing enqueued.  The
+ * pages have no counterpart; it names the kernel for profiling and reports.
+ * With num_splits > 1 a second, small kernel (art_combine_kernel) follows. */
+const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_q8, int32_t with_art);
+
 /* Static, human-readable name of a status code. */
 const char* art_status_string(art_status status);
 

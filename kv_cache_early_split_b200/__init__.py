@@ -13,7 +13,7 @@ from dataclasses import dataclass
 from . import capi
 from .capi import ArtError
 
-__all__ = ["capi", "ArtError", "DeviceProblem", "upload", "decode"]
+__all__ = ["capi", "ArtError", "DeviceProblem", "upload", "decode", "kernel_name"]
 
 
 @dataclass
@@ -133,6 +133,15 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
     if check and rc != capi.ART_OK:
         raise ArtError(rc, name)
     return rc
+
+
+def kernel_name(dp: DeviceProblem, mode: str) -> str:
+    """Base name of the main CUDA kernel decode(dp, mode) launches (art_kernel_name)."""
+    dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
+    name = capi.art_kernel_name(dp.shape, dtype, mode.startswith("q8"), mode in ("art", "q8_art"))
+    if name is None:
+        raise ArtError(capi.ART_ERR_UNSUPPORTED, "art_kernel_name")
+    return name
 
 
 def device_status(dp: DeviceProblem, stream=None) -> int:

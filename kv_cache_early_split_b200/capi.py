@@ -34,6 +34,7 @@ EXPORTS = (
     "art_decode_attn_q8_skipv",
     "art_read_device_status",
     "art_status_string",
+    "art_kernel_name",
 )
 
 
@@ -97,6 +98,8 @@ def lib() -> ctypes.CDLL:
             L.art_read_device_status.argtypes = [_P, _P]
             L.art_status_string.restype = ctypes.c_char_p
             L.art_status_string.argtypes = [ctypes.c_int]
+            L.art_kernel_name.restype = ctypes.c_char_p
+            L.art_kernel_name.argtypes = [_SH, ctypes.c_int, ctypes.c_int32, ctypes.c_int32]
             _lib = L
     return _lib
 
@@ -145,6 +148,12 @@ def art_read_device_status(ws, stream) -> int:
 
 def art_status_string(code: int) -> str:
     return lib().art_status_string(int(code)).decode()
+
+
+def art_kernel_name(shape, dtype, kv_q8, with_art):
+    """Base name of the main kernel a call with this shape launches, or None if unsupported."""
+    r = lib().art_kernel_name(ctypes.byref(shape), int(dtype), int(bool(kv_q8)), int(bool(with_art)))
+    return None if r is None else r.decode()
 
 
 def make_params(eps_scale: float, eps_dir: float, patience: int, lanes) -> art_params:

@@ -585,6 +585,23 @@ art_status art_read_device_status(void* ws, void* stream) {
   return ART_OK;
 }
 
+const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_q8, int32_t with_art) {
+  if (!shape_ok(shape)) return nullptr;
+  int kind, mode;
+  if (kv_q8) {
+    kind = artk::KV_Q8;
+    mode = with_art ? artk::MODE_SKIP_ART : artk::MODE_SKIP;
+  } else {
+    if (dtype != ART_F32 && dtype != ART_BF16) return nullptr;
+    kind = dtype == ART_F32 ? artk::KV_F32 : artk::KV_BF16;
+    mode = with_art ? artk::MODE_ART : artk::MODE_FULL;
+  }
+  if (tc_eligible(kind, mode, shape)) return "art_decode_tc_kernel";
+  KernelInfo ki;
+  if (!pick_kernel(kind, mode, shape->d, shape->Hq / shape->Hkv, &ki)) return nullptr;
+  return "art_decode_kernel";
+}
+
 const char* art_status_string(art_status status) {
   switch (status) {
     case ART_OK: return "ART_OK";

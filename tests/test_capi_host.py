@@ -123,3 +123,18 @@ def test_invalid_arguments_q8(L):
 
 def test_read_status_rejects_null(L):
     assert capi.art_read_device_status(None, None) == capi.ART_ERR_INVALID_ARG
+
+
+def test_kernel_name_query(L):
+    """The selection query follows the documented tensor-core eligibility rule."""
+    tc = shape(Hq=32, Hkv=8, d=128, tile=64)
+    assert capi.art_kernel_name(tc, capi.ART_BF16, False, True) == "art_decode_tc_kernel"
+    assert capi.art_kernel_name(tc, capi.ART_BF16, False, False) == "art_decode_tc_kernel"
+    assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=128, tile=128), capi.ART_BF16, 0, 1) == "art_decode_tc_kernel"
+    assert capi.art_kernel_name(tc, capi.ART_F32, False, True) == "art_decode_kernel"
+    assert capi.art_kernel_name(tc, capi.ART_BF16, True, True) == "art_decode_kernel"
+    assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=64, tile=64), capi.ART_BF16, 0, 1) == "art_decode_kernel"
+    assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=128, tile=32), capi.ART_BF16, 0, 1) == "art_decode_kernel"
+    assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=96, tile=64), capi.ART_BF16, 0, 1) is None
+    assert capi.art_kernel_name(shape(Hq=32, Hkv=2, d=128, tile=64), capi.ART_BF16, 0, 1) is None
+    assert capi.art_kernel_name(shape(B=0), capi.ART_BF16, 0, 1) is None
