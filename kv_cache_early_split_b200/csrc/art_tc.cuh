@@ -354,6 +354,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     const uint32_t lane_base = static_cast<uint32_t>(32 * wq) << 16;
     const int w_n = TE / 32;           // warps per tile
     const int w_lo = (er / TE) * w_n;  // first warp of this row's tile
+    // reductions over the warps of one tile run over all four warps with a predicate
+    // (fixed trip count, no loop branches)
+    auto in_tile = [&](int w, int lo) { return w >= lo && w < lo + w_n; };
     auto epi_wait = [&](uint32_t bb_, uint32_t parity, bool watch_exit) -> bool {
       bool ok = true;
       if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status, false);
@@ -420,7 +423,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float mt = -INFINITY;
-        for (int w = w_lo; w < w_lo + w_n; ++w) mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (in_tile(w, w_lo)) mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
         red[g] = pw[g] = (s2[g] == -INFINITY) ? 0.f : ex2_fast(s2[g] - mt);
       }
       {
@@ -468,20 +473,30 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       }
       tc_fence_before();
       mbar_arrive(bar(B_OFREE + bb));
-#pragma unroll
-      for (int i = 0; i < KT_MAX; ++i) {
-        if (i >= ntl) continue;
-        const int lo_w = i * w_n;
+      if (!ART) {  // the block is one tile: every thread merges it into its own state
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
           float mt = -INFINITY, lt = 0.f;
-          for (int w = lo_w; w < lo_w + w_n; ++w) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
             mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
             lt += wsum[(bb * 4 + w) * GMAX + g];
           }
-          if (!ART) {
-            if (g < G) merge_tile(g, mt, lt, ot[i][g]);
-          } else if (leader) {
+          if (g < G) merge_tile(g, mt, lt, ot[0][g]);
+        }
+      } else if (leader) {  // tile statistics for the round's publication and merge
+#pragma unroll
+        for (int i = 0; i < KT_MAX; ++i) {
+          if (i >= ntl) continue;
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            float mt = -INFINITY, lt = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              if (in_tile(w, i * w_n)) {
+                mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
+                lt += wsum[(bb * 4 + w) * GMAX + g];
+              }
             tst[((jl % NSLOT) * KT_MAX + i) * GMAX * 2 + g * 2 + 0] = mt;
             tst[((jl % NSLOT) * KT_MAX + i) * GMAX * 2 + g * 2 + 1] = lt;
           }
