@@ -534,16 +534,18 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         }
         return true;
       };
-      // stop once the controller has ended the run: merge every round it decided, then leave
-      if (named_barrier_or(BAR_EPI, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]))) {
+      // Once the controller has ended the run, merge every round it decided and leave.
+      // Otherwise publish round r, then merge round r - LAG by its decision (after the last
+      // round, everything still pending).  Both paths share one merge call site.
+      const bool leaving = named_barrier_or(BAR_EPI, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]));
+      int m_hi;
+      if (leaving) {
         const bool aborted = named_barrier_or(BAR_EPI, 128, leader && ctl[CTL_ABORT] != 0);
         const int er_round = ctl[CTL_EXIT_ROUND];  // written before the exit flag, never changed after
-        if (!aborted) merge_span(max(0, r - LAG), min(r, er_round));
-        break;
-      }
-      // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
-      const int sl = r % NSLOT;
-      {
+        m_hi = aborted ? -1 : min(r, er_round);
+      } else {
+        // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
+        const int sl = r % NSLOT;
         float* ps = pub + sl * (PUB_SLOT / 4);
         const int pi = l2p[er];
 #pragma unroll
@@ -566,10 +568,10 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           fence_acq_rel_cluster();
           mbar_arrive_cluster_relaxed(map_to_rank(bar(B_XFULL + sl), er));
         }
+        m_hi = (r == iters - 1) ? r : r - LAG;
       }
-      // merge round r - LAG by its decision; after the last round, everything still pending
-      // (no decision: the run ended, and the exit path above merges what was decided)
-      merge_span(max(0, r - LAG), (r == iters - 1) ? r : r - LAG);
+      merge_span(max(0, r - LAG), m_hi);
+      if (leaving) break;
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i)
 #pragma unroll
