@@ -15,22 +15,26 @@
 // Full attention treats a whole 128-position block as one tile (the tile size
 // has no effect on its result); ART keeps the caller's tiles.
 //
-// Warp roles (224 threads, one CTA per SM):
-//   warp 0      TMA producer: K/V blocks (4 tiled 3-D TMA loads, 64 KiB) into a 3-deep ring
-//   warp 1      MMA issuer (one lane) and tensor-memory owner
-//   warps 2..5  epilogue: scores -> per-tile max / weights -> P^T in smem; O readback
-//               (thread = d row) -> online merge in registers; ART publication.
-//               The scores step of block j+1 runs before the readback of block j.
-//   warp 6      ART controller: per round, reads all CTAs' publications through
-//               distributed shared memory and replays the rule in tile order.
-// Blocks are dealt round-robin over the cluster exactly as in art_decode_kernel.
+// Warp roles (384 threads, one CTA per SM):
+//   warp 0       TMA producer: K/V blocks (4 tiled 3-D TMA loads, 64 KiB) into a 3-deep ring
+//   warp 1       MMA issuer (one lane) and tensor-memory owner
+//   warp 2       ART controller: per round, reads all CTAs' publications through
+//                distributed shared memory and replays the rule in tile order.
+//   warp 3       idle
+//   warps 4..11  two epilogue warpgroups (thread = TMEM lane); warpgroup wg takes the
+//                CTA's own blocks wg, wg + 2, ...: scores -> per-tile max / weights ->
+//                P^T in smem; O readback (thread = d row) -> online merge in registers;
+//                ART publication.  While one warpgroup waits on a barrier or the tensor
+//                cores, the other works on the next block.
+// Blocks are dealt round-robin over the cluster exactly as in art_decode_kernel; the
+// CTA's own block r belongs to ART round r.
 //
-// ART exchange without back-pressure barriers: rounds cycle through NSLOT = 6
-// publication slots and the epilogue merges round r - LAG (LAG = 2) after
-// publishing round r.  Before a CTA publishes round x it has merged round
-// x-1-LAG, so its controller has decided that round, so every CTA had published
-// it, so every CTA had merged round x-2-2*LAG, so every controller had decided
-// -- and finished reading -- round x-2-2*LAG = x-NSLOT: the slot is free.
+// ART exchange without back-pressure barriers: rounds cycle through NSLOT publication
+// slots and a warpgroup merges round r - LAG after publishing round r (LAG = NWG = 2:
+// its own previous round).  Before a warpgroup publishes round x it has merged round
+// x-NWG-LAG, so its controller has decided that round, so every CTA had published it,
+// so every CTA had merged round x-2*NWG-2*LAG, so every controller had decided -- and
+// finished reading -- every round up to x-2*NWG-2*LAG = x-NSLOT: the slot is free.
 #pragma once
 
 #include <cuda.h>
@@ -47,15 +51,17 @@ namespace tc {
 constexpr int BLK = 128;  // positions per block (= MMA M for the scores)
 constexpr int D = 128;
 constexpr int NSTG = 3;
-constexpr int NWARP = 7;
+constexpr int NWG = 2;  // epilogue warpgroups, taking alternate blocks
+constexpr int NWARP = 4 + 4 * NWG;
 constexpr int NTHR = NWARP * 32;
 constexpr int KT_MAX = 2;  // ART tiles per block (tile 64)
 constexpr int STAGE_BYTES = 4 * 16384;
 constexpr uint32_t TMEM_COLS = 128;
-constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_CTL = 6;
-constexpr int BAR_EPI = 1;  // named barrier of the 128 epilogue threads
-constexpr int LAG = 2;
-constexpr int NSLOT = 2 + 2 * LAG;
+constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_CTL = 2, WARP_EPI0 = 4;
+constexpr int BAR_EPI = 1;  // named barriers BAR_EPI + wg: the 128 threads of epilogue warpgroup wg
+constexpr int LAG = 2;      // a round is merged LAG rounds after it was published (LAG % NWG == 0)
+constexpr int NSLOT = 2 * NWG + 2 * LAG;
+static_assert(LAG % NWG == 0, "a warpgroup merges its own rounds");
 
 struct TcParams {
   CUtensorMap tmK;  // 64-byte aligned (first members)
@@ -83,23 +89,30 @@ enum : int {
   B_OFULL = B_PFULL + 2, B_OFREE = B_OFULL + 2, B_XFULL = B_OFREE + 2, B_DEC = B_XFULL + NSLOT,
   B_DRAIN = B_DEC + NSLOT, B_COUNT = B_DRAIN + 1
 };
-static_assert(B_COUNT * 8 <= 256, "barrier area");
-constexpr uint32_t OFF_WRED = OFF_BAR + 256;                           // [2][4][GMAX] per-warp maxima
+static_assert(B_COUNT * 8 <= 512, "barrier area");
+constexpr uint32_t OFF_WRED = OFF_BAR + 512;                           // [2][4][GMAX] per-warp maxima
 constexpr uint32_t OFF_WSUM = OFF_WRED + 4 * 2 * 4 * GMAX;             // [2][4][GMAX] per-warp sums
 constexpr uint32_t OFF_TST = OFF_WSUM + 4 * 2 * 4 * GMAX;              // [NSLOT][KT][GMAX][2] tile (m, l)
-constexpr uint32_t OFF_PUB = OFF_TST + 4 * NSLOT * KT_MAX * GMAX * 2;  // [NSLOT][KT][GMAX][2+PMAX]
-constexpr uint32_t PUB_ENTRY = 2 + PMAX;
-constexpr uint32_t PUB_SLOT = 4 * KT_MAX * GMAX * PUB_ENTRY;
-constexpr uint32_t OFF_DEC = OFF_PUB + NSLOT * PUB_SLOT;  // [NSLOT][GMAX] int
-constexpr uint32_t OFF_CTL = OFF_DEC + 4 * NSLOT * GMAX;  // [16] int
-constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;             // [GMAX][RF_SIZE] float
-constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;  // [GMAX][RI_SIZE] int
-constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;  // [D] int8
-constexpr uint32_t SMEM_USED = OFF_L2P + D;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
-static_assert(SMEM_BYTES <= 232448, "shared memory per block");
-// final reduction (aliases stage 0 after the pipeline has drained)
-constexpr uint32_t OFF_RED = 0;  // [GMAX][D] numerators, then [GMAX] m, [GMAX] l, [4] ints
+constexpr uint32_t OFF_DEC = OFF_TST + 4 * NSLOT * KT_MAX * GMAX * 2;  // [NSLOT][GMAX] int
+constexpr uint32_t OFF_CTL = OFF_DEC + 4 * NSLOT * GMAX;               // [16] int
+constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;                          // [GMAX][RF_SIZE] float
+constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;               // [GMAX][RI_SIZE] int
+constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;              // [D] int8
+constexpr uint32_t OFF_PUB = OFF_L2P + D;  // [NSLOT][KT][GP][2+PC] float, sized per kernel (Pub)
+// Publication slots of a kernel with GP heads per kv head and probe capacity PC:
+// per tile and head, (m_t, l_t) then the PC probe lanes of O_t.
+template <int GP, int PC>
+struct Pub {
+  static constexpr uint32_t ENTRY = 2 + PC;
+  static constexpr uint32_t SLOT = 4 * KT_MAX * GP * ENTRY;
+  static constexpr uint32_t SMEM_BYTES = OFF_PUB + NSLOT * SLOT + 1024;  // + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "shared memory per block");
+};
+constexpr uint32_t SMEM_BYTES = Pub<GMAX, PMAX>::SMEM_BYTES;  // the largest instantiation
+// final reduction (aliases stage 0 after the pipeline has drained):
+// [NWG][GMAX][D] numerators, then [NWG][GMAX] m, [NWG][GMAX] l, [4] ints
+constexpr uint32_t OFF_RED = 0;
+constexpr uint32_t RED_M = NWG * GMAX * D, RED_L = RED_M + NWG * GMAX, RED_I = RED_L + NWG * GMAX;
 enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, CTL_TREAD, CTL_TMEM };
 
 __device__ __forceinline__ uint32_t s_col(int b) { return 16u * b; }
@@ -160,6 +173,7 @@ __device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parit
 template <int GP, int MODE, int PC>
 __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
+  using PB = Pub<GP, PC>;
   static_assert(GP >= 1 && GP <= 8, "up to 8 query heads per kv head");
   static_assert(PC == 16 || PC == 32, "probe capacity");
   extern __shared__ uint8_t smem_raw[];
@@ -233,7 +247,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   for (int i = tid; i < D; i += NTHR) l2p[i] = -1;
   for (int i = tid; i < 8192 / 16; i += NTHR) reinterpret_cast<uint4*>(sm + OFF_P)[i] = make_uint4(0, 0, 0, 0);
   if (ART)
-    for (int i = tid; i < static_cast<int>(NSLOT * PUB_SLOT / 16); i += NTHR)
+    for (int i = tid; i < static_cast<int>(NSLOT * PB::SLOT / 16); i += NTHR)
       reinterpret_cast<uint4*>(sm + OFF_PUB)[i] = make_uint4(0, 0, 0, 0);
   if (tid < GMAX) {
     float* r = rf + tid * RF_SIZE;
@@ -344,10 +358,14 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       wait_phase(bar(B_DRAIN), 0, ctl, false, p.ws_status, false);
     }
     __syncwarp();
-  } else if (warp < WARP_CTL) {
-    // ------------------------------------------------------------ epilogue warpgroup
-    // All 128 threads take every branch together: mbarrier waits are done by one
-    // leader thread and their outcome is shared with a reducing named barrier.
+  } else if (warp >= WARP_EPI0) {
+    // ------------------------------------------------------------ epilogue warpgroups
+    // Warpgroup wg takes the own blocks jl = wg, wg + NWG, ... (TMEM and smem buffers
+    // bb = jl & 1 = wg).  All 128 threads of a warpgroup take every branch together:
+    // mbarrier waits are done by one leader thread and their outcome is shared with a
+    // reducing named barrier of that warpgroup.
+    const int wg = (warp - WARP_EPI0) >> 2;
+    const int bar_epi = BAR_EPI + wg;
     const int wq = warp & 3;
     const int er = 32 * wq + lane;  // TMEM lane: position row of S, d row of O
     const bool leader = (er == 0);
@@ -360,14 +378,17 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     auto epi_wait = [&](uint32_t bb_, uint32_t parity, bool watch_exit) -> bool {
       bool ok = true;
       if (leader) ok = wait_phase(bb_, parity, ctl, watch_exit, p.ws_status, false);
-      return named_barrier_and(BAR_EPI, 128, ok);
+      return named_barrier_and(bar_epi, 128, ok);
     };
-    float ot[KT_MAX][GP], pend1[KT_MAX][GP], pend2[KT_MAX][GP];
+    // ot: this block's tile outputs; pnd: the warpgroup's previous round (published, not
+    // merged yet: a round is merged LAG = NWG rounds, i.e. one own round, after publication)
+    static_assert(LAG == NWG, "one pending own round");
+    float ot[KT_MAX][GP], pnd[KT_MAX][GP];
 #pragma unroll
     for (int i = 0; i < KT_MAX; ++i)
 #pragma unroll
-      for (int g = 0; g < GP; ++g) ot[i][g] = pend1[i][g] = pend2[i][g] = 0.f;
-    int ntl1 = 0, ntl2 = 0;
+      for (int g = 0; g < GP; ++g) ot[i][g] = pnd[i][g] = 0.f;
+    int ntl_p = 0;
     auto merge_tile = [&](int g, float mt, float lt, float o) {
       const float M = fmaxf(m_own[g], mt);
       const float a = rescale_fast(m_own[g], M), bt = rescale_fast(mt, M);
@@ -396,7 +417,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     auto wait_decision = [&](int rp) -> bool {
       bool got = true;
       if (leader) got = wait_decision_phase(bar(B_DEC + rp % NSLOT), (rp / NSLOT) & 1, rp, ctl, p.ws_status);
-      return named_barrier_and(BAR_EPI, 128, got);
+      return named_barrier_and(bar_epi, 128, got);
     };
 
     // scores -> weights -> P^T (hi, lo) in smem for own block jl; false if the run ended
@@ -419,7 +440,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         const float wm = warp_reduce_heads<GP, true>(red, lane);
         if ((lane & (32 / GP - 1)) == 0) wred[(bb * 4 + wq) * GMAX + lane / (32 / GP)] = wm;
       }
-      named_barrier(BAR_EPI, 128);
+      named_barrier(bar_epi, 128);
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         float mt = -INFINITY;
@@ -507,46 +528,43 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 
     const int iters = ART ? R : my_blocks;
     bool streaming = true;
-    for (int it = -1; it < iters; ++it) {
-      // scores of the next own block first, then the readback of this one
-      if (it + 1 < my_blocks && streaming) streaming = s_phase(it + 1);
-      if (it < 0) continue;
+    for (int r = wg; r < iters; r += NWG) {  // own block r of the CTA = ART round r
       int ntl = 0;
-      if (it < my_blocks && streaming) streaming = o_phase(it, ntl);
+      if (r < my_blocks && streaming) streaming = s_phase(r);
+      if (r < my_blocks && streaming) streaming = o_phase(r, ntl);
       if (!ART) {
-        if (!streaming && it + 1 < iters) break;  // aborted
+        if (!streaming) break;  // aborted
         continue;
       }
-      const int r = it;
-      // Merge, in order, the pending rounds lo..hi (a subset of r-2, r-1, r held in pend2,
-      // pend1, ot) by their decisions.  A single call site keeps the loop body small.
+      // Merge, in order, the warpgroup's rounds lo, lo + NWG, .., hi (r - LAG held in pnd,
+      // r in ot) by their decisions.  A single call site keeps the loop body small.
       auto merge_span = [&](int lo, int hi) -> bool {
 #pragma unroll 1
-        for (int rk = lo; rk <= hi; ++rk) {
+        for (int rk = lo; rk <= hi; rk += NWG) {
           if (!wait_decision(rk)) return false;
-          const int k = rk - (r - 2);
+          const bool cur = (rk == r);
           float tmp[KT_MAX][GP];
 #pragma unroll
           for (int i = 0; i < KT_MAX; ++i)
 #pragma unroll
-            for (int g = 0; g < GP; ++g) tmp[i][g] = (k == 0) ? pend2[i][g] : ((k == 1) ? pend1[i][g] : ot[i][g]);
-          merge_round(rk, tmp, (k == 0) ? ntl2 : ((k == 1) ? ntl1 : ntl));
+            for (int g = 0; g < GP; ++g) tmp[i][g] = cur ? ot[i][g] : pnd[i][g];
+          merge_round(rk, tmp, cur ? ntl : ntl_p);
         }
         return true;
       };
       // Once the controller has ended the run, merge every round it decided and leave.
-      // Otherwise publish round r, then merge round r - LAG by its decision (after the last
-      // round, everything still pending).  Both paths share one merge call site.
-      const bool leaving = named_barrier_or(BAR_EPI, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]));
+      // Otherwise publish round r, then merge round r - LAG by its decision (after the
+      // warpgroup's last round, everything still pending).  Both paths share one merge site.
+      const bool leaving = named_barrier_or(bar_epi, 128, leader && (ctl[CTL_EXIT] || ctl[CTL_ABORT]));
       int m_hi;
       if (leaving) {
-        const bool aborted = named_barrier_or(BAR_EPI, 128, leader && ctl[CTL_ABORT] != 0);
+        const bool aborted = named_barrier_or(bar_epi, 128, leader && ctl[CTL_ABORT] != 0);
         const int er_round = ctl[CTL_EXIT_ROUND];  // written before the exit flag, never changed after
         m_hi = aborted ? -1 : min(r, er_round);
       } else {
         // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
         const int sl = r % NSLOT;
-        float* ps = pub + sl * (PUB_SLOT / 4);
+        float* ps = pub + sl * (PB::SLOT / 4);
         const int pi = l2p[er];
 #pragma unroll
         for (int i = 0; i < KT_MAX; ++i) {
@@ -554,7 +572,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
           for (int g = 0; g < GP; ++g) {
             if (g < G) {
-              float* e = ps + (i * GMAX + g) * PUB_ENTRY;
+              float* e = ps + (i * GP + g) * PB::ENTRY;
               if (leader) {
                 e[0] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2];
                 e[1] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2 + 1];
@@ -563,26 +581,22 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
             }
           }
         }
-        named_barrier(BAR_EPI, 128);
+        named_barrier(bar_epi, 128);
         if (er < C) {  // one thread per peer: make the slot visible, then signal that CTA
           fence_acq_rel_cluster();
           mbar_arrive_cluster_relaxed(map_to_rank(bar(B_XFULL + sl), er));
         }
-        m_hi = (r == iters - 1) ? r : r - LAG;
+        m_hi = (r + NWG >= iters) ? r : r - LAG;
       }
-      merge_span(max(0, r - LAG), m_hi);
+      merge_span(r >= LAG ? r - LAG : r, m_hi);
       if (leaving) break;
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i)
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          pend2[i][g] = pend1[i][g];
-          pend1[i][g] = ot[i][g];
-        }
-      ntl2 = ntl1;
-      ntl1 = ntl;
+        for (int g = 0; g < GP; ++g) pnd[i][g] = ot[i][g];
+      ntl_p = ntl;
     }
-  } else {
+  } else if (warp == WARP_CTL) {
     // ------------------------------------------------------------ ART controller
     if constexpr (ART) {
       const int TQ = C * KT;    // tiles per round (power of two <= 32)
@@ -596,7 +610,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r / NSLOT) & 1, ctl, false, p.ws_status, true);
         if (!__shfl_sync(0xffffffffu, okw, 0)) break;
         const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
-        const uint32_t slot_base = smem_u32(pub) + sl * PUB_SLOT;
+        const uint32_t slot_base = smem_u32(pub) + sl * PB::SLOT;
         for (int g0 = 0; g0 < G; g0 += HPP) {
           const int g = g0 + hh;
           const bool active = g < G;
@@ -609,7 +623,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
           for (int k = 0; k < PC; ++k) a[k] = 0.f;
           if (valid) {  // this tile's (m, l, probe) from the CTA that computed it
-            const uint32_t src = map_to_rank(slot_base + ((i * GMAX + g) * PUB_ENTRY) * 4, c);
+            const uint32_t src = map_to_rank(slot_base + ((i * GP + g) * PB::ENTRY) * 4, c);
             ld_dsmem_v2(src, m, l);
 #pragma unroll
             for (int k = 0; k < PC; k += 2) ld_dsmem_v2(src + 8 + 4 * k, a[k], a[k + 1]);
@@ -731,17 +745,18 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   }
   __syncthreads();  // (2) the ring is quiet: stage 0 can hold the final reduction
   float* red = reinterpret_cast<float*>(sm + OFF_RED);
-  int* redi = reinterpret_cast<int*>(sm + OFF_RED + 4 * (GMAX * D + 2 * GMAX));
-  if (warp >= 2 && warp < WARP_CTL) {
+  int* redi = reinterpret_cast<int*>(sm + OFF_RED + 4 * RED_I);
+  if (warp >= WARP_EPI0) {  // each warpgroup leaves its own online-softmax state
+    const int wg = (warp - WARP_EPI0) >> 2;
     const int er = 32 * (warp & 3) + lane;
 #pragma unroll
     for (int g = 0; g < GP; ++g)
-      if (g < G) red[g * D + er] = acc[g];
+      if (g < G) red[(wg * GMAX + g) * D + er] = acc[g];
     if (er == 0) {
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
-        red[GMAX * D + g] = m_own[g];
-        red[GMAX * D + GMAX + g] = l_own[g];
+        red[RED_M + wg * GMAX + g] = m_own[g];
+        red[RED_L + wg * GMAX + g] = l_own[g];
       }
     }
   }
@@ -753,27 +768,26 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     const uint32_t rb = smem_u32(red);
     for (int idx = tid; idx < G * D; idx += NTHR) {
       const int g = idx / D, dd = idx % D;
+      // the C x NWG partial states of head g (C > 1: read from each rank's shared memory)
+      auto part_f = [&](int cc, uint32_t off) -> float {
+        return (C > 1) ? ld_dsmem_f32(map_to_rank(rb + 4 * off, cc)) : red[off];
+      };
       float M = -INFINITY;
-      for (int cc = 0; cc < C; ++cc) {
-        const float mc = (C > 1) ? ld_dsmem_f32(map_to_rank(rb + 4 * (GMAX * D + g), cc)) : red[GMAX * D + g];
-        M = fmaxf(M, mc);
-      }
+      for (int cc = 0; cc < C; ++cc)
+#pragma unroll
+        for (int w = 0; w < NWG; ++w) M = fmaxf(M, part_f(cc, RED_M + w * GMAX + g));
       float den = 0.f, num = 0.f;
       for (int cc = 0; cc < C; ++cc) {
-        float mc, lc, ac;
-        if (C > 1) {
-          mc = ld_dsmem_f32(map_to_rank(rb + 4 * (GMAX * D + g), cc));
-          lc = ld_dsmem_f32(map_to_rank(rb + 4 * (GMAX * D + GMAX + g), cc));
-          ac = ld_dsmem_f32(map_to_rank(rb + 4 * (g * D + dd), cc));
-        } else {
-          mc = red[GMAX * D + g];
-          lc = red[GMAX * D + GMAX + g];
-          ac = red[g * D + dd];
+#pragma unroll
+        for (int w = 0; w < NWG; ++w) {
+          const float mc = part_f(cc, RED_M + w * GMAX + g);
+          if (mc == -INFINITY) continue;
+          const float lc = part_f(cc, RED_L + w * GMAX + g);
+          const float ac = part_f(cc, (w * GMAX + g) * D + dd);
+          const float wt = exp2f(mc - M);
+          den += wt * lc;
+          num += wt * ac;
         }
-        if (mc == -INFINITY) continue;
-        const float w = exp2f(mc - M);
-        den += w * lc;
-        num += w * ac;
       }
       const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + g;
       if (p.S == 1) {
