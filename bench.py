@@ -55,6 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOADS)
     ap.add_argument("--mode", default=None, choices=("art", "full", "q8", "q8_art"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweeps", action="store_true", help="skip the ART scaling / overhead sweeps")
     a = ap.parse_args(argv)
     if a.mode is None:
         a.mode = "q8_art" if a.workload.startswith("q8") else "art"
@@ -286,13 +287,50 @@ def run_reference(args):
     return 0
 
 
+def art_sweeps(K, dp, w, args, stream):
+    """Two sweeps of the ART path on the same buffers (ART modes only).
+
+    scaling: thresholds +inf and patience k stop every (head, split) after exactly min(k, n)
+    tiles, so time against tiles read should be a line with a small intercept.
+    overhead: thresholds 0 never stop, so ART reads every tile; its time against full
+    attention is the cost of the probe, the exchange and the rule."""
+    import torch
+
+    if args.mode not in ("art", "q8_art"):
+        return None
+    full_mode = "full" if args.mode == "art" else "q8"
+    n = int(-(-int(w.seq_lens.max()) // w.tile)) // max(1, w.num_splits)
+    ks = sorted({1, max(1, n // 8), max(1, n // 4), max(1, n // 2), n})
+    steps = max(3, min(args.steps, 10))
+    pts = []
+    for k in ks:
+        art = dict(w.art, eps_scale=float("inf"), eps_dir=float("inf"), patience=k)
+        _, launch = time_mode(K, dp, args.mode, steps, 2, stream, art=art)
+        rb = bytes_read(w, dp.tiles_read().cpu().numpy())
+        pts.append({"patience": k, "tiles_frac": float(dp.tiles.float().mean().item()) / (n * w.num_splits),
+                     "ms": launch, "kv_bytes_read": rb})
+    x = np.array([p["kv_bytes_read"] for p in pts], dtype=np.float64)
+    y = np.array([p["ms"] for p in pts], dtype=np.float64)
+    slope, icpt = np.polyfit(x, y, 1) if len(pts) > 1 else (0.0, float(y[0]))
+    eps0 = dict(w.art, eps_scale=0.0, eps_dir=0.0)
+    _, ms_eps0 = time_mode(K, dp, args.mode, steps, 2, stream, art=eps0)
+    _, ms_full = time_mode(K, dp, full_mode, steps, 2, stream)
+    torch.cuda.synchronize()
+    return {
+        "scaling": {"points": pts, "fit_ms": {"intercept": float(icpt), "per_gb": float(slope) * 1e9},
+                    "note": "eps = +inf, patience k: exactly min(k, n) tiles per (head, split)"},
+        "overhead_eps0": {"ms_art_eps0": ms_eps0, "ms_full": ms_full, "ratio": ms_eps0 / ms_full,
+                          "note": "eps = 0: ART never stops and reads every tile"},
+    }
+
+
 # ----------------------------------------------------------------------------- our arm
-def time_mode(K, dp, mode, steps, warmup, stream):
+def time_mode(K, dp, mode, steps, warmup, stream, art=None):
     """Device time of `steps` calls: (total ms, mean per-launch ms from per-launch events)."""
     import torch
 
     for _ in range(warmup):
-        K.decode(dp, mode, stream=stream.cuda_stream)
+        K.decode(dp, mode, art=art, stream=stream.cuda_stream)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -301,7 +339,7 @@ def time_mode(K, dp, mode, steps, warmup, stream):
     start.record(stream)
     for i in range(steps):
         ev[i][0].record(stream)
-        K.decode(dp, mode, stream=stream.cuda_stream)
+        K.decode(dp, mode, art=art, stream=stream.cuda_stream)
         ev[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
@@ -367,6 +405,8 @@ def run_ours(args):
                 "kv_bytes_read": o_read},
     }
 
+    sweeps = art_sweeps(K, dp, w, args, stream) if not args.no_sweeps else None
+
     # end to end through the public call: the step's query in from pinned host memory, O and tiles back out
     q_host = dp.q.cpu().pin_memory()
     o_host = torch.empty_like(dp.o, device="cpu").pin_memory()
@@ -416,6 +456,7 @@ def run_ours(args):
                      "peak_source": f"{peak_kind} hbm_gbs (copy)", "traffic": traffic,
                      "kernel": kernel, "bytes_per_launch": rb, "launch_ms": launch_ms},
         "modes": modes,
+        "art_sweeps": sweeps,
         "e2e": e2e,
         "gpu_launches": gpu_launches,
         "clocks": clocks,
