@@ -81,6 +81,9 @@ def _load():
                 ctypes.POINTER(_Art), ctypes.c_double, ctypes.c_void_p, ctypes.c_int,
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
             ]
+            lib.oracle_decode_ordered.restype = ctypes.c_int
+            lib.oracle_decode_ordered.argtypes = lib.oracle_decode.argtypes[:12] + [ctypes.c_void_p] + \
+                lib.oracle_decode.argtypes[12:]
             lib.oracle_bf16_to_double.restype = ctypes.c_double
             lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
             lib.oracle_f16_to_double.restype = ctypes.c_double
@@ -125,6 +128,7 @@ def decode(
     no_break: bool = False,
     want_metrics: bool = False,
     n_threads: int = 1,
+    tile_order: np.ndarray | None = None,
 ) -> OracleResult:
     """Run the oracle.
 
@@ -132,6 +136,8 @@ def decode(
     k, v: float32 / uint16 bf16 bits / int8, [B,Hkv,L_max,d].
     k_scale, v_scale: uint16 fp16 bits [B,Hkv,L_max,d/32] (KV_Q8 only).
     art: None for plain attention, else dict(eps_scale, eps_dir, patience, lanes).
+    tile_order: None (natural order) or int32 [B,Hkv,ceil(L_max/tile)]: each (batch, kv head)'s
+      traversal sequence; split s walks positions [s*n/S, (s+1)*n/S) of it (see orders.py).
     """
     lib = _load()
     B, Hq, d = q.shape
@@ -161,9 +167,13 @@ def decode(
     tiles = np.zeros((B, Hq), np.int32)
     n_tiles_max = (L_max + tile - 1) // tile
     metrics = np.zeros((B, Hq, n_tiles_max, 2), np.float64) if want_metrics else None
-    rc = lib.oracle_decode(
+    order = None
+    if tile_order is not None:
+        order = np.ascontiguousarray(tile_order, dtype=np.int32)
+        assert order.shape == (B, Hkv, n_tiles_max), order.shape
+    rc = lib.oracle_decode_ordered(
         ctypes.byref(sh), kind, _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale), _ptr(seq),
-        ctypes.byref(art_s) if art_s is not None else None, float(tau), _ptr(fu), int(no_break),
+        ctypes.byref(art_s) if art_s is not None else None, float(tau), _ptr(fu), int(no_break), _ptr(order),
         _ptr(o), _ptr(used), _ptr(tiles), _ptr(metrics), int(n_threads),
     )
     if rc != 0:

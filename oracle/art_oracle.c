@@ -23,7 +23,9 @@
  *               thresholds (tau, phi) at the same time.
  *          S2.3 patience p: the criterion must hold on p consecutive tiles.
  *          S2.4 block 0 is always evaluated before any termination; tile
- *               order does not change full attention.
+ *               order does not change full attention; the traversal order
+ *               of the KV blocks may be changed (recency first, importance
+ *               first) and ART then watches the probe along that order.
  *   [SKIP] "La paradoja de la eficiencia: como omitir redefine la velocidad
  *          de los LLM", puntofijo.es, section "La Elegancia de la Omision":
  *          the flash kernel knows the softmax weights before it touches V,
@@ -43,6 +45,10 @@
  *     numerator when exp(s_j - m') < tau, m' the running maximum of the
  *     split after the current tile; its weight stays in the denominator.
  *   - q8 value = int8 * (fp16 scale of its 32-element block).
+ *   - traversal order (S2.4): an explicit per-(batch, kv head) sequence of
+ *     tile indices; the split structure applies to positions in the
+ *     sequence, and each split's segment must be a permutation of that
+ *     split's own tiles.  Without a sequence the order is 0, 1, ..., n-1.
  */
 #include <math.h>
 #include <stdint.h>
@@ -133,13 +139,15 @@ static double l2norm(const double* x, int n) {
 
 /*
  * One (batch, query head).  Returns 0 or a negative error.
- * o: [d]; used: [S]; metrics: NULL or [n_tiles_max][2] (d_scale, d_dir) by tile index.
+ * o: [d]; used: [S]; metrics: NULL or [n_tiles_max][2] (d_scale, d_dir) by position in
+ * the traversal sequence; seq: NULL (natural order) or this kv head's [n_tiles_max]
+ * traversal sequence.
  */
 static int decode_one_head(const oracle_shape* sh, int kind, const void* q, const void* k,
                            const void* v, const uint16_t* k_scale, const uint16_t* v_scale,
                            int L, int b, int hq, const oracle_art* art, double tau,
-                           const int32_t* forced_used, int no_break, double* o, int32_t* used,
-                           double* metrics, int n_tiles_max) {
+                           const int32_t* forced_used, int no_break, const int32_t* seq,
+                           double* o, int32_t* used, double* metrics, int n_tiles_max) {
   const int d = sh->d, T = sh->tile, S = sh->num_splits;
   const int G = sh->Hq / sh->Hkv;
   const int kvh = hq / G;
@@ -191,8 +199,14 @@ static int decode_one_head(const oracle_shape* sh, int kind, const void* q, cons
     int run = 0, stopped = 0;
     const int forced = forced_used ? forced_used[s] : -1;
 
-    for (int t = ta; t < tb; ++t) {
+    for (int kpos = ta; kpos < tb; ++kpos) {
       if (forced >= 0 && cur.used >= forced) break;
+      const int t = seq ? seq[kpos] : kpos; /* the tile at this position of the sequence */
+      if (t < ta || t >= tb) {
+        free(qv); free(kr); free(vr); free(sc); free(x); free(xprev);
+        free(part_m); free(part_l); free(part_acc); free(cur.acc); free(snap.acc);
+        return ORACLE_ERR_ARG;
+      }
       const int j0 = t * T;
       const int j1 = (j0 + T < L) ? j0 + T : L;
 
@@ -238,9 +252,9 @@ static int decode_one_head(const oracle_shape* sh, int kind, const void* q, cons
           d_dir = 1.0 - dot / (a * bn);
           if (d_dir < 0.0) d_dir = 0.0;
         }
-        if (metrics && t < n_tiles_max) {
-          metrics[2 * t + 0] = d_scale;
-          metrics[2 * t + 1] = d_dir;
+        if (metrics && kpos < n_tiles_max) {
+          metrics[2 * kpos + 0] = d_scale;
+          metrics[2 * kpos + 1] = d_dir;
         }
         /* S2.2 + S2.3: both below threshold, on p consecutive tiles. */
         const int hold = (d_scale < art->eps_scale) && (d_dir < art->eps_dir);
@@ -280,7 +294,7 @@ static int decode_one_head(const oracle_shape* sh, int kind, const void* q, cons
 }
 
 /*
- * Decode every (batch, query head).
+ * Decode every (batch, query head), tiles in the traversal order `tile_order`.
  *   q        f32 [B,Hq,d] for ORACLE_KV_F32, else bf16 bits [B,Hq,d]
  *   k, v     f32 / bf16 bits / int8, [B,Hkv,L_max,d]
  *   k_scale, v_scale  q8 only: fp16 bits [B,Hkv,L_max,d/32]
@@ -294,13 +308,19 @@ static int decode_one_head(const oracle_shape* sh, int kind, const void* q, cons
  *   o        [B,Hq,d] doubles
  *   used     [B,Hq,S] tiles consumed per split
  *   tiles    [B,Hq] sum of used over splits
- *   metrics  NULL or [B,Hq,n_tiles_max,2]; NaN where no rule was evaluated
+ *   metrics  NULL or [B,Hq,n_tiles_max,2] by position in the traversal sequence;
+ *            NaN where no rule was evaluated
+ *   tile_order  NULL (natural order) or [B,Hkv,n_tiles_max]: the traversal sequence
+ *            of each (batch, kv head); entries at positions >= ceil(L_b/T) are ignored
  *   n_threads  OpenMP threads over (batch, query head); <= 0: library default
+ * A sequence entry outside its split's tiles gives ORACLE_ERR_ARG.
  */
-int oracle_decode(const oracle_shape* sh, int kind, const void* q, const void* k, const void* v,
-                  const uint16_t* k_scale, const uint16_t* v_scale, const int32_t* seq_lens,
-                  const oracle_art* art, double tau, const int32_t* forced_used, int no_break,
-                  double* o, int32_t* used, int32_t* tiles, double* metrics, int n_threads) {
+int oracle_decode_ordered(const oracle_shape* sh, int kind, const void* q, const void* k,
+                          const void* v, const uint16_t* k_scale, const uint16_t* v_scale,
+                          const int32_t* seq_lens, const oracle_art* art, double tau,
+                          const int32_t* forced_used, int no_break, const int32_t* tile_order,
+                          double* o, int32_t* used, int32_t* tiles, double* metrics,
+                          int n_threads) {
   if (!sh || !q || !k || !v || !seq_lens || !o || !used || !tiles) return ORACLE_ERR_ARG;
   if (sh->B < 1 || sh->Hq < 1 || sh->Hkv < 1 || sh->d < 1 || sh->L_max < 1 || sh->tile < 1 ||
       sh->num_splits < 1)
@@ -330,8 +350,10 @@ int oracle_decode(const oracle_shape* sh, int kind, const void* q, const void* k
 #endif
   for (int bh = 0; bh < nheads; ++bh) {
     const int b = bh / sh->Hq, hq = bh % sh->Hq;
+    const int kvh = hq / (sh->Hq / sh->Hkv);
+    const int32_t* seq = tile_order ? tile_order + ((long)b * sh->Hkv + kvh) * n_tiles_max : NULL;
     int r = decode_one_head(sh, kind, q, k, v, k_scale, v_scale, seq_lens[b], b, hq, art, tau,
-                            forced_used ? forced_used + (long)bh * S : NULL, no_break,
+                            forced_used ? forced_used + (long)bh * S : NULL, no_break, seq,
                             o + (long)bh * sh->d, used + (long)bh * S,
                             metrics ? metrics + (long)bh * n_tiles_max * 2 : NULL, n_tiles_max);
     if (r < err) err = r;
@@ -340,4 +362,13 @@ int oracle_decode(const oracle_shape* sh, int kind, const void* q, const void* k
     tiles[bh] = sum;
   }
   return err;
+}
+
+/* Natural tile order (0, 1, ..., n-1 in every split). */
+int oracle_decode(const oracle_shape* sh, int kind, const void* q, const void* k, const void* v,
+                  const uint16_t* k_scale, const uint16_t* v_scale, const int32_t* seq_lens,
+                  const oracle_art* art, double tau, const int32_t* forced_used, int no_break,
+                  double* o, int32_t* used, int32_t* tiles, double* metrics, int n_threads) {
+  return oracle_decode_ordered(sh, kind, q, k, v, k_scale, v_scale, seq_lens, art, tau, forced_used,
+                               no_break, NULL, o, used, tiles, metrics, n_threads);
 }
