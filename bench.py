@@ -287,6 +287,40 @@ def run_reference(args):
     return 0
 
 
+ABLATION_GRID = {
+    # criterion family -> (eps_scale, eps_dir) pairs, loosest last
+    "both": [(1e-4, 1e-5), (1e-3, 1e-4), (1e-2, 1e-3), (1e-1, 1e-2)],
+    "scale_only": [(1e-4, float("inf")), (1e-3, float("inf")), (1e-2, float("inf")), (1e-1, float("inf"))],
+    "direction_only": [(float("inf"), 1e-5), (float("inf"), 1e-4), (float("inf"), 1e-3), (float("inf"), 1e-2)],
+}
+
+
+def art_ablation(K, dp, w, args):
+    """Premature-stop error against tiles saved for each criterion family and patience 1, 2, 4:
+    per query head, ||O_ART - O_full|| / ||O_full|| (L2 over d), on the bench's own buffers."""
+    import torch
+
+    mode = args.mode
+    full_mode = "full" if mode == "art" else "q8"
+    K.decode(dp, full_mode)
+    o_full = dp.o.clone()
+    nrm = torch.linalg.vector_norm(o_full, dim=-1).clamp_min(1e-30)
+    n_tot = float((-(-w.seq_lens.astype(np.int64) // w.tile)).mean())
+    rows = []
+    for fam, pairs in ABLATION_GRID.items():
+        for pat in (1, 2, 4):
+            for es, ed in pairs:
+                K.decode(dp, mode, art=dict(w.art, eps_scale=es, eps_dir=ed, patience=pat))
+                rel = torch.linalg.vector_norm(dp.o - o_full, dim=-1) / nrm
+                rows.append({"criterion": fam, "patience": pat,  # null threshold: criterion off (+inf)
+                             "eps_scale": None if es == float("inf") else es,
+                             "eps_dir": None if ed == float("inf") else ed,
+                             "tiles_saved": 1.0 - float(dp.tiles.float().mean().item()) / n_tot,
+                             "rel_err_mean": float(rel.mean().item()), "rel_err_max": float(rel.max().item())})
+    torch.cuda.synchronize()
+    return rows
+
+
 def art_sweeps(K, dp, w, args, stream):
     """Two sweeps of the ART path on the same buffers (ART modes only).
 
@@ -312,6 +346,7 @@ def art_sweeps(K, dp, w, args, stream):
     x = np.array([p["kv_bytes_read"] for p in pts], dtype=np.float64)
     y = np.array([p["ms"] for p in pts], dtype=np.float64)
     slope, icpt = np.polyfit(x, y, 1) if len(pts) > 1 else (0.0, float(y[0]))
+    ablation = art_ablation(K, dp, w, args)
     eps0 = dict(w.art, eps_scale=0.0, eps_dir=0.0)
     _, ms_eps0 = time_mode(K, dp, args.mode, steps, 2, stream, art=eps0)
     _, ms_full = time_mode(K, dp, full_mode, steps, 2, stream)
@@ -321,6 +356,7 @@ def art_sweeps(K, dp, w, args, stream):
                     "note": "eps = +inf, patience k: exactly min(k, n) tiles per (head, split)"},
         "overhead_eps0": {"ms_art_eps0": ms_eps0, "ms_full": ms_full, "ratio": ms_eps0 / ms_full,
                           "note": "eps = 0: ART never stops and reads every tile"},
+        "ablation": ablation,
     }
 
 

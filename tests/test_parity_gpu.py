@@ -110,6 +110,8 @@ ART_SETTINGS = [
     dict(eps_scale=5e-2, eps_dir=2e-2, patience=3),
     dict(eps_scale=float("inf"), eps_dir=float("inf"), patience=2),
     dict(eps_scale=0.0, eps_dir=0.0, patience=1),
+    dict(eps_scale=2e-2, eps_dir=float("inf"), patience=2),  # magnitude criterion only
+    dict(eps_scale=float("inf"), eps_dir=5e-3, patience=4),  # direction criterion only
 ]
 
 
@@ -122,7 +124,7 @@ def test_art_small(case, setting):
     g, exact, amb = check_art(w, mode, art=a, tau=(1e-6 if w.kind == "q8" else None))
     n = n_tiles(w, w.tile)
     S = w.num_splits
-    if a["eps_scale"] == float("inf"):
+    if a["eps_scale"] == float("inf") and a["eps_dir"] == float("inf"):
         for b in range(w.B):
             lens = [((s + 1) * n[b]) // S - (s * n[b]) // S for s in range(S)]
             assert np.array_equal(g["used"][b], np.tile([min(a["patience"], x) for x in lens], (w.Hq, 1)))
