@@ -321,6 +321,60 @@ def art_ablation(K, dp, w, args):
     return rows
 
 
+def art_orders(K, dp, w, args, stream):
+    """ART with the configured thresholds along each traversal order (natural, recency first,
+    importance first): time per call, tiles read, error against full attention, and the time to
+    build the sequence on the GPU per step (importance: scoring and sort; the per-tile key summary
+    is built once, as a cache would maintain it when keys are appended, and timed apart)."""
+    import torch
+
+    if args.mode != "art" or w.kind not in ("f32", "bf16"):
+        return None
+    steps = max(3, min(args.steps, 10))
+    K.decode(dp, "full")
+    o_full = dp.o.clone()
+    nrm = torch.linalg.vector_norm(o_full, dim=-1).clamp_min(1e-30)
+    n_tot = float((-(-w.seq_lens.astype(np.int64) // w.tile)).mean())
+    out = {}
+    summary = K.key_summary(dp, stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        summary = K.key_summary(dp, stream=stream.cuda_stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    out["key_summary_ms"] = e0.elapsed_time(e1) / steps
+    for kind in ("natural", "recency", "importance"):
+        order = None
+        build_ms = 0.0
+        if kind != "natural":
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            order = K.tile_order(dp, kind, stream=stream.cuda_stream, summary=summary)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(steps):
+                order = K.tile_order(dp, kind, stream=stream.cuda_stream, summary=summary)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            build_ms = e0.elapsed_time(e1) / steps
+        for _ in range(2):
+            K.decode(dp, "art", order=order, stream=stream.cuda_stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            K.decode(dp, "art", order=order, stream=stream.cuda_stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rel = torch.linalg.vector_norm(dp.o - o_full, dim=-1) / nrm
+        out[kind] = {"ms": e0.elapsed_time(e1) / steps, "order_build_ms": build_ms,
+                     "tiles_frac": float(dp.tiles.float().mean().item()) / n_tot,
+                     "kv_bytes_read": bytes_read(w, dp.tiles_read().cpu().numpy()),
+                     "rel_err_mean": float(rel.mean().item()), "rel_err_max": float(rel.max().item())}
+    return out
+
+
 def art_sweeps(K, dp, w, args, stream):
     """Two sweeps of the ART path on the same buffers (ART modes only).
 
@@ -347,6 +401,7 @@ def art_sweeps(K, dp, w, args, stream):
     y = np.array([p["ms"] for p in pts], dtype=np.float64)
     slope, icpt = np.polyfit(x, y, 1) if len(pts) > 1 else (0.0, float(y[0]))
     ablation = art_ablation(K, dp, w, args)
+    trav = art_orders(K, dp, w, args, stream)
     eps0 = dict(w.art, eps_scale=0.0, eps_dir=0.0)
     _, ms_eps0 = time_mode(K, dp, args.mode, steps, 2, stream, art=eps0)
     _, ms_full = time_mode(K, dp, full_mode, steps, 2, stream)
@@ -357,6 +412,7 @@ def art_sweeps(K, dp, w, args, stream):
         "overhead_eps0": {"ms_art_eps0": ms_eps0, "ms_full": ms_full, "ratio": ms_eps0 / ms_full,
                           "note": "eps = 0: ART never stops and reads every tile"},
         "ablation": ablation,
+        "orders": trav,
     }
 
 

@@ -79,7 +79,8 @@ typedef enum {
   ART_ERR_WORKSPACE = -3,   /* ws NULL or smaller than art_workspace_bytes() */
   ART_ERR_CUDA = -4,        /* a CUDA runtime call failed (launch, attribute) */
   ART_ERR_TIMEOUT = -5,     /* device: a bounded wait gave up (status word) */
-  ART_ERR_SEQLEN = -6       /* device: a seq_len outside [1, L_max] (status word) */
+  ART_ERR_SEQLEN = -6,      /* device: a seq_len outside [1, L_max] (status word) */
+  ART_ERR_ORDER = -7        /* device: a tile_order entry outside its split (status word) */
 } art_status;
 
 typedef enum { ART_F32 = 0, ART_BF16 = 1 } art_dtype;
@@ -167,9 +168,60 @@ art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, 
                                     float tau, const art_params* params, float* o, int32_t* tiles,
                                     void* ws, size_t ws_bytes, void* stream);
 
+/* ---- KV tile traversal orders ("Resumen Tecnico: ART", S2.4: ART composes with
+ * other KV-cache policies by reordering the traversal sequence of the KV blocks,
+ * "recency first" or "importance first"; reordering does not change full
+ * attention; block 0 comes first).  The page names the orders without defining
+ * them; this library's readings:
+ *   - A traversal sequence is an int32 array tile_order[B, Hkv, n_max],
+ *     n_max = ceil(L_max / tile), DEVICE memory, one sequence per (batch, kv
+ *     head).  With num_splits = S, split s of a sequence of n = ceil(L_b/tile)
+ *     tiles walks positions [floor(s*n/S), floor((s+1)*n/S)), and those
+ *     positions must hold a permutation of split s's own tiles (the same
+ *     index range).  Positions >= n are ignored (the builders write -1).
+ *   - recency first: each split's first tile, then its other tiles from the
+ *     newest back to the oldest.
+ *   - importance first: each split's first tile, then its other tiles by the
+ *     score max over the kv head's query heads g of q_g . mu_t (mu_t the mean
+ *     key of tile t, art_tile_key_summary), highest first, ties to the lower
+ *     tile index; scores are computed in fp32.
+ * The builders read seq_lens on the device; a sequence whose seq_len is
+ * outside [1, L_max] gets -1 everywhere.  They allocate nothing and only
+ * enqueue work on `stream`. */
+
+/* Recency-first sequences for every (batch, kv head) into tile_order. */
+art_status art_tile_order_recency(const art_shape* shape, const int32_t* seq_lens, int32_t* tile_order,
+                                  void* stream);
+
+/* Per-tile key summary: summary[B, Hkv, n_max, d] fp32 (DEVICE) = mean of K over
+ * each tile's positions [t*tile, min((t+1)*tile, L_b)); 0 for tiles past L_b.
+ * k as in the decode calls (fp32 or bf16, [B, Hkv, L_max, d]); d in {64, 128}. */
+art_status art_tile_key_summary(const art_shape* shape, art_dtype dtype, const void* k, const int32_t* seq_lens,
+                                float* summary, void* stream);
+
+/* Importance-first sequences from the query q[B, Hq, d] (fp32 or bf16) and a
+ * key summary.  One thread block per (batch, kv head) holds n_max scores in
+ * shared memory: shapes needing more than 200 KiB give ART_ERR_UNSUPPORTED. */
+art_status art_tile_order_importance(const art_shape* shape, art_dtype dtype, const void* q, const float* summary,
+                                     const int32_t* seq_lens, int32_t* tile_order, void* stream);
+
+/* Decode attention with ART along caller-given traversal sequences ("Resumen
+ * Tecnico: ART", S2.2-S2.4): as art_decode_attn_terminate, but split s of each
+ * (batch, kv head) consumes the tiles listed at its positions of tile_order, in
+ * that order, and the rule watches the probe along that sequence; `tiles` and the
+ * per-split counters count tiles consumed.  With both thresholds 0 it is full
+ * attention in any order.  tile_order is DEVICE memory (4-byte aligned).  An
+ * entry outside its split is replaced by the natural tile at that position and
+ * flags ART_ERR_ORDER in the status word (results of that call are then
+ * unspecified); duplicate entries inside the split's range are not detected. */
+art_status art_decode_attn_terminate_ordered(const art_shape* shape, art_dtype dtype, const void* q,
+                                             const void* k, const void* v, const int32_t* seq_lens,
+                                             const art_params* params, const int32_t* tile_order, float* o,
+                                             int32_t* tiles, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, read the sticky status word of ws, clear it, and
- * return ART_OK, ART_ERR_SEQLEN or ART_ERR_TIMEOUT (ART_ERR_CUDA if the
- * synchronisation or copy failed). */
+ * return ART_OK, ART_ERR_SEQLEN, ART_ERR_TIMEOUT or ART_ERR_ORDER (ART_ERR_CUDA
+ * if the synchronisation or copy failed). */
 art_status art_read_device_status(void* ws, void* stream);
 
 /* Base name of the CUDA kernel a call with this shape would launch for its

@@ -13,7 +13,7 @@ from dataclasses import dataclass
 from . import capi
 from .capi import ArtError
 
-__all__ = ["capi", "ArtError", "DeviceProblem", "upload", "decode", "kernel_name"]
+__all__ = ["capi", "ArtError", "DeviceProblem", "upload", "decode", "kernel_name", "tile_order", "key_summary"]
 
 
 @dataclass
@@ -99,15 +99,19 @@ def _ptr(t):
 
 
 def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float | None = None, stream=None,
-           check: bool = True) -> int:
+           check: bool = True, order=None) -> int:
     """Launch one decode call on dp's buffers.
 
     mode: "full" | "art" (art_decode_attn_terminate) | "q8" (q8_skipv without ART) |
-          "q8_art" (q8_skipv with ART).  Returns the C status code; raises
+          "q8_art" (q8_skipv with ART).  order: None, or an int32 device tensor
+    [B, Hkv, ceil(L_max/tile)] of tile traversal sequences (mode "art" only:
+    art_decode_attn_terminate_ordered).  Returns the C status code; raises
     ArtError on a non-zero code when check is True.
     """
     import torch
 
+    if order is not None and mode != "art":
+        raise ValueError("a traversal order applies to mode 'art' only")
     st = torch.cuda.current_stream().cuda_stream if stream is None else stream
     a = dp.art if art is None else art
     dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
@@ -115,6 +119,12 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
         rc = capi.art_decode_attn_full(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens),
                                        _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
         name = "art_decode_attn_full"
+    elif mode == "art" and order is not None:
+        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+        rc = capi.art_decode_attn_terminate_ordered(
+            dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens), params, _ptr(order),
+            _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
+        name = "art_decode_attn_terminate_ordered"
     elif mode == "art":
         params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
         rc = capi.art_decode_attn_terminate(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens),
@@ -133,6 +143,48 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
     if check and rc != capi.ART_OK:
         raise ArtError(rc, name)
     return rc
+
+
+def tile_order(dp: DeviceProblem, kind: str, *, stream=None, summary=None):
+    """Build tile traversal sequences on the GPU: kind "recency" or "importance" (the latter from dp's
+    query and a per-tile key summary, computed here unless given).  Returns int32 [B, Hkv, n_max]."""
+    import torch
+
+    s = dp.shape
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    n_max = -(-s.L_max // s.tile)
+    out = torch.empty((s.B, s.Hkv, n_max), dtype=torch.int32, device=dp.k.device)
+    if kind == "recency":
+        rc = capi.art_tile_order_recency(s, _ptr(dp.seq_lens), _ptr(out), st)
+        name = "art_tile_order_recency"
+    elif kind == "importance":
+        if dp.kind not in ("f32", "bf16"):
+            raise ValueError("importance order needs fp32 or bf16 keys")
+        dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
+        if summary is None:
+            summary = key_summary(dp, stream=st)
+        rc = capi.art_tile_order_importance(s, dtype, _ptr(dp.q), _ptr(summary), _ptr(dp.seq_lens), _ptr(out), st)
+        name = "art_tile_order_importance"
+    else:
+        raise ValueError(kind)
+    if rc != capi.ART_OK:
+        raise ArtError(rc, name)
+    return out
+
+
+def key_summary(dp: DeviceProblem, *, stream=None):
+    """Mean key per tile, fp32 [B, Hkv, n_max, d] (art_tile_key_summary)."""
+    import torch
+
+    s = dp.shape
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    n_max = -(-s.L_max // s.tile)
+    out = torch.empty((s.B, s.Hkv, n_max, s.d), dtype=torch.float32, device=dp.k.device)
+    dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
+    rc = capi.art_tile_key_summary(s, dtype, _ptr(dp.k), _ptr(dp.seq_lens), _ptr(out), st)
+    if rc != capi.ART_OK:
+        raise ArtError(rc, "art_tile_key_summary")
+    return out
 
 
 def kernel_name(dp: DeviceProblem, mode: str) -> str:

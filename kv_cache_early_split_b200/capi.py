@@ -20,6 +20,7 @@ ART_ERR_WORKSPACE = -3
 ART_ERR_CUDA = -4
 ART_ERR_TIMEOUT = -5
 ART_ERR_SEQLEN = -6
+ART_ERR_ORDER = -7
 ART_F32 = 0
 ART_BF16 = 1
 
@@ -35,6 +36,10 @@ EXPORTS = (
     "art_read_device_status",
     "art_status_string",
     "art_kernel_name",
+    "art_tile_order_recency",
+    "art_tile_key_summary",
+    "art_tile_order_importance",
+    "art_decode_attn_terminate_ordered",
 )
 
 
@@ -98,6 +103,15 @@ def lib() -> ctypes.CDLL:
             L.art_read_device_status.argtypes = [_P, _P]
             L.art_status_string.restype = ctypes.c_char_p
             L.art_status_string.argtypes = [ctypes.c_int]
+            L.art_tile_order_recency.restype = ctypes.c_int
+            L.art_tile_order_recency.argtypes = [_SH, _P, _P, _P]
+            L.art_tile_key_summary.restype = ctypes.c_int
+            L.art_tile_key_summary.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P]
+            L.art_tile_order_importance.restype = ctypes.c_int
+            L.art_tile_order_importance.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _P]
+            L.art_decode_attn_terminate_ordered.restype = ctypes.c_int
+            L.art_decode_attn_terminate_ordered.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, _P,
+                                                            ctypes.c_size_t, _P]
             L.art_kernel_name.restype = ctypes.c_char_p
             L.art_kernel_name.argtypes = [_SH, ctypes.c_int, ctypes.c_int32, ctypes.c_int32]
             _lib = L
@@ -148,6 +162,24 @@ def art_read_device_status(ws, stream) -> int:
 
 def art_status_string(code: int) -> str:
     return lib().art_status_string(int(code)).decode()
+
+
+def art_tile_order_recency(shape, seq_lens, tile_order, stream) -> int:
+    return int(lib().art_tile_order_recency(ctypes.byref(shape), seq_lens, tile_order, stream))
+
+
+def art_tile_key_summary(shape, dtype, k, seq_lens, summary, stream) -> int:
+    return int(lib().art_tile_key_summary(ctypes.byref(shape), dtype, k, seq_lens, summary, stream))
+
+
+def art_tile_order_importance(shape, dtype, q, summary, seq_lens, tile_order, stream) -> int:
+    return int(lib().art_tile_order_importance(ctypes.byref(shape), dtype, q, summary, seq_lens, tile_order, stream))
+
+
+def art_decode_attn_terminate_ordered(shape, dtype, q, k, v, seq_lens, params, tile_order, o, tiles, ws, ws_bytes,
+                                      stream) -> int:
+    return int(lib().art_decode_attn_terminate_ordered(
+        ctypes.byref(shape), dtype, q, k, v, seq_lens, _ref(params), tile_order, o, tiles, ws, ws_bytes, stream))
 
 
 def art_kernel_name(shape, dtype, kv_q8, with_art):

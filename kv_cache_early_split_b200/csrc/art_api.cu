@@ -10,6 +10,7 @@
 
 #include "art_decode.h"
 #include "art_kernels.cuh"
+#include "art_order.cuh"
 #include "art_tc.cuh"
 
 namespace {
@@ -237,13 +238,14 @@ bool tc_eligible(int kind, int mode, const art_shape* s) {
          (s->tile == 64 || s->tile == 128) && G >= 1 && G <= 8;
 }
 
-// K/V [B*Hkv][L_max][128] bf16 as a 3-D tensor map; box = 64 d x 128 positions, 128-byte swizzle.
-bool make_kv_map(CUtensorMap* m, const void* base, const art_shape* s) {
+// K/V [B*Hkv][L_max][128] bf16 as a 3-D tensor map; box = 64 d x `rows` positions (128 or 64),
+// 128-byte swizzle.
+bool make_kv_map(CUtensorMap* m, const void* base, const art_shape* s, unsigned rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(s->L_max), static_cast<cuuint64_t>(s->B) * s->Hkv};
   const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(s->L_max) * 256};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, rows, 1};
   const cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -266,8 +268,8 @@ TcFn tc_pick(int mode, int G, int n_probe) {
 }
 
 art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k, const void* v,
-                     const int32_t* seq_lens, const art_params* a, float* o, int32_t* tiles, void* ws,
-                     void* stream) {
+                     const int32_t* seq_lens, const art_params* a, const int32_t* order, float* o,
+                     int32_t* tiles, void* ws, void* stream) {
   const int G = s->Hq / s->Hkv;
   const TcFn fn = tc_pick(mode, G, a ? a->n_probe : 0);
   artk::tc::TcParams p;
@@ -283,6 +285,10 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
     for (int i = 0; i < a->n_probe; ++i) p.lanes[i] = static_cast<int8_t>(a->probe_lanes[i]);
   }
   if (!make_kv_map(&p.tmK, k, s) || !make_kv_map(&p.tmV, v, s)) return ART_ERR_CUDA;
+  if (order && s->tile == 64 && (!make_kv_map(&p.tmK64, k, s, 64) || !make_kv_map(&p.tmV64, v, s, 64)))
+    return ART_ERR_CUDA;
+  p.order = order;
+  p.n_max = (s->L_max + s->tile - 1) / s->tile;
   int sms = 0;
   art_status st = prepare(reinterpret_cast<KernelFn>(fn), &sms);
   if (st != ART_OK) return st;
@@ -390,9 +396,9 @@ art_status validate_params(const art_params* a, int d, int epc, int* emask) {
 
 art_status launch(int kind, int mode, const art_shape* s, const void* q, const void* k, const void* v,
                   const uint16_t* ks, const uint16_t* vs, const int32_t* seq_lens, const art_params* a,
-                  float tau, float* o, int32_t* tiles, void* ws, void* stream) {
+                  float tau, float* o, int32_t* tiles, void* ws, void* stream, const int32_t* order = nullptr) {
   const int G = s->Hq / s->Hkv;
-  if (tc_eligible(kind, mode, s)) return launch_tc(mode, s, q, k, v, seq_lens, a, o, tiles, ws, stream);
+  if (tc_eligible(kind, mode, s)) return launch_tc(mode, s, q, k, v, seq_lens, a, order, o, tiles, ws, stream);
   KernelInfo ki;
   if (!pick_kernel(kind, mode, s->d, G, &ki)) return ART_ERR_UNSUPPORTED;
   Params p;
@@ -440,6 +446,8 @@ art_status launch(int kind, int mode, const art_shape* s, const void* q, const v
   p.nstage = cfg.nstage;
   p.qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(s->d)));
   p.tau = tau;
+  p.order = order;
+  p.n_max = max_tiles;
 
   cudaLaunchConfig_t lc;
   memset(&lc, 0, sizeof lc);
@@ -572,6 +580,79 @@ art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, 
                 tiles, ws, stream);
 }
 
+art_status art_decode_attn_terminate_ordered(const art_shape* shape, art_dtype dtype, const void* q,
+                                             const void* k, const void* v, const int32_t* seq_lens,
+                                             const art_params* params, const int32_t* tile_order, float* o,
+                                             int32_t* tiles, void* ws, size_t ws_bytes, void* stream) {
+  art_status st = validate_common(shape, q, k, v, seq_lens, o, ws, ws_bytes);
+  if (st != ART_OK) return st;
+  if (dtype != ART_F32 && dtype != ART_BF16) return ART_ERR_INVALID_ARG;
+  if (!params || !tile_order || (reinterpret_cast<uintptr_t>(tile_order) & 3u)) return ART_ERR_INVALID_ARG;
+  const int kind = dtype == ART_F32 ? artk::KV_F32 : artk::KV_BF16;
+  return launch(kind, artk::MODE_ART, shape, q, k, v, nullptr, nullptr, seq_lens, params, 0.f, o, tiles, ws,
+                stream, tile_order);
+}
+
+art_status art_tile_order_recency(const art_shape* shape, const int32_t* seq_lens, int32_t* tile_order,
+                                  void* stream) {
+  if (!shape_ok(shape) || !seq_lens || !tile_order) return ART_ERR_INVALID_ARG;
+  const int n_max = (shape->L_max + shape->tile - 1) / shape->tile;
+  const unsigned grid = static_cast<unsigned>(shape->B) * shape->Hkv;
+  artk::ord::tile_order_recency_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      seq_lens, shape->Hkv, shape->L_max, shape->tile, shape->num_splits, n_max, tile_order);
+  return cudaGetLastError() == cudaSuccess ? ART_OK : ART_ERR_CUDA;
+}
+
+art_status art_tile_key_summary(const art_shape* shape, art_dtype dtype, const void* k, const int32_t* seq_lens,
+                                float* summary, void* stream) {
+  if (!shape_ok(shape) || !k || !seq_lens || !summary) return ART_ERR_INVALID_ARG;
+  if (shape->d != 64 && shape->d != 128) return ART_ERR_UNSUPPORTED;
+  const int n_max = (shape->L_max + shape->tile - 1) / shape->tile;
+  constexpr int kTilesPerBlock = 8;
+  const dim3 grid(static_cast<unsigned>(shape->B) * shape->Hkv, (n_max + kTilesPerBlock - 1) / kTilesPerBlock);
+  if (grid.y > 65535u) return ART_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == ART_F32)
+    artk::ord::tile_key_summary_kernel<float><<<grid, shape->d, 0, st>>>(
+        static_cast<const float*>(k), seq_lens, shape->Hkv, shape->L_max, shape->d, shape->tile, n_max,
+        kTilesPerBlock, summary);
+  else if (dtype == ART_BF16)
+    artk::ord::tile_key_summary_kernel<__nv_bfloat16><<<grid, shape->d, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), seq_lens, shape->Hkv, shape->L_max, shape->d, shape->tile, n_max,
+        kTilesPerBlock, summary);
+  else
+    return ART_ERR_INVALID_ARG;
+  return cudaGetLastError() == cudaSuccess ? ART_OK : ART_ERR_CUDA;
+}
+
+art_status art_tile_order_importance(const art_shape* shape, art_dtype dtype, const void* q, const float* summary,
+                                     const int32_t* seq_lens, int32_t* tile_order, void* stream) {
+  if (!shape_ok(shape) || !q || !summary || !seq_lens || !tile_order) return ART_ERR_INVALID_ARG;
+  if (shape->Hq % shape->Hkv != 0) return ART_ERR_INVALID_ARG;
+  if (dtype != ART_F32 && dtype != ART_BF16) return ART_ERR_INVALID_ARG;
+  const int n_max = (shape->L_max + shape->tile - 1) / shape->tile;
+  const size_t smem = 4 * (static_cast<size_t>(shape->Hq / shape->Hkv) * shape->d + n_max);
+  if (smem > 200 * 1024) return ART_ERR_UNSUPPORTED;
+  const unsigned grid = static_cast<unsigned>(shape->B) * shape->Hkv;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == ART_F32) {
+    auto fn = &artk::ord::tile_order_importance_kernel<float>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+      return ART_ERR_CUDA;
+    fn<<<grid, artk::ord::kImpThreads, smem, st>>>(static_cast<const float*>(q), summary, seq_lens, shape->Hq, shape->Hkv,
+                                shape->L_max, shape->d, shape->tile, shape->num_splits, n_max, tile_order);
+  } else {
+    auto fn = &artk::ord::tile_order_importance_kernel<__nv_bfloat16>;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+      return ART_ERR_CUDA;
+    fn<<<grid, artk::ord::kImpThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q), summary, seq_lens, shape->Hq, shape->Hkv,
+                                shape->L_max, shape->d, shape->tile, shape->num_splits, n_max, tile_order);
+  }
+  return cudaGetLastError() == cudaSuccess ? ART_OK : ART_ERR_CUDA;
+}
+
 art_status art_read_device_status(void* ws, void* stream) {
   if (!ws) return ART_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -582,6 +663,7 @@ art_status art_read_device_status(void* ws, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return ART_ERR_CUDA;
   if (h & artk::kStatusSeqLen) return ART_ERR_SEQLEN;
   if (h & artk::kStatusTimeout) return ART_ERR_TIMEOUT;
+  if (h & artk::kStatusOrder) return ART_ERR_ORDER;
   return ART_OK;
 }
 
@@ -611,6 +693,7 @@ const char* art_status_string(art_status status) {
     case ART_ERR_CUDA: return "ART_ERR_CUDA";
     case ART_ERR_TIMEOUT: return "ART_ERR_TIMEOUT";
     case ART_ERR_SEQLEN: return "ART_ERR_SEQLEN";
+    case ART_ERR_ORDER: return "ART_ERR_ORDER";
   }
   return "ART_ERR_UNKNOWN";
 }

@@ -11,6 +11,7 @@ namespace artk {
 // Device status bits (sticky word in the workspace).
 constexpr int kStatusSeqLen = 1;
 constexpr int kStatusTimeout = 2;
+constexpr int kStatusOrder = 4;  // a traversal-sequence entry outside its split
 
 // A wait gives up after this many nanoseconds of %globaltimer time.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;

@@ -65,6 +65,8 @@ struct Params {
   int32_t* ws_used;    // [B*Hq*S] tiles consumed per split
   int32_t* ws_tiles_read;  // [B*Hkv*S]
   int32_t* ws_status;
+  const int32_t* order;  // NULL or [B*Hkv][n_max] tile traversal sequences
+  int n_max;             // ceil(L_max / T)
   int B, Hq, Hkv, L_max, T, S, G, C, nstage, n_probe, patience;
   float qscale;  // log2(e)/sqrt(d): scores live in the log2 domain
   float eps_scale, eps_dir, tau;
@@ -291,6 +293,14 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
   const int ns = t1 - t0;
   const int my_tiles = ns > rank ? (ns - rank + C - 1) / C : 0;
   const int rounds = (MODE == MODE_FULL) ? my_tiles : (ns + C - 1) / C;
+  // Tile at position q of this split's traversal sequence (the natural order without one).  An
+  // entry outside the split is replaced by the natural tile (the producer flags it).
+  const int32_t* ord_seq = p.order ? p.order + (static_cast<long long>(b) * p.Hkv + kvh) * p.n_max : nullptr;
+  auto phys_of = [&](int q) -> int {
+    if (!ord_seq) return q;
+    const int e = __ldg(ord_seq + q);
+    return (e >= t0 && e < t1) ? e : q;
+  };
 
   // ---- shared-memory initialisation
   if (tid == 0) {
@@ -327,7 +337,9 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
   const long long slab_row0 = (static_cast<long long>(b) * p.Hkv + kvh) * p.L_max;
   auto issue = [&](int ord) -> bool {
     if (ord >= my_tiles) return false;
-    const int t = t0 + ord * C + rank;
+    const int tq = t0 + ord * C + rank;
+    const int t = phys_of(tq);
+    if (ord_seq && t != __ldg(ord_seq + tq)) atomicOr(p.ws_status, kStatusOrder);
     const int rows = min(T, L - t * T);
     const int stage = ord % p.nstage;
     const uint32_t bar = bar0 + 8 * stage;
@@ -399,7 +411,7 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
   for (int r = 0; r < rounds; ++r) {
     const int t = t0 + r * C + rank;
     const bool have = (MODE == MODE_FULL) ? true : (t < t1);
-    const int rows = have ? min(T, L - t * T) : 0;
+    const int rows = have ? min(T, L - phys_of(t) * T) : 0;
     const int stage = r % p.nstage;
     const int slot = r & 1;
     const uint8_t* st = smem + stage * Ly.stage;

@@ -64,8 +64,12 @@ constexpr int NSLOT = 2 * NWG + 2 * LAG;
 static_assert(LAG % NWG == 0, "a warpgroup merges its own rounds");
 
 struct TcParams {
-  CUtensorMap tmK;  // 64-byte aligned (first members)
+  CUtensorMap tmK;  // 64-byte aligned (first members); box 64 d x 128 positions
   CUtensorMap tmV;
+  CUtensorMap tmK64;  // box 64 d x 64 positions (ordered traversal with tile 64)
+  CUtensorMap tmV64;
+  const int32_t* order;  // NULL or [B*Hkv][n_max] tile traversal sequences (ART only)
+  int n_max;
   const uint16_t* q;
   const int32_t* seq_lens;
   float* o;
@@ -203,6 +207,14 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   const int my_blocks = nblk > rank ? (nblk - rank + C - 1) / C : 0;
   const int R = (nblk + C - 1) / C;
   const int zc = b * p.Hkv + kvh;
+  // Tile at position q of this split's traversal sequence (ART with a sequence; natural order
+  // otherwise).  An entry outside the split is replaced by the natural tile (the producer flags it).
+  const int32_t* ord_seq = (ART && p.order) ? p.order + static_cast<long long>(zc) * p.n_max : nullptr;
+  auto phys_of = [&](int q) -> int {
+    if (!ord_seq) return q;
+    const int e = __ldg(ord_seq + q);
+    return (e >= t0 && e < t1) ? e : q;
+  };
   // tiles of own block jl that lie inside the split
   auto block_tiles = [&](int jl) -> int {
     if (!ART) return 1;
@@ -296,14 +308,35 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         const int stage = jl % NSTG;
         if (jl >= NSTG && !wait_phase(bar(B_EMPTY + stage), ((jl / NSTG) - 1) & 1, ctl, ART, p.ws_status, false)) break;
         const int j = jl * C + rank;
-        const int p0 = pbeg + j * BLK;
         const uint32_t fb = bar(B_FULL + stage);
         const uint32_t st = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES);
-        mbar_arrive_expect_tx(fb, STAGE_BYTES);
-        tma_load_3d(st, &p.tmK, fb, 0, p0, zc);
-        tma_load_3d(st + 16384, &p.tmK, fb, 64, p0, zc);
-        tma_load_3d(st + 32768, &p.tmV, fb, 0, p0, zc);
-        tma_load_3d(st + 49152, &p.tmV, fb, 64, p0, zc);
+        if (!ord_seq || T == BLK) {  // one 128-position run: the block, or its one (reordered) tile
+          int p0 = pbeg + j * BLK;
+          if (ord_seq) {
+            const int ph = phys_of(t0 + j);
+            if (ph != __ldg(ord_seq + t0 + j)) atomicOr(p.ws_status, kStatusOrder);
+            p0 = ph * BLK;
+          }
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          tma_load_3d(st, &p.tmK, fb, 0, p0, zc);
+          tma_load_3d(st + 16384, &p.tmK, fb, 64, p0, zc);
+          tma_load_3d(st + 32768, &p.tmV, fb, 0, p0, zc);
+          tma_load_3d(st + 49152, &p.tmV, fb, 64, p0, zc);
+        } else {  // tile 64 in a sequence: each tile of the block into its half of the stage
+          const int nt = min(KT, t1 - (t0 + j * KT));
+          mbar_arrive_expect_tx(fb, nt * (STAGE_BYTES / 2));
+          for (int i = 0; i < nt; ++i) {
+            const int tq = t0 + j * KT + i;
+            const int ph = phys_of(tq);
+            if (ph != __ldg(ord_seq + tq)) atomicOr(p.ws_status, kStatusOrder);
+            const int r0 = ph * 64;
+            const uint32_t off = i * 8192;  // 64 rows of 128 bytes: whole swizzle atoms
+            tma_load_3d(st + off, &p.tmK64, fb, 0, r0, zc);
+            tma_load_3d(st + 16384 + off, &p.tmK64, fb, 64, r0, zc);
+            tma_load_3d(st + 32768 + off, &p.tmV64, fb, 0, r0, zc);
+            tma_load_3d(st + 49152 + off, &p.tmV64, fb, 64, r0, zc);
+          }
+        }
         ++issued;
         tiles_read += min(BLK / T, t1 - (t0 + j * (BLK / T)));
       }
@@ -424,6 +457,9 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     auto s_phase = [&](int jl) -> bool {
       const int bb = jl & 1, stage = jl % NSTG;
       const int j = jl * C + rank;
+      // this row's KV position (the load is issued before the wait and used after it)
+      const int tq = t0 + j * KT + er / TE;
+      const int ph = (ord_seq && tq < t1) ? phys_of(tq) : 0;
       if (!epi_wait(bar(B_SFULL + bb), (jl >> 1) & 1, ART)) return false;
       tc_fence_after();
       float sv[8];
@@ -431,8 +467,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(bar(B_SFREE + bb));
-      const int pos = pbeg + j * BLK + er;
-      const bool valid = pos < pend;
+      const int pos = ord_seq ? ph * T + (er % TE) : pbeg + j * BLK + er;
+      const bool valid = ord_seq ? (tq < t1 && pos < L) : (pos < pend);
       float s2[GP], red[GP], pw[GP];
 #pragma unroll
       for (int g = 0; g < GP; ++g) red[g] = s2[g] = (valid && g < G) ? sv[g] * p.qscale : -INFINITY;

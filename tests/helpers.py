@@ -18,7 +18,7 @@ KIND = {"f32": oracle.KV_F32, "bf16": oracle.KV_BF16, "q8": oracle.KV_Q8}
 
 
 def oracle_run(w, mode, *, num_splits=None, tile=None, forced_used=None, metrics=False, art=None, tau=None,
-               n_threads=8):
+               n_threads=8, tile_order=None):
     a = (art or w.art) if mode in ("art", "q8_art") else None
     t = w.tau if tau is None else tau
     return oracle.decode(
@@ -26,6 +26,7 @@ def oracle_run(w, mode, *, num_splits=None, tile=None, forced_used=None, metrics
         tile=w.tile if tile is None else tile, num_splits=w.num_splits if num_splits is None else num_splits,
         art=a, tau=(t if mode in ("q8", "q8_art") else 0.0), forced_used=forced_used,
         no_break=metrics and a is not None, want_metrics=metrics and a is not None, n_threads=n_threads,
+        tile_order=tile_order,
     )
 
 
