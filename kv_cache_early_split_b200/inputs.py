@@ -278,3 +278,53 @@ def workload(name: str, *, keys_b=None, keys_h=None) -> Workload:
             kind="q8", B=2, Hq=32, Hkv=8, d=128, L_max=32768, tile=64, tau=1e-6, art=dict(ART_C2), **kw,
         )
     raise ValueError(name)
+
+
+# ----------------------------------------------------------------------------- paged layout
+@dataclass
+class PagedKV:
+    """A workload's K/V (and q8 scales) scattered into a page pool [num_pages, Hkv, page_size, ...].
+
+    block_table[b, i] is the page holding positions [i*page_size, (i+1)*page_size) of sequence b;
+    entries past the sequence are -1.  Pages that no sequence uses hold NaN (fp16 NaN scales for q8),
+    so a read of a wrong page shows up in the output."""
+
+    page_size: int
+    num_pages: int
+    block_table: np.ndarray  # int32 [B, max_pages]
+    k: np.ndarray
+    v: np.ndarray
+    k_scale: np.ndarray | None
+    v_scale: np.ndarray | None
+
+
+def paginate(w: Workload, page_size: int, seed: int = 0, spare_pages: int = 3) -> PagedKV:
+    B, Hkv, L_max = w.B, w.Hkv, w.L_max
+    max_pages = -(-L_max // page_size)
+    need = [-(-int(L) // page_size) for L in w.seq_lens]
+    num_pages = sum(need) + spare_pages
+    perm = np.random.default_rng(seed).permutation(num_pages).astype(np.int32)
+    table = np.full((B, max_pages), -1, np.int32)
+    nxt = 0
+    for b in range(B):
+        table[b, :need[b]] = perm[nxt:nxt + need[b]]
+        nxt += need[b]
+
+    def scatter(x, fill):
+        if x is None:
+            return None
+        tail = x.shape[3:]
+        pool = np.empty((num_pages, Hkv, page_size) + tail, dtype=x.dtype)
+        pool[...] = fill
+        for b in range(B):
+            for i in range(need[b]):
+                j0 = i * page_size
+                j1 = min(j0 + page_size, L_max)
+                pool[table[b, i], :, :j1 - j0] = x[b, :, j0:j1]
+        return pool
+
+    nan = {np.dtype(np.float32): np.float32(np.nan), np.dtype(np.uint16): np.uint16(0x7FC0),
+           np.dtype(np.int8): np.int8(0)}[w.k.dtype]
+    return PagedKV(page_size=page_size, num_pages=num_pages, block_table=table,
+                   k=scatter(w.k, nan), v=scatter(w.v, nan),
+                   k_scale=scatter(w.k_scale, np.uint16(0x7E00)), v_scale=scatter(w.v_scale, np.uint16(0x7E00)))
