@@ -375,6 +375,31 @@ def art_orders(K, dp, w, args, stream):
     return out
 
 
+def paged_sweep(K, w, args, stream):
+    """The same step over a paged copy of the cache (random page placement, block table per
+    sequence), page sizes 64 and 256: ms per call in both modes, and KV bytes read."""
+    import torch
+
+    modes = ("q8", "q8_art") if w.kind == "q8" else ("full", "art")
+    steps = max(3, min(args.steps, 10))
+    out = {}
+    for page in (64, 256):
+        if page % w.tile:
+            continue
+        pg = I.paginate(w, page, seed=1)
+        dpp = K.upload(w, paged=pg)
+        row = {"kernel": K.kernel_name(dpp, modes[1])}
+        for m in modes:
+            _, launch = time_mode(K, dpp, m, steps, 2, stream)
+            row[m] = {"ms": launch, "kv_bytes_read": bytes_read(w, dpp.tiles_read().cpu().numpy())}
+        if K.device_status(dpp) != 0:
+            raise RuntimeError("device status not OK after the paged sweep")
+        out[f"page_{page}"] = row
+        del dpp
+        torch.cuda.empty_cache()
+    return out
+
+
 def art_sweeps(K, dp, w, args, stream):
     """Two sweeps of the ART path on the same buffers (ART modes only).
 
@@ -498,6 +523,7 @@ def run_ours(args):
     }
 
     sweeps = art_sweeps(K, dp, w, args, stream) if not args.no_sweeps else None
+    paged = paged_sweep(K, w, args, stream) if not args.no_sweeps else None
 
     # end to end through the public call: the step's query in from pinned host memory, O and tiles back out
     q_host = dp.q.cpu().pin_memory()
@@ -549,6 +575,7 @@ def run_ours(args):
                      "kernel": kernel, "bytes_per_launch": rb, "launch_ms": launch_ms},
         "modes": modes,
         "art_sweeps": sweeps,
+        "paged": paged,
         "e2e": e2e,
         "gpu_launches": gpu_launches,
         "clocks": clocks,

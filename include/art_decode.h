@@ -80,7 +80,8 @@ typedef enum {
   ART_ERR_CUDA = -4,        /* a CUDA runtime call failed (launch, attribute) */
   ART_ERR_TIMEOUT = -5,     /* device: a bounded wait gave up (status word) */
   ART_ERR_SEQLEN = -6,      /* device: a seq_len outside [1, L_max] (status word) */
-  ART_ERR_ORDER = -7        /* device: a tile_order entry outside its split (status word) */
+  ART_ERR_ORDER = -7,       /* device: a tile_order entry outside its split (status word) */
+  ART_ERR_PAGE = -8         /* device: a block_table entry outside [0, num_pages) (status word) */
 } art_status;
 
 typedef enum { ART_F32 = 0, ART_BF16 = 1 } art_dtype;
@@ -219,9 +220,43 @@ art_status art_decode_attn_terminate_ordered(const art_shape* shape, art_dtype d
                                              const art_params* params, const int32_t* tile_order, float* o,
                                              int32_t* tiles, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- Paged KV cache.  The serving stack the pages measure against (vLLM; the
+ * intelligenzai.it page on random-attention eviction quotes its step latencies on an
+ * H200) keeps the cache in fixed-size pages behind a per-sequence block table.  Position j of
+ * sequence b lives in page block_table[b][j / page_size], row j % page_size, of
+ * page pools laid out [num_pages][Hkv][page_size][d] (q8 scales
+ * [num_pages][Hkv][page_size][d/32]).  Pages may be shared between sequences.
+ * Entries of a block-table row past ceil(L_b / page_size) are never read.  An
+ * entry outside [0, num_pages) is replaced by page 0 and flags ART_ERR_PAGE in
+ * the status word (results of that call are then unspecified). */
+typedef struct {
+  int32_t page_size;         /* positions per page: a multiple of shape->tile (the tensor-core
+                                kernel needs a multiple of 64; others use the CUDA-core kernel) */
+  int32_t num_pages;         /* pages in each pool */
+  int32_t max_pages_per_seq; /* columns of block_table; shape->L_max <= max_pages_per_seq * page_size */
+  const int32_t* block_table; /* DEVICE int32 [B][max_pages_per_seq] */
+} art_paged_kv;
+
+/* Decode attention over a paged cache: full attention (params == NULL) or ART
+ * (params != NULL), optionally along traversal sequences (tile_order != NULL,
+ * ART only; see art_decode_attn_terminate_ordered).  Same outputs, workspace and
+ * errors as the contiguous entry points; k_pages / v_pages are the pools. */
+art_status art_decode_attn_paged(const art_shape* shape, art_dtype dtype, const void* q, const void* k_pages,
+                                 const void* v_pages, const art_paged_kv* pages, const int32_t* seq_lens,
+                                 const art_params* params, const int32_t* tile_order, float* o, int32_t* tiles,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* art_decode_attn_q8_skipv over a paged q8 cache (pools of int8 codes and fp16
+ * scales); params == NULL runs without ART. */
+art_status art_decode_attn_q8_skipv_paged(const art_shape* shape, const void* q_bf16, const int8_t* k_q_pages,
+                                          const uint16_t* k_scale_pages, const int8_t* v_q_pages,
+                                          const uint16_t* v_scale_pages, const art_paged_kv* pages,
+                                          const int32_t* seq_lens, float tau, const art_params* params, float* o,
+                                          int32_t* tiles, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream`, read the sticky status word of ws, clear it, and
- * return ART_OK, ART_ERR_SEQLEN, ART_ERR_TIMEOUT or ART_ERR_ORDER (ART_ERR_CUDA
- * if the synchronisation or copy failed). */
+ * return ART_OK, ART_ERR_SEQLEN, ART_ERR_TIMEOUT, ART_ERR_ORDER or ART_ERR_PAGE
+ * (ART_ERR_CUDA if the synchronisation or copy failed). */
 art_status art_read_device_status(void* ws, void* stream);
 
 /* Base name of the CUDA kernel a call with this shape would launch for its

@@ -33,6 +33,8 @@ class DeviceProblem:
     ws: object
     art: dict
     tau: float
+    pages: object = None  # paged cache: capi.art_paged_kv (k, v, scales are then page pools)
+    block_table: object = None
 
     @property
     def ws_bytes(self) -> int:
@@ -72,8 +74,10 @@ def _t(torch, arr, device, dtype=None):
     return t.to(device)
 
 
-def upload(w, device="cuda", num_splits=None, tile=None):
-    """Copy a kv_cache_early_split_b200.inputs.Workload to the GPU and allocate o / tiles / workspace."""
+def upload(w, device="cuda", num_splits=None, tile=None, paged=None):
+    """Copy a kv_cache_early_split_b200.inputs.Workload to the GPU and allocate o / tiles / workspace.
+    paged: None, or an inputs.PagedKV of the same workload: its page pools and block table are
+    uploaded instead of the contiguous K/V."""
     import torch
 
     S = w.num_splits if num_splits is None else int(num_splits)
@@ -82,10 +86,17 @@ def upload(w, device="cuda", num_splits=None, tile=None):
     wsb = capi.art_workspace_bytes(shape)
     if wsb == 0:
         raise ArtError(capi.ART_ERR_INVALID_ARG, "art_workspace_bytes")
+    src = w if paged is None else paged
+    bt = None
+    pg = None
+    if paged is not None:
+        bt = _t(torch, paged.block_table, device, torch.int32)
+        pg = capi.art_paged_kv(paged.page_size, paged.num_pages, paged.block_table.shape[1], bt.data_ptr())
     return DeviceProblem(
         kind=w.kind, shape=shape,
-        q=_t(torch, w.q, device), k=_t(torch, w.k, device), v=_t(torch, w.v, device),
-        k_scale=_t(torch, w.k_scale, device), v_scale=_t(torch, w.v_scale, device),
+        q=_t(torch, w.q, device), k=_t(torch, src.k, device), v=_t(torch, src.v, device),
+        k_scale=_t(torch, src.k_scale, device), v_scale=_t(torch, src.v_scale, device),
+        pages=pg, block_table=bt,
         seq_lens=_t(torch, w.seq_lens, device, torch.int32),
         o=torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=device),
         tiles=torch.empty((w.B, w.Hq), dtype=torch.int32, device=device),
@@ -115,6 +126,8 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
     st = torch.cuda.current_stream().cuda_stream if stream is None else stream
     a = dp.art if art is None else art
     dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
+    if dp.pages is not None:
+        return _decode_paged(dp, mode, a, tau, st, check, order)
     if mode == "full":
         rc = capi.art_decode_attn_full(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens),
                                        _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
@@ -138,6 +151,29 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
             dp.shape, _ptr(dp.q), _ptr(dp.k), _ptr(dp.k_scale), _ptr(dp.v), _ptr(dp.v_scale), _ptr(dp.seq_lens),
             dp.tau if tau is None else tau, params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
         name = "art_decode_attn_q8_skipv"
+    else:
+        raise ValueError(mode)
+    if check and rc != capi.ART_OK:
+        raise ArtError(rc, name)
+    return rc
+
+
+def _decode_paged(dp, mode, a, tau, st, check, order):
+    params = None
+    if mode in ("art", "q8_art"):
+        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+    if mode in ("full", "art"):
+        dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
+        rc = capi.art_decode_attn_paged(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), dp.pages,
+                                        _ptr(dp.seq_lens), params, _ptr(order), _ptr(dp.o), _ptr(dp.tiles),
+                                        _ptr(dp.ws), dp.ws_bytes, st)
+        name = "art_decode_attn_paged"
+    elif mode in ("q8", "q8_art"):
+        rc = capi.art_decode_attn_q8_skipv_paged(
+            dp.shape, _ptr(dp.q), _ptr(dp.k), _ptr(dp.k_scale), _ptr(dp.v), _ptr(dp.v_scale), dp.pages,
+            _ptr(dp.seq_lens), dp.tau if tau is None else tau, params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws),
+            dp.ws_bytes, st)
+        name = "art_decode_attn_q8_skipv_paged"
     else:
         raise ValueError(mode)
     if check and rc != capi.ART_OK:
@@ -173,8 +209,11 @@ def tile_order(dp: DeviceProblem, kind: str, *, stream=None, summary=None):
 
 
 def key_summary(dp: DeviceProblem, *, stream=None):
-    """Mean key per tile, fp32 [B, Hkv, n_max, d] (art_tile_key_summary)."""
+    """Mean key per tile, fp32 [B, Hkv, n_max, d] (art_tile_key_summary; contiguous K only)."""
     import torch
+
+    if dp.pages is not None:
+        raise ValueError("the key summary reads a contiguous cache")
 
     s = dp.shape
     st = torch.cuda.current_stream().cuda_stream if stream is None else stream
@@ -193,6 +232,8 @@ def kernel_name(dp: DeviceProblem, mode: str) -> str:
     name = capi.art_kernel_name(dp.shape, dtype, mode.startswith("q8"), mode in ("art", "q8_art"))
     if name is None:
         raise ArtError(capi.ART_ERR_UNSUPPORTED, "art_kernel_name")
+    if dp.pages is not None and dp.pages.page_size % 64 and name == "art_decode_tc_kernel":
+        name = "art_decode_kernel"  # the tensor-core path takes pages of a multiple of 64 positions
     return name
 
 

@@ -21,6 +21,7 @@ ART_ERR_CUDA = -4
 ART_ERR_TIMEOUT = -5
 ART_ERR_SEQLEN = -6
 ART_ERR_ORDER = -7
+ART_ERR_PAGE = -8
 ART_F32 = 0
 ART_BF16 = 1
 
@@ -40,6 +41,8 @@ EXPORTS = (
     "art_tile_key_summary",
     "art_tile_order_importance",
     "art_decode_attn_terminate_ordered",
+    "art_decode_attn_paged",
+    "art_decode_attn_q8_skipv_paged",
 )
 
 
@@ -57,6 +60,15 @@ class art_params(ctypes.Structure):
     ]
 
 
+class art_paged_kv(ctypes.Structure):
+    _fields_ = [
+        ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("block_table", ctypes.c_void_p),
+    ]
+
+
 class ArtError(RuntimeError):
     def __init__(self, code: int, where: str):
         super().__init__(f"{where}: {art_status_string(code)} ({code})")
@@ -69,6 +81,7 @@ _lib = None
 _P = ctypes.c_void_p
 _SH = ctypes.POINTER(art_shape)
 _PA = ctypes.POINTER(art_params)
+_PG = ctypes.POINTER(art_paged_kv)
 
 
 def lib() -> ctypes.CDLL:
@@ -112,6 +125,12 @@ def lib() -> ctypes.CDLL:
             L.art_decode_attn_terminate_ordered.restype = ctypes.c_int
             L.art_decode_attn_terminate_ordered.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, _P,
                                                             ctypes.c_size_t, _P]
+            L.art_decode_attn_paged.restype = ctypes.c_int
+            L.art_decode_attn_paged.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _PG, _P, _PA, _P, _P, _P, _P,
+                                                ctypes.c_size_t, _P]
+            L.art_decode_attn_q8_skipv_paged.restype = ctypes.c_int
+            L.art_decode_attn_q8_skipv_paged.argtypes = [_SH, _P, _P, _P, _P, _P, _PG, _P, ctypes.c_float, _PA, _P,
+                                                         _P, _P, ctypes.c_size_t, _P]
             L.art_kernel_name.restype = ctypes.c_char_p
             L.art_kernel_name.argtypes = [_SH, ctypes.c_int, ctypes.c_int32, ctypes.c_int32]
             _lib = L
@@ -180,6 +199,20 @@ def art_decode_attn_terminate_ordered(shape, dtype, q, k, v, seq_lens, params, t
                                       stream) -> int:
     return int(lib().art_decode_attn_terminate_ordered(
         ctypes.byref(shape), dtype, q, k, v, seq_lens, _ref(params), tile_order, o, tiles, ws, ws_bytes, stream))
+
+
+def art_decode_attn_paged(shape, dtype, q, k_pages, v_pages, pages, seq_lens, params, tile_order, o, tiles, ws,
+                          ws_bytes, stream) -> int:
+    return int(lib().art_decode_attn_paged(
+        ctypes.byref(shape), dtype, q, k_pages, v_pages, _ref(pages), seq_lens, _ref(params), tile_order, o, tiles,
+        ws, ws_bytes, stream))
+
+
+def art_decode_attn_q8_skipv_paged(shape, q_bf16, k_q_pages, k_scale_pages, v_q_pages, v_scale_pages, pages, seq_lens,
+                                   tau, params, o, tiles, ws, ws_bytes, stream) -> int:
+    return int(lib().art_decode_attn_q8_skipv_paged(
+        ctypes.byref(shape), q_bf16, k_q_pages, k_scale_pages, v_q_pages, v_scale_pages, _ref(pages), seq_lens,
+        float(tau), _ref(params), o, tiles, ws, ws_bytes, stream))
 
 
 def art_kernel_name(shape, dtype, kv_q8, with_art):

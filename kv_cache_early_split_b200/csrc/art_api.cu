@@ -232,10 +232,24 @@ EncodeTiledFn encode_fn() {
   return g_encode;
 }
 
-bool tc_eligible(int kind, int mode, const art_shape* s) {
+bool tc_eligible(int kind, int mode, const art_shape* s, const art_paged_kv* pg = nullptr) {
   const int G = s->Hq / s->Hkv;
   return kind == artk::KV_BF16 && (mode == artk::MODE_FULL || mode == artk::MODE_ART) && s->d == 128 &&
-         (s->tile == 64 || s->tile == 128) && G >= 1 && G <= 8;
+         (s->tile == 64 || s->tile == 128) && G >= 1 && G <= 8 && (!pg || pg->page_size % 64 == 0);
+}
+
+// A bf16 page pool [num_pages*Hkv][page_size][128] as a 3-D tensor map; box = 64 d x 64 positions.
+bool make_pool_map(CUtensorMap* m, const void* base, const art_shape* s, const art_paged_kv* pg) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(pg->page_size),
+                              static_cast<cuuint64_t>(pg->num_pages) * s->Hkv};
+  const cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(pg->page_size) * 256};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // K/V [B*Hkv][L_max][128] bf16 as a 3-D tensor map; box = 64 d x `rows` positions (128 or 64),
@@ -269,7 +283,7 @@ TcFn tc_pick(int mode, int G, int n_probe) {
 
 art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k, const void* v,
                      const int32_t* seq_lens, const art_params* a, const int32_t* order, float* o,
-                     int32_t* tiles, void* ws, void* stream) {
+                     int32_t* tiles, void* ws, void* stream, const art_paged_kv* pg) {
   const int G = s->Hq / s->Hkv;
   const TcFn fn = tc_pick(mode, G, a ? a->n_probe : 0);
   artk::tc::TcParams p;
@@ -284,9 +298,17 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
     p.n_probe = a->n_probe;
     for (int i = 0; i < a->n_probe; ++i) p.lanes[i] = static_cast<int8_t>(a->probe_lanes[i]);
   }
-  if (!make_kv_map(&p.tmK, k, s) || !make_kv_map(&p.tmV, v, s)) return ART_ERR_CUDA;
-  if (order && s->tile == 64 && (!make_kv_map(&p.tmK64, k, s, 64) || !make_kv_map(&p.tmV64, v, s, 64)))
-    return ART_ERR_CUDA;
+  if (pg) {  // the paged path loads 64-position halves from the page pools
+    if (!make_pool_map(&p.tmK64, k, s, pg) || !make_pool_map(&p.tmV64, v, s, pg)) return ART_ERR_CUDA;
+    p.block_table = pg->block_table;
+    p.page_size = pg->page_size;
+    p.max_pages = pg->max_pages_per_seq;
+    p.num_pages = pg->num_pages;
+  } else {
+    if (!make_kv_map(&p.tmK, k, s) || !make_kv_map(&p.tmV, v, s)) return ART_ERR_CUDA;
+    if (order && s->tile == 64 && (!make_kv_map(&p.tmK64, k, s, 64) || !make_kv_map(&p.tmV64, v, s, 64)))
+      return ART_ERR_CUDA;
+  }
   p.order = order;
   p.n_max = (s->L_max + s->tile - 1) / s->tile;
   int sms = 0;
@@ -379,6 +401,15 @@ art_status validate_common(const art_shape* s, const void* q, const void* k, con
   return ART_OK;
 }
 
+art_status validate_paged(const art_shape* s, const art_paged_kv* pg) {
+  if (!pg || !pg->block_table || (reinterpret_cast<uintptr_t>(pg->block_table) & 3u)) return ART_ERR_INVALID_ARG;
+  if (pg->page_size < 1 || pg->num_pages < 1 || pg->max_pages_per_seq < 1) return ART_ERR_INVALID_ARG;
+  if (pg->page_size % s->tile != 0) return ART_ERR_UNSUPPORTED;
+  if (1LL * pg->max_pages_per_seq * pg->page_size < s->L_max) return ART_ERR_INVALID_ARG;
+  if (1LL * pg->num_pages * s->Hkv * pg->page_size > 0x7fffffffLL) return ART_ERR_UNSUPPORTED;
+  return ART_OK;
+}
+
 art_status validate_params(const art_params* a, int d, int epc, int* emask) {
   if (!a || !a->probe_lanes) return ART_ERR_INVALID_ARG;
   if (a->n_probe < 1 || a->n_probe > artk::PMAX || a->patience < 1) return ART_ERR_INVALID_ARG;
@@ -396,9 +427,11 @@ art_status validate_params(const art_params* a, int d, int epc, int* emask) {
 
 art_status launch(int kind, int mode, const art_shape* s, const void* q, const void* k, const void* v,
                   const uint16_t* ks, const uint16_t* vs, const int32_t* seq_lens, const art_params* a,
-                  float tau, float* o, int32_t* tiles, void* ws, void* stream, const int32_t* order = nullptr) {
+                  float tau, float* o, int32_t* tiles, void* ws, void* stream, const int32_t* order = nullptr,
+                  const art_paged_kv* pg = nullptr) {
   const int G = s->Hq / s->Hkv;
-  if (tc_eligible(kind, mode, s)) return launch_tc(mode, s, q, k, v, seq_lens, a, order, o, tiles, ws, stream);
+  if (tc_eligible(kind, mode, s, pg))
+    return launch_tc(mode, s, q, k, v, seq_lens, a, order, o, tiles, ws, stream, pg);
   KernelInfo ki;
   if (!pick_kernel(kind, mode, s->d, G, &ki)) return ART_ERR_UNSUPPORTED;
   Params p;
@@ -448,6 +481,12 @@ art_status launch(int kind, int mode, const art_shape* s, const void* q, const v
   p.tau = tau;
   p.order = order;
   p.n_max = max_tiles;
+  if (pg) {
+    p.block_table = pg->block_table;
+    p.page_size = pg->page_size;
+    p.max_pages = pg->max_pages_per_seq;
+    p.num_pages = pg->num_pages;
+  }
 
   cudaLaunchConfig_t lc;
   memset(&lc, 0, sizeof lc);
@@ -593,6 +632,41 @@ art_status art_decode_attn_terminate_ordered(const art_shape* shape, art_dtype d
                 stream, tile_order);
 }
 
+art_status art_decode_attn_paged(const art_shape* shape, art_dtype dtype, const void* q, const void* k_pages,
+                                 const void* v_pages, const art_paged_kv* pages, const int32_t* seq_lens,
+                                 const art_params* params, const int32_t* tile_order, float* o, int32_t* tiles,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  art_status st = validate_common(shape, q, k_pages, v_pages, seq_lens, o, ws, ws_bytes);
+  if (st != ART_OK) return st;
+  if (dtype != ART_F32 && dtype != ART_BF16) return ART_ERR_INVALID_ARG;
+  st = validate_paged(shape, pages);
+  if (st != ART_OK) return st;
+  if (tile_order && (!params || (reinterpret_cast<uintptr_t>(tile_order) & 3u))) return ART_ERR_INVALID_ARG;
+  const int kind = dtype == ART_F32 ? artk::KV_F32 : artk::KV_BF16;
+  return launch(kind, params ? artk::MODE_ART : artk::MODE_FULL, shape, q, k_pages, v_pages, nullptr, nullptr,
+                seq_lens, params, 0.f, o, tiles, ws, stream, tile_order, pages);
+}
+
+art_status art_decode_attn_q8_skipv_paged(const art_shape* shape, const void* q_bf16, const int8_t* k_q_pages,
+                                          const uint16_t* k_scale_pages, const int8_t* v_q_pages,
+                                          const uint16_t* v_scale_pages, const art_paged_kv* pages,
+                                          const int32_t* seq_lens, float tau, const art_params* params, float* o,
+                                          int32_t* tiles, void* ws, size_t ws_bytes, void* stream) {
+  art_status st = validate_common(shape, q_bf16, k_q_pages, v_q_pages, seq_lens, o, ws, ws_bytes);
+  if (st != ART_OK) return st;
+  if (!k_scale_pages || !v_scale_pages) return ART_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(k_scale_pages) & 15u) || (reinterpret_cast<uintptr_t>(v_scale_pages) & 15u))
+    return ART_ERR_INVALID_ARG;
+  if (isnan(tau)) return ART_ERR_INVALID_ARG;
+  st = validate_paged(shape, pages);
+  if (st != ART_OK) return st;
+  // every tile's scale run starts on a 16-byte boundary: page_size * (d/32) * 2 bytes per page slab
+  if ((1LL * pages->page_size * (shape->d / 32) * 2) % 16 != 0) return ART_ERR_UNSUPPORTED;
+  const int mode = params ? artk::MODE_SKIP_ART : artk::MODE_SKIP;
+  return launch(artk::KV_Q8, mode, shape, q_bf16, k_q_pages, v_q_pages, k_scale_pages, v_scale_pages, seq_lens,
+                params, tau, o, tiles, ws, stream, nullptr, pages);
+}
+
 art_status art_tile_order_recency(const art_shape* shape, const int32_t* seq_lens, int32_t* tile_order,
                                   void* stream) {
   if (!shape_ok(shape) || !seq_lens || !tile_order) return ART_ERR_INVALID_ARG;
@@ -664,6 +738,7 @@ art_status art_read_device_status(void* ws, void* stream) {
   if (h & artk::kStatusSeqLen) return ART_ERR_SEQLEN;
   if (h & artk::kStatusTimeout) return ART_ERR_TIMEOUT;
   if (h & artk::kStatusOrder) return ART_ERR_ORDER;
+  if (h & artk::kStatusPage) return ART_ERR_PAGE;
   return ART_OK;
 }
 
@@ -694,6 +769,7 @@ const char* art_status_string(art_status status) {
     case ART_ERR_TIMEOUT: return "ART_ERR_TIMEOUT";
     case ART_ERR_SEQLEN: return "ART_ERR_SEQLEN";
     case ART_ERR_ORDER: return "ART_ERR_ORDER";
+    case ART_ERR_PAGE: return "ART_ERR_PAGE";
   }
   return "ART_ERR_UNKNOWN";
 }

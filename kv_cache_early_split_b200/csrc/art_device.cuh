@@ -12,6 +12,7 @@ namespace artk {
 constexpr int kStatusSeqLen = 1;
 constexpr int kStatusTimeout = 2;
 constexpr int kStatusOrder = 4;  // a traversal-sequence entry outside its split
+constexpr int kStatusPage = 8;   // a block-table entry outside the page pool
 
 // A wait gives up after this many nanoseconds of %globaltimer time.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;

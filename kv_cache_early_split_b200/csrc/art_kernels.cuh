@@ -67,6 +67,10 @@ struct Params {
   int32_t* ws_status;
   const int32_t* order;  // NULL or [B*Hkv][n_max] tile traversal sequences
   int n_max;             // ceil(L_max / T)
+  // paged cache: NULL, or [B][max_pages] page of each page_size run of positions; K/V (and q8
+  // scales) are then page pools [num_pages][Hkv][page_size][...]
+  const int32_t* block_table;
+  int page_size, max_pages, num_pages;
   int B, Hq, Hkv, L_max, T, S, G, C, nstage, n_probe, patience;
   float qscale;  // log2(e)/sqrt(d): scores live in the log2 domain
   float eps_scale, eps_dir, tau;
@@ -344,7 +348,16 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
     const int stage = ord % p.nstage;
     const uint32_t bar = bar0 + 8 * stage;
     uint8_t* st = smem + stage * Ly.stage;
-    const long long row = slab_row0 + static_cast<long long>(t) * T;
+    long long row = slab_row0 + static_cast<long long>(t) * T;
+    if (p.block_table) {  // the tile lies inside one page (page_size is a multiple of T)
+      const int pos0 = t * T;
+      int pg = __ldg(p.block_table + static_cast<long long>(b) * p.max_pages + pos0 / p.page_size);
+      if (pg < 0 || pg >= p.num_pages) {
+        atomicOr(p.ws_status, kStatusPage);
+        pg = 0;
+      }
+      row = (static_cast<long long>(pg) * p.Hkv + kvh) * p.page_size + pos0 % p.page_size;
+    }
     uint32_t bytes = 2u * rows * ROWB;
     uint32_t sbytes = 0;
     if constexpr (KIND == KV_Q8) {

@@ -70,6 +70,10 @@ struct TcParams {
   CUtensorMap tmV64;
   const int32_t* order;  // NULL or [B*Hkv][n_max] tile traversal sequences (ART only)
   int n_max;
+  // paged cache: NULL, or [B][max_pages] page of each page_size run of positions; tmK64/tmV64 then
+  // map the page pools [num_pages*Hkv][page_size][128] (page_size a multiple of 64)
+  const int32_t* block_table;
+  int page_size, max_pages, num_pages;
   const uint16_t* q;
   const int32_t* seq_lens;
   float* o;
@@ -310,7 +314,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         const int j = jl * C + rank;
         const uint32_t fb = bar(B_FULL + stage);
         const uint32_t st = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES);
-        if (!ord_seq || T == BLK) {  // one 128-position run: the block, or its one (reordered) tile
+        if (!p.block_table && (!ord_seq || T == BLK)) {
+          // one 128-position run: the block, or its one (reordered) tile of 128
           int p0 = pbeg + j * BLK;
           if (ord_seq) {
             const int ph = phys_of(t0 + j);
@@ -322,19 +327,49 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           tma_load_3d(st + 16384, &p.tmK, fb, 64, p0, zc);
           tma_load_3d(st + 32768, &p.tmV, fb, 0, p0, zc);
           tma_load_3d(st + 49152, &p.tmV, fb, 64, p0, zc);
-        } else {  // tile 64 in a sequence: each tile of the block into its half of the stage
-          const int nt = min(KT, t1 - (t0 + j * KT));
-          mbar_arrive_expect_tx(fb, nt * (STAGE_BYTES / 2));
-          for (int i = 0; i < nt; ++i) {
-            const int tq = t0 + j * KT + i;
-            const int ph = phys_of(tq);
-            if (ph != __ldg(ord_seq + tq)) atomicOr(p.ws_status, kStatusOrder);
-            const int r0 = ph * 64;
-            const uint32_t off = i * 8192;  // 64 rows of 128 bytes: whole swizzle atoms
-            tma_load_3d(st + off, &p.tmK64, fb, 0, r0, zc);
-            tma_load_3d(st + 16384 + off, &p.tmK64, fb, 64, r0, zc);
-            tma_load_3d(st + 32768 + off, &p.tmV64, fb, 0, r0, zc);
-            tma_load_3d(st + 49152 + off, &p.tmV64, fb, 64, r0, zc);
+        } else {
+          // two 64-position halves, each from its own place (a tile of a traversal sequence, a
+          // page of a paged cache), loaded when it starts inside the sequence; rows not loaded
+          // are masked by the epilogue
+          int lp[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (ord_seq && T != BLK) {
+              const int tq = t0 + j * KT + h;
+              lp[h] = -1;
+              if (tq < t1) {
+                const int ph = phys_of(tq);
+                if (ph != __ldg(ord_seq + tq)) atomicOr(p.ws_status, kStatusOrder);
+                lp[h] = ph * 64;
+              }
+            } else if (ord_seq) {
+              const int ph = phys_of(t0 + j);
+              if (h == 0 && ph != __ldg(ord_seq + t0 + j)) atomicOr(p.ws_status, kStatusOrder);
+              lp[h] = ph * BLK + 64 * h;
+            } else {
+              lp[h] = pbeg + j * BLK + 64 * h;
+            }
+            if (lp[h] >= L) lp[h] = -1;
+          }
+          mbar_arrive_expect_tx(fb, ((lp[0] >= 0) + (lp[1] >= 0)) * (STAGE_BYTES / 2));
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (lp[h] < 0) continue;
+            int r = lp[h], z = zc;
+            if (p.block_table) {
+              int pg = __ldg(p.block_table + static_cast<long long>(b) * p.max_pages + lp[h] / p.page_size);
+              if (pg < 0 || pg >= p.num_pages) {
+                atomicOr(p.ws_status, kStatusPage);
+                pg = 0;
+              }
+              r = lp[h] % p.page_size;
+              z = pg * p.Hkv + kvh;
+            }
+            const uint32_t off = h * 8192;  // 64 rows of 128 bytes: whole swizzle atoms
+            tma_load_3d(st + off, &p.tmK64, fb, 0, r, z);
+            tma_load_3d(st + 16384 + off, &p.tmK64, fb, 64, r, z);
+            tma_load_3d(st + 32768 + off, &p.tmV64, fb, 0, r, z);
+            tma_load_3d(st + 49152 + off, &p.tmV64, fb, 64, r, z);
           }
         }
         ++issued;
