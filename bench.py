@@ -375,6 +375,42 @@ def art_orders(K, dp, w, args, stream):
     return out
 
 
+def evict_sweep(K, dp, w, args, stream):
+    """Random eviction to a quarter of the cache (sink L/128, recent window L/32, the rest drawn
+    uniformly), then full attention and ART on the packed cache: time of the selection, the packing
+    and the decodes, KV bytes read, and error against full attention over the whole cache."""
+    import torch
+
+    L = int(w.L_max)
+    budget, sink, recent = L // 4, L // 128, L // 32
+    if budget < sink + recent + 1:
+        return None
+    steps = max(3, min(args.steps, 10))
+    full_mode, art_mode = ("q8", "q8_art") if w.kind == "q8" else ("full", "art")
+    K.decode(dp, full_mode)
+    o_full = dp.o.clone()
+    nrm = torch.linalg.vector_norm(o_full, dim=-1).clamp_min(1e-30)
+    gen = torch.Generator(device=dp.k.device).manual_seed(1234)
+    keys = torch.randint(-2**31, 2**31 - 1, (w.B, w.Hkv, L), dtype=torch.int32, device=dp.k.device, generator=gen)
+    dp2, kept = K.evict_random(dp, keys, sink, recent, budget, stream=stream.cuda_stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):  # selection + packing of K and V into the same buffers (no allocation)
+        K.evict_random_into(dp, dp2, kept, keys, sink, recent, stream=stream.cuda_stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    out = {"budget": budget, "n_sink": sink, "n_recent": recent, "select_and_pack_ms": e0.elapsed_time(e1) / steps}
+    for m in (full_mode, art_mode):
+        _, launch = time_mode(K, dp2, m, steps, 2, stream)
+        rel = torch.linalg.vector_norm(dp2.o - o_full, dim=-1) / nrm
+        out[m] = {"ms": launch, "kv_bytes_read": bytes_read(w, dp2.tiles_read().cpu().numpy()),
+                  "rel_err_mean": float(rel.mean().item()), "rel_err_max": float(rel.max().item())}
+    if K.device_status(dp2) != 0:
+        raise RuntimeError("device status not OK after the eviction sweep")
+    return out
+
+
 def paged_sweep(K, w, args, stream):
     """The same step over a paged copy of the cache (random page placement, block table per
     sequence), page sizes 64 and 256: ms per call in both modes, and KV bytes read."""
@@ -524,6 +560,7 @@ def run_ours(args):
 
     sweeps = art_sweeps(K, dp, w, args, stream) if not args.no_sweeps else None
     paged = paged_sweep(K, w, args, stream) if not args.no_sweeps else None
+    evicted = evict_sweep(K, dp, w, args, stream) if not args.no_sweeps else None
 
     # end to end through the public call: the step's query in from pinned host memory, O and tiles back out
     q_host = dp.q.cpu().pin_memory()
@@ -576,6 +613,7 @@ def run_ours(args):
         "modes": modes,
         "art_sweeps": sweeps,
         "paged": paged,
+        "eviction": evicted,
         "e2e": e2e,
         "gpu_launches": gpu_launches,
         "clocks": clocks,

@@ -254,6 +254,36 @@ art_status art_decode_attn_q8_skipv_paged(const art_shape* shape, const void* q_
                                           const int32_t* seq_lens, float tau, const art_params* params, float* o,
                                           int32_t* tiles, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- Random KV eviction ahead of ART (intelligenzai.it page on arXiv 2609.03430,
+ * Random Attention: keep the initial prompt and the most recent window, drop the
+ * rest uniformly at random inside each head; "Resumen Tecnico: ART" S2.4: ART runs
+ * on what a cache policy keeps).  This library's reading, per (batch, kv head):
+ * a sequence of length L <= budget keeps every position; otherwise it keeps
+ * [0, n_sink), [L - n_recent, L) and the m = budget - n_sink - n_recent middle
+ * positions j whose (rand_keys[b][h][j], j) pairs are the m smallest (a uniform
+ * draw without replacement when the keys are uniform and independent).  The
+ * caller supplies the random keys, so the draw is reproducible.  The kept rows
+ * are then packed (art_evict_compact) into a cache of L_max = budget, and any
+ * decode entry point runs on it with seq_lens = kept_lens. */
+typedef enum { ART_KV_F32 = 0, ART_KV_BF16 = 1, ART_KV_Q8 = 2 } art_kv_format;
+
+/* kept[B][Hkv][budget] int32 (DEVICE): the kept positions in increasing order,
+ * -1 past min(L_b, budget); kept_lens[B] (DEVICE) = min(L_b, budget) (0 for a
+ * seq_len outside [1, L_max]).  rand_keys: DEVICE uint32 [B][Hkv][L_max].
+ * Requires n_sink >= 0, n_recent >= 0, budget >= max(1, n_sink + n_recent). */
+art_status art_evict_random_select(const art_shape* shape, const int32_t* seq_lens, const uint32_t* rand_keys,
+                                   int32_t n_sink, int32_t n_recent, int32_t budget, int32_t* kept,
+                                   int32_t* kept_lens, void* stream);
+
+/* Pack rows: dst[b][h][i] = src[b][h][kept[b][h][i]] for the [B][Hkv][L_max][d]
+ * cache `src` of the given format into dst [B][Hkv][budget][d]; q8 also packs its
+ * scales (src_scale [B][Hkv][L_max][d/32] -> dst_scale [B][Hkv][budget][d/32];
+ * pass NULL for both otherwise).  Rows whose index is -1 (or outside [0, L_max))
+ * are written as zeros.  Call once for K and once for V. */
+art_status art_evict_compact(const art_shape* shape, art_kv_format format, const void* src,
+                             const uint16_t* src_scale, const int32_t* kept, int32_t budget, void* dst,
+                             uint16_t* dst_scale, void* stream);
+
 /* Synchronise `stream`, read the sticky status word of ws, clear it, and
  * return ART_OK, ART_ERR_SEQLEN, ART_ERR_TIMEOUT, ART_ERR_ORDER or ART_ERR_PAGE
  * (ART_ERR_CUDA if the synchronisation or copy failed). */

@@ -13,7 +13,8 @@ from dataclasses import dataclass
 from . import capi
 from .capi import ArtError
 
-__all__ = ["capi", "ArtError", "DeviceProblem", "upload", "decode", "kernel_name", "tile_order", "key_summary"]
+__all__ = ["capi", "ArtError", "DeviceProblem", "upload", "decode", "kernel_name", "tile_order", "key_summary",
+           "evict_random", "evict_random_into"]
 
 
 @dataclass
@@ -206,6 +207,55 @@ def tile_order(dp: DeviceProblem, kind: str, *, stream=None, summary=None):
     if rc != capi.ART_OK:
         raise ArtError(rc, name)
     return out
+
+
+def evict_random(dp: DeviceProblem, rand_keys, n_sink: int, n_recent: int, budget: int, *, stream=None):
+    """Random eviction on the GPU (art_evict_random_select + art_evict_compact): returns (the
+    DeviceProblem of the packed cache, L_max = budget, seq_lens = kept lengths; kept positions
+    int32 [B, Hkv, budget]).  rand_keys: device tensor of 32-bit keys [B, Hkv, L_max] (int32 or
+    uint32 bits)."""
+    import torch
+
+    if dp.pages is not None:
+        raise ValueError("eviction packs a contiguous cache")
+    s = dp.shape
+    dev = dp.k.device
+    shape2 = capi.art_shape(s.B, s.Hq, s.Hkv, s.d, budget, s.tile, s.num_splits)
+
+    def like(x, rows_last):
+        return None if x is None else torch.empty((s.B, s.Hkv, budget, rows_last), dtype=x.dtype, device=dev)
+
+    dp2 = DeviceProblem(
+        kind=dp.kind, shape=shape2, q=dp.q, k=like(dp.k, s.d), v=like(dp.v, s.d),
+        k_scale=like(dp.k_scale, s.d // 32), v_scale=like(dp.v_scale, s.d // 32),
+        seq_lens=torch.empty((s.B,), dtype=torch.int32, device=dev), o=torch.empty_like(dp.o),
+        tiles=torch.empty_like(dp.tiles), ws=torch.zeros(capi.art_workspace_bytes(shape2), dtype=torch.uint8,
+                                                         device=dev),
+        art=dict(dp.art), tau=dp.tau)
+    kept = torch.empty((s.B, s.Hkv, budget), dtype=torch.int32, device=dev)
+    evict_random_into(dp, dp2, kept, rand_keys, n_sink, n_recent, stream=stream)
+    return dp2, kept
+
+
+def evict_random_into(dp: DeviceProblem, dp2: DeviceProblem, kept, rand_keys, n_sink: int, n_recent: int, *,
+                      stream=None) -> None:
+    """evict_random into the buffers of an existing packed problem (no allocation): kept positions
+    into `kept`, kept lengths into dp2.seq_lens, packed rows into dp2.k / dp2.v (and scales)."""
+    import torch
+
+    s = dp.shape
+    budget = dp2.shape.L_max
+    st = torch.cuda.current_stream().cuda_stream if stream is None else stream
+    rc = capi.art_evict_random_select(s, _ptr(dp.seq_lens), _ptr(rand_keys), n_sink, n_recent, budget, _ptr(kept),
+                                      _ptr(dp2.seq_lens), st)
+    if rc != capi.ART_OK:
+        raise ArtError(rc, "art_evict_random_select")
+    fmt = {"f32": capi.ART_KV_F32, "bf16": capi.ART_KV_BF16, "q8": capi.ART_KV_Q8}[dp.kind]
+    for name in ("k", "v"):
+        rc = capi.art_evict_compact(s, fmt, _ptr(getattr(dp, name)), _ptr(getattr(dp, name + "_scale")), _ptr(kept),
+                                    budget, _ptr(getattr(dp2, name)), _ptr(getattr(dp2, name + "_scale")), st)
+        if rc != capi.ART_OK:
+            raise ArtError(rc, "art_evict_compact")
 
 
 def key_summary(dp: DeviceProblem, *, stream=None):

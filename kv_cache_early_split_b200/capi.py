@@ -24,6 +24,7 @@ ART_ERR_ORDER = -7
 ART_ERR_PAGE = -8
 ART_F32 = 0
 ART_BF16 = 1
+ART_KV_F32, ART_KV_BF16, ART_KV_Q8 = 0, 1, 2
 
 # every symbol the header declares
 EXPORTS = (
@@ -43,6 +44,8 @@ EXPORTS = (
     "art_decode_attn_terminate_ordered",
     "art_decode_attn_paged",
     "art_decode_attn_q8_skipv_paged",
+    "art_evict_random_select",
+    "art_evict_compact",
 )
 
 
@@ -131,6 +134,11 @@ def lib() -> ctypes.CDLL:
             L.art_decode_attn_q8_skipv_paged.restype = ctypes.c_int
             L.art_decode_attn_q8_skipv_paged.argtypes = [_SH, _P, _P, _P, _P, _P, _PG, _P, ctypes.c_float, _PA, _P,
                                                          _P, _P, ctypes.c_size_t, _P]
+            L.art_evict_random_select.restype = ctypes.c_int
+            L.art_evict_random_select.argtypes = [_SH, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                                                  _P]
+            L.art_evict_compact.restype = ctypes.c_int
+            L.art_evict_compact.argtypes = [_SH, ctypes.c_int, _P, _P, _P, ctypes.c_int32, _P, _P, _P]
             L.art_kernel_name.restype = ctypes.c_char_p
             L.art_kernel_name.argtypes = [_SH, ctypes.c_int, ctypes.c_int32, ctypes.c_int32]
             _lib = L
@@ -213,6 +221,16 @@ def art_decode_attn_q8_skipv_paged(shape, q_bf16, k_q_pages, k_scale_pages, v_q_
     return int(lib().art_decode_attn_q8_skipv_paged(
         ctypes.byref(shape), q_bf16, k_q_pages, k_scale_pages, v_q_pages, v_scale_pages, _ref(pages), seq_lens,
         float(tau), _ref(params), o, tiles, ws, ws_bytes, stream))
+
+
+def art_evict_random_select(shape, seq_lens, rand_keys, n_sink, n_recent, budget, kept, kept_lens, stream) -> int:
+    return int(lib().art_evict_random_select(ctypes.byref(shape), seq_lens, rand_keys, int(n_sink), int(n_recent),
+                                             int(budget), kept, kept_lens, stream))
+
+
+def art_evict_compact(shape, fmt, src, src_scale, kept, budget, dst, dst_scale, stream) -> int:
+    return int(lib().art_evict_compact(ctypes.byref(shape), int(fmt), src, src_scale, kept, int(budget), dst,
+                                       dst_scale, stream))
 
 
 def art_kernel_name(shape, dtype, kv_q8, with_art):

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "art_decode.h"
+#include "art_evict.cuh"
 #include "art_kernels.cuh"
 #include "art_order.cuh"
 #include "art_tc.cuh"
@@ -665,6 +666,43 @@ art_status art_decode_attn_q8_skipv_paged(const art_shape* shape, const void* q_
   const int mode = params ? artk::MODE_SKIP_ART : artk::MODE_SKIP;
   return launch(artk::KV_Q8, mode, shape, q_bf16, k_q_pages, v_q_pages, k_scale_pages, v_scale_pages, seq_lens,
                 params, tau, o, tiles, ws, stream, nullptr, pages);
+}
+
+art_status art_evict_random_select(const art_shape* shape, const int32_t* seq_lens, const uint32_t* rand_keys,
+                                   int32_t n_sink, int32_t n_recent, int32_t budget, int32_t* kept,
+                                   int32_t* kept_lens, void* stream) {
+  if (!shape_ok(shape) || !seq_lens || !rand_keys || !kept || !kept_lens) return ART_ERR_INVALID_ARG;
+  if (n_sink < 0 || n_recent < 0 || budget < 1 || 1LL * n_sink + n_recent > budget) return ART_ERR_INVALID_ARG;
+  const unsigned grid = static_cast<unsigned>(shape->B) * shape->Hkv;
+  artk::evict::evict_select_kernel<<<grid, artk::evict::kSelThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      seq_lens, rand_keys, shape->Hkv, shape->L_max, n_sink, n_recent, budget, kept, kept_lens);
+  return cudaGetLastError() == cudaSuccess ? ART_OK : ART_ERR_CUDA;
+}
+
+art_status art_evict_compact(const art_shape* shape, art_kv_format format, const void* src,
+                             const uint16_t* src_scale, const int32_t* kept, int32_t budget, void* dst,
+                             uint16_t* dst_scale, void* stream) {
+  if (!shape_ok(shape) || !src || !kept || !dst || budget < 1) return ART_ERR_INVALID_ARG;
+  if (format != ART_KV_F32 && format != ART_KV_BF16 && format != ART_KV_Q8) return ART_ERR_INVALID_ARG;
+  const bool q8 = format == ART_KV_Q8;
+  if (q8 != (src_scale != nullptr) || q8 != (dst_scale != nullptr)) return ART_ERR_INVALID_ARG;
+  if (q8 && shape->d % 32 != 0) return ART_ERR_UNSUPPORTED;
+  const int esz = format == ART_KV_F32 ? 4 : (format == ART_KV_BF16 ? 2 : 1);
+  const int row_bytes = shape->d * esz;
+  if (row_bytes % 16 != 0) return ART_ERR_UNSUPPORTED;
+  auto mis = [](const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
+  if (mis(src, 16) || mis(dst, 16) || (q8 && (mis(src_scale, 4) || mis(dst_scale, 4)))) return ART_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  constexpr int kWarps = 8;
+  const dim3 grid(static_cast<unsigned>(shape->B) * shape->Hkv, (budget + kWarps - 1) / kWarps);
+  if (grid.y > 65535u) return ART_ERR_UNSUPPORTED;
+  artk::evict::evict_compact_kernel<uint4><<<grid, 32 * kWarps, 0, st>>>(
+      static_cast<const uint8_t*>(src), kept, shape->L_max, budget, row_bytes, static_cast<uint8_t*>(dst));
+  if (q8)
+    artk::evict::evict_compact_kernel<uint32_t><<<grid, 32 * kWarps, 0, st>>>(
+        reinterpret_cast<const uint8_t*>(src_scale), kept, shape->L_max, budget, (shape->d / 32) * 2,
+        reinterpret_cast<uint8_t*>(dst_scale));
+  return cudaGetLastError() == cudaSuccess ? ART_OK : ART_ERR_CUDA;
 }
 
 art_status art_tile_order_recency(const art_shape* shape, const int32_t* seq_lens, int32_t* tile_order,

@@ -307,6 +307,19 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   if (warp == WARP_TMA) {
     if (lane == 0) {
       int issued = 0, tiles_read = 0;
+      // paged cache in natural order: the page ids of a block follow from its position, so those of
+      // the next block are loaded while this one's copies are issued and the next stage frees up
+      const bool pg_ahead = p.block_table && !ord_seq;
+      const int32_t* bt_row = p.block_table ? p.block_table + static_cast<long long>(b) * p.max_pages : nullptr;
+      auto page_ids = [&](int jl, int (&pg)[2]) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int lp = pbeg + (jl * C + rank) * BLK + 64 * h;
+          pg[h] = (jl < my_blocks && lp < L) ? __ldg(bt_row + lp / p.page_size) : 0;
+        }
+      };
+      int pg_cur[2] = {0, 0}, pg_next[2] = {0, 0};
+      if (pg_ahead) page_ids(0, pg_cur);
       for (int jl = 0; jl < my_blocks; ++jl) {
         if (ART && ctl[CTL_EXIT]) break;
         const int stage = jl % NSTG;
@@ -357,7 +370,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
             if (lp[h] < 0) continue;
             int r = lp[h], z = zc;
             if (p.block_table) {
-              int pg = __ldg(p.block_table + static_cast<long long>(b) * p.max_pages + lp[h] / p.page_size);
+              int pg = pg_ahead ? pg_cur[h] : __ldg(bt_row + lp[h] / p.page_size);
               if (pg < 0 || pg >= p.num_pages) {
                 atomicOr(p.ws_status, kStatusPage);
                 pg = 0;
@@ -371,6 +384,11 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
             tma_load_3d(st + 32768 + off, &p.tmV64, fb, 0, r, z);
             tma_load_3d(st + 49152 + off, &p.tmV64, fb, 64, r, z);
           }
+        }
+        if (pg_ahead) {
+          page_ids(jl + 1, pg_next);
+          pg_cur[0] = pg_next[0];
+          pg_cur[1] = pg_next[1];
         }
         ++issued;
         tiles_read += min(BLK / T, t1 - (t0 + j * (BLK / T)));
