@@ -269,24 +269,30 @@ bool make_kv_map(CUtensorMap* m, const void* base, const art_shape* s, unsigned 
 
 using TcFn = void (*)(artk::tc::TcParams);
 
-template <int MODE, int PC>
+template <int MODE, int PC, bool GEN>
 TcFn tc_pick_gp(int G) {
-  if (G == 1) return &artk::tc::art_decode_tc_kernel<1, MODE, PC>;
-  if (G == 2) return &artk::tc::art_decode_tc_kernel<2, MODE, PC>;
-  if (G <= 4) return &artk::tc::art_decode_tc_kernel<4, MODE, PC>;
-  return &artk::tc::art_decode_tc_kernel<8, MODE, PC>;
+  if (G == 1) return &artk::tc::art_decode_tc_kernel<1, MODE, PC, GEN>;
+  if (G == 2) return &artk::tc::art_decode_tc_kernel<2, MODE, PC, GEN>;
+  if (G <= 4) return &artk::tc::art_decode_tc_kernel<4, MODE, PC, GEN>;
+  return &artk::tc::art_decode_tc_kernel<8, MODE, PC, GEN>;
 }
 
-TcFn tc_pick(int mode, int G, int n_probe) {
-  if (mode != artk::MODE_ART) return tc_pick_gp<artk::MODE_FULL, 16>(G);
-  return n_probe <= 16 ? tc_pick_gp<artk::MODE_ART, 16>(G) : tc_pick_gp<artk::MODE_ART, 32>(G);
+template <bool GEN>
+TcFn tc_pick_gen(int mode, int G, int n_probe) {
+  if (mode != artk::MODE_ART) return tc_pick_gp<artk::MODE_FULL, 16, GEN>(G);
+  return n_probe <= 16 ? tc_pick_gp<artk::MODE_ART, 16, GEN>(G) : tc_pick_gp<artk::MODE_ART, 32, GEN>(G);
+}
+
+// gen: a traversal sequence or a paged cache (the general-addressing instantiations)
+TcFn tc_pick(int mode, int G, int n_probe, bool gen) {
+  return gen ? tc_pick_gen<true>(mode, G, n_probe) : tc_pick_gen<false>(mode, G, n_probe);
 }
 
 art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k, const void* v,
                      const int32_t* seq_lens, const art_params* a, const int32_t* order, float* o,
                      int32_t* tiles, void* ws, void* stream, const art_paged_kv* pg) {
   const int G = s->Hq / s->Hkv;
-  const TcFn fn = tc_pick(mode, G, a ? a->n_probe : 0);
+  const TcFn fn = tc_pick(mode, G, a ? a->n_probe : 0, order != nullptr || pg != nullptr);
   artk::tc::TcParams p;
   memset(&p, 0, sizeof p);
   if (a) {

@@ -178,7 +178,9 @@ __device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parit
 
 // GP: query heads per kv head (padded to 1, 2, 4 or 8); MODE: full or ART;
 // PC: probe-lane capacity of the rule replay (16 or 32, lanes beyond n_probe are zero).
-template <int GP, int MODE, int PC>
+// GEN: general addressing (a traversal sequence or a paged cache); without it the kernel carries
+// none of that code (smaller instruction footprint on the contiguous, natural-order path).
+template <int GP, int MODE, int PC, bool GEN>
 __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
   using PB = Pub<GP, PC>;
@@ -213,7 +215,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   const int zc = b * p.Hkv + kvh;
   // Tile at position q of this split's traversal sequence (ART with a sequence; natural order
   // otherwise).  An entry outside the split is replaced by the natural tile (the producer flags it).
-  const int32_t* ord_seq = (ART && p.order) ? p.order + static_cast<long long>(zc) * p.n_max : nullptr;
+  const int32_t* ord_seq = (GEN && ART && p.order) ? p.order + static_cast<long long>(zc) * p.n_max : nullptr;
+  const int32_t* const btab = GEN ? p.block_table : nullptr;
   auto phys_of = [&](int q) -> int {
     if (!ord_seq) return q;
     const int e = __ldg(ord_seq + q);
@@ -309,8 +312,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       int issued = 0, tiles_read = 0;
       // paged cache in natural order: the page ids of a block follow from its position, so those of
       // the next block are loaded while this one's copies are issued and the next stage frees up
-      const bool pg_ahead = p.block_table && !ord_seq;
-      const int32_t* bt_row = p.block_table ? p.block_table + static_cast<long long>(b) * p.max_pages : nullptr;
+      const bool pg_ahead = btab && !ord_seq;
+      const int32_t* bt_row = btab ? btab + static_cast<long long>(b) * p.max_pages : nullptr;
       auto page_ids = [&](int jl, int (&pg)[2]) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -327,7 +330,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         const int j = jl * C + rank;
         const uint32_t fb = bar(B_FULL + stage);
         const uint32_t st = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES);
-        if (!p.block_table && (!ord_seq || T == BLK)) {
+        if (!btab && (!ord_seq || T == BLK)) {
           // one 128-position run: the block, or its one (reordered) tile of 128
           int p0 = pbeg + j * BLK;
           if (ord_seq) {
@@ -369,7 +372,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           for (int h = 0; h < 2; ++h) {
             if (lp[h] < 0) continue;
             int r = lp[h], z = zc;
-            if (p.block_table) {
+            if (btab) {
               int pg = pg_ahead ? pg_cur[h] : __ldg(bt_row + lp[h] / p.page_size);
               if (pg < 0 || pg >= p.num_pages) {
                 atomicOr(p.ws_status, kStatusPage);
