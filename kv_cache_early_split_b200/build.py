@@ -16,7 +16,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libart_decode.so")
-SOURCES = [os.path.join(CSRC, "art_api.cu")]
+# art_api.cu holds the C ABI and the CUDA-core kernels; art_tc_gp*.cu the tensor-core instantiations
+SOURCES = [os.path.join(CSRC, f) for f in ("art_api.cu", "art_tc_gp1.cu", "art_tc_gp2.cu", "art_tc_gp4.cu",
+                                           "art_tc_gp8.cu")]
 DEPS = SOURCES + [
     os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cuh", ".h"))
 ] + [os.path.join(INCLUDE, "art_decode.h")]
@@ -24,7 +26,7 @@ DEPS = SOURCES + [
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-fPIC",
     "-Xptxas", "-v",
     "--expt-relaxed-constexpr",
 ]
@@ -45,20 +47,35 @@ def needs_build() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object (in parallel), then link the shared library."""
+    from concurrent.futures import ThreadPoolExecutor
+
     if not force and not needs_build():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, *SOURCES, "-o", tmp]
-    r = subprocess.run(cmd, capture_output=True, text=True)
+    tag = f".tmp{os.getpid()}"
+    objs = [os.path.join(PKG, os.path.basename(src)[:-3] + tag + ".o") for src in SOURCES]
+    cmds = [[nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj] for src, obj in zip(SOURCES, objs)]
+    with ThreadPoolExecutor(len(cmds)) as ex:
+        results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds))
+    tmp = LIB + tag
+    link = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", tmp]
+    if all(r.returncode == 0 for r in results):
+        results.append(subprocess.run(link, capture_output=True, text=True))
+        cmds.append(link)
     log = os.path.join(PKG, "build.log")
     with open(log, "w") as f:
-        f.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)
-    if r.returncode != 0:
-        sys.stderr.write(r.stdout + r.stderr)
+        for c, r in zip(cmds, results):
+            f.write(" ".join(c) + "\n" + r.stdout + r.stderr)
+    for o in objs:
+        if os.path.exists(o):
+            os.remove(o)
+    bad = [r for r in results if r.returncode != 0]
+    if bad:
+        sys.stderr.write(bad[0].stdout + bad[0].stderr)
         raise RuntimeError(f"nvcc failed (log: {log})")
     os.replace(tmp, LIB)
     if verbose:
-        sys.stdout.write(r.stderr)
+        sys.stdout.write("".join(r.stderr for r in results))
     return LIB
 
 

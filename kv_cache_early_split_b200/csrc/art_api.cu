@@ -12,7 +12,7 @@
 #include "art_evict.cuh"
 #include "art_kernels.cuh"
 #include "art_order.cuh"
-#include "art_tc.cuh"
+#include "art_tc_pick.cuh"
 
 namespace {
 
@@ -267,32 +267,32 @@ bool make_kv_map(CUtensorMap* m, const void* base, const art_shape* s, unsigned 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-using TcFn = void (*)(artk::tc::TcParams);
+using artk::tc::TcFn;
 
-template <int MODE, int PC, bool GEN>
-TcFn tc_pick_gp(int G) {
-  if (G == 1) return &artk::tc::art_decode_tc_kernel<1, MODE, PC, GEN>;
-  if (G == 2) return &artk::tc::art_decode_tc_kernel<2, MODE, PC, GEN>;
-  if (G <= 4) return &artk::tc::art_decode_tc_kernel<4, MODE, PC, GEN>;
-  return &artk::tc::art_decode_tc_kernel<8, MODE, PC, GEN>;
+// The tensor-core kernel for G heads per kv head; gen: a traversal sequence or a paged cache;
+// ncw: ART controller warps.
+TcFn tc_pick(int mode, int G, int n_probe, bool gen, int ncw) {
+  const int pc = n_probe <= 16 ? 16 : 32;
+  if (G == 1) return artk::tc::kernel_gp1(mode, pc, gen, ncw);
+  if (G == 2) return artk::tc::kernel_gp2(mode, pc, gen, ncw);
+  if (G <= 4) return artk::tc::kernel_gp4(mode, pc, gen, ncw);
+  return artk::tc::kernel_gp8(mode, pc, gen, ncw);
 }
 
-template <bool GEN>
-TcFn tc_pick_gen(int mode, int G, int n_probe) {
-  if (mode != artk::MODE_ART) return tc_pick_gp<artk::MODE_FULL, 16, GEN>(G);
-  return n_probe <= 16 ? tc_pick_gp<artk::MODE_ART, 16, GEN>(G) : tc_pick_gp<artk::MODE_ART, 32, GEN>(G);
-}
-
-// gen: a traversal sequence or a paged cache (the general-addressing instantiations)
-TcFn tc_pick(int mode, int G, int n_probe, bool gen) {
-  return gen ? tc_pick_gen<true>(mode, G, n_probe) : tc_pick_gen<false>(mode, G, n_probe);
+// ART controller warps for cluster size C: two when one round's rule replay needs two or more
+// passes of a warp over the heads (a pass covers 32 / (C * tiles per block) heads).
+int tc_ncw(int mode, int G, int C, int kt) {
+  if (mode != artk::MODE_ART) return 1;
+  const int hpp = 32 / (C * kt);
+  return (G + hpp - 1) / hpp >= 2 ? 2 : 1;
 }
 
 art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k, const void* v,
                      const int32_t* seq_lens, const art_params* a, const int32_t* order, float* o,
                      int32_t* tiles, void* ws, void* stream, const art_paged_kv* pg) {
   const int G = s->Hq / s->Hkv;
-  const TcFn fn = tc_pick(mode, G, a ? a->n_probe : 0, order != nullptr || pg != nullptr);
+  const bool gen = order != nullptr || pg != nullptr;
+  const int n_probe = a ? a->n_probe : 0;
   artk::tc::TcParams p;
   memset(&p, 0, sizeof p);
   if (a) {
@@ -319,7 +319,7 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   p.order = order;
   p.n_max = (s->L_max + s->tile - 1) / s->tile;
   int sms = 0;
-  art_status st = prepare(reinterpret_cast<KernelFn>(fn), &sms);
+  art_status st = prepare(reinterpret_cast<KernelFn>(tc_pick(mode, G, n_probe, gen, 1)), &sms);
   if (st != ART_OK) return st;
   // one CTA per SM; cluster size C: power of two, units*C <= SMs, C*tiles_per_block <= 32 (one rule lane
   // per tile of a round), and no more CTAs than 128-position blocks in a split.
@@ -329,7 +329,12 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   const long long max_blocks = ((max_tiles + s->num_splits - 1) / s->num_splits * s->tile + 127) / 128;
   int C = 1;
   while (C < artk::CMAX && 1LL * units * (2 * C) <= sms && 2 * C * kt <= 32 && 2 * C <= max_blocks) C *= 2;
-  while (C > 1) {
+  TcFn fn = nullptr;
+  while (true) {  // the largest C whose clusters fit, with the kernel variant for that C
+    fn = tc_pick(mode, G, n_probe, gen, tc_ncw(mode, G, C, kt));
+    st = prepare(reinterpret_cast<KernelFn>(fn), &sms);
+    if (st != ART_OK) return st;
+    if (C == 1) break;
     cudaLaunchConfig_t lc;
     memset(&lc, 0, sizeof lc);
     cudaLaunchAttribute attr[1];

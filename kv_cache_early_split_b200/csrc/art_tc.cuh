@@ -20,7 +20,8 @@
 //   warp 1       MMA issuer (one lane) and tensor-memory owner
 //   warp 2       ART controller: per round, reads all CTAs' publications through
 //                distributed shared memory and replays the rule in tile order.
-//   warp 3       idle
+//   warp 3       second ART controller when the replay of a round needs two or more
+//                passes over the heads (each warp takes half of them); idle otherwise
 //   warps 4..11  two epilogue warpgroups (thread = TMEM lane); warpgroup wg takes the
 //                CTA's own blocks wg, wg + 2, ...: scores -> per-tile max / weights ->
 //                P^T in smem; O readback (thread = d row) -> online merge in registers;
@@ -59,6 +60,7 @@ constexpr int STAGE_BYTES = 4 * 16384;
 constexpr uint32_t TMEM_COLS = 128;
 constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_CTL = 2, WARP_EPI0 = 4;
 constexpr int BAR_EPI = 1;  // named barriers BAR_EPI + wg: the 128 threads of epilogue warpgroup wg
+constexpr int BAR_CTL = 3;  // named barrier of the two controller warps
 constexpr int LAG = 2;      // a round is merged LAG rounds after it was published (LAG % NWG == 0)
 constexpr int NSLOT = 2 * NWG + 2 * LAG;
 static_assert(LAG % NWG == 0, "a warpgroup merges its own rounds");
@@ -121,7 +123,8 @@ constexpr uint32_t SMEM_BYTES = Pub<GMAX, PMAX>::SMEM_BYTES;  // the largest ins
 // [NWG][GMAX][D] numerators, then [NWG][GMAX] m, [NWG][GMAX] l, [4] ints
 constexpr uint32_t OFF_RED = 0;
 constexpr uint32_t RED_M = NWG * GMAX * D, RED_L = RED_M + NWG * GMAX, RED_I = RED_L + NWG * GMAX;
-enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, CTL_TREAD, CTL_TMEM };
+enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, CTL_TREAD, CTL_TMEM,
+             CTL_STOPFLAG = 8 };  // [2 rounds][2 controller warps]: all of the warp's heads stopped
 
 __device__ __forceinline__ uint32_t s_col(int b) { return 16u * b; }
 __device__ __forceinline__ uint32_t o_col(int b, int i) { return 32u + 32u * b + 16u * i; }
@@ -180,7 +183,8 @@ __device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parit
 // PC: probe-lane capacity of the rule replay (16 or 32, lanes beyond n_probe are zero).
 // GEN: general addressing (a traversal sequence or a paged cache); without it the kernel carries
 // none of that code (smaller instruction footprint on the contiguous, natural-order path).
-template <int GP, int MODE, int PC, bool GEN>
+// NCW: ART controller warps (2 when a round's replay needs two or more passes over the heads).
+template <int GP, int MODE, int PC, bool GEN, int NCW>
 __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
   using PB = Pub<GP, PC>;
@@ -688,11 +692,13 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         for (int g = 0; g < GP; ++g) pnd[i][g] = ot[i][g];
       ntl_p = ntl;
     }
-  } else if (warp == WARP_CTL) {
-    // ------------------------------------------------------------ ART controller
-    if constexpr (ART) {
-      const int TQ = C * KT;    // tiles per round (power of two <= 32)
-      const int HPP = 32 / TQ;  // heads per pass
+  } else if (warp == WARP_CTL || (NCW == 2 && warp == WARP_CTL + 1)) {
+    // ------------------------------------------------------------ ART controller(s)
+    const int TQ = C * KT;    // tiles per round (power of two <= 32)
+    const int HPP = 32 / TQ;  // heads per pass
+    constexpr int ncw = NCW;  // the host picks 2 when a round needs two or more passes over the heads
+    const int cw = (NCW == 1) ? 0 : warp - WARP_CTL;
+    if (ART && cw < ncw) {
       const int hh = lane / TQ, q = lane % TQ;
       const int c = q / KT, i = q % KT;
       const unsigned segmask = (TQ == 32) ? 0xffffffffu : ((1u << TQ) - 1u);
@@ -700,10 +706,12 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         const int sl = r % NSLOT;
         int okw = 1;
         if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r / NSLOT) & 1, ctl, false, p.ws_status, true);
-        if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if constexpr (NCW == 2) okw = named_barrier_and(BAR_CTL, 64, okw != 0);  // both warps leave together
+        if (!okw) break;
         const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
         const uint32_t slot_base = smem_u32(pub) + sl * PB::SLOT;
-        for (int g0 = 0; g0 < G; g0 += HPP) {
+        for (int g0 = cw * HPP; g0 < G; g0 += ncw * HPP) {
           const int g = g0 + hh;
           const bool active = g < G;
           const int gs = active ? g : 0;
@@ -812,19 +820,43 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           if (active && q == 0) dec[sl * GMAX + g] = stopped_before ? -2 : stop;
           __syncwarp();
         }
-        if (lane == 0) {
-          bool all = true;
-          for (int g = 0; g < G; ++g) all &= (ri[g * RI_SIZE + RI_STOPPED] != 0);
-          __threadfence_block();
-          mbar_arrive(bar(B_DEC + sl));
-          if (all) {
-            ctl[CTL_EXIT_ROUND] = r;
+        if constexpr (NCW == 1) {
+          if (lane == 0) {
+            bool all = true;
+            for (int g = 0; g < G; ++g) all &= (ri[g * RI_SIZE + RI_STOPPED] != 0);
             __threadfence_block();
-            ctl[CTL_EXIT] = 1;
+            mbar_arrive(bar(B_DEC + sl));
+            if (all) {
+              ctl[CTL_EXIT_ROUND] = r;
+              __threadfence_block();
+              ctl[CTL_EXIT] = 1;
+            }
           }
+          __syncwarp();
+          if (ctl[CTL_EXIT]) break;
+        } else {
+          // this warp's heads all stopped?  (flags double-buffered by round: the named barrier
+          // keeps the two warps within one round of each other)
+          if (lane == 0) {
+            bool mine = true;
+            for (int g0 = cw * HPP; g0 < G; g0 += NCW * HPP)
+              for (int g = g0; g < min(G, g0 + HPP); ++g) mine &= (ri[g * RI_SIZE + RI_STOPPED] != 0);
+            ctl[CTL_STOPFLAG + 2 * (r & 1) + cw] = mine ? 1 : 0;
+          }
+          named_barrier(BAR_CTL, 64);  // both warps' decisions and flags are written
+          const bool all = ctl[CTL_STOPFLAG + 2 * (r & 1)] && ctl[CTL_STOPFLAG + 2 * (r & 1) + 1];
+          if (cw == 0 && lane == 0) {
+            __threadfence_block();
+            mbar_arrive(bar(B_DEC + sl));
+            if (all) {
+              ctl[CTL_EXIT_ROUND] = r;
+              __threadfence_block();
+              ctl[CTL_EXIT] = 1;
+            }
+          }
+          __syncwarp();
+          if (all) break;
         }
-        __syncwarp();
-        if (ctl[CTL_EXIT]) break;
       }
     }
   }

@@ -1,0 +1,8 @@
+// Tensor-core decode kernel instantiations for 4 query head(s) per kv head.
+#include "art_tc_pick.cuh"
+
+namespace artk {
+namespace tc {
+TcFn kernel_gp4(int mode, int pc, bool gen, int ncw) { return pick_gp<4>(mode, pc, gen, ncw); }
+}  // namespace tc
+}  // namespace artk
