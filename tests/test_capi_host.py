@@ -138,3 +138,70 @@ def test_kernel_name_query(L):
     assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=96, tile=64), capi.ART_BF16, 0, 1) is None
     assert capi.art_kernel_name(shape(Hq=32, Hkv=2, d=128, tile=64), capi.ART_BF16, 0, 1) is None
     assert capi.art_kernel_name(shape(B=0), capi.ART_BF16, 0, 1) is None
+
+
+def test_status_strings_new_codes(L):
+    assert capi.art_status_string(capi.ART_ERR_ORDER) == "ART_ERR_ORDER"
+    assert capi.art_status_string(capi.ART_ERR_PAGE) == "ART_ERR_PAGE"
+
+
+def test_invalid_arguments_orders(L):
+    s = shape()
+    assert capi.art_tile_order_recency(s, None, A, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_tile_order_recency(shape(B=0), A, A * 2, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_tile_key_summary(s, capi.ART_BF16, None, A, A * 2, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_tile_key_summary(shape(d=96), capi.ART_BF16, A, A * 2, A * 3, None) == capi.ART_ERR_UNSUPPORTED
+    assert capi.art_tile_key_summary(s, 7, A, A * 2, A * 3, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_tile_order_importance(shape(Hq=30), capi.ART_BF16, A, A * 2, A * 3, A * 4,
+                                          None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_tile_order_importance(s, 7, A, A * 2, A * 3, A * 4, None) == capi.ART_ERR_INVALID_ARG
+    big = shape(L_max=1 << 26, tile=16)  # 4M tiles of scores would not fit one block's shared memory
+    assert capi.art_tile_order_importance(big, capi.ART_BF16, A, A * 2, A * 3, A * 4,
+                                          None) == capi.ART_ERR_UNSUPPORTED
+    ok = capi.make_params(1e-3, 1e-4, 1, [0, 8])
+    wsb = capi.art_workspace_bytes(s)
+
+    def ordered(params, order):
+        return capi.art_decode_attn_terminate_ordered(s, capi.ART_BF16, A, A * 2, A * 3, A * 4, params, order,
+                                                      A * 5, A * 6, A * 7, wsb, None)
+
+    assert ordered(None, A * 8) == capi.ART_ERR_INVALID_ARG
+    assert ordered(ok, None) == capi.ART_ERR_INVALID_ARG
+    assert ordered(ok, A * 8 + 2) == capi.ART_ERR_INVALID_ARG  # misaligned sequence array
+
+
+def test_invalid_arguments_paged(L):
+    s = shape(L_max=4096, tile=64)
+    wsb = capi.art_workspace_bytes(s)
+
+    def paged(pages, params=None, order=None):
+        return capi.art_decode_attn_paged(s, capi.ART_BF16, A, A * 2, A * 3, pages, A * 4, params, order, A * 5,
+                                          A * 6, A * 7, wsb, None)
+
+    good = capi.art_paged_kv(128, 200, 32, A * 8)
+    assert paged(None) == capi.ART_ERR_INVALID_ARG
+    assert paged(capi.art_paged_kv(128, 200, 32, None)) == capi.ART_ERR_INVALID_ARG
+    assert paged(capi.art_paged_kv(96, 200, 64, A * 8)) == capi.ART_ERR_UNSUPPORTED  # not a multiple of the tile
+    assert paged(capi.art_paged_kv(128, 200, 16, A * 8)) == capi.ART_ERR_INVALID_ARG  # 16 * 128 < L_max
+    assert paged(capi.art_paged_kv(128, 0, 32, A * 8)) == capi.ART_ERR_INVALID_ARG
+    assert paged(capi.art_paged_kv(128, 1 << 30, 32, A * 8)) == capi.ART_ERR_UNSUPPORTED  # pool index overflow
+    assert paged(good, params=None, order=A * 9) == capi.ART_ERR_INVALID_ARG  # a sequence needs ART
+    assert capi.art_decode_attn_q8_skipv_paged(s, A, A * 2, None, A * 3, A * 4, good, A * 5, 1e-6, None, A * 6,
+                                               A * 7, A * 9, wsb, None) == capi.ART_ERR_INVALID_ARG
+
+
+def test_invalid_arguments_eviction(L):
+    s = shape(L_max=4096)
+    assert capi.art_evict_random_select(s, A, None, 4, 8, 64, A * 2, A * 3, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_evict_random_select(s, A, A * 2, 40, 40, 64, A * 3, A * 4, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_evict_random_select(s, A, A * 2, -1, 8, 64, A * 3, A * 4, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_evict_random_select(s, A, A * 2, 0, 0, 0, A * 3, A * 4, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_evict_compact(s, 7, A, None, A * 2, 64, A * 3, None, None) == capi.ART_ERR_INVALID_ARG
+    assert capi.art_evict_compact(s, capi.ART_KV_Q8, A, None, A * 2, 64, A * 3, None,
+                                  None) == capi.ART_ERR_INVALID_ARG  # q8 needs its scales
+    assert capi.art_evict_compact(s, capi.ART_KV_BF16, A, A * 4, A * 2, 64, A * 3, A * 5,
+                                  None) == capi.ART_ERR_INVALID_ARG  # scales only with q8
+    assert capi.art_evict_compact(s, capi.ART_KV_BF16, A, None, A * 2, 64, A * 3 + 8, None,
+                                  None) == capi.ART_ERR_INVALID_ARG  # misaligned destination
+    assert capi.art_evict_compact(shape(d=4), capi.ART_KV_BF16, A, None, A * 2, 64, A * 3, None,
+                                  None) == capi.ART_ERR_UNSUPPORTED  # 8-byte rows
