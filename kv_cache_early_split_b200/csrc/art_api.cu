@@ -269,14 +269,14 @@ bool make_kv_map(CUtensorMap* m, const void* base, const art_shape* s, unsigned 
 
 using artk::tc::TcFn;
 
-// The tensor-core kernel for G heads per kv head; gen: a traversal sequence or a paged cache;
+// The tensor-core kernel for G heads per kv head; ord: a traversal sequence; paged: a paged cache;
 // ncw: ART controller warps.
-TcFn tc_pick(int mode, int G, int n_probe, bool gen, int ncw) {
+TcFn tc_pick(int mode, int G, int n_probe, bool ord, bool paged, int ncw) {
   const int pc = n_probe <= 16 ? 16 : 32;
-  if (G == 1) return artk::tc::kernel_gp1(mode, pc, gen, ncw);
-  if (G == 2) return artk::tc::kernel_gp2(mode, pc, gen, ncw);
-  if (G <= 4) return artk::tc::kernel_gp4(mode, pc, gen, ncw);
-  return artk::tc::kernel_gp8(mode, pc, gen, ncw);
+  if (G == 1) return artk::tc::kernel_gp1(mode, pc, ord, paged, ncw);
+  if (G == 2) return artk::tc::kernel_gp2(mode, pc, ord, paged, ncw);
+  if (G <= 4) return artk::tc::kernel_gp4(mode, pc, ord, paged, ncw);
+  return artk::tc::kernel_gp8(mode, pc, ord, paged, ncw);
 }
 
 // ART controller warps for cluster size C: two when one round's rule replay needs two or more
@@ -291,7 +291,7 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
                      const int32_t* seq_lens, const art_params* a, const int32_t* order, float* o,
                      int32_t* tiles, void* ws, void* stream, const art_paged_kv* pg) {
   const int G = s->Hq / s->Hkv;
-  const bool gen = order != nullptr || pg != nullptr;
+  const bool ord = order != nullptr, paged = pg != nullptr;
   const int n_probe = a ? a->n_probe : 0;
   artk::tc::TcParams p;
   memset(&p, 0, sizeof p);
@@ -319,7 +319,7 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   p.order = order;
   p.n_max = (s->L_max + s->tile - 1) / s->tile;
   int sms = 0;
-  art_status st = prepare(reinterpret_cast<KernelFn>(tc_pick(mode, G, n_probe, gen, 1)), &sms);
+  art_status st = prepare(reinterpret_cast<KernelFn>(tc_pick(mode, G, n_probe, ord, paged, 1)), &sms);
   if (st != ART_OK) return st;
   // one CTA per SM; cluster size C: power of two, units*C <= SMs, C*tiles_per_block <= 32 (one rule lane
   // per tile of a round), and no more CTAs than 128-position blocks in a split.
@@ -331,7 +331,7 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   while (C < artk::CMAX && 1LL * units * (2 * C) <= sms && 2 * C * kt <= 32 && 2 * C <= max_blocks) C *= 2;
   TcFn fn = nullptr;
   while (true) {  // the largest C whose clusters fit, with the kernel variant for that C
-    fn = tc_pick(mode, G, n_probe, gen, tc_ncw(mode, G, C, kt));
+    fn = tc_pick(mode, G, n_probe, ord, paged, tc_ncw(mode, G, C, kt));
     st = prepare(reinterpret_cast<KernelFn>(fn), &sms);
     if (st != ART_OK) return st;
     if (C == 1) break;

@@ -181,10 +181,10 @@ __device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parit
 
 // GP: query heads per kv head (padded to 1, 2, 4 or 8); MODE: full or ART;
 // PC: probe-lane capacity of the rule replay (16 or 32, lanes beyond n_probe are zero).
-// GEN: general addressing (a traversal sequence or a paged cache); without it the kernel carries
-// none of that code (smaller instruction footprint on the contiguous, natural-order path).
+// ORD / PAGED: a traversal sequence / a paged cache; a kernel without them carries none of that
+// code (the ART epilogue and the producer are sensitive to their instruction footprint).
 // NCW: ART controller warps (2 when a round's replay needs two or more passes over the heads).
-template <int GP, int MODE, int PC, bool GEN, int NCW>
+template <int GP, int MODE, int PC, bool ORD, bool PAGED, int NCW>
 __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
   using PB = Pub<GP, PC>;
@@ -219,8 +219,8 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   const int zc = b * p.Hkv + kvh;
   // Tile at position q of this split's traversal sequence (ART with a sequence; natural order
   // otherwise).  An entry outside the split is replaced by the natural tile (the producer flags it).
-  const int32_t* ord_seq = (GEN && ART && p.order) ? p.order + static_cast<long long>(zc) * p.n_max : nullptr;
-  const int32_t* const btab = GEN ? p.block_table : nullptr;
+  const int32_t* ord_seq = (ORD && ART && p.order) ? p.order + static_cast<long long>(zc) * p.n_max : nullptr;
+  const int32_t* const btab = PAGED ? p.block_table : nullptr;
   auto phys_of = [&](int q) -> int {
     if (!ord_seq) return q;
     const int e = __ldg(ord_seq + q);

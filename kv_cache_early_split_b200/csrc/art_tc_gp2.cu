@@ -3,6 +3,8 @@
 
 namespace artk {
 namespace tc {
-TcFn kernel_gp2(int mode, int pc, bool gen, int ncw) { return pick_gp<2>(mode, pc, gen, ncw); }
+TcFn kernel_gp2(int mode, int pc, bool ord, bool paged, int ncw) {
+  return pick_gp<2>(mode, pc, ord, paged, ncw);
+}
 }  // namespace tc
 }  // namespace artk

@@ -3,6 +3,8 @@
 
 namespace artk {
 namespace tc {
-TcFn kernel_gp8(int mode, int pc, bool gen, int ncw) { return pick_gp<8>(mode, pc, gen, ncw); }
+TcFn kernel_gp8(int mode, int pc, bool ord, bool paged, int ncw) {
+  return pick_gp<8>(mode, pc, ord, paged, ncw);
+}
 }  // namespace tc
 }  // namespace artk
