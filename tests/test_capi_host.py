@@ -205,3 +205,21 @@ def test_invalid_arguments_eviction(L):
                                   None) == capi.ART_ERR_INVALID_ARG  # misaligned destination
     assert capi.art_evict_compact(shape(d=4), capi.ART_KV_BF16, A, None, A * 2, 64, A * 3, None,
                                   None) == capi.ART_ERR_UNSUPPORTED  # 8-byte rows
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback: with the CUDA library absent, the first call raises instead of computing anything."""
+    import subprocess
+    import sys
+
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from kv_cache_early_split_b200 import capi\n"
+        "capi.LIB_PATH = %r\n"
+        "try:\n"
+        "    capi.art_workspace_bytes(capi.art_shape(1, 1, 1, 64, 64, 64, 1))\n"
+        "except OSError as e:\n"
+        "    print('raised', 'no fallback' in str(e))\n"
+    ) % (os.path.dirname(os.path.dirname(os.path.abspath(__file__))), str(tmp_path / "absent.so"))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.stdout.strip() == "raised True", r.stdout + r.stderr
