@@ -185,7 +185,8 @@ bool choose_config(const KernelInfo& ki, const art_shape* s, int sms, int max_ti
   const int target = sms * (per_sm > 2 ? 2 : per_sm);
   int C = 1;
   while (C < artk::CMAX && units * (2 * C) <= target && 2 * C <= max_tiles_per_split) C *= 2;
-  // shrink the cluster until the runtime can co-schedule one of that size
+  // shrink the cluster until every cluster of the grid is resident at once (one wave): a cluster of
+  // C CTAs needs C free SMs in one GPC, so large clusters can leave a tail wave behind
   while (C > 1) {
     cudaLaunchConfig_t lc;
     memset(&lc, 0, sizeof lc);
@@ -200,7 +201,7 @@ bool choose_config(const KernelInfo& ki, const art_shape* s, int sms, int max_ti
     lc.attrs = attr;
     lc.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, ki.fn, &lc) == cudaSuccess && nclusters > 0) break;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, ki.fn, &lc) == cudaSuccess && nclusters >= units) break;
     cudaGetLastError();  // clear a sticky-free query error
     C /= 2;
   }
@@ -330,7 +331,7 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   int C = 1;
   while (C < artk::CMAX && 1LL * units * (2 * C) <= sms && 2 * C * kt <= 32 && 2 * C <= max_blocks) C *= 2;
   TcFn fn = nullptr;
-  while (true) {  // the largest C whose clusters fit, with the kernel variant for that C
+  while (true) {  // the largest C whose clusters are all resident at once, with the kernel variant for that C
     fn = tc_pick(mode, G, n_probe, ord, paged, tc_ncw(mode, G, C, kt));
     st = prepare(reinterpret_cast<KernelFn>(fn), &sms);
     if (st != ART_OK) return st;
@@ -348,7 +349,7 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
     lc.attrs = attr;
     lc.numAttrs = 1;
     int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, fn, &lc) == cudaSuccess && nclusters > 0) break;
+    if (cudaOccupancyMaxActiveClusters(&nclusters, fn, &lc) == cudaSuccess && nclusters >= units) break;
     cudaGetLastError();
     C /= 2;
   }
