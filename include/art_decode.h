@@ -104,7 +104,10 @@ typedef struct {
   int32_t n_probe;
 } art_params;
 
-/* Bytes of workspace a call with this shape needs (0 on an invalid shape). */
+/* Bytes of workspace a call with this shape needs (0 on an invalid shape).  With one split it
+ * includes room for full attention to run as up to 4 internal splits of each sequence (same
+ * result; chosen by the library when that keeps more SMs busy); the caller-visible arrays below
+ * keep the caller's split layout either way. */
 size_t art_workspace_bytes(const art_shape* shape);
 
 /* Byte offset inside ws of the int32 array tiles_read[B, Hkv, num_splits]:

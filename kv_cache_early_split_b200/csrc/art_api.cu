@@ -26,8 +26,12 @@ constexpr int kSmemReservedPerBlock = 1024;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Full attention with one caller split may run as up to this many internal splits (same result:
+// attention does not depend on how the positions are grouped) when that fills more SMs.
+constexpr int kFullSplitsMax = 4;
+
 struct WsLayout {
-  size_t tiles_read, used, partial, total;
+  size_t tiles_read, used, partial, int_tiles_read, int_used, int_partial, total;
 };
 
 bool shape_ok(const art_shape* s) {
@@ -42,7 +46,13 @@ WsLayout ws_layout(const art_shape* s) {
   w.tiles_read = kWsHeader;
   w.used = align256(w.tiles_read + 4 * units);
   w.partial = align256(w.used + 4 * heads);
-  w.total = align256(w.partial + 4 * heads * (size_t(s->d) + 2));
+  // internal splits of full attention (one caller split, up to kFullSplitsMax parts per sequence)
+  const size_t iunits = size_t(s->B) * s->Hkv * kFullSplitsMax, iheads = size_t(s->B) * s->Hq * kFullSplitsMax;
+  w.int_tiles_read = align256(w.partial + 4 * heads * (size_t(s->d) + 2));
+  w.int_used = align256(w.int_tiles_read + 4 * iunits);
+  w.int_partial = align256(w.int_used + 4 * iheads);
+  w.total = (s->num_splits == 1) ? align256(w.int_partial + 4 * iheads * (size_t(s->d) + 2))
+                                 : w.int_tiles_read;
   return w;
 }
 
@@ -323,36 +333,64 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   art_status st = prepare(reinterpret_cast<KernelFn>(tc_pick(mode, G, n_probe, ord, paged, 1)), &sms);
   if (st != ART_OK) return st;
   // one CTA per SM; cluster size C: power of two, units*C <= SMs, C*tiles_per_block <= 32 (one rule lane
-  // per tile of a round), and no more CTAs than 128-position blocks in a split.
-  const int units = s->B * s->Hkv * s->num_splits;
+  // per tile of a round), no more CTAs than 128-position blocks in a split, and every cluster resident
+  // at once (a cluster of C CTAs needs C free SMs of one GPC, so large clusters can leave a tail wave)
   const int kt = 128 / s->tile;
   const long long max_tiles = (s->L_max + s->tile - 1) / s->tile;
-  const long long max_blocks = ((max_tiles + s->num_splits - 1) / s->num_splits * s->tile + 127) / 128;
-  int C = 1;
-  while (C < artk::CMAX && 1LL * units * (2 * C) <= sms && 2 * C * kt <= 32 && 2 * C <= max_blocks) C *= 2;
-  TcFn fn = nullptr;
-  while (true) {  // the largest C whose clusters are all resident at once, with the kernel variant for that C
-    fn = tc_pick(mode, G, n_probe, ord, paged, tc_ncw(mode, G, C, kt));
-    st = prepare(reinterpret_cast<KernelFn>(fn), &sms);
-    if (st != ART_OK) return st;
-    if (C == 1) break;
-    cudaLaunchConfig_t lc;
-    memset(&lc, 0, sizeof lc);
-    cudaLaunchAttribute attr[1];
-    lc.gridDim = dim3(static_cast<unsigned>(units * C), 1, 1);
-    lc.blockDim = dim3(artk::tc::NTHR, 1, 1);
-    lc.dynamicSmemBytes = artk::tc::SMEM_BYTES;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    lc.attrs = attr;
-    lc.numAttrs = 1;
-    int nclusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&nclusters, fn, &lc) == cudaSuccess && nclusters >= units) break;
-    cudaGetLastError();
-    C /= 2;
+  struct Pick {
+    int C, units;
+    TcFn fn;
+  };
+  auto choose = [&](int S_, Pick* out) -> art_status {
+    const int units_ = s->B * s->Hkv * S_;
+    const long long max_blocks = ((max_tiles + S_ - 1) / S_ * s->tile + 127) / 128;
+    int C_ = 1;
+    while (C_ < artk::CMAX && 1LL * units_ * (2 * C_) <= sms && 2 * C_ * kt <= 32 && 2 * C_ <= max_blocks) C_ *= 2;
+    TcFn fn_ = nullptr;
+    while (true) {
+      fn_ = tc_pick(mode, G, n_probe, ord, paged, tc_ncw(mode, G, C_, kt));
+      const art_status st_ = prepare(reinterpret_cast<KernelFn>(fn_), &sms);
+      if (st_ != ART_OK) return st_;
+      if (C_ == 1) break;
+      cudaLaunchConfig_t lc;
+      memset(&lc, 0, sizeof lc);
+      cudaLaunchAttribute attr[1];
+      lc.gridDim = dim3(static_cast<unsigned>(units_ * C_), 1, 1);
+      lc.blockDim = dim3(artk::tc::NTHR, 1, 1);
+      lc.dynamicSmemBytes = artk::tc::SMEM_BYTES;
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = C_;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      lc.attrs = attr;
+      lc.numAttrs = 1;
+      int nclusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&nclusters, fn_, &lc) == cudaSuccess && nclusters >= units_) break;
+      cudaGetLastError();
+      C_ /= 2;
+    }
+    *out = Pick{C_, units_, fn_};
+    return ART_OK;
+  };
+  Pick pk;
+  st = choose(s->num_splits, &pk);
+  if (st != ART_OK) return st;
+  // Full attention with one caller split: split each sequence internally when that puts more CTAs to
+  // work at once (the combine kernel merges the parts and reports the caller's counters).
+  int S_run = s->num_splits;
+  if (mode == artk::MODE_FULL && s->num_splits == 1) {
+    for (int f = 2; f <= kFullSplitsMax && f <= max_tiles; f *= 2) {
+      Pick q2;
+      st = choose(f, &q2);
+      if (st != ART_OK) return st;
+      if (1LL * q2.units * q2.C > 1LL * pk.units * pk.C && 1LL * q2.units * q2.C <= sms) {
+        pk = q2;
+        S_run = f;
+      }
+    }
   }
+  const int C = pk.C, units = pk.units;
+  const TcFn fn = pk.fn;
   const WsLayout w = ws_layout(s);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   p.q = static_cast<const uint16_t*>(q);
@@ -360,15 +398,16 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   p.o = o;
   p.tiles = tiles;
   p.ws_status = reinterpret_cast<int32_t*>(wsb);
-  p.ws_tiles_read = reinterpret_cast<int32_t*>(wsb + w.tiles_read);
-  p.ws_used = reinterpret_cast<int32_t*>(wsb + w.used);
-  p.ws_partial = reinterpret_cast<float*>(wsb + w.partial);
+  const bool internal = S_run != s->num_splits;  // full attention split internally
+  p.ws_tiles_read = reinterpret_cast<int32_t*>(wsb + (internal ? w.int_tiles_read : w.tiles_read));
+  p.ws_used = reinterpret_cast<int32_t*>(wsb + (internal ? w.int_used : w.used));
+  p.ws_partial = reinterpret_cast<float*>(wsb + (internal ? w.int_partial : w.partial));
   p.B = s->B;
   p.Hq = s->Hq;
   p.Hkv = s->Hkv;
   p.L_max = s->L_max;
   p.T = s->tile;
-  p.S = s->num_splits;
+  p.S = S_run;
   p.G = G;
   p.C = C;
   p.qscale = static_cast<float>(1.4426950408889634 / sqrt(128.0));
@@ -387,10 +426,15 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   lc.attrs = attr;
   lc.numAttrs = 1;
   if (cudaLaunchKernelEx(&lc, fn, p) != cudaSuccess) return ART_ERR_CUDA;
-  if (s->num_splits > 1) {
+  if (S_run > 1) {
     const int heads = s->B * s->Hq;
-    artk::art_combine_kernel<128><<<(heads + 7) / 8, 256, 0, lc.stream>>>(p.ws_partial, p.ws_used, o, tiles, heads,
-                                                                           s->num_splits);
+    if (internal)  // also the caller's one-split counters
+      artk::art_combine_kernel<128><<<(heads + 7) / 8, 256, 0, lc.stream>>>(
+          p.ws_partial, p.ws_used, o, tiles, heads, S_run, reinterpret_cast<int32_t*>(wsb + w.used),
+          p.ws_tiles_read, reinterpret_cast<int32_t*>(wsb + w.tiles_read), G);
+    else
+      artk::art_combine_kernel<128><<<(heads + 7) / 8, 256, 0, lc.stream>>>(p.ws_partial, p.ws_used, o, tiles,
+                                                                             heads, S_run);
     if (cudaGetLastError() != cudaSuccess) return ART_ERR_CUDA;
   }
   return ART_OK;

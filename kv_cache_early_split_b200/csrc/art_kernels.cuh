@@ -829,12 +829,17 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
 
 // ------------------------------------------------------------------ split combine
 // One warp per (batch, query head): O = sum_s 2^(m_s-M) acc_s / sum_s 2^(m_s-M) l_s.
+// With internal splits of one caller split (full attention only), also the caller's per-split
+// counters: used_out[hq] = tiles consumed, tread_out[b*Hkv + kvh] = the sum of tread_in over the splits.
 template <int D>
 __global__ void __launch_bounds__(256) art_combine_kernel(const float* __restrict__ part,
                                                           const int32_t* __restrict__ used,
                                                           float* __restrict__ o,
                                                           int32_t* __restrict__ tiles, int n_heads,
-                                                          int S) {
+                                                          int S, int32_t* __restrict__ used_out = nullptr,
+                                                          const int32_t* __restrict__ tread_in = nullptr,
+                                                          int32_t* __restrict__ tread_out = nullptr,
+                                                          int G = 1) {
   const int hq = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (hq >= n_heads) return;
@@ -858,6 +863,13 @@ __global__ void __launch_bounds__(256) art_combine_kernel(const float* __restric
 #pragma unroll
   for (int i = 0; i < D / 32; ++i) o[static_cast<long long>(hq) * D + lane + 32 * i] = num[i] / den;
   if (lane == 0 && tiles) tiles[hq] = tsum;
+  if (lane == 0 && used_out) used_out[hq] = tsum;
+  if (lane == 0 && tread_out && hq % G == 0) {
+    const int bk = hq / G;  // batch * Hkv + kv head
+    int t = 0;
+    for (int s2 = 0; s2 < S; ++s2) t += tread_in[static_cast<long long>(bk) * S + s2];
+    tread_out[bk] = t;
+  }
 }
 
 }  // namespace artk
