@@ -110,6 +110,12 @@ typedef struct {
  * keep the caller's split layout either way. */
 size_t art_workspace_bytes(const art_shape* shape);
 
+/* Bytes of workspace art_decode_attn_q8_skipv needs to run full attention (params == NULL) as
+ * two streaming passes: art_workspace_bytes(shape) plus scores [B, Hkv, L_max, Hq/Hkv] fp32,
+ * tile and chunk maxima and per-chunk partial states (0 on an invalid shape).  The offsets below
+ * hold for this larger workspace too. */
+size_t art_q8_workspace_bytes(const art_shape* shape);
+
 /* Byte offset inside ws of the int32 array tiles_read[B, Hkv, num_splits]:
  * KV tiles actually fetched from HBM for each (batch, kv head, split) by the
  * last call, speculative prefetch included.  Written by every call. */
@@ -165,7 +171,13 @@ art_status art_decode_attn_terminate_noalloc(const art_shape* shape, art_dtype d
  * scale each (q8_0 style; value = code * scale), bf16 query.  V rows whose
  * weight exp(s_j - m') is below tau are neither dequantised nor accumulated
  * (puntofijo.es, "La Elegancia de la Omision").  params == NULL runs without
- * ART; otherwise ART as in art_decode_attn_terminate. */
+ * ART; otherwise ART as in art_decode_attn_terminate.
+ * Without ART and with ws_bytes >= art_q8_workspace_bytes(shape) (and B*Hkv*num_splits
+ * <= 65535) the call runs as two streaming passes over the whole GPU: scores and tile maxima
+ * from K, then the running maxima m', the skip test and the V products (a tile whose rows all
+ * fail the test for every head is not read), then a combine.  Same rule, same outputs and
+ * counters; a tile counts as read either way.  With a smaller workspace one pass deals the
+ * tiles of a split over a thread-block cluster and exchanges tile maxima every round. */
 art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
                                     const uint16_t* k_scale_f16, const int8_t* v_q,
                                     const uint16_t* v_scale_f16, const int32_t* seq_lens,
@@ -297,7 +309,8 @@ art_status art_read_device_status(void* ws, void* stream);
  * tile 64 or 128, Hq/Hkv <= 8, full or ART) or "art_decode_kernel" (CUDA-core
  * path, everything else); NULL for an invalid or unsupported shape.  kv_q8 != 0
  * asks about art_decode_attn_q8_skipv (dtype is then ignored); with_art != 0
- * about the ART variant.  A query only: no CUDA call, nothing enqueued.  The
+ * about the ART variant.  q8 without ART names "q8_pv_kernel", the second of
+ * the two passes that run when the workspace holds art_q8_workspace_bytes.  A query only: no CUDA call, nothing enqueued.  The
  * pages have no counterpart; it names the kernel for profiling and reports.
  * With num_splits > 1 a second, small kernel (art_combine_kernel) follows. */
 const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_q8, int32_t with_art);

@@ -75,16 +75,24 @@ def _t(torch, arr, device, dtype=None):
     return t.to(device)
 
 
-def upload(w, device="cuda", num_splits=None, tile=None, paged=None):
+def _ws_bytes(kind: str, shape, paged: bool, q8_two_pass: bool) -> int:
+    """Workspace for a problem: the q8 two-pass arrays too for a contiguous q8 cache."""
+    if kind == "q8" and not paged and q8_two_pass:
+        return capi.art_q8_workspace_bytes(shape)
+    return capi.art_workspace_bytes(shape)
+
+
+def upload(w, device="cuda", num_splits=None, tile=None, paged=None, q8_two_pass=True):
     """Copy a kv_cache_early_split_b200.inputs.Workload to the GPU and allocate o / tiles / workspace.
     paged: None, or an inputs.PagedKV of the same workload: its page pools and block table are
-    uploaded instead of the contiguous K/V."""
+    uploaded instead of the contiguous K/V.  q8_two_pass: for a contiguous q8 cache, size the
+    workspace for the two-pass full-attention path (False: the one-pass cluster kernel)."""
     import torch
 
     S = w.num_splits if num_splits is None else int(num_splits)
     T = w.tile if tile is None else int(tile)
     shape = capi.art_shape(w.B, w.Hq, w.Hkv, w.d, w.L_max, T, S)
-    wsb = capi.art_workspace_bytes(shape)
+    wsb = _ws_bytes(w.kind, shape, paged is not None, q8_two_pass)
     if wsb == 0:
         raise ArtError(capi.ART_ERR_INVALID_ARG, "art_workspace_bytes")
     src = w if paged is None else paged
@@ -229,8 +237,9 @@ def evict_random(dp: DeviceProblem, rand_keys, n_sink: int, n_recent: int, budge
         kind=dp.kind, shape=shape2, q=dp.q, k=like(dp.k, s.d), v=like(dp.v, s.d),
         k_scale=like(dp.k_scale, s.d // 32), v_scale=like(dp.v_scale, s.d // 32),
         seq_lens=torch.empty((s.B,), dtype=torch.int32, device=dev), o=torch.empty_like(dp.o),
-        tiles=torch.empty_like(dp.tiles), ws=torch.zeros(capi.art_workspace_bytes(shape2), dtype=torch.uint8,
-                                                         device=dev),
+        tiles=torch.empty_like(dp.tiles),
+        ws=torch.zeros(_ws_bytes(dp.kind, shape2, False, dp.ws_bytes > capi.art_workspace_bytes(s)),
+                       dtype=torch.uint8, device=dev),
         art=dict(dp.art), tau=dp.tau)
     kept = torch.empty((s.B, s.Hkv, budget), dtype=torch.int32, device=dev)
     evict_random_into(dp, dp2, kept, rand_keys, n_sink, n_recent, stream=stream)

@@ -29,6 +29,7 @@ ART_KV_F32, ART_KV_BF16, ART_KV_Q8 = 0, 1, 2
 # every symbol the header declares
 EXPORTS = (
     "art_workspace_bytes",
+    "art_q8_workspace_bytes",
     "art_workspace_tiles_read_offset",
     "art_workspace_split_tiles_offset",
     "art_decode_attn_full",
@@ -100,6 +101,8 @@ def lib() -> ctypes.CDLL:
             L = ctypes.CDLL(LIB_PATH)
             L.art_workspace_bytes.restype = ctypes.c_size_t
             L.art_workspace_bytes.argtypes = [_SH]
+            L.art_q8_workspace_bytes.restype = ctypes.c_size_t
+            L.art_q8_workspace_bytes.argtypes = [_SH]
             L.art_workspace_tiles_read_offset.restype = ctypes.c_size_t
             L.art_workspace_tiles_read_offset.argtypes = [_SH]
             L.art_workspace_split_tiles_offset.restype = ctypes.c_size_t
@@ -151,6 +154,10 @@ def _ref(x):
 
 def art_workspace_bytes(shape: art_shape) -> int:
     return int(lib().art_workspace_bytes(ctypes.byref(shape)))
+
+
+def art_q8_workspace_bytes(shape: art_shape) -> int:
+    return int(lib().art_q8_workspace_bytes(ctypes.byref(shape)))
 
 
 def art_workspace_tiles_read_offset(shape: art_shape) -> int:

@@ -12,6 +12,7 @@
 #include "art_evict.cuh"
 #include "art_kernels.cuh"
 #include "art_order.cuh"
+#include "art_q8_two.cuh"
 #include "art_tc_pick.cuh"
 
 namespace {
@@ -573,6 +574,28 @@ art_status launch(int kind, int mode, const art_shape* s, const void* q, const v
   return ART_OK;
 }
 
+// Two-pass q8 decode (full attention with the V skip): the kernels, their workspace arrays (after
+// the common ones) and their launch shape live in art_q8_two.cuh.
+artk::q8two::Dims q8_dims(const art_shape* s) {
+  return artk::q8two::Dims{s->B, s->Hq, s->Hkv, s->d, s->L_max, s->tile, s->num_splits};
+}
+
+size_t q8_ws_total(const art_shape* s) { return artk::q8two::workspace_end(q8_dims(s), ws_layout(s).total); }
+
+bool q8two_eligible(const art_shape* s, const art_params* params, size_t ws_bytes) {
+  return !params && ws_bytes >= q8_ws_total(s) && artk::q8two::grid_ok(q8_dims(s));
+}
+
+art_status launch_q8two(const art_shape* s, const void* q, const int8_t* k, const uint16_t* ks, const int8_t* v,
+                        const uint16_t* vs, const int32_t* seq_lens, float tau, float* o, int32_t* tiles, void* ws,
+                        void* stream) {
+  const WsLayout w = ws_layout(s);
+  const cudaError_t e = artk::q8two::launch(q8_dims(s), static_cast<const uint16_t*>(q), k, ks, v, vs, seq_lens,
+                                            tau, o, tiles, static_cast<uint8_t*>(ws), w.tiles_read, w.used, w.total,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? ART_OK : ART_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Scratch memory for art_decode_attn_terminate_noalloc.  The array is a
 // file-scope device variable: every GPU that loads this library holds it until
@@ -606,6 +629,11 @@ extern "C" {
 size_t art_workspace_bytes(const art_shape* shape) {
   if (!shape_ok(shape)) return 0;
   return ws_layout(shape).total;
+}
+
+size_t art_q8_workspace_bytes(const art_shape* shape) {
+  if (!shape_ok(shape)) return 0;
+  return q8_ws_total(shape);
 }
 
 size_t art_workspace_tiles_read_offset(const art_shape* shape) {
@@ -671,6 +699,8 @@ art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, 
   if (isnan(tau)) return ART_ERR_INVALID_ARG;
   const long long scale_row_bytes = (shape->d / 32) * 2;
   if ((1LL * shape->L_max * scale_row_bytes) % 16 != 0) return ART_ERR_UNSUPPORTED;
+  if (q8two_eligible(shape, params, ws_bytes))
+    return launch_q8two(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, o, tiles, ws, stream);
   const int mode = params ? artk::MODE_SKIP_ART : artk::MODE_SKIP;
   return launch(artk::KV_Q8, mode, shape, q_bf16, k_q, v_q, k_scale_f16, v_scale_f16, seq_lens, params, tau, o,
                 tiles, ws, stream);
@@ -848,6 +878,9 @@ const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_
     mode = with_art ? artk::MODE_ART : artk::MODE_FULL;
   }
   if (tc_eligible(kind, mode, shape)) return "art_decode_tc_kernel";
+  if (mode == artk::MODE_SKIP && (shape->d == 64 || shape->d == 128) && shape->Hq % shape->Hkv == 0 &&
+      shape->Hq / shape->Hkv <= artk::GMAX)
+    return "q8_pv_kernel";
   KernelInfo ki;
   if (!pick_kernel(kind, mode, shape->d, shape->Hq / shape->Hkv, &ki)) return nullptr;
   return "art_decode_kernel";

@@ -1,0 +1,688 @@
+// Two-pass decode attention over a q8 cache with the exact V skip (full attention, no ART).
+//
+// The skip rule (puntofijo.es, "La Elegancia de la Omision") leaves row j of tile t out of the
+// numerator when exp(s_j - m'_t) < tau, m'_t the running maximum of the split's scores after tile
+// t.  In one pass, m'_t needs the maxima of every earlier tile of the split, which a CTA that
+// deals tiles with its neighbours only learns by waiting on them.  Split into passes instead:
+//
+//   pass 1 (q8_scores_kernel): s_j = q.k_j / sqrt(d) (log2 domain) for every row, the maximum of
+//          every tile and of every chunk of CT tiles.  Reads K once, writes the scores.
+//   pass 2 (q8_pv_kernel): m'_t = max(chunk maxima before the chunk, tile maxima of the chunk up
+//          to t); weights p_j = 2^(s_j - m'_t) for the skip test, numerator and denominator taken
+//          relative to the chunk's own reference max; V rows with every head below tau are not
+//          dequantised, tiles with every row of every head below tau are not even read.
+//   combine (q8_combine_kernel): the chunk states of every split merged per query head.
+//
+// Every step is a plain streaming kernel over the whole grid: no cluster barriers, no waits on
+// other CTAs.  Each warp walks its rows in groups of RPI (one row per TPR lanes) and stages them
+// through a ring of P groups in shared memory with cp.async, so that P groups per warp are in
+// flight without holding registers.  Bytes: K and V (+ scales) once, plus 2 x 4 x GP bytes of
+// scores per row.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "art_kernels.cuh"
+
+namespace artk {
+namespace q8two {
+
+constexpr int NT = 256;  // threads per CTA
+constexpr int NW = NT / 32;
+constexpr int P = 8;       // ring slots per warp (row groups in flight)
+constexpr int CTMAX = 32;  // tiles per chunk at most (one lane per tile in the in-chunk prefix)
+
+struct Params {
+  const uint16_t* q;   // [B, Hq, D] bf16 bits
+  const int8_t* k;     // [B, Hkv, L_max, D] codes
+  const uint16_t* ks;  // [B, Hkv, L_max, D/32] fp16 bits
+  const int8_t* v;
+  const uint16_t* vs;
+  const int32_t* seq_lens;  // [B]
+  float* o;                 // [B, Hq, D]
+  int32_t* tiles;           // [B, Hq] or NULL
+  int32_t* ws_status;
+  int32_t* ws_tiles_read;  // [B*Hkv*S]
+  int32_t* ws_used;        // [B*Hq*S]
+  float* scores;           // [B*Hkv][L_max][GP]  log2-domain scores (heads padded to GP)
+  float* tmax;             // [B*Hkv][n_max][G]  tile maxima
+  float* cmax;             // [B*Hkv*S][CPS][G]  chunk maxima
+  float* part;             // [B*Hq*S][CPS][2 + D]  chunk states (m, l, acc)
+  int B, Hq, Hkv, L_max, T, S, G, GP, CT, CPS, n_max;
+  float qscale, tau;
+};
+
+// Smallest chunk: at least 128 rows per warp where that stays within CTMAX tiles.
+__host__ __device__ inline int chunk_tiles_min(int T) {
+  int ct = NW * (T >= 128 ? 1 : 128 / T);
+  return ct > CTMAX ? CTMAX : ct;
+}
+
+__host__ __device__ constexpr int gp_of(int G) { return G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8)); }
+
+template <int D, int GP>
+struct Geom {
+  static constexpr int EPT = GP <= 4 ? 16 : 8;  // codes per thread of a row
+  static constexpr int TPR = D / EPT;           // threads per row
+  static constexpr int RPI = 32 / TPR;          // rows per group (one warp iteration)
+  static constexpr int NB = D / 32;             // scale blocks per row
+  static constexpr int HMASK = (TPR - 1) & ~(TPR / GP - 1);  // lane bits that name the head
+  // one ring slot: codes [RPI][D] bytes, scales [RPI][NB] fp16, scores [RPI][GP] fp32 (pass 2)
+  static constexpr int SLOT_CODES = RPI * D;
+  static constexpr int SLOT_SCALES = RPI * NB * 2;
+  static constexpr int SLOT_SCORES = RPI * GP * 4;
+  static constexpr int SLOT = SLOT_CODES + SLOT_SCALES + SLOT_SCORES;
+  static_assert(TPR >= GP && TPR <= 32 && 32 % TPR == 0, "a row must split evenly over a warp");
+  static_assert(SLOT_CODES % 16 == 0 && SLOT_SCALES % 16 == 0 && SLOT_SCORES % 16 == 0, "16-byte slots");
+};
+
+// Head whose total transpose_reduce<GP, RL> leaves in this lane.
+template <int GP, int RL>
+__device__ __forceinline__ int head_of_lane(int lane) {
+  int head = 0;
+#pragma unroll
+  for (int h = GP / 2, off = RL / 2; h >= 1; h >>= 1, off >>= 1)
+    if (lane & off) head += h;
+  return head;
+}
+
+// ---- cp.async (global -> shared, completion tracked per thread in commit groups)
+template <int BYTES>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void* src) {
+  if constexpr (BYTES == 16)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+  else
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(BYTES) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Codes as float pairs (exponent-field insertion as in s8x8_to_f32; the subtraction is exact).
+template <int EPT>
+__device__ __forceinline__ void codes_to_f2(const uint32_t (&w)[EPT / 4], float2 (&f)[EPT / 2]) {
+  const float2 bias = make_float2(-8388736.0f, -8388736.0f);
+#pragma unroll
+  for (int i = 0; i < EPT / 4; ++i) {
+    const uint32_t u = w[i] ^ 0x80808080u;
+    const float2 lo = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u)),
+                                  __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541u)));
+    const float2 hi = make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542u)),
+                                  __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543u)));
+    f[2 * i] = __fadd2_rn(lo, bias);
+    f[2 * i + 1] = __fadd2_rn(hi, bias);
+  }
+}
+
+// EPT codes of this lane from a ring slot
+template <int EPT>
+__device__ __forceinline__ void lds_codes(const uint8_t* p, uint32_t (&w)[EPT / 4]) {
+  if constexpr (EPT == 16) {
+    const uint4 x = *reinterpret_cast<const uint4*>(p);
+    w[0] = x.x;
+    w[1] = x.y;
+    w[2] = x.z;
+    w[3] = x.w;
+  } else {
+    const uint2 x = *reinterpret_cast<const uint2*>(p);
+    w[0] = x.x;
+    w[1] = x.y;
+  }
+}
+
+struct Range {
+  int L, t0, t1, c0, c1;
+};
+
+// Sequence, split and chunk of this CTA (blockIdx.x = chunk, blockIdx.y = (batch, kv head, split)).
+// An invalid length reads as an empty sequence (the combine kernel reports it).
+__device__ __forceinline__ Range cta_range(const Params& p) {
+  Range r;
+  const int unit = blockIdx.y;
+  const int b = unit / p.S / p.Hkv;
+  const int split = unit % p.S;
+  r.L = p.seq_lens[b];
+  if (r.L < 1 || r.L > p.L_max) r.L = 0;
+  const int n_tiles = (r.L + p.T - 1) / p.T;
+  r.t0 = static_cast<int>((static_cast<long long>(split) * n_tiles) / p.S);
+  r.t1 = static_cast<int>((static_cast<long long>(split + 1) * n_tiles) / p.S);
+  r.c0 = r.t0 + static_cast<int>(blockIdx.x) * p.CT;
+  r.c1 = min(r.c0 + p.CT, r.t1);
+  return r;
+}
+
+// The row groups of one warp, in order: tiles c0 + warp, c0 + warp + NW, ... of the chunk, ipt =
+// T / RPI groups per tile.  The current group starts at row `row0` of tile `t` (group `ik` of the
+// tile), whose rows end at `rend`.  Advanced incrementally: no divisions per group.
+struct Walk {
+  int t, row0, rend, ik;
+  __device__ __forceinline__ void start(const Range& r, int warp, int T) {
+    t = r.c0 + warp;
+    row0 = t * T;
+    rend = min(row0 + T, r.L);
+    ik = 0;
+  }
+  __device__ __forceinline__ void next(const Range& r, int T, int ipt, int rpi) {
+    row0 += rpi;
+    if (++ik == ipt) {
+      ik = 0;
+      t += NW;
+      row0 = t * T;
+      rend = min(row0 + T, r.L);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ pass 1: scores and maxima
+template <int D, int GP>
+__global__ void __launch_bounds__(NT, 2) q8_scores_kernel(const __grid_constant__ Params p) {
+  using Gm = Geom<D, GP>;
+  constexpr int EPT = Gm::EPT, TPR = Gm::TPR, RPI = Gm::RPI, NB = Gm::NB;
+  constexpr int SLOT = Gm::SLOT_CODES + Gm::SLOT_SCALES;  // no scores in this pass's ring
+  __shared__ __align__(16) uint8_t s_ring[NW][P][SLOT];
+  __shared__ float s_cm[NW][GP];
+  const Range r = cta_range(p);
+  if (r.c0 >= r.t1) return;  // empty chunk
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % TPR, rsub = lane / TPR;
+  const int unit = blockIdx.y;
+  const int bk = unit / p.S;
+  const int b = bk / p.Hkv, kvh = bk % p.Hkv;
+  const int T = p.T, G = p.G;
+  const int head = head_of_lane<GP, TPR>(lane);
+  const bool writer = (sub % (TPR / GP)) == 0 && head < G;
+
+  // query elements [sub*EPT, sub*EPT + EPT) of every head, scaled into the log2 domain
+  float2 q2[GP][EPT / 2];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+#pragma unroll
+    for (int h = 0; h < EPT / 8; ++h) {
+      float f[8];
+      if (g < G) {
+        const long long qrow = static_cast<long long>(b) * p.Hq + kvh * G + g;
+        bf16x8_to_f32(*reinterpret_cast<const uint4*>(p.q + qrow * D + sub * EPT + 8 * h), f);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) q2[g][4 * h + e] = make_float2(f[2 * e] * p.qscale, f[2 * e + 1] * p.qscale);
+    }
+  }
+
+  const int8_t* kb = p.k + static_cast<long long>(bk) * p.L_max * D;
+  const uint16_t* ksb = p.ks + static_cast<long long>(bk) * p.L_max * NB;
+  float* scb = p.scores + static_cast<long long>(bk) * p.L_max * GP;
+  const int ipt = T / RPI;
+  const int nct = r.c1 - r.c0;
+  const int niter = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ipt;
+  const uint32_t ring = smem_u32(&s_ring[warp][0][0]);
+  // rows past the end are not copied; their slot bytes are stale and their results unused
+  Walk wi, wc;
+  wi.start(r, warp, T);
+  wc = wi;
+  int ki = 0;
+  auto issue = [&]() {
+    if (ki < niter) {
+      const int row = wi.row0 + rsub;
+      if (row < wi.rend) {
+        const uint32_t slot = ring + (ki & (P - 1)) * SLOT;
+        cp_async<EPT>(slot + rsub * D + sub * EPT, kb + static_cast<long long>(row) * D + sub * EPT);
+        if (sub == 0) cp_async<NB * 2>(slot + Gm::SLOT_CODES + rsub * NB * 2, ksb + static_cast<long long>(row) * NB);
+      }
+      wi.next(r, T, ipt, RPI);
+    }
+    ++ki;
+    cp_async_commit();
+  };
+
+  float cm = -INFINITY, tm = -INFINITY;
+  auto body = [&](int k) {
+    const int row = wc.row0 + rsub;
+    const uint8_t* slot = &s_ring[warp][k & (P - 1)][0];
+    uint32_t cw[EPT / 4];
+    lds_codes<EPT>(slot + rsub * D + sub * EPT, cw);
+    const float sc = __half2float(
+        __ushort_as_half(reinterpret_cast<const uint16_t*>(slot + Gm::SLOT_CODES)[rsub * NB + (sub * EPT) / 32]));
+    float2 kf[EPT / 2];
+    codes_to_f2<EPT>(cw, kf);
+    float part[GP];
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+      float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < EPT / 2; ++i) a = __ffma2_rn(q2[h][i], kf[i], a);
+      part[h] = (a.x + a.y) * sc;
+    }
+    int hd;
+    const float tot = transpose_reduce<GP, TPR>(part, lane, hd);
+    if (row < wc.rend) {
+      tm = fmaxf(tm, tot);
+      if (writer) scb[static_cast<long long>(row) * GP + head] = tot;
+    }
+    if (wc.ik == ipt - 1) {
+      // last group of tile wc.t: its maximum per head over the lanes that hold that head
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1)
+        if (!(off & Gm::HMASK)) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, off));
+      if (lane < TPR && writer) p.tmax[(static_cast<long long>(bk) * p.n_max + wc.t) * G + head] = tm;
+      cm = fmaxf(cm, tm);
+      tm = -INFINITY;
+    }
+    wc.next(r, T, ipt, RPI);
+  };
+
+  // two groups per step (niter is a multiple of ipt, which is even): their chains interleave
+#pragma unroll 1
+  for (int k = 0; k < P - 2; ++k) issue();
+#pragma unroll 1
+  for (int k = 0; k < niter; k += 2) {
+    issue();
+    issue();
+    cp_async_wait<P - 2>();  // groups k, k + 1 have landed (this lane's copies) ...
+    __syncwarp();            // ... and every lane's
+    body(k);
+    body(k + 1);
+    __syncwarp();  // every lane is done with these slots before they are refilled
+  }
+  cp_async_wait<0>();
+  if (lane < TPR && (sub % (TPR / GP)) == 0) s_cm[warp][head] = cm;
+  __syncthreads();
+  if (static_cast<int>(threadIdx.x) < G) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) m = fmaxf(m, s_cm[w][threadIdx.x]);
+    p.cmax[(static_cast<long long>(unit) * p.CPS + blockIdx.x) * G + threadIdx.x] = m;
+  }
+}
+
+// ------------------------------------------------------------------ pass 2: weights, skip, PV
+template <int D, int GP>
+__global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Params p) {
+  using Gm = Geom<D, GP>;
+  constexpr int EPT = Gm::EPT, TPR = Gm::TPR, RPI = Gm::RPI, NB = Gm::NB, SLOT = Gm::SLOT;
+  constexpr int RING = NW * P * SLOT, ACC = NW * GP * D * 4;
+  // the ring while the rows stream, then the warps' accumulators
+  __shared__ __align__(16) uint8_t s_buf[RING > ACC ? RING : ACC];
+  __shared__ float s_mp[CTMAX][GP], s_ref[GP];
+  __shared__ int s_live[CTMAX];
+  __shared__ float s_l[NW][GP];
+  const Range r = cta_range(p);
+  if (r.c0 >= r.t1) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane % TPR, rsub = lane / TPR;
+  const int unit = blockIdx.y;
+  const int bk = unit / p.S, split = unit % p.S;
+  const int b = bk / p.Hkv, kvh = bk % p.Hkv;
+  const int T = p.T, G = p.G;
+  const float tau = p.tau;
+  const int nct = r.c1 - r.c0;  // <= CTMAX
+
+  // Running maxima m'_t of the chunk's tiles (lane j: tile c0 + j): the maximum of the split's
+  // chunks before this one, then the inclusive prefix maximum of the chunk's tile maxima.  ref
+  // (m' at the chunk's last tile) is the reference of the chunk's weights.  A tile whose own
+  // maximum already fails the skip test for every head has every row skipped: its V rows are not
+  // read at all (the scores still feed the denominator).
+  if (warp == 0) {
+    const float* cm = p.cmax + static_cast<long long>(unit) * p.CPS * G;
+    bool live = false;
+    for (int g = 0; g < G; ++g) {
+      float m = -INFINITY;
+      for (int c = lane; c < static_cast<int>(blockIdx.x); c += 32) m = fmaxf(m, cm[c * G + g]);
+      m = warp_max(m);
+      const float own = lane < nct ? p.tmax[(static_cast<long long>(bk) * p.n_max + r.c0 + lane) * G + g]
+                                   : -INFINITY;
+      float x = own;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x = fmaxf(x, y);
+      }
+      const float mpj = fmaxf(m, x);
+      if (lane < nct) {
+        s_mp[lane][g] = mpj;
+        if (!(exp2f(own - mpj) < tau)) live = true;
+      }
+      if (lane == 31) s_ref[g] = mpj;
+    }
+    if (lane < nct) s_live[lane] = live ? 1 : 0;
+  }
+  __syncthreads();
+
+  const int8_t* vb = p.v + static_cast<long long>(bk) * p.L_max * D;
+  const uint16_t* vsb = p.vs + static_cast<long long>(bk) * p.L_max * NB;
+  const float* scb = p.scores + static_cast<long long>(bk) * p.L_max * GP;
+  const int ipt = T / RPI;
+  const int niter = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ipt;
+  uint8_t* ring = s_buf + warp * P * SLOT;
+  const uint32_t ring_a = smem_u32(ring);
+  // rows past the end are not copied (stale slot bytes, zero weight); dead tiles copy scores only
+  Walk wi, wc;
+  wi.start(r, warp, T);
+  wc = wi;
+  int ki = 0;
+  auto issue = [&]() {
+    if (ki < niter) {
+      const int row = wi.row0 + rsub;
+      if (row < wi.rend) {
+        const uint32_t slot = ring_a + (ki & (P - 1)) * SLOT;
+        if (sub == 0) {
+          const float* src = scb + static_cast<long long>(row) * GP;
+          const uint32_t dst = slot + Gm::SLOT_CODES + Gm::SLOT_SCALES + rsub * GP * 4;
+          if constexpr (GP == 8) {
+            cp_async<16>(dst, src);
+            cp_async<16>(dst + 16, src + 4);
+          } else {
+            cp_async<GP * 4>(dst, src);
+          }
+        }
+        if (s_live[wi.t - r.c0]) {
+          cp_async<EPT>(slot + rsub * D + sub * EPT, vb + static_cast<long long>(row) * D + sub * EPT);
+          if (sub == 0) cp_async<NB * 2>(slot + Gm::SLOT_CODES + rsub * NB * 2, vsb + static_cast<long long>(row) * NB);
+        }
+      }
+      wi.next(r, T, ipt, RPI);
+    }
+    ++ki;
+    cp_async_commit();
+  };
+
+  // Weights: lane (pr, ph) = (lane / GP, lane % GP) forms the weight of head ph of row pr of each
+  // group (RPI * GP <= 32 pairs) and accumulates that head's denominator; the lanes of a row then
+  // fetch the row's weights by shuffle.
+  constexpr int NPAIR = RPI * GP;
+  static_assert(NPAIR <= 32, "one lane per (row, head) of a group");
+  const int pr = lane / GP, ph = lane % GP;
+  const bool pair = lane < NPAIR && ph < G;
+  float2 acc[GP][EPT / 2];
+#pragma unroll
+  for (int h = 0; h < GP; ++h)
+#pragma unroll
+    for (int i = 0; i < EPT / 2; ++i) acc[h][i] = make_float2(0.f, 0.f);
+  float l = 0.f, mp = 0.f, fac = 0.f;
+  bool live = false;
+  auto body = [&](int k) {
+    if (wc.ik == 0) {
+      // a new tile: m'_t of this lane's head; fac = 2^(m'_t - ref) turns a skip-test weight into
+      // a numerator weight
+      const int j = wc.t - r.c0;
+      mp = pair ? s_mp[j][ph] : 0.f;
+      fac = pair ? exp2f(mp - s_ref[ph]) : 0.f;
+      live = s_live[j] != 0;
+    }
+    const uint8_t* slot = ring + (k & (P - 1)) * SLOT;
+    float wk = 0.f;
+    {
+      const bool ok = pair && wc.row0 + pr < wc.rend;
+      const float sj = ok ? reinterpret_cast<const float*>(slot + Gm::SLOT_CODES + Gm::SLOT_SCALES)[lane] : -INFINITY;
+      const float pj = exp2f(sj - mp);  // 0 for rows past the end and padded heads
+      const float wj = pj * fac;
+      l += wj;  // skipped rows stay in the denominator
+      wk = (live && !(pj < tau) && pj > 0.f) ? wj : 0.f;
+    }
+    float w[GP];
+    bool any = false;
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+      w[h] = __shfl_sync(0xffffffffu, wk, rsub * GP + h);
+      any |= w[h] > 0.f;
+    }
+    if (any) {  // otherwise the row is not dequantised
+      uint32_t cw[EPT / 4];
+      lds_codes<EPT>(slot + rsub * D + sub * EPT, cw);
+      const float vsc = __half2float(
+          __ushort_as_half(reinterpret_cast<const uint16_t*>(slot + Gm::SLOT_CODES)[rsub * NB + (sub * EPT) / 32]));
+      float2 vf[EPT / 2];
+      codes_to_f2<EPT>(cw, vf);
+#pragma unroll
+      for (int h = 0; h < GP; ++h) {
+        const float wv = w[h] * vsc;
+        const float2 w2 = make_float2(wv, wv);
+#pragma unroll
+        for (int i = 0; i < EPT / 2; ++i) acc[h][i] = __ffma2_rn(w2, vf[i], acc[h][i]);
+      }
+    }
+    wc.next(r, T, ipt, RPI);
+  };
+
+  // two groups per step (niter is a multiple of ipt, which is even): their chains interleave
+#pragma unroll 1
+  for (int k = 0; k < P - 2; ++k) issue();
+#pragma unroll 1
+  for (int k = 0; k < niter; k += 2) {
+    issue();
+    issue();
+    cp_async_wait<P - 2>();
+    __syncwarp();
+    body(k);
+    body(k + 1);
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+
+  // sum over the row groups of the warp, then over the warps
+#pragma unroll
+  for (int off = GP; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);  // lane h < GP: head h
+#pragma unroll
+  for (int off = TPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+#pragma unroll
+      for (int i = 0; i < EPT / 2; ++i) {
+        acc[h][i].x += __shfl_xor_sync(0xffffffffu, acc[h][i].x, off);
+        acc[h][i].y += __shfl_xor_sync(0xffffffffu, acc[h][i].y, off);
+      }
+    }
+  }
+  __syncthreads();  // every warp is done with its ring before the accumulators overwrite it
+  float* s_acc = reinterpret_cast<float*>(s_buf);  // [NW][GP][D]
+  if (lane < TPR) {
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+#pragma unroll
+      for (int i = 0; i < EPT / 2; ++i)
+        *reinterpret_cast<float2*>(&s_acc[(warp * GP + h) * D + sub * EPT + 2 * i]) = acc[h][i];
+    }
+  }
+  if (lane < GP) s_l[warp][lane] = l;
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * D; idx += NT) {
+    const int h = idx / D, dd = idx % D;
+    float a = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < NW; ++w2) a += s_acc[(w2 * GP + h) * D + dd];
+    const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + h;
+    float* dst = p.part + ((hq * p.S + split) * p.CPS + blockIdx.x) * (2 + D);
+    dst[2 + dd] = a;
+    if (dd == 0) {
+      float lsum = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < NW; ++w2) lsum += s_l[w2][h];
+      dst[0] = s_ref[h];
+      dst[1] = lsum;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ combine
+// One CTA of D threads per (batch, query head), thread = output element: the chunk states of every
+// split merged online (running maximum, rescaled sums), loads of 8 chunks in flight at a time;
+// then the per-split counters of the caller's split layout.
+template <int D>
+__global__ void __launch_bounds__(D) q8_combine_kernel(const __grid_constant__ Params p) {
+  constexpr int CU = 8;
+  const int hq = blockIdx.x;
+  const int dd = threadIdx.x;
+  const int b = hq / p.Hq, h = hq % p.Hq;
+  const int bk = b * p.Hkv + h / p.G;
+  int L = p.seq_lens[b];
+  const bool bad = (L < 1 || L > p.L_max);
+  if (bad) L = 0;
+  const int n_tiles = (L + p.T - 1) / p.T;
+  const float* ph = p.part + static_cast<long long>(hq) * p.S * p.CPS * (2 + D);
+  float M = -INFINITY, den = 0.f, num = 0.f;
+  for (int s = 0; s < p.S; ++s) {
+    const int ns = static_cast<int>((static_cast<long long>(s + 1) * n_tiles) / p.S) -
+                   static_cast<int>((static_cast<long long>(s) * n_tiles) / p.S);
+    const int nch = (ns + p.CT - 1) / p.CT;
+    const float* pc = ph + static_cast<long long>(s) * p.CPS * (2 + D);
+    for (int c0 = 0; c0 < nch; c0 += CU) {
+      float m[CU], lc[CU], ac[CU];
+#pragma unroll
+      for (int u = 0; u < CU; ++u) {
+        const bool in = c0 + u < nch;
+        m[u] = in ? pc[(c0 + u) * (2 + D)] : -INFINITY;
+        lc[u] = in ? pc[(c0 + u) * (2 + D) + 1] : 0.f;
+        ac[u] = in ? pc[(c0 + u) * (2 + D) + 2 + dd] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < CU; ++u) {
+        if (m[u] == -INFINITY) continue;
+        if (m[u] > M) {
+          const float r = exp2f(M - m[u]);
+          den *= r;
+          num *= r;
+          M = m[u];
+        }
+        const float w = exp2f(m[u] - M);
+        den += w * lc[u];
+        num += w * ac[u];
+      }
+    }
+    if (dd == 0) {
+      p.ws_used[static_cast<long long>(hq) * p.S + s] = ns;
+      if (h % p.G == 0) p.ws_tiles_read[static_cast<long long>(bk) * p.S + s] = ns;
+    }
+  }
+  p.o[static_cast<long long>(hq) * D + dd] = bad ? __int_as_float(0x7fc00000) : num / den;
+  if (dd == 0) {
+    if (p.tiles) p.tiles[hq] = n_tiles;
+    if (bad && h == 0) atomicOr(p.ws_status, kStatusSeqLen);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+struct Dims {
+  int B, Hq, Hkv, d, L_max, T, S;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace arrays after the common ones (which end at `base`), sized for the smallest chunk.
+struct Layout2 {
+  size_t scores, tmax, cmax, part, end;
+  int n_max, CT, CPS;
+};
+
+inline Layout2 layout2(const Dims& s, size_t base) {
+  Layout2 q;
+  const int G = s.Hq / s.Hkv;
+  q.n_max = (s.L_max + s.T - 1) / s.T;
+  q.CT = chunk_tiles_min(s.T);
+  const int per_split = (q.n_max + s.S - 1) / s.S;
+  q.CPS = (per_split + q.CT - 1) / q.CT;
+  const size_t bk = size_t(s.B) * s.Hkv, units = bk * s.S;
+  q.scores = align256(base);
+  q.tmax = align256(q.scores + 4 * bk * size_t(s.L_max) * gp_of(G));
+  q.cmax = align256(q.tmax + 4 * bk * size_t(q.n_max) * G);
+  q.part = align256(q.cmax + 4 * units * size_t(q.CPS) * G);
+  q.end = align256(q.part + 4 * units * G * size_t(q.CPS) * (size_t(s.d) + 2));
+  return q;
+}
+
+inline size_t workspace_end(const Dims& s, size_t base) { return layout2(s, base).end; }
+
+// (batch, kv head, split) units index blockIdx.y
+inline bool grid_ok(const Dims& s) { return 1LL * s.B * s.Hkv * s.S <= 65535; }
+
+// Tiles per chunk: the one in [smallest, CTMAX] whose grid (2 CTAs per SM) finishes soonest,
+// counting a CTA's time as its tile count and the waves it takes.
+inline int choose_ct(const Dims& s, int sms) {
+  const int n_max = (s.L_max + s.T - 1) / s.T;
+  const int per_split = (n_max + s.S - 1) / s.S;
+  const long long units = 1LL * s.B * s.Hkv * s.S, slots = 2LL * sms;
+  int best = chunk_tiles_min(s.T);
+  long long best_cost = -1;
+  for (int ct = best; ct <= CTMAX; ++ct) {
+    const long long ctas = units * ((per_split + ct - 1) / ct);
+    const long long cost = ((ctas + slots - 1) / slots) * ct;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = ct;
+    }
+  }
+  return best;
+}
+
+template <int D, int GP>
+cudaError_t launch_dg(const Params& p, cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>(p.CPS), static_cast<unsigned>(p.B * p.Hkv * p.S));
+  q8_scores_kernel<D, GP><<<grid, NT, 0, st>>>(p);
+  q8_pv_kernel<D, GP><<<grid, NT, 0, st>>>(p);
+  q8_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const Params& p, cudaStream_t st) {
+  if (p.GP == 1) return launch_dg<D, 1>(p, st);
+  if (p.GP == 2) return launch_dg<D, 2>(p, st);
+  if (p.GP == 4) return launch_dg<D, 4>(p, st);
+  return launch_dg<D, 8>(p, st);
+}
+
+// Enqueue the three kernels.  ws: the caller's workspace; tiles_read_off / used_off: the common
+// per-split counters inside it; base: where the common arrays end.
+inline cudaError_t launch(const Dims& s, const uint16_t* q, const int8_t* k, const uint16_t* ks, const int8_t* v,
+                          const uint16_t* vs, const int32_t* seq_lens, float tau, float* o, int32_t* tiles,
+                          uint8_t* ws, size_t tiles_read_off, size_t used_off, size_t base, cudaStream_t st) {
+  static int sms_of[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (sms_of[dev] == 0) {
+    int v_ = 0;
+    e = cudaDeviceGetAttribute(&v_, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    sms_of[dev] = v_;
+  }
+  const Layout2 ql = layout2(s, base);
+  Params p;
+  p.q = q;
+  p.k = k;
+  p.ks = ks;
+  p.v = v;
+  p.vs = vs;
+  p.seq_lens = seq_lens;
+  p.o = o;
+  p.tiles = tiles;
+  p.ws_status = reinterpret_cast<int32_t*>(ws);
+  p.ws_tiles_read = reinterpret_cast<int32_t*>(ws + tiles_read_off);
+  p.ws_used = reinterpret_cast<int32_t*>(ws + used_off);
+  p.scores = reinterpret_cast<float*>(ws + ql.scores);
+  p.tmax = reinterpret_cast<float*>(ws + ql.tmax);
+  p.cmax = reinterpret_cast<float*>(ws + ql.cmax);
+  p.part = reinterpret_cast<float*>(ws + ql.part);
+  p.B = s.B;
+  p.Hq = s.Hq;
+  p.Hkv = s.Hkv;
+  p.L_max = s.L_max;
+  p.T = s.T;
+  p.S = s.S;
+  p.G = s.Hq / s.Hkv;
+  p.GP = gp_of(p.G);
+  p.CT = choose_ct(s, sms_of[dev]);  // >= the layout's chunk, so at most its chunk count
+  p.CPS = ((ql.n_max + s.S - 1) / s.S + p.CT - 1) / p.CT;
+  p.n_max = ql.n_max;
+  p.qscale = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(s.d)));
+  p.tau = tau;
+  return s.d == 64 ? launch_d<64>(p, st) : launch_d<128>(p, st);
+}
+
+}  // namespace q8two
+}  // namespace artk

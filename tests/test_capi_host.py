@@ -59,6 +59,23 @@ def test_workspace_sizes(L):
     assert capi.art_workspace_bytes(shape(num_splits=0)) == 0
 
 
+def test_q8_workspace_sizes(L):
+    """The two-pass q8 workspace extends the common one: scores [B, Hkv, L_max, G] fp32, tile and
+    chunk maxima, and a (2 + d)-float state per query head and chunk of every split."""
+    for kw in (dict(), dict(num_splits=3), dict(d=64, tile=16), dict(Hq=8, Hkv=8, tile=256), dict(B=1, L_max=1)):
+        s = shape(**kw)
+        base, q8 = capi.art_workspace_bytes(s), capi.art_q8_workspace_bytes(s)
+        n_max = -(-s.L_max // s.tile)
+        assert q8 >= base + 4 * s.B * s.Hq * s.L_max + 4 * s.B * s.Hq * n_max
+        chunks = -(-n_max // s.num_splits)  # chunks of at least one tile per split
+        ct = min(32, 8 * max(1, 128 // s.tile))
+        assert q8 >= base + 4 * s.B * s.Hq * s.num_splits * -(-chunks // ct) * (s.d + 2)
+    assert capi.art_q8_workspace_bytes(shape(B=0)) == 0
+    # the default q8 workload: 2 x 8 kv heads x 32768 positions x 4 heads of scores = 8 MiB and change
+    s = shape(B=2)
+    assert capi.art_q8_workspace_bytes(s) - capi.art_workspace_bytes(s) < 12 << 20
+
+
 A = 0x100000  # fake 16-byte aligned device addresses (never dereferenced)
 
 

@@ -20,8 +20,8 @@ from helpers import TOL, check_tiles, oracle_run  # noqa: E402
 pytestmark = pytest.mark.gpu
 
 
-def gpu(w, mode, *, tile=None, S=None, art=None, tau=None, stream=None):
-    dp = K.upload(w, num_splits=S, tile=tile)
+def gpu(w, mode, *, tile=None, S=None, art=None, tau=None, stream=None, two_pass=True):
+    dp = K.upload(w, num_splits=S, tile=tile, q8_two_pass=two_pass)
     K.decode(dp, mode, art=art, tau=tau, stream=stream)
     st = K.device_status(dp, stream=stream)
     return dict(
@@ -34,10 +34,10 @@ def n_tiles(w, tile):
     return -(-w.seq_lens.astype(np.int64) // tile)
 
 
-def check_full(w, mode="full", tile=None, S=None, tau=None):
+def check_full(w, mode="full", tile=None, S=None, tau=None, two_pass=True):
     tile = tile or w.tile
     S = S or w.num_splits
-    g = gpu(w, mode, tile=tile, S=S, tau=tau)
+    g = gpu(w, mode, tile=tile, S=S, tau=tau, two_pass=two_pass)
     assert g["status"] == capi.ART_OK
     r = oracle_run(w, mode, tile=tile, num_splits=S, tau=tau)
     err = np.max(np.abs(g["o"] - r.o))
@@ -99,8 +99,9 @@ def make_small(kind, d, Hq, Hkv, B, L_max, lens, tile, S, seed=0, **kw):
 def test_full_small(case):
     w = make_small(*case)
     if w.kind == "q8":
-        check_full(w, "q8", tau=0.0)
-        check_full(w, "q8", tau=1e-6)
+        for two_pass in (True, False):  # two streaming passes / one pass over a cluster
+            check_full(w, "q8", tau=0.0, two_pass=two_pass)
+            check_full(w, "q8", tau=1e-6, two_pass=two_pass)
     else:
         check_full(w)
 
@@ -147,10 +148,48 @@ def test_vskip_actually_skips_and_matches():
     w = I.make_workload(kind="q8", B=1, Hq=4, Hkv=1, d=128, L_max=2048, tile=64, seed=5, gumbel_scale=6.0,
                         q_scale=2.0)
     for tau in (1e-3, 1e-6, 0.0, 2.0):
-        check_full(w, "q8", tau=tau)
+        for two_pass in (True, False):
+            check_full(w, "q8", tau=tau, two_pass=two_pass)
     full = oracle_run(w, "q8", tau=0.0)
     skip = oracle_run(w, "q8", tau=1e-3)
     assert np.max(np.abs(full.o - skip.o)) > 1e-6  # the skip changed something measurable
+
+
+Q8_TWO_PASS = [
+    # d, Hq, Hkv, B, L_max, lens, tile, S: every head-group width (1, 2, 3 -> 4, 4, 8), d = 64 / 128,
+    # chunks of 32 / 16 / 8 tiles (several per split), ragged tails, length 1, empty splits
+    (128, 8, 8, 2, 4096, [4096, 1], 16, 1),
+    (64, 8, 4, 2, 3000, [2999, 1500], 32, 3),
+    (128, 6, 2, 1, 5000, [4937], 64, 2),
+    (128, 8, 2, 2, 4500, [4500, 2047], 64, 1),
+    (64, 16, 2, 3, 2500, [2500, 777, 3], 128, 4),
+    (128, 8, 1, 1, 4096, [4096], 256, 1),
+    (128, 32, 8, 1, 2048, [2000], 64, 8),
+]
+
+
+@pytest.mark.parametrize("case", Q8_TWO_PASS, ids=lambda c: f"d{c[0]}-g{c[1] // c[2]}-T{c[6]}-S{c[7]}")
+def test_q8_two_pass_shapes(case):
+    d, Hq, Hkv, B, L_max, lens, tile, S = case
+    w = I.make_workload(kind="q8", B=B, Hq=Hq, Hkv=Hkv, d=d, L_max=L_max, tile=tile, num_splits=S,
+                        seq_lens=lens, seed=77 + tile, gumbel_scale=3.0, q_scale=1.5)
+    for tau in (0.0, 1e-4):
+        check_full(w, "q8", tau=tau)
+
+
+def test_q8_two_pass_skips_whole_tiles():
+    """A sink key far above every other score: after its tile almost every row of every head
+    falls below tau, so the two-pass path leaves whole V tiles unread; outputs still match the
+    oracle's row rule, and the same call over a one-pass workspace agrees."""
+    w = I.make_workload(kind="q8", B=2, Hq=8, Hkv=2, d=128, L_max=4096, tile=64, seq_lens=[4096, 3001],
+                        seed=11, sink=40.0)
+    for tau in (1e-6, 1e-3):
+        g2 = check_full(w, "q8", tau=tau, two_pass=True)
+        g1 = check_full(w, "q8", tau=tau, two_pass=False)
+        assert np.max(np.abs(g1["o"] - g2["o"])) <= TOL["q8"]
+    r = oracle_run(w, "q8", tau=1e-6)
+    r0 = oracle_run(w, "q8", tau=0.0)
+    assert np.max(np.abs(r.o - r0.o)) > 0.0  # rows were skipped
 
 
 def test_empty_splits_and_tiny_lengths():
