@@ -111,8 +111,9 @@ typedef struct {
 size_t art_workspace_bytes(const art_shape* shape);
 
 /* Bytes of workspace art_decode_attn_q8_skipv needs to run full attention (params == NULL) as
- * two streaming passes: art_workspace_bytes(shape) plus scores [B, Hkv, L_max, Hq/Hkv] fp32,
- * tile and chunk maxima and per-chunk partial states (0 on an invalid shape).  The offsets below
+ * two streaming passes: art_workspace_bytes(shape) plus scores [B, Hkv, L_max, GP] fp32 (GP the
+ * next power of two >= Hq/Hkv), tile and chunk maxima and per-chunk partial states (0 on an
+ * invalid shape).  The offsets below
  * hold for this larger workspace too. */
 size_t art_q8_workspace_bytes(const art_shape* shape);
 
