@@ -94,7 +94,7 @@ def term(s, params, **kw):
 
 
 def q8(s, params=None, tau=1e-6, **kw):
-    wsb = capi.art_workspace_bytes(s) or (1 << 20)
+    wsb = kw.get("ws_bytes", capi.art_workspace_bytes(s) or (1 << 20))
     return capi.art_decode_attn_q8_skipv(s, A, A * 2, kw.get("ks", A * 8), A * 3, kw.get("vs", A * 9), A * 4, tau,
                                          params, A * 5, A * 6, A * 7, wsb, None)
 
@@ -136,6 +136,14 @@ def test_invalid_arguments_q8(L):
     assert q8(s, tau=float("nan")) == capi.ART_ERR_INVALID_ARG
     assert q8(shape(L_max=32767)) == capi.ART_ERR_UNSUPPORTED  # scale rows not 16-byte granular
     assert q8(s, params=capi.make_params(1e-3, 1e-4, 1, [200])) == capi.ART_ERR_INVALID_ARG
+    # the same checks, synchronously and before any launch, with a two-pass workspace
+    big = capi.art_q8_workspace_bytes(s)
+    assert q8(s, ks=None, ws_bytes=big) == capi.ART_ERR_INVALID_ARG
+    assert q8(s, vs=A + 2, ws_bytes=big) == capi.ART_ERR_INVALID_ARG
+    assert q8(s, tau=float("nan"), ws_bytes=big) == capi.ART_ERR_INVALID_ARG
+    s2 = shape(L_max=32767)
+    assert q8(s2, ws_bytes=capi.art_q8_workspace_bytes(s2)) == capi.ART_ERR_UNSUPPORTED
+    assert q8(s, ws_bytes=capi.art_workspace_bytes(s) - 16) == capi.ART_ERR_WORKSPACE
 
 
 def test_read_status_rejects_null(L):
