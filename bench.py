@@ -2,22 +2,25 @@
 """Benchmark: single-token decode attention with ART on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--mode art|full|q8|q8_art]
+                    [--workload NAME] [--mode art|full|q8|q8_art] [--no-sweeps]
 
 A step is one decode call over the whole batch of the workload (default: GQA
-bf16, B=4, Hq=32, Hkv=8, d=128, L=32768, tile 64 -- the long-context decode
-shape the pages' results are quoted on): Q load, K/V tile stream, scores,
-online softmax, PV, the ART probe and rule, the early-exit vote and the
-epilogue, all in one kernel launch.  The KV cache (512 MiB) is larger than L2,
-so no flush is needed between steps.
+bf16, B=16, Hq=32, Hkv=8, d=128, per-sequence lengths uniform in [8192, 65536],
+tile 64, 8 KV splits + combine -- the largest of the five long-context decode
+shapes, 2.25 GiB of K/V): Q load, K/V tile stream, scores, online softmax, PV,
+the ART probe and rule, the early-exit vote, the epilogue and the split
+combine.  The KV cache is larger than L2, so no flush is needed between steps.
 
 Prints ONE JSON line (rank 0).  `value` is decoded query-heads per second over
 all ranks, device-timed with CUDA events; `e2e` times the same call with the
 step's query copied from pinned host memory and its result copied back; the
 `roofline` object rates the decode kernel on the KV bytes it actually read
-(device counters) against the measured HBM copy bandwidth.  With N > 1 every
-rank decodes its own batch of the same shape (weak scaling, no collective in
-the data path); timing is the max over ranks.
+(device counters) against the measured HBM copy bandwidth.  `workloads` holds
+the same measurements for all five workloads (full and ART modes, bytes read
+and consumed, the thresholds-0 overhead and the thresholds-+inf scaling sweep),
+`vskip` the q8 V-skip threshold sweep.  With N > 1 every rank decodes its own
+batch of the same shape (weak scaling, no collective in the data path); timing
+is the max over ranks.
 """
 from __future__ import annotations
 
@@ -40,7 +43,9 @@ from kv_cache_early_split_b200 import inputs as I  # noqa: E402
 
 METRIC = "decode attention query-heads/s and KV GB/s (fraction of HBM peak), full vs ART"
 UNIT = "query-heads/s"
-DEFAULT_WORKLOAD = "gqa_b4_h32x8_d128_L32k"
+DEFAULT_WORKLOAD = "split_b16_h32x8_d128_Lvar"
+# workload of the ablation, traversal-order, paged-cache and eviction sweeps
+EXTRAS_WORKLOAD = "gqa_b4_h32x8_d128_L32k"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
 FALLBACK_HBM_GBS = 6650.0
@@ -55,7 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOADS)
     ap.add_argument("--mode", default=None, choices=("art", "full", "q8", "q8_art"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-sweeps", action="store_true", help="skip the ART scaling / overhead sweeps")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="time the workload's two modes only (no other workloads, sweeps or extras)")
     a = ap.parse_args(argv)
     if a.mode is None:
         a.mode = "q8_art" if a.workload.startswith("q8") else "art"
@@ -316,12 +322,11 @@ ABLATION_GRID = {
 }
 
 
-def art_ablation(K, dp, w, args):
+def art_ablation(K, dp, w, mode):
     """Premature-stop error against tiles saved for each criterion family and patience 1, 2, 4:
     per query head, ||O_ART - O_full|| / ||O_full|| (L2 over d), on the bench's own buffers."""
     import torch
 
-    mode = args.mode
     full_mode = "full" if mode == "art" else "q8"
     K.decode(dp, full_mode)
     o_full = dp.o.clone()
@@ -342,16 +347,15 @@ def art_ablation(K, dp, w, args):
     return rows
 
 
-def art_orders(K, dp, w, args, stream):
+def art_orders(K, dp, w, steps, stream):
     """ART with the configured thresholds along each traversal order (natural, recency first,
     importance first): time per call, tiles read, error against full attention, and the time to
     build the sequence on the GPU per step (importance: scoring and sort; the per-tile key summary
     is built once, as a cache would maintain it when keys are appended, and timed apart)."""
     import torch
 
-    if args.mode != "art" or w.kind not in ("f32", "bf16"):
+    if w.kind not in ("f32", "bf16"):
         return None
-    steps = max(3, min(args.steps, 10))
     K.decode(dp, "full")
     o_full = dp.o.clone()
     nrm = torch.linalg.vector_norm(o_full, dim=-1).clamp_min(1e-30)
@@ -396,7 +400,7 @@ def art_orders(K, dp, w, args, stream):
     return out
 
 
-def evict_sweep(K, dp, w, args, stream):
+def evict_sweep(K, dp, w, steps, stream):
     """Random eviction to a quarter of the cache (sink L/128, recent window L/32, the rest drawn
     uniformly), then full attention and ART on the packed cache: time of the selection, the packing
     and the decodes, KV bytes read, and error against full attention over the whole cache."""
@@ -406,7 +410,6 @@ def evict_sweep(K, dp, w, args, stream):
     budget, sink, recent = L // 4, L // 128, L // 32
     if budget < sink + recent + 1:
         return None
-    steps = max(3, min(args.steps, 10))
     full_mode, art_mode = ("q8", "q8_art") if w.kind == "q8" else ("full", "art")
     K.decode(dp, full_mode)
     o_full = dp.o.clone()
@@ -432,13 +435,12 @@ def evict_sweep(K, dp, w, args, stream):
     return out
 
 
-def paged_sweep(K, w, args, stream):
+def paged_sweep(K, w, steps, stream):
     """The same step over a paged copy of the cache (random page placement, block table per
     sequence), page sizes 64 and 256: ms per call in both modes, and KV bytes read."""
     import torch
 
     modes = ("q8", "q8_art") if w.kind == "q8" else ("full", "art")
-    steps = max(3, min(args.steps, 10))
     out = {}
     for page in (64, 256):
         if page % w.tile:
@@ -457,45 +459,111 @@ def paged_sweep(K, w, args, stream):
     return out
 
 
-def art_sweeps(K, dp, w, args, stream):
-    """Two sweeps of the ART path on the same buffers (ART modes only).
-
-    scaling: thresholds +inf and patience k stop every (head, split) after exactly min(k, n)
-    tiles, so time against tiles read should be a line with a small intercept.
-    overhead: thresholds 0 never stop, so ART reads every tile; its time against full
-    attention is the cost of the probe, the exchange and the rule."""
-    import torch
-
-    if args.mode not in ("art", "q8_art"):
-        return None
-    full_mode = "full" if args.mode == "art" else "q8"
+def scaling_sweep(K, dp, w, mode, steps, stream):
+    """Thresholds +inf and patience k stop every (head, split) after exactly min(k, n) tiles, so the
+    time per call against KV bytes read should be a line with a small intercept."""
     n = int(-(-int(w.seq_lens.max()) // w.tile)) // max(1, w.num_splits)
-    ks = sorted({1, max(1, n // 8), max(1, n // 4), max(1, n // 2), n})
-    steps = max(3, min(args.steps, 10))
+    ks = sorted({1, max(1, n // 8), max(1, n // 4), max(1, n // 2), max(1, n)})
+    n_all = float((-(-w.seq_lens.astype(np.int64) // w.tile)).sum() * w.Hq)
+    flush = needs_flush(w)
     pts = []
     for k in ks:
         art = dict(w.art, eps_scale=float("inf"), eps_dir=float("inf"), patience=k)
-        _, launch = time_mode(K, dp, args.mode, steps, 2, stream, art=art)
+        _, launch = time_mode(K, dp, mode, steps, 2, stream, art=art, flush=flush)
         rb = bytes_read(w, dp.tiles_read().cpu().numpy())
-        pts.append({"patience": k, "tiles_frac": float(dp.tiles.float().mean().item()) / (n * w.num_splits),
-                     "ms": launch, "kv_bytes_read": rb})
+        cb = bytes_consumed(w, dp.split_tiles().cpu().numpy())
+        pts.append({"patience": k, "tiles_frac": float(dp.tiles.double().sum().item()) / n_all,
+                    "ms": launch, "kv_bytes_read": rb, "kv_bytes_consumed": cb, "read_over_consumed": rb / cb})
     x = np.array([p["kv_bytes_read"] for p in pts], dtype=np.float64)
     y = np.array([p["ms"] for p in pts], dtype=np.float64)
     slope, icpt = np.polyfit(x, y, 1) if len(pts) > 1 else (0.0, float(y[0]))
-    ablation = art_ablation(K, dp, w, args)
-    trav = art_orders(K, dp, w, args, stream)
-    eps0 = dict(w.art, eps_scale=0.0, eps_dir=0.0)
-    _, ms_eps0 = time_mode(K, dp, args.mode, steps, 2, stream, art=eps0)
-    _, ms_full = time_mode(K, dp, full_mode, steps, 2, stream)
-    torch.cuda.synchronize()
-    return {
-        "scaling": {"points": pts, "fit_ms": {"intercept": float(icpt), "per_gb": float(slope) * 1e9},
-                    "note": "eps = +inf, patience k: exactly min(k, n) tiles per (head, split)"},
-        "overhead_eps0": {"ms_art_eps0": ms_eps0, "ms_full": ms_full, "ratio": ms_eps0 / ms_full,
-                          "note": "eps = 0: ART never stops and reads every tile"},
-        "ablation": ablation,
-        "orders": trav,
-    }
+    return {"points": pts, "fit_ms": {"intercept": float(icpt), "per_gb": float(slope) * 1e9},
+            "note": "eps = +inf, patience k: exactly min(k, n) tiles per (head, split)"}
+
+
+def mode_row(K, dp, w, mode, steps, stream, peak, art=None):
+    """Time one mode on a workload's buffers; throughput, KV bytes read (device counters) and
+    consumed (the slowest head of each kv head), and tile counts of the last call."""
+    flush = needs_flush(w)
+    _, launch = time_mode(K, dp, mode, steps, 2, stream, art=art, flush=flush)
+    if K.device_status(dp) != 0:
+        raise RuntimeError(f"device status not OK after {w.name} {mode}")
+    n_full = -(-w.seq_lens.astype(np.int64) // w.tile)
+    rb = bytes_read(w, dp.tiles_read().cpu().numpy())
+    cb = bytes_consumed(w, dp.split_tiles().cpu().numpy())
+    tiles = dp.tiles.cpu().numpy()
+    gbs = rb / (launch / 1e3) / 1e9
+    return {"ms": launch, "query_heads_per_s": w.B * w.Hq / (launch / 1e3), "kv_bytes_read": rb,
+            "kv_bytes_consumed": cb, "kv_gbs_read": gbs, "frac_of_hbm": gbs / peak,
+            "kv_gbs_consumed": cb / (launch / 1e3) / 1e9, "read_over_consumed": rb / cb,
+            "mean_tiles_frac": float(tiles.mean() / n_full.mean())}
+
+
+def measure_workload(K, w, dp, args, stream, peak, sweeps=True):
+    """Full and ART modes of one workload: time per call, GB/s read and consumed, fraction of HBM;
+    ART time per consumed KV byte against full attention's per byte; the thresholds-0 overhead and
+    the thresholds-+inf scaling sweep."""
+    full_mode, art_mode = ("q8", "q8_art") if w.kind == "q8" else ("full", "art")
+    steps = max(3, min(args.steps, 10))
+    out = {"kernel": {full_mode: K.kernel_name(dp, full_mode), art_mode: K.kernel_name(dp, art_mode)},
+           "kv_cache_bytes": kv_cache_bytes(w),
+           "l2": "flushed before every timed launch" if needs_flush(w) else "KV larger than L2, no flush"}
+    out[full_mode] = mode_row(K, dp, w, full_mode, steps, stream, peak)
+    out[art_mode] = mode_row(K, dp, w, art_mode, steps, stream, peak)
+    f, a = out[full_mode], out[art_mode]
+    out["art_over_full_time"] = a["ms"] / f["ms"]
+    # time per consumed byte, ART over full (1.0: ART time follows what it consumed exactly)
+    out["art_per_consumed_byte_over_full"] = (a["ms"] / a["kv_bytes_consumed"]) / (f["ms"] / f["kv_bytes_read"])
+    if sweeps:
+        eps0 = dict(w.art, eps_scale=0.0, eps_dir=0.0)
+        e = mode_row(K, dp, w, art_mode, steps, stream, peak, art=eps0)
+        out["overhead_eps0"] = {"ms": e["ms"], "ratio_to_full": e["ms"] / f["ms"],
+                                "note": "eps = 0: ART never stops and reads every tile"}
+        out["scaling"] = scaling_sweep(K, dp, w, art_mode, steps, stream)
+    return out
+
+
+def vskip_sweep(K, args, stream, device):
+    """The q8 V-dequant skip threshold tau in {0, 1e-6, 1e-3} on the q8 workload (N(0,1) keys) and on
+    its skewed variant (attention sink, Gumbel key offsets, log-normal V norms): ms per call with and
+    without ART.  tau = 0 skips nothing, so the time differences are the skip's saving."""
+    import torch
+
+    steps = max(3, min(args.steps, 10))
+    out = {"context": "pages: -22.8% decode time at 32K (turbo3 KV, Apple M5 Max), +5% with q8_0 KV "
+                      "(M5 Max / M2 Pro); other hardware and formats, not a target"}
+    for name in ("q8_b2_h32x8_d128_L32k", "q8_b2_h32x8_d128_L32k_skewed"):
+        w = I.workload(name)
+        dp = K.upload(w, device=device)
+        rows = {}
+        for tau in (0.0, 1e-6, 1e-3):
+            row = {}
+            for mode in ("q8", "q8_art"):
+                for _ in range(2):
+                    K.decode(dp, mode, tau=tau, stream=stream.cuda_stream)
+                torch.cuda.synchronize()
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+                for e0, e1 in ev:
+                    l2_flush(stream)
+                    e0.record(stream)
+                    K.decode(dp, mode, tau=tau, stream=stream.cuda_stream)
+                    e1.record(stream)
+                torch.cuda.synchronize()
+                row[mode] = {"ms": sum(a.elapsed_time(b) for a, b in ev) / steps,
+                             "kv_bytes_read": bytes_read(w, dp.tiles_read().cpu().numpy()),
+                             "mean_tiles_frac": float(dp.tiles.float().mean().item())
+                             / float((-(-w.seq_lens.astype(np.int64) // w.tile)).mean())}
+            rows[f"tau_{tau:g}"] = row
+        if K.device_status(dp) != 0:
+            raise RuntimeError("device status not OK after the V-skip sweep")
+        for mode in ("q8", "q8_art"):
+            base = rows["tau_0"][mode]["ms"]
+            for t in ("tau_1e-06", "tau_0.001"):
+                rows[t][mode]["time_saved_vs_tau0"] = 1.0 - rows[t][mode]["ms"] / base
+        out[name] = rows
+        del dp
+        torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -598,20 +666,44 @@ def run_ours(args):
     other = {"art": "full", "full": "art", "q8": "q8_art", "q8_art": "q8"}[args.mode]
     o_total, o_launch = time_mode(K, dp, other, args.steps, args.warmup, stream, flush=flush)
     o_read = bytes_read(w, dp.tiles_read().cpu().numpy())
+    o_cons = bytes_consumed(w, dp.split_tiles().cpu().numpy())
     o_max, _ = aggregate(o_total, 0)
     modes = {
         args.mode: {"query_heads_per_s": value, "ms_per_step": max_ms / args.steps,
                     "kv_gbs_read": achieved, "frac_of_hbm": achieved / peak,
-                    "kv_bytes_read": rb, "kv_bytes_consumed": cb,
+                    "kv_bytes_read": rb, "kv_bytes_consumed": cb, "read_over_consumed": rb / cb,
                     "mean_tiles_frac": float(tiles.mean() / n_full.mean())},
         other: {"query_heads_per_s": heads * world * args.steps / (o_max / 1e3), "ms_per_step": o_max / args.steps,
                 "kv_gbs_read": o_read / (o_launch / 1e3) / 1e9, "frac_of_hbm": o_read / (o_launch / 1e3) / 1e9 / peak,
-                "kv_bytes_read": o_read},
+                "kv_bytes_read": o_read, "kv_bytes_consumed": o_cons},
     }
 
-    sweeps = art_sweeps(K, dp, w, args, stream) if not args.no_sweeps else None
-    paged = paged_sweep(K, w, args, stream) if not args.no_sweeps else None
-    evicted = evict_sweep(K, dp, w, args, stream) if not args.no_sweeps else None
+    workloads = vskip = extras = None
+    if not args.no_sweeps:
+        # every workload, full and ART, with the overhead and scaling sweeps
+        workloads = {}
+        for name in I.WORKLOADS:
+            if name == w.name:
+                workloads[name] = measure_workload(K, w, dp, args, stream, peak)
+                continue
+            wl = I.workload(name)
+            dpl = K.upload(wl, device=dev)
+            workloads[name] = measure_workload(K, wl, dpl, args, stream, peak)
+            del dpl, wl
+            torch.cuda.empty_cache()
+        vskip = vskip_sweep(K, args, stream, dev)
+        # ablation, traversal orders, paged cache and eviction on the 32K GQA workload
+        steps_x = max(3, min(args.steps, 10))
+        we = w if w.name == EXTRAS_WORKLOAD else I.workload(EXTRAS_WORKLOAD)
+        dpe = dp if we is w else K.upload(we, device=dev)
+        extras = {"workload": we.name, "ablation": art_ablation(K, dpe, we, "art"),
+                  "orders": art_orders(K, dpe, we, steps_x, stream),
+                  "paged": paged_sweep(K, we, steps_x, stream),
+                  "eviction": evict_sweep(K, dpe, we, steps_x, stream)}
+        if dpe is not dp:
+            del dpe
+        del we
+        torch.cuda.empty_cache()
 
     # end to end through the public call: the step's query in from pinned host memory, O and tiles back out
     q_host = dp.q.cpu().pin_memory()
@@ -655,6 +747,8 @@ def run_ours(args):
     traffic = measured_traffic(w.name, args.mode, kernel)
     if launches_per_call(K, dp, w, args.mode) == 3:
         kernel = "q8_scores_kernel + q8_pv_kernel + q8_combine_kernel (timed as one call)"
+    elif w.num_splits > 1:
+        kernel += " (timed with its split combine kernel)"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -664,9 +758,9 @@ def run_ours(args):
                      "peak_source": f"{peak_kind} hbm_gbs (copy)", "traffic": traffic,
                      "kernel": kernel, "bytes_per_launch": rb, "launch_ms": launch_ms},
         "modes": modes,
-        "art_sweeps": sweeps,
-        "paged": paged,
-        "eviction": evicted,
+        "workloads": workloads,
+        "vskip": vskip,
+        "extras": extras,
         "e2e": e2e,
         "gpu_launches": gpu_launches,
         "clocks": clocks,

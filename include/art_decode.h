@@ -155,14 +155,22 @@ art_status art_decode_attn_terminate(const art_shape* shape, art_dtype dtype, co
  *   - Calls no cudaMalloc / cudaFree and no allocating library routine.  The
  *     first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture on that device.
+ *     stream capture on that device.  The cached address belongs to the
+ *     device's current context: after cudaDeviceReset (or anything else that
+ *     destroys and recreates the primary context) the array lives at a new
+ *     address and the cache is stale, so do not call this entry point again
+ *     in that process after a reset.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind.  No word of it has to start at zero (the kernels write all they
  *     read), so nothing is cleared between calls.  Calls whose executions
  *     overlap on the GPU (different streams, or concurrent host threads) race
  *     on the array: serialise them.
  *   - Device-side errors (a seq_len outside [1, L_max]) show as NaN outputs
- *     and 0 tiles for that sequence; there is no status to read back. */
+ *     and 0 tiles for that sequence; there is no status to read back.  A
+ *     bounded wait that gives up inside a kernel (a hung copy; it never
+ *     happens in normal operation) is not reported either, and leaves the
+ *     outputs of the affected sequences unspecified: callers that must
+ *     detect it use art_decode_attn_terminate and art_read_device_status. */
 art_status art_decode_attn_terminate_noalloc(const art_shape* shape, art_dtype dtype, const void* q,
                                              const void* k, const void* v, const int32_t* seq_lens,
                                              const art_params* params, float* o, int32_t* tiles,

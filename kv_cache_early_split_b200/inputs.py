@@ -27,6 +27,8 @@ discuss, 32K-128K positions; the pages' own benchmark suites are not used):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -199,32 +201,42 @@ def make_workload(
     if kind == "q8":
         k_scale = np.zeros((B, Hkv, L_max, d // 32), np.uint16)
         v_scale = np.zeros((B, Hkv, L_max, d // 32), np.uint16)
-    for bi, b in enumerate(kb):
-        for hi, h in enumerate(kh):
-            kf = _normal_slab(seed, _T_K, b, h, L_max, d)
-            if lognormal_v:
-                vf = _normal_slab(seed, _T_V, b, h, L_max, d)
-                vf /= np.linalg.norm(vf, axis=1, keepdims=True)
-                vf *= _rng(seed, _T_VNORM, b, h).lognormal(0.0, 1.0, size=(L_max, 1)).astype(np.float32)
-            else:
-                vf = _normal_slab(seed, _T_V, b, h, L_max, d)
-            if sink or gumbel_scale:
-                mean_q = q_used[bi, hi * G:(hi + 1) * G].mean(axis=0)
-                nrm = float(np.linalg.norm(mean_q))
-                u = mean_q / nrm if nrm > 0 else np.zeros(d, np.float32)
-                if gumbel_scale:
-                    g = _rng(seed, _T_GUMBEL, b, h).gumbel(0.0, gumbel_scale, size=(L_max, 1)).astype(np.float32)
-                    kf += g * u[None, :]
-                if sink:
-                    kf[0] += np.float32(sink) * u
-            # storage format of this slab
-            if kind == "f32":
-                k[bi, hi], v[bi, hi] = kf, vf
-            elif kind == "bf16":
-                k[bi, hi], v[bi, hi] = bf16_bits(kf), bf16_bits(vf)
-            else:
-                k[bi, hi], k_scale[bi, hi] = quantize_q8(kf)
-                v[bi, hi], v_scale[bi, hi] = quantize_q8(vf)
+    def build_slab(bi, b, hi, h):
+        kf = _normal_slab(seed, _T_K, b, h, L_max, d)
+        if lognormal_v:
+            vf = _normal_slab(seed, _T_V, b, h, L_max, d)
+            vf /= np.linalg.norm(vf, axis=1, keepdims=True)
+            vf *= _rng(seed, _T_VNORM, b, h).lognormal(0.0, 1.0, size=(L_max, 1)).astype(np.float32)
+        else:
+            vf = _normal_slab(seed, _T_V, b, h, L_max, d)
+        if sink or gumbel_scale:
+            mean_q = q_used[bi, hi * G:(hi + 1) * G].mean(axis=0)
+            nrm = float(np.linalg.norm(mean_q))
+            u = mean_q / nrm if nrm > 0 else np.zeros(d, np.float32)
+            if gumbel_scale:
+                g = _rng(seed, _T_GUMBEL, b, h).gumbel(0.0, gumbel_scale, size=(L_max, 1)).astype(np.float32)
+                kf += g * u[None, :]
+            if sink:
+                kf[0] += np.float32(sink) * u
+        # storage format of this slab
+        if kind == "f32":
+            k[bi, hi], v[bi, hi] = kf, vf
+        elif kind == "bf16":
+            k[bi, hi], v[bi, hi] = bf16_bits(kf), bf16_bits(vf)
+        else:
+            k[bi, hi], k_scale[bi, hi] = quantize_q8(kf)
+            v[bi, hi], v_scale[bi, hi] = quantize_q8(vf)
+
+    # Every slab has its own random stream and its own output rows, so the slabs are built in
+    # parallel threads (numpy's generators and array kernels release the GIL); the result is the
+    # same as building them one after another.
+    slabs = [(bi, b, hi, h) for bi, b in enumerate(kb) for hi, h in enumerate(kh)]
+    if len(slabs) > 1 and L_max * d >= (1 << 16):
+        with ThreadPoolExecutor(max_workers=min(len(slabs), os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda a: build_slab(*a), slabs))
+    else:
+        for a in slabs:
+            build_slab(*a)
     if art is None:
         art = dict(eps_scale=1e-3, eps_dir=1e-4, patience=1, lanes=probe_lanes_strided(d, 16 if d >= 128 else 8))
     return Workload(
@@ -245,12 +257,26 @@ WORKLOADS = (
 )
 
 
+# Variants used by the benchmark's sweeps (not among the five workloads):
+#   q8_b2_h32x8_d128_L32k_skewed  the q8 workload's shape with skewed logits: attention sink
+#                                 (key 0 moved 8 units along the group's mean query), keys shifted
+#                                 along that direction by Gumbel(0, 2), V rows = unit directions
+#                                 times LogNormal(0, 1) norms -- so that many softmax weights fall
+#                                 below the V-skip threshold.
+VARIANTS = ("q8_b2_h32x8_d128_L32k_skewed",)
+
+
 def workload(name: str, *, keys_b=None, keys_h=None) -> Workload:
-    """The five named synthetic workloads (seed 20260000 + index).
+    """The five named synthetic workloads (seed 20260000 + index), or a variant of VARIANTS.
 
     keys_b / keys_h select a slice (batches, kv heads) of the same problem; the
     selected slabs are bit-identical to those of the full workload.
     """
+    if name == VARIANTS[0]:
+        return make_workload(
+            name=name, kind="q8", B=2, Hq=32, Hkv=8, d=128, L_max=32768, tile=64, tau=1e-6, sink=8.0,
+            gumbel_scale=2.0, lognormal_v=True, art=dict(ART_C2), seed=20260104, keys_b=keys_b, keys_h=keys_h,
+        )
     i = WORKLOADS.index(name)
     seed = 20260000 + i
     kw = dict(name=name, seed=seed, keys_b=keys_b, keys_h=keys_h)

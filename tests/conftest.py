@@ -9,3 +9,15 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Parity counts the GPU tests collected (stop-tile agreement, errors), one line each."""
+    try:
+        from helpers import REPORT
+    except ImportError:
+        return
+    if REPORT:
+        terminalreporter.write_sep("-", "parity report")
+        for line in REPORT:
+            terminalreporter.write_line(line)

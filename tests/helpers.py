@@ -13,6 +13,8 @@ import numpy as np
 import oracle
 
 WINDOW = 1e-4
+# Lines the GPU tests want shown at the end of the pytest run (see conftest.py).
+REPORT = []
 TOL = {"f32": 1e-5, "bf16": 2e-3, "q8": 2e-3}
 KIND = {"f32": oracle.KV_F32, "bf16": oracle.KV_BF16, "q8": oracle.KV_Q8}
 

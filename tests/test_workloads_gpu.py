@@ -1,9 +1,20 @@
 """The five synthetic workloads at their full sizes, in the launch configuration
-the benchmark times.  The GPU runs the whole problem; outputs of sampled
-(batch, kv head) slabs are checked element by element against the oracle on
-the same slab (built bit-identically by the seeded generator), and properties
-that hold at any size are checked on every head.
+the benchmark times, checked on EVERY (batch, query head, split) against the
+oracle run over the whole problem on all host cores:
+
+* full attention: every output element within the tolerance, every tile count
+  equal to the oracle's;
+* ART: every stop tile accepted by the rule's acceptance DP (a tile whose oracle
+  metric lies within 1e-4 of its threshold may count either way), every output
+  element within the tolerance of the oracle re-run to the GPU's own stop tiles,
+  and the GPU's stop tile equal to the oracle's own stop tile on at least
+  AGREE_FLOOR of the (head, split) pairs -- so the ambiguity window cannot hide
+  a drift of the stop tiles.
+
+The exact / ambiguous / agreeing counts are reported at the end of the pytest run.
 """
+import os
+
 import numpy as np
 import pytest
 
@@ -12,32 +23,30 @@ torch = pytest.importorskip("torch")
 import kv_cache_early_split_b200 as K  # noqa: E402
 from kv_cache_early_split_b200 import capi  # noqa: E402
 from kv_cache_early_split_b200 import inputs as I  # noqa: E402
-from helpers import TOL, check_tiles, oracle_run  # noqa: E402
+from helpers import REPORT, TOL, check_tiles, oracle_run  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 
-# (workload, modes, sampled (b, kvh) slabs)
 CASES = [
-    ("fp32_b1_h1_d64_L4k", ("full", "art"), [(0, 0)]),
-    ("gqa_b4_h32x8_d128_L32k", ("full", "art"), [(0, 0), (3, 5)]),
-    ("gqa_b1_h32x8_d128_L128k", ("full", "art"), [(0, 2)]),
-    ("split_b16_h32x8_d128_Lvar", ("full", "art"), [(2, 1), (11, 7)]),
-    ("q8_b2_h32x8_d128_L32k", ("q8", "q8_art"), [(1, 3)]),
+    ("fp32_b1_h1_d64_L4k", ("full", "art")),
+    ("gqa_b4_h32x8_d128_L32k", ("full", "art")),
+    ("gqa_b1_h32x8_d128_L128k", ("full", "art")),
+    ("split_b16_h32x8_d128_Lvar", ("full", "art")),
+    ("q8_b2_h32x8_d128_L32k", ("q8", "q8_art")),
 ]
 
-_cache = {}
+# Fraction of (head, split) pairs whose GPU stop tile must equal the oracle's own stop tile.  The
+# GPU evaluates the metrics in fp32 from fp32 accumulations (bf16 inputs, bf16 hi + lo weights on
+# the tensor cores), the oracle in fp64; a stop moves only where a metric lies within the fp32
+# evaluation error (~1e-7 absolute for d_dir near 1e-4) of its threshold.
+AGREE_FLOOR = 0.99
+
+THREADS = max(1, os.cpu_count() or 1)
 
 
-def full_workload(name):
-    if name not in _cache:
-        _cache.clear()
-        _cache[name] = I.workload(name)
-    return _cache[name]
-
-
-@pytest.mark.parametrize("name,modes,slabs", CASES, ids=[c[0] for c in CASES])
-def test_workload(name, modes, slabs):
-    w = full_workload(name)
+@pytest.mark.parametrize("name,modes", CASES, ids=[c[0] for c in CASES])
+def test_workload_every_unit(name, modes):
+    w = I.workload(name)
     dp = K.upload(w)
     n = -(-w.seq_lens.astype(np.int64) // w.tile)
     S, G = w.num_splits, w.G
@@ -51,25 +60,27 @@ def test_workload(name, modes, slabs):
         assert np.all(np.isfinite(o))
         assert np.array_equal(used.sum(axis=2), tiles)
         assert np.all(tiles >= 1) and np.all(tiles <= n[:, None])
-        art_mode = mode in ("art", "q8_art")
-        if not art_mode:
-            assert np.array_equal(tiles, np.repeat(n[:, None], w.Hq, axis=1))
         for b in range(w.B):
             for h in range(w.Hkv):
                 need = used[b, h * G:(h + 1) * G].max(axis=0)
                 assert np.all(read[b, h] >= need)
-        for (b, h) in slabs:
-            ws = I.workload(name, keys_b=[b], keys_h=[h])
-            assert np.array_equal(ws.k[0, 0], w.k[b, h]) and np.array_equal(ws.q[0], w.q[b, h * G:(h + 1) * G])
-            sl = slice(h * G, (h + 1) * G)
-            if art_mode:
-                ref = oracle_run(ws, mode, metrics=True)
-                exact, amb = check_tiles(ws, ref.metrics, used[b:b + 1, sl], ws.art, ws.tile, S)
-                forced = oracle_run(ws, "q8" if mode == "q8_art" else "full", forced_used=used[b:b + 1, sl])
-                err = np.max(np.abs(o[b, sl] - forced.o[0]))
-                print(f"{name} {mode} slab ({b},{h}): tiles {tiles[b, sl]} of {n[b]} exact={exact} amb={amb} err={err:.2e}")
-            else:
-                ref = oracle_run(ws, mode)
-                err = np.max(np.abs(o[b, sl] - ref.o[0]))
-                print(f"{name} {mode} slab ({b},{h}): err={err:.2e}")
-            assert err <= TOL[w.kind]
+        art_mode = mode in ("art", "q8_art")
+        if not art_mode:
+            ref = oracle_run(w, mode, n_threads=THREADS)
+            assert np.array_equal(tiles, np.repeat(n[:, None], w.Hq, axis=1))
+            assert np.array_equal(used, ref.used)
+            err = float(np.max(np.abs(o - ref.o)))
+            REPORT.append(f"{name} {mode}: {w.B * w.Hq} heads, max abs err {err:.2e}")
+            assert err <= TOL[w.kind], err
+            continue
+        ref = oracle_run(w, mode, metrics=True, n_threads=THREADS)
+        exact, amb = check_tiles(w, ref.metrics, used, w.art, w.tile, S)
+        agree = float(np.mean(used == ref.used))
+        forced = oracle_run(w, "q8" if mode == "q8_art" else "full", forced_used=used, n_threads=THREADS)
+        err = float(np.max(np.abs(o - forced.o)))
+        REPORT.append(
+            f"{name} {mode}: {used.size} (head, split) stops: {exact} unambiguous, {amb} inside the 1e-4 window, "
+            f"{agree:.4f} equal to the oracle's own stop; tiles consumed {tiles.sum() / (n.sum() * w.Hq):.3f} "
+            f"of all; max abs err {err:.2e}")
+        assert err <= TOL[w.kind], err
+        assert agree >= AGREE_FLOOR, agree
