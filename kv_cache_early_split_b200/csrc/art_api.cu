@@ -291,10 +291,12 @@ TcFn tc_pick(int mode, int G, int n_probe, bool ord, bool paged, int ncw) {
   return artk::tc::kernel_gp8(mode, pc, ord, paged, ncw);
 }
 
-// ART controller warps for cluster size C: two when one round's rule replay needs two or more
-// passes of a warp over the heads (a pass covers 32 / (C * tiles per block) heads).
+// ART controller for cluster size C: 0 (the sequential controller) for a single CTA; else the scan
+// controller, on two warps when one round's rule replay needs two or more passes of a warp over the
+// heads (a pass covers 32 / (C * tiles per block) heads).
 int tc_ncw(int mode, int G, int C, int kt) {
   if (mode != artk::MODE_ART) return 1;
+  if (C == 1) return 0;
   const int hpp = 32 / (C * kt);
   return (G + hpp - 1) / hpp >= 2 ? 2 : 1;
 }

@@ -333,3 +333,30 @@ __device__ __forceinline__ bool mbar_try_wait_cluster_sleep(uint32_t bar, uint32
   return ok != 0;
 }
 }  // namespace artk
+
+namespace artk {
+// Four consecutive floats of shared memory: of this CTA (cluster = false, `addr` a CTA-local
+// shared address) or of any CTA of the cluster (`addr` from map_to_rank).
+__device__ __forceinline__ float4 ld_smem_v4(uint32_t addr, bool cluster) {
+  float4 v;
+  if (cluster)
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+  else
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr)
+                 : "memory");
+  return v;
+}
+__device__ __forceinline__ float ld_smem_f32(uint32_t addr, bool cluster) {
+  float v;
+  if (cluster)
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  else
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+}  // namespace artk

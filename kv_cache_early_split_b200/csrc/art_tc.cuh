@@ -108,21 +108,31 @@ constexpr uint32_t OFF_CTL = OFF_DEC + 4 * NSLOT * GMAX;               // [16] i
 constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;                          // [GMAX][RF_SIZE] float
 constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;               // [GMAX][RI_SIZE] int
 constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;              // [D] int8
-constexpr uint32_t OFF_PUB = OFF_L2P + D;  // [NSLOT][KT][GP][2+PC] float, sized per kernel (Pub)
-// Publication slots of a kernel with GP heads per kv head and probe capacity PC:
-// per tile and head, (m_t, l_t) then the PC probe lanes of O_t.
+constexpr uint32_t OFF_PUB = OFF_L2P + D;  // [NSLOT] publication slots, sized per kernel (Pub)
+static_assert(OFF_RF % 16 == 0 && OFF_PUB % 16 == 0 && OFF_TST % 16 == 0 && OFF_DEC % 16 == 0, "vector access");
+// Publication slot of a kernel with GP heads per kv head and probe capacity PC, one entry per
+// (tile i of the block, head g), e = i * GP + g:  m_t[KT_MAX * GP], l_t[KT_MAX * GP], then the PC
+// probe lanes of O_t per entry (rows of PC floats, 16-byte aligned for vector loads).
 template <int GP, int PC>
 struct Pub {
-  static constexpr uint32_t ENTRY = 2 + PC;
-  static constexpr uint32_t SLOT = 4 * KT_MAX * GP * ENTRY;
+  static constexpr uint32_t NE = KT_MAX * GP;
+  static constexpr uint32_t OFF_L = NE, OFF_X = 2 * NE;  // float offsets inside a slot
+  static constexpr uint32_t SLOT = 4 * NE * (2 + PC);
   static constexpr uint32_t SMEM_BYTES = OFF_PUB + NSLOT * SLOT + 1024;  // + alignment slack
+  static_assert((4 * OFF_X) % 16 == 0 && SLOT % 16 == 0, "probe rows 16-byte aligned");
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 };
 constexpr uint32_t SMEM_BYTES = Pub<GMAX, PMAX>::SMEM_BYTES;  // the largest instantiation
 // final reduction (aliases stage 0 after the pipeline has drained):
-// [NWG][GMAX][D] numerators, then [NWG][GMAX] m, [NWG][GMAX] l, [4] ints
+// [NWG][GMAX][D] numerators, then [NWG][GMAX] m, [NWG][GMAX] l, [4] ints (slot 0 ends up holding
+// the CTA's combined state)
 constexpr uint32_t OFF_RED = 0;
 constexpr uint32_t RED_M = NWG * GMAX * D, RED_L = RED_M + NWG * GMAX, RED_I = RED_L + NWG * GMAX;
+// merge tables (floats): [CMAX][GMAX] per-rank maxima / weights, [CMAX][GMAX] per-rank
+// denominators, [GMAX] merged max, [GMAX] merged denominators
+constexpr uint32_t RED_W = RED_I + 8, RED_LT = RED_W + CMAX * GMAX, RED_MG = RED_LT + CMAX * GMAX,
+                   RED_DN = RED_MG + GMAX;
+static_assert(4 * (RED_DN + GMAX) <= STAGE_BYTES, "final reduction fits stage 0");
 enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, CTL_TREAD, CTL_TMEM,
              CTL_STOPFLAG = 8 };  // [2 rounds][2 controller warps]: all of the warp's heads stopped
 
@@ -183,7 +193,8 @@ __device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parit
 // PC: probe-lane capacity of the rule replay (16 or 32, lanes beyond n_probe are zero).
 // ORD / PAGED: a traversal sequence / a paged cache; a kernel without them carries none of that
 // code (the ART epilogue and the producer are sensitive to their instruction footprint).
-// NCW: ART controller warps (2 when a round's replay needs two or more passes over the heads).
+// NCW: the ART controller: 0 = the sequential controller of a single-CTA cluster, 1 or 2 = the scan
+// controller warps of a cluster (2 when a round's replay needs two or more passes over the heads).
 template <int GP, int MODE, int PC, bool ORD, bool PAGED, int NCW>
 __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
@@ -489,20 +500,50 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       l_own[g] = a * l_own[g] + bt * lt;
       m_own[g] = M;
     };
-    // merge the pending tiles `pt` (ntlp of them) of round rp by that round's decision
+    // merge the pending tiles `pt` (ntlp of them) of round rp by that round's decision.  The
+    // decisions and tile statistics are loaded first (vector loads), then every (tile, head) is
+    // merged without branches: a tile past its head's stop tile merges with weight 0.
     auto merge_round = [&](int rp, const float (&pt)[KT_MAX][GP], int ntlp) {
       const int sp = rp % NSLOT;
+      int dv[GP];
+      float tm[KT_MAX][GP], tl[KT_MAX][GP];
+      if constexpr (GP >= 4) {
+#pragma unroll
+        for (int g = 0; g < GP; g += 4) {
+          const int4 d4 = *reinterpret_cast<const int4*>(dec + sp * GMAX + g);
+          dv[g] = d4.x, dv[g + 1] = d4.y, dv[g + 2] = d4.z, dv[g + 3] = d4.w;
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < GP; ++g) dv[g] = dec[sp * GMAX + g];
+      }
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i) {
-        if (i < ntlp) {
-          const int q = rank * KT + i;
+        const float* ts = tst + (sp * KT_MAX + i) * GMAX * 2;
+        if constexpr (GP >= 2) {
 #pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            const int d = dec[sp * GMAX + g];
-            if (g < G && (d == -1 || (d >= 0 && q <= d)))
-              merge_tile(g, tst[(sp * KT_MAX + i) * GMAX * 2 + g * 2], tst[(sp * KT_MAX + i) * GMAX * 2 + g * 2 + 1],
-                         pt[i][g]);
+          for (int g = 0; g < GP; g += 2) {
+            const float4 v = *reinterpret_cast<const float4*>(ts + 2 * g);
+            tm[i][g] = v.x, tl[i][g] = v.y, tm[i][g + 1] = v.z, tl[i][g + 1] = v.w;
           }
+        } else {
+          tm[i][0] = ts[0], tl[i][0] = ts[1];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < KT_MAX; ++i) {
+        const int q = rank * KT + i;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          const int d = dv[g];
+          const bool take = i < ntlp && g < G && (d == -1 || (d >= 0 && q <= d));
+          // statistics of a tile that is not taken may be stale or unset: select, never scale by 0
+          const float M = fmaxf(m_own[g], tm[i][g]);
+          const float a = rescale_fast(m_own[g], M), bt = rescale_fast(tm[i][g], M);
+          const float na = a * acc[g] + bt * pt[i][g], nl = a * l_own[g] + bt * tl[i][g];
+          acc[g] = take ? na : acc[g];
+          l_own[g] = take ? nl : l_own[g];
+          m_own[g] = take ? M : m_own[g];
         }
       }
     };
@@ -601,12 +642,17 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           }
           if (g < G) merge_tile(g, mt, lt, ot[0][g]);
         }
-      } else if (leader) {  // tile statistics for the round's publication and merge
-#pragma unroll
-        for (int i = 0; i < KT_MAX; ++i) {
-          if (i >= ntl) continue;
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
+      } else {
+        // ART: this block's tiles go to publication slot jl % NSLOT.  One thread per (tile, head)
+        // forms the tile's (m_t, l_t) from the per-warp maxima and sums and writes it to the slot
+        // and to the CTA's own copy (tst, read by the merge); the threads of the probe lanes write
+        // their lanes of O_t.  The warpgroup barrier that follows orders these writes before the
+        // round is signalled.
+        const int sl = jl % NSLOT;
+        float* ps = pub + sl * (PB::SLOT / 4);
+        if (er < KT_MAX * GP) {
+          const int i = er / GP, g = er % GP;
+          if (i < ntl && g < G) {
             float mt = -INFINITY, lt = 0.f;
 #pragma unroll
             for (int w = 0; w < 4; ++w)
@@ -614,9 +660,19 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
                 mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
                 lt += wsum[(bb * 4 + w) * GMAX + g];
               }
-            tst[((jl % NSLOT) * KT_MAX + i) * GMAX * 2 + g * 2 + 0] = mt;
-            tst[((jl % NSLOT) * KT_MAX + i) * GMAX * 2 + g * 2 + 1] = lt;
+            tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2 + 0] = mt;
+            tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2 + 1] = lt;
+            ps[er] = mt;
+            ps[PB::OFF_L + er] = lt;
           }
+        }
+        const int pi = l2p[er];
+        if (pi >= 0) {
+#pragma unroll
+          for (int i = 0; i < KT_MAX; ++i)
+#pragma unroll
+            for (int g = 0; g < GP; ++g)
+              if (i < ntl && g < G) ps[PB::OFF_X + (i * GP + g) * PC + pi] = ot[i][g];
         }
       }
       return true;
@@ -658,29 +714,18 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         const int er_round = ctl[CTL_EXIT_ROUND];  // written before the exit flag, never changed after
         m_hi = aborted ? -1 : min(r, er_round);
       } else {
-        // publish round r: (m_t, l_t, probe lanes of O_t) of this CTA's tiles
+        // round r is in its publication slot (written by o_phase; the barrier above ordered the
+        // warpgroup's writes): signal every CTA's controller.  Across CTAs the slot is read through
+        // distributed shared memory, so the signalling thread first fences at cluster scope; a
+        // single CTA needs only the barrier's own release.
         const int sl = r % NSLOT;
-        float* ps = pub + sl * (PB::SLOT / 4);
-        const int pi = l2p[er];
-#pragma unroll
-        for (int i = 0; i < KT_MAX; ++i) {
-          if (i >= ntl) continue;
-#pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            if (g < G) {
-              float* e = ps + (i * GP + g) * PB::ENTRY;
-              if (leader) {
-                e[0] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2];
-                e[1] = tst[(sl * KT_MAX + i) * GMAX * 2 + g * 2 + 1];
-              }
-              if (pi >= 0) e[2 + pi] = ot[i][g];
-            }
+        if (er < C) {
+          if (C > 1) {
+            fence_acq_rel_cluster();
+            mbar_arrive_cluster_relaxed(map_to_rank(bar(B_XFULL + sl), er));
+          } else {
+            mbar_arrive(bar(B_XFULL + sl));
           }
-        }
-        named_barrier(bar_epi, 128);
-        if (er < C) {  // one thread per peer: make the slot visible, then signal that CTA
-          fence_acq_rel_cluster();
-          mbar_arrive_cluster_relaxed(map_to_rank(bar(B_XFULL + sl), er));
         }
         m_hi = (r + NWG >= iters) ? r : r - LAG;
       }
@@ -693,15 +738,118 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       ntl_p = ntl;
     }
   } else if (warp == WARP_CTL || (NCW == 2 && warp == WARP_CTL + 1)) {
+    // NCW = 0: the sequential controller of a single-CTA cluster; 1 or 2: the scan controller(s)
+    // of a cluster (two warps when a round's replay needs two or more passes over the heads)
     // ------------------------------------------------------------ ART controller(s)
     const int TQ = C * KT;    // tiles per round (power of two <= 32)
     const int HPP = 32 / TQ;  // heads per pass
-    constexpr int ncw = NCW;  // the host picks 2 when a round needs two or more passes over the heads
+    constexpr int ncw = NCW > 0 ? NCW : 1;  // the host picks 2 when a round needs two or more passes over the heads
     const int cw = (NCW == 1) ? 0 : warp - WARP_CTL;
-    if (ART && cw < ncw) {
+    if constexpr (ART && NCW == 0) {
+      // Single-CTA cluster: a round is this CTA's KT tiles, replayed one after another.  Head g
+      // owns LPH lanes holding CPL probe lanes each; its carried state (m, l, probe accumulators,
+      // previous probe and norm, run) lives in registers across rounds.  Norms and the direction
+      // change are reduced over the head's lanes with xor shuffles.
+      constexpr int LPH = (32 / GP) < PC ? (32 / GP) : PC;
+      constexpr int CPL = PC / LPH;
+      const int g = lane / LPH, j = lane % LPH;
+      const bool active = g < G;
+      const int gs = active ? g : 0;
+      float m = -INFINITY, l = 0.f, nrmp = 0.f, a[CPL], xp[CPL];
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) a[k] = xp[k] = 0.f;
+      int run = 0;
+      bool stopped = !active;
+      auto group_sum = [&](float v) {
+#pragma unroll
+        for (int o = LPH / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        return v;
+      };
+#pragma unroll 1
+      for (int r = 0; r < R; ++r) {
+        const int sl = r % NSLOT;
+        int okw = 1;
+        if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r / NSLOT) & 1, ctl, false, p.ws_status, false);
+        if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+        const int nv = max(0, min(KT, t1 - (t0 + r * KT)));
+        const float* ps = pub + sl * (PB::SLOT / 4);
+        const bool was_stopped = stopped;
+        int stop_q = -1;
+#pragma unroll 1
+        for (int q = 0; q < nv; ++q) {
+          const int e = q * GP + gs;
+          const float mt = ps[e], lt = ps[PB::OFF_L + e];
+          float at[CPL];
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) at[k] = ps[PB::OFF_X + e * PC + j * CPL + k];
+          const float M = fmaxf(m, mt);
+          const float al = rescale_fast(m, M), be = rescale_fast(mt, M);
+          const float nl = al * l + be * lt;
+          const float inv_l = __fdividef(1.f, nl);
+          float na[CPL], x[CPL], sq = 0.f;
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            na[k] = al * a[k] + be * at[k];
+            x[k] = na[k] * inv_l;
+            sq = fmaf(x[k], x[k], sq);
+          }
+          const float nrm = __fsqrt_rn(group_sum(sq));
+          const bool both = nrm > 0.f && nrmp > 0.f;
+          const float in = both ? __fdividef(1.f, nrm) : 0.f, ip = both ? __fdividef(1.f, nrmp) : 0.f;
+          float dq = 0.f;
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const float dl = x[k] * in - xp[k] * ip;
+            dq = fmaf(dl, dl, dq);
+          }
+          const float dd2 = group_sum(dq);
+          const float d_scale = fabsf(nrm - nrmp);
+          const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd2);
+          const bool hold = (d_scale < p.eps_scale) && (d_dir < p.eps_dir);
+          if (!stopped) {  // a stopped head keeps its state (it still takes part in the shuffles)
+            m = M;
+            l = nl;
+            nrmp = nrm;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+              a[k] = na[k];
+              xp[k] = x[k];
+            }
+            run = hold ? run + 1 : 0;
+            if (run >= p.patience) {
+              stopped = true;
+              stop_q = q;
+            }
+          }
+        }
+        if (active && j == 0) {
+          dec[sl * GMAX + g] = was_stopped ? -2 : stop_q;
+          if (stop_q >= 0) {
+            ri[g * RI_SIZE + RI_STOPPED] = 1;
+            ri[g * RI_SIZE + RI_USED] = r * KT + stop_q + 1;
+          }
+        }
+        const bool all = __ballot_sync(0xffffffffu, active && !stopped) == 0u;
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence_block();
+          mbar_arrive(bar(B_DEC + sl));
+          if (all) {
+            ctl[CTL_EXIT_ROUND] = r;
+            __threadfence_block();
+            ctl[CTL_EXIT] = 1;
+          }
+        }
+        __syncwarp();
+        if (all) break;
+      }
+    } else if (ART && cw < ncw) {
       const int hh = lane / TQ, q = lane % TQ;
       const int c = q / KT, i = q % KT;
+      const int seg0 = hh * TQ;  // first lane of this head's segment
       const unsigned segmask = (TQ == 32) ? 0xffffffffu : ((1u << TQ) - 1u);
+      const bool remote = C > 1;  // the tile's publication lives in CTA c of the cluster
+      const uint32_t pub_c = remote ? map_to_rank(smem_u32(pub), c) : smem_u32(pub);
       for (int r = 0; r < R; ++r) {
         const int sl = r % NSLOT;
         int okw = 1;
@@ -710,7 +858,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         if constexpr (NCW == 2) okw = named_barrier_and(BAR_CTL, 64, okw != 0);  // both warps leave together
         if (!okw) break;
         const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
-        const uint32_t slot_base = smem_u32(pub) + sl * PB::SLOT;
+        const uint32_t slot = pub_c + sl * PB::SLOT;
         for (int g0 = cw * HPP; g0 < G; g0 += ncw * HPP) {
           const int g = g0 + hh;
           const bool active = g < G;
@@ -723,10 +871,15 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
           for (int k = 0; k < PC; ++k) a[k] = 0.f;
           if (valid) {  // this tile's (m, l, probe) from the CTA that computed it
-            const uint32_t src = map_to_rank(slot_base + ((i * GP + g) * PB::ENTRY) * 4, c);
-            ld_dsmem_v2(src, m, l);
+            const uint32_t e = static_cast<uint32_t>(i * GP + g);
+            m = ld_smem_f32(slot + 4 * e, remote);
+            l = ld_smem_f32(slot + 4 * (PB::OFF_L + e), remote);
+            const uint32_t px = slot + 4 * (PB::OFF_X + e * PC);
 #pragma unroll
-            for (int k = 0; k < PC; k += 2) ld_dsmem_v2(src + 8 + 4 * k, a[k], a[k + 1]);
+            for (int k = 0; k < PC; k += 4) {
+              const float4 v = ld_smem_v4(px + 4 * k, remote);
+              a[k] = v.x, a[k + 1] = v.y, a[k + 2] = v.z, a[k + 3] = v.w;
+            }
           }
           // inclusive scan of the merge over the round's tiles (segments of TQ lanes)
           float cs[5], co[5];
@@ -759,59 +912,68 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
             }
           }
           // prepend the state carried over from earlier rounds
-          const float mR = R_f[RF_M], lR = R_f[RF_L];
+          const float4 st = *reinterpret_cast<const float4*>(R_f);  // m, l, |x_prev|, -
+          const float mR = st.x, lR = st.y;
           const float Mf = fmaxf(mR, m);
           const float aR = rescale_fast(mR, Mf), aS = rescale_fast(m, Mf);
           l = aR * lR + aS * l;
           m = Mf;
           const float inv_l = __fdividef(1.f, l);
-          float x[PC], nrm2 = 0.f;
+          float x[PC], sq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int k = 0; k < PC; ++k) {
-            a[k] = aR * R_f[RF_A + k] + aS * a[k];
-            x[k] = a[k] * inv_l;
-            nrm2 = fmaf(x[k], x[k], nrm2);
+          for (int k = 0; k < PC; k += 4) {
+            const float4 ar = *reinterpret_cast<const float4*>(R_f + RF_A + k);
+            a[k] = aR * ar.x + aS * a[k];
+            a[k + 1] = aR * ar.y + aS * a[k + 1];
+            a[k + 2] = aR * ar.z + aS * a[k + 2];
+            a[k + 3] = aR * ar.w + aS * a[k + 3];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              x[k + u] = a[k + u] * inv_l;
+              sq[u] = fmaf(x[k + u], x[k + u], sq[u]);
+            }
           }
-          const float nrm = __fsqrt_rn(nrm2);
+          const float nrm = __fsqrt_rn((sq[0] + sq[1]) + (sq[2] + sq[3]));
           float nrmp = __shfl_up_sync(0xffffffffu, nrm, 1, TQ);
-          if (q == 0) nrmp = R_f[RF_NRM];
+          if (q == 0) nrmp = st.z;
           const bool both = nrm > 0.f && nrmp > 0.f;
           const float in = both ? __fdividef(1.f, nrm) : 0.f, ip = both ? __fdividef(1.f, nrmp) : 0.f;
-          float dd2 = 0.f;
+          float dq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int k = 0; k < PC; ++k) {
-            float xp = __shfl_up_sync(0xffffffffu, x[k], 1, TQ);
-            if (q == 0) xp = R_f[RF_XP + k];
-            const float dl = x[k] * in - xp * ip;
-            dd2 = fmaf(dl, dl, dd2);
+          for (int k = 0; k < PC; k += 4) {
+            const float4 xr = *reinterpret_cast<const float4*>(R_f + RF_XP + k);
+            const float xrv[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float xp = __shfl_up_sync(0xffffffffu, x[k + u], 1, TQ);
+              if (q == 0) xp = xrv[u];
+              const float dl = x[k + u] * in - xp * ip;
+              dq[u] = fmaf(dl, dl, dq[u]);
+            }
           }
+          const float dd2 = (dq[0] + dq[1]) + (dq[2] + dq[3]);
           const float d_scale = fabsf(nrm - nrmp);
           const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd2);
           const bool hold = valid && (d_scale < p.eps_scale) && (d_dir < p.eps_dir);
-          const unsigned seg = (__ballot_sync(0xffffffffu, hold) >> (hh * TQ)) & segmask;
-          int run = stopped_before ? 0 : R_i[RI_RUN];
-          int stop = -1;
-          if (!stopped_before) {
-            for (int qq = 0; qq < nv; ++qq) {
-              run = ((seg >> qq) & 1u) ? run + 1 : 0;
-              if (run >= p.patience) {
-                stop = qq;
-                break;
-              }
-            }
-          }
-          __syncwarp();
+          // patience, for every tile of the round at once: the run ending at tile q is the number
+          // of consecutive holding tiles up to q (plus the carried run when they reach back to the
+          // round's first tile); the head stops at the first tile whose run reaches the patience.
+          const unsigned hbits = (__ballot_sync(0xffffffffu, hold) >> seg0) & segmask;
+          const int run0 = stopped_before ? 0 : R_i[RI_RUN];
+          const unsigned zeros = ~hbits & ((1u << q) - 1u);
+          const int runq = !((hbits >> q) & 1u) ? 0 : (zeros == 0u ? run0 + q + 1 : q - (31 - __clz(zeros)));
+          const bool reach = hold && runq >= p.patience;
+          const unsigned rbits = (__ballot_sync(0xffffffffu, reach) >> seg0) & segmask;
+          const int stop = (!stopped_before && rbits != 0u) ? __ffs(rbits) - 1 : -1;
           const int srcq = (stop >= 0) ? stop : nv - 1;
           if (active && !stopped_before && nv > 0 && q == srcq) {
-            R_f[RF_M] = m;
-            R_f[RF_L] = l;
-            R_f[RF_NRM] = nrm;
+            *reinterpret_cast<float4*>(R_f) = make_float4(m, l, nrm, 0.f);
 #pragma unroll
-            for (int k = 0; k < PC; ++k) {
-              R_f[RF_A + k] = a[k];
-              R_f[RF_XP + k] = x[k];
+            for (int k = 0; k < PC; k += 4) {
+              *reinterpret_cast<float4*>(R_f + RF_A + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
+              *reinterpret_cast<float4*>(R_f + RF_XP + k) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
             }
-            R_i[RI_RUN] = run;
+            R_i[RI_RUN] = runq;
             if (stop >= 0) {
               R_i[RI_STOPPED] = 1;
               R_i[RI_USED] = r * TQ + stop + 1;
@@ -870,61 +1032,88 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   __syncthreads();  // (2) the ring is quiet: stage 0 can hold the final reduction
   float* red = reinterpret_cast<float*>(sm + OFF_RED);
   int* redi = reinterpret_cast<int*>(sm + OFF_RED + 4 * RED_I);
-  if (warp >= WARP_EPI0) {  // each warpgroup leaves its own online-softmax state
-    const int wg = (warp - WARP_EPI0) >> 2;
-    const int er = 32 * (warp & 3) + lane;
+  // 1. the CTA's two warpgroup states become one (warpgroup 1 hands its state to warpgroup 0)
+  const int er_ = 32 * (warp & 3) + lane;
+  if (warp >= WARP_EPI0 + 4) {
 #pragma unroll
     for (int g = 0; g < GP; ++g)
-      if (g < G) red[(wg * GMAX + g) * D + er] = acc[g];
-    if (er == 0) {
+      if (g < G) red[(GMAX + g) * D + er_] = acc[g];
+    if (er_ == 0) {
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
-        red[RED_M + wg * GMAX + g] = m_own[g];
-        red[RED_L + wg * GMAX + g] = l_own[g];
+        red[RED_M + GMAX + g] = m_own[g];
+        red[RED_L + GMAX + g] = l_own[g];
       }
     }
   }
   if (tid == 0) redi[0] = ctl[CTL_TREAD];
-
-  // ---------------------------------------------------------------- cluster merge and output
-  if (C > 1) cluster_sync_all(); else __syncthreads();
-  if (rank == 0) {
-    const uint32_t rb = smem_u32(red);
-    for (int idx = tid; idx < G * D; idx += NTHR) {
-      const int g = idx / D, dd = idx % D;
-      // the C x NWG partial states of head g (C > 1: read from each rank's shared memory)
-      auto part_f = [&](int cc, uint32_t off) -> float {
-        return (C > 1) ? ld_dsmem_f32(map_to_rank(rb + 4 * off, cc)) : red[off];
-      };
-      float M = -INFINITY;
-      for (int cc = 0; cc < C; ++cc)
+  __syncthreads();
+  if (warp >= WARP_EPI0 && warp < WARP_EPI0 + 4) {
 #pragma unroll
-        for (int w = 0; w < NWG; ++w) M = fmaxf(M, part_f(cc, RED_M + w * GMAX + g));
-      float den = 0.f, num = 0.f;
-      for (int cc = 0; cc < C; ++cc) {
-#pragma unroll
-        for (int w = 0; w < NWG; ++w) {
-          const float mc = part_f(cc, RED_M + w * GMAX + g);
-          if (mc == -INFINITY) continue;
-          const float lc = part_f(cc, RED_L + w * GMAX + g);
-          const float ac = part_f(cc, (w * GMAX + g) * D + dd);
-          const float wt = exp2f(mc - M);
-          den += wt * lc;
-          num += wt * ac;
-        }
-      }
-      const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + g;
-      if (p.S == 1) {
-        p.o[hq * D + dd] = bad_len ? __int_as_float(0x7fc00000) : num / den;
-      } else {
-        float* part = p.ws_partial + (hq * p.S + split) * (D + 2);
-        if (dd == 0) {
-          part[0] = M;
-          part[1] = den;
-        }
-        part[2 + dd] = num;
+    for (int g = 0; g < GP; ++g) {
+      if (g >= G) continue;
+      const float m1 = red[RED_M + GMAX + g], l1 = red[RED_L + GMAX + g];
+      const float M = fmaxf(m_own[g], m1);
+      const float w0 = rescale_fast(m_own[g], M), w1 = rescale_fast(m1, M);
+      red[g * D + er_] = w0 * acc[g] + w1 * red[(GMAX + g) * D + er_];
+      if (er_ == 0) {
+        red[RED_M + g] = M;
+        red[RED_L + g] = w0 * l_own[g] + w1 * l1;
       }
     }
+  }
+
+  // ---------------------------------------------------------------- cluster merge and output
+  // 2. every CTA of the cluster merges a share of the (head, d) outputs over the C states: the
+  //    per-rank weights 2^(m_c - M) and the denominators are tabulated once, then each output
+  //    element takes C loads from the ranks' shared memory
+  if (C > 1) cluster_sync_all(); else __syncthreads();
+  const uint32_t rb = smem_u32(red);
+  float* wt = red + RED_W;    // [CMAX][GMAX]: the ranks' maxima, then their weights 2^(m_c - M)
+  float* lt = red + RED_LT;   // [CMAX][GMAX] the ranks' denominators
+  float* mg = red + RED_MG;   // [GMAX] merged max
+  float* den = red + RED_DN;  // [GMAX] merged denominator
+  if (tid < C * G) {
+    const int cc = tid / G, g = tid % G;
+    wt[cc * GMAX + g] = (C > 1) ? ld_dsmem_f32(map_to_rank(rb + 4 * (RED_M + g), cc)) : red[RED_M + g];
+    lt[cc * GMAX + g] = (C > 1) ? ld_dsmem_f32(map_to_rank(rb + 4 * (RED_L + g), cc)) : red[RED_L + g];
+  }
+  __syncthreads();
+  if (tid < G) {
+    float M = -INFINITY;
+    for (int cc = 0; cc < C; ++cc) M = fmaxf(M, wt[cc * GMAX + tid]);
+    float dsum = 0.f;
+    for (int cc = 0; cc < C; ++cc) {
+      const float w = rescale_fast(wt[cc * GMAX + tid], M);
+      wt[cc * GMAX + tid] = w;
+      dsum += w * lt[cc * GMAX + tid];
+    }
+    mg[tid] = M;
+    den[tid] = dsum;
+  }
+  __syncthreads();
+  const int share = (G * D + C - 1) / C;
+  for (int idx = rank * share + tid; idx < min(G * D, (rank + 1) * share); idx += NTHR) {
+    const int g = idx / D, dd = idx % D;
+    float num = 0.f;
+#pragma unroll 4
+    for (int cc = 0; cc < C; ++cc) {
+      const float ac = (C > 1) ? ld_dsmem_f32(map_to_rank(rb + 4 * (g * D + dd), cc)) : red[g * D + dd];
+      num = fmaf(wt[cc * GMAX + g], ac, num);
+    }
+    const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + g;
+    if (p.S == 1) {
+      p.o[hq * D + dd] = bad_len ? __int_as_float(0x7fc00000) : num / den[g];
+    } else {
+      float* part = p.ws_partial + (hq * p.S + split) * (D + 2);
+      if (dd == 0) {
+        part[0] = mg[g];
+        part[1] = den[g];
+      }
+      part[2 + dd] = num;
+    }
+  }
+  if (rank == 0) {
     if (tid < G) {
       const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + tid;
       const int used = bad_len ? 0 : (ART ? ri[tid * RI_SIZE + RI_USED] : ns);

@@ -10,9 +10,11 @@ namespace tc {
 using TcFn = void (*)(TcParams);
 
 // The kernel for GP heads per kv head: mode MODE_FULL / MODE_ART, probe capacity pc (16 or 32, ART),
-// a traversal sequence (ord, ART only), a paged cache (paged), ncw ART controller warps (1 or 2).
+// a traversal sequence (ord, ART only), a paged cache (paged), the ART controller ncw (0: sequential,
+// single-CTA cluster; 1 or 2: scan controller warps).
 template <int GP, int MODE, int PC, bool ORD, bool PAGED>
 TcFn pick_ncw(int ncw) {
+  if (ncw == 0) return &art_decode_tc_kernel<GP, MODE, PC, ORD, PAGED, 0>;
   return ncw == 2 ? &art_decode_tc_kernel<GP, MODE, PC, ORD, PAGED, 2> : &art_decode_tc_kernel<GP, MODE, PC, ORD, PAGED, 1>;
 }
 
