@@ -360,3 +360,19 @@ __device__ __forceinline__ float ld_smem_f32(uint32_t addr, bool cluster) {
   return v;
 }
 }  // namespace artk
+
+namespace artk {
+// Non-blocking check of phase `parity` (mbarrier.test_wait never suspends the thread, unlike
+// try_wait): for a thread that polls several barriers.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+}  // namespace artk

@@ -95,9 +95,10 @@ constexpr uint32_t OFF_Q = NSTG * STAGE_BYTES;  // 2 halves x 2 KiB
 constexpr uint32_t OFF_P = OFF_Q + 4096;        // 2 buffers x 4 KiB
 constexpr uint32_t OFF_BAR = OFF_P + 8192;      // mbarriers
 enum : int {
-  B_FULL = 0, B_EMPTY = B_FULL + NSTG, B_SFULL = B_EMPTY + NSTG, B_SFREE = B_SFULL + 2, B_PFULL = B_SFREE + 2,
-  B_OFULL = B_PFULL + 2, B_OFREE = B_OFULL + 2, B_XFULL = B_OFREE + 2, B_DEC = B_XFULL + NSLOT,
-  B_DRAIN = B_DEC + NSLOT, B_COUNT = B_DRAIN + 1
+  B_FULL = 0, B_EMPTY = B_FULL + NSTG, B_SFULL = B_EMPTY + NSTG, B_SFREE = B_SFULL + 2,
+  B_OFULL = B_SFREE + 2, B_XFULL = B_OFULL + 2, B_DEC = B_XFULL + NSLOT,
+  B_DRAIN = B_DEC + NSLOT,  // [3]: tensor-core ops of the MMA warp, of warpgroup 0's and 1's leaders
+  B_COUNT = B_DRAIN + 3
 };
 static_assert(B_COUNT * 8 <= 512, "barrier area");
 constexpr uint32_t OFF_WRED = OFF_BAR + 512;                           // [2][4][GMAX] per-warp maxima
@@ -137,6 +138,9 @@ enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, 
              CTL_STOPFLAG = 8 };  // [2 rounds][2 controller warps]: all of the warp's heads stopped
 
 __device__ __forceinline__ uint32_t s_col(int b) { return 16u * b; }
+// instruction descriptors: scores S^T = K . Q^T (both K-major); output O_t^T = V_t^T . P_t^T (both MN-major)
+constexpr uint32_t idS = idesc_bf16(128, 16, false, false);
+constexpr uint32_t idO = idesc_bf16(128, 16, true, true);
 __device__ __forceinline__ uint32_t o_col(int b, int i) { return 32u + 32u * b + 16u * i; }
 
 // A wait gives up after this many SM clock cycles (about one second at B200 clocks).
@@ -164,6 +168,20 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
       atomicOr(status, kStatusTimeout);
       ctl[CTL_ABORT] = 1;
       return false;
+    }
+  }
+}
+
+// Wait for asynchronous work the CTA has in flight (copies into its shared memory, tensor-core
+// ops on its tensor memory) before that memory is reused or released.  Bounded by the wait limit
+// only: a CTA that aborted still waits for what it issued.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_sleep(bar, parity, kSuspendNs)) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(status, kStatusTimeout);
+      return;
     }
   }
 }
@@ -265,15 +283,13 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_SFULL + s), 1);
       mbar_init(bar(B_SFREE + s), 128);
-      mbar_init(bar(B_PFULL + s), 128);
       mbar_init(bar(B_OFULL + s), 1);
-      mbar_init(bar(B_OFREE + s), 128);
     }
     for (int s = 0; s < NSLOT; ++s) {
       mbar_init(bar(B_XFULL + s), C);
       mbar_init(bar(B_DEC + s), 1);
     }
-    mbar_init(bar(B_DRAIN), 1);
+    for (int s = 0; s < 3; ++s) mbar_init(bar(B_DRAIN + s), 1);
     fence_mbar_init();
     if (bad_len && rank == 0) atomicOr(p.ws_status, kStatusSeqLen);
   }
@@ -416,50 +432,34 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, 16, false, false);
-      constexpr uint32_t idO = idesc_bf16(128, 16, true, true);
       const uint32_t q_addr = smem_u32(sm + OFF_Q);
+      // The scores of every own block, in order: K/V landed, S buffer free.  (The PV product of
+      // a block is issued by the leader of the epilogue warpgroup that wrote its weights.)
+      // Descriptors are built once per operand buffer and stepped by constant offsets: the
+      // address field (bits 0-13, 16-byte units) of a shared-memory address below 256 KB never
+      // carries into the next field.
+      const uint64_t qd0 = smem_desc(q_addr, 16, 1024, 2);
       int consumed = 0;
-      auto issue_scores = [&](int jl) -> bool {
+      for (int jl = 0; jl < my_blocks; ++jl) {
         const int stage = jl % NSTG, bb = jl & 1;
-        if (!wait_phase(bar(B_FULL + stage), (jl / NSTG) & 1, ctl, ART, p.ws_status, false)) return false;
+        if (!wait_phase(bar(B_FULL + stage), (jl / NSTG) & 1, ctl, ART, p.ws_status, false)) break;
         consumed = jl + 1;
-        if (jl >= 2 && !wait_phase(bar(B_SFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status, false)) return false;
+        if (jl >= 2 && !wait_phase(bar(B_SFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status, false)) break;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES);
+        const uint64_t kd0 = smem_desc(smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES), 16, 1024, 2);
+        const uint32_t dcol = tmem + s_col(bb);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t h = kk >> 2, off = (kk & 3) * 32;
-          umma_bf16(tmem + s_col(bb), smem_desc(k_addr + h * 16384 + off, 16, 1024, 2),
-                    smem_desc(q_addr + h * 2048 + off, 16, 1024, 2), idS, kk > 0);
+          constexpr uint32_t kq[8] = {0, 2, 4, 6, 1024, 1026, 1028, 1030};  // (h * 16384 + (kk & 3) * 32) / 16
+          constexpr uint32_t qq[8] = {0, 2, 4, 6, 128, 130, 132, 134};      // (h * 2048 + (kk & 3) * 32) / 16
+          umma_bf16(dcol, kd0 + kq[kk], qd0 + qq[kk], idS, kk > 0);
         }
         umma_commit(bar(B_SFULL + bb));
-        return true;
-      };
-      bool ok = (my_blocks == 0) || issue_scores(0);
-      for (int jl = 0; ok && jl < my_blocks; ++jl) {
-        if (jl + 1 < my_blocks && !issue_scores(jl + 1)) break;
-        const int stage = jl % NSTG, bb = jl & 1;
-        if (!wait_phase(bar(B_PFULL + bb), (jl >> 1) & 1, ctl, ART, p.ws_status, false)) break;
-        if (jl >= 2 && !wait_phase(bar(B_OFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status, false)) break;
-        tc_fence_after();
-        const int ntl = block_tiles(jl);
-        const uint32_t v_addr = smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES + 32768);
-        const uint32_t p_addr = smem_u32(sm + OFF_P + bb * 4096);
-        for (int i = 0; i < ntl; ++i) {
-          for (int s = 0; s < TE / 16; ++s) {
-            const int pos0 = i * TE + s * 16;
-            umma_bf16(tmem + o_col(bb, i), smem_desc(v_addr + pos0 * 128, 16384, 1024, 2),
-                      smem_desc(p_addr + (pos0 / 8) * 256, 256, 128, 0), idO, s > 0);
-          }
-        }
-        umma_commit(bar(B_OFULL + bb));
-        umma_commit(bar(B_EMPTY + stage));
       }
       ctl[CTL_CONSUMED] = consumed;
-      // every issued tensor-core op has completed before the drain barrier fires
+      // every tensor-core op this thread issued has completed before the drain barrier fires
       umma_commit(bar(B_DRAIN));
-      wait_phase(bar(B_DRAIN), 0, ctl, false, p.ws_status, false);
+      drain_wait(bar(B_DRAIN), 0, p.ws_status);
     }
     __syncwarp();
   } else if (warp >= WARP_EPI0) {
@@ -606,8 +606,25 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           reinterpret_cast<uint4*>(vrow + 16384)[c] = make_uint4(0, 0, 0, 0);
         }
       }
+      // every thread's weights (and zeroed V rows) are written: the leader issues the PV product
       fence_proxy_async_smem();
-      mbar_arrive(bar(B_PFULL + bb));
+      named_barrier(bar_epi, 128);
+      if (leader) {
+        tc_fence_after();
+        const int ntl = block_tiles(jl);
+        const uint64_t vd0 = smem_desc(smem_u32(sm + OFF_STAGE + stage * STAGE_BYTES + 32768), 16384, 1024, 2);
+        const uint64_t pd0 = smem_desc(smem_u32(sm + OFF_P + bb * 4096), 256, 128, 0);
+        // 8 MMAs of 16 positions each, unrolled so that the operand offsets are constants; MMA u
+        // belongs to tile u * 16 / TE and starts that tile's accumulator when it is its first
+        const int tsh = (TE == 64) ? 6 : 7;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = (u * 16) >> tsh;
+          if (i < ntl) umma_bf16(tmem + o_col(bb, i), vd0 + (u * 128u), pd0 + (u * 32u), idO, ((u * 16) & (TE - 1)) != 0);
+        }
+        umma_commit(bar(B_OFULL + bb));
+        umma_commit(bar(B_EMPTY + stage));
+      }
       return true;
     };
     // O_t readback (thread = d row) for own block jl into ot; tile stats to tst; false if the run ended
@@ -629,8 +646,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
           for (int g = 0; g < GP; ++g) ot[i][g] = ov[g] + ov[8 + g];
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(B_OFREE + bb));
+      tc_fence_before();  // O of buffer bb is read: the next PV into it comes after a warpgroup barrier
       if (!ART) {  // the block is one tile: every thread merges it into its own state
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
@@ -736,6 +752,11 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
         for (int g = 0; g < GP; ++g) pnd[i][g] = ot[i][g];
       ntl_p = ntl;
+    }
+    // every PV product this warpgroup's leader issued has completed before the CTA moves on
+    if (leader) {
+      umma_commit(bar(B_DRAIN + 1 + wg));
+      drain_wait(bar(B_DRAIN + 1 + wg), 0, p.ws_status);
     }
   } else if (warp == WARP_CTL || (NCW == 2 && warp == WARP_CTL + 1)) {
     // NCW = 0: the sequential controller of a single-CTA cluster; 1 or 2: the scan controller(s)
@@ -1027,7 +1048,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   // drain: copies that were issued but never consumed still land in shared memory
   if (warp == WARP_TMA && lane == 0) {
     for (int ord = ctl[CTL_CONSUMED]; ord < ctl[CTL_ISSUED]; ++ord)
-      wait_phase(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, ctl, false, p.ws_status, false);
+      drain_wait(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, p.ws_status);
   }
   __syncthreads();  // (2) the ring is quiet: stage 0 can hold the final reduction
   float* red = reinterpret_cast<float*>(sm + OFF_RED);
