@@ -166,7 +166,7 @@ def hbm_peak():
 # Sources each timed kernel is compiled from, with the C-ABI file that sets its launch shape.
 KERNEL_SOURCES = {
     "art_decode_tc_kernel": ("art_api.cu", "art_device.cuh", "art_kernels.cuh", "art_tc.cuh", "art_tc_pick.cuh",
-                             "art_tc_gp1.cu", "art_tc_gp2.cu", "art_tc_gp4.cu", "art_tc_gp8.cu"),
+                             "art_tc_gp1.cu", "art_tc_gp2.cu", "art_tc_gp4.cu", "art_tc_gp8.cu", "art_tc_q8.cu"),
     "art_decode_kernel": ("art_api.cu", "art_device.cuh", "art_kernels.cuh"),
     "q8_two_pass": ("art_api.cu", "art_device.cuh", "art_kernels.cuh", "art_q8_two.cuh"),
 }

@@ -181,17 +181,41 @@ art_status art_decode_attn_terminate_noalloc(const art_shape* shape, art_dtype d
  * weight exp(s_j - m') is below tau are neither dequantised nor accumulated
  * (puntofijo.es, "La Elegancia de la Omision").  params == NULL runs without
  * ART; otherwise ART as in art_decode_attn_terminate.
- * Without ART and with ws_bytes >= art_q8_workspace_bytes(shape) (and B*Hkv*num_splits
- * <= 65535) the call runs as two streaming passes over the whole GPU: scores and tile maxima
- * from K, then the running maxima m', the skip test and the V products (a tile whose rows all
- * fail the test for every head is not read), then a combine.  Same rule, same outputs and
- * counters; a tile counts as read either way.  With a smaller workspace one pass deals the
- * tiles of a split over a thread-block cluster and exchanges tile maxima every round. */
+ * The library picks one of three implementations (same rule, same outputs within rounding,
+ * same counters; a tile counts as read when it was fetched):
+ *   - without ART and with ws_bytes >= art_q8_workspace_bytes(shape) (and B*Hkv*num_splits
+ *     <= 65535), two streaming passes over the whole GPU: scores and tile maxima from K, then
+ *     the running maxima m', the skip test and the V products (a tile whose rows all fail the
+ *     test for every head is not read), then a combine;
+ *   - otherwise on the tensor cores when d = 128, 3 or 4 query heads per kv head, tile 64 or
+ *     128 and L_max even: int8 codes become f16 MMA operands exactly, the scores take the K
+ *     scales per 32-element block in fp32, the V scales are folded into the weights, and the
+ *     running maxima m' of the V skip are exchanged between the CTAs of a cluster every round;
+ *   - otherwise one pass on the CUDA cores that deals the tiles of a split over a
+ *     thread-block cluster and exchanges tile maxima every round. */
 art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
                                     const uint16_t* k_scale_f16, const int8_t* v_q,
                                     const uint16_t* v_scale_f16, const int32_t* seq_lens,
                                     float tau, const art_params* params, float* o, int32_t* tiles,
                                     void* ws, size_t ws_bytes, void* stream);
+
+/* Implementations of art_decode_attn_q8_skipv, for art_decode_attn_q8_skipv_path. */
+typedef enum {
+  ART_Q8_AUTO = 0,         /* the library's choice (as art_decode_attn_q8_skipv) */
+  ART_Q8_TENSOR_CORE = 1,  /* tcgen05 tensor cores */
+  ART_Q8_TWO_PASS = 2,     /* two streaming passes + combine (no ART; q8 workspace) */
+  ART_Q8_CLUSTER = 3       /* one pass on the CUDA cores over a thread-block cluster */
+} art_q8_path;
+
+/* art_decode_attn_q8_skipv on a named implementation (testing, benchmarking, or pinning one
+ * kernel in production).  Same arguments, plus `path`; ART_ERR_UNSUPPORTED (nothing enqueued)
+ * when that implementation does not take the shape or mode (see art_decode_attn_q8_skipv),
+ * ART_ERR_INVALID_ARG for an unknown path. */
+art_status art_decode_attn_q8_skipv_path(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
+                                         const uint16_t* k_scale_f16, const int8_t* v_q,
+                                         const uint16_t* v_scale_f16, const int32_t* seq_lens, float tau,
+                                         const art_params* params, float* o, int32_t* tiles, void* ws,
+                                         size_t ws_bytes, int32_t path, void* stream);
 
 /* ---- KV tile traversal orders ("Resumen Tecnico: ART", S2.4: ART composes with
  * other KV-cache policies by reordering the traversal sequence of the KV blocks,

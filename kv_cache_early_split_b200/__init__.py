@@ -118,15 +118,21 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
+Q8_PATHS = {"auto": capi.ART_Q8_AUTO, "tensor_core": capi.ART_Q8_TENSOR_CORE, "two_pass": capi.ART_Q8_TWO_PASS,
+            "cluster": capi.ART_Q8_CLUSTER}
+
+
 def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float | None = None, stream=None,
-           check: bool = True, order=None) -> int:
+           check: bool = True, order=None, q8_path: str = "auto") -> int:
     """Launch one decode call on dp's buffers.
 
     mode: "full" | "art" (art_decode_attn_terminate) | "q8" (q8_skipv without ART) |
           "q8_art" (q8_skipv with ART).  order: None, or an int32 device tensor
     [B, Hkv, ceil(L_max/tile)] of tile traversal sequences (mode "art" only:
-    art_decode_attn_terminate_ordered).  Returns the C status code; raises
-    ArtError on a non-zero code when check is True.
+    art_decode_attn_terminate_ordered).  q8_path: for the q8 modes, "auto" (the library's choice)
+    or one implementation, "tensor_core" / "two_pass" / "cluster"
+    (art_decode_attn_q8_skipv_path).  Returns the C status code; raises ArtError on a non-zero
+    code when check is True.
     """
     import torch
 
@@ -156,10 +162,11 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
         params = None
         if mode == "q8_art":
             params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
-        rc = capi.art_decode_attn_q8_skipv(
+        rc = capi.art_decode_attn_q8_skipv_path(
             dp.shape, _ptr(dp.q), _ptr(dp.k), _ptr(dp.k_scale), _ptr(dp.v), _ptr(dp.v_scale), _ptr(dp.seq_lens),
-            dp.tau if tau is None else tau, params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
-        name = "art_decode_attn_q8_skipv"
+            dp.tau if tau is None else tau, params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes,
+            Q8_PATHS[q8_path], st)
+        name = "art_decode_attn_q8_skipv_path"
     else:
         raise ValueError(mode)
     if check and rc != capi.ART_OK:

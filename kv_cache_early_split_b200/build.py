@@ -16,9 +16,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libart_decode.so")
-# art_api.cu holds the C ABI and the CUDA-core kernels; art_tc_gp*.cu the tensor-core instantiations
+# art_api.cu holds the C ABI and the CUDA-core kernels; art_tc_gp*.cu / art_tc_q8.cu the tensor-core
+# instantiations (bf16 per head count, q8)
 SOURCES = [os.path.join(CSRC, f) for f in ("art_api.cu", "art_tc_gp1.cu", "art_tc_gp2.cu", "art_tc_gp4.cu",
-                                           "art_tc_gp8.cu")]
+                                           "art_tc_gp8.cu", "art_tc_q8.cu")]
 DEPS = SOURCES + [
     os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".cuh", ".h"))
 ] + [os.path.join(INCLUDE, "art_decode.h")]

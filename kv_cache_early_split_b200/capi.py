@@ -25,6 +25,7 @@ ART_ERR_PAGE = -8
 ART_F32 = 0
 ART_BF16 = 1
 ART_KV_F32, ART_KV_BF16, ART_KV_Q8 = 0, 1, 2
+ART_Q8_AUTO, ART_Q8_TENSOR_CORE, ART_Q8_TWO_PASS, ART_Q8_CLUSTER = 0, 1, 2, 3
 
 # every symbol the header declares
 EXPORTS = (
@@ -36,6 +37,7 @@ EXPORTS = (
     "art_decode_attn_terminate",
     "art_decode_attn_terminate_noalloc",
     "art_decode_attn_q8_skipv",
+    "art_decode_attn_q8_skipv_path",
     "art_read_device_status",
     "art_status_string",
     "art_kernel_name",
@@ -118,6 +120,9 @@ def lib() -> ctypes.CDLL:
             L.art_decode_attn_q8_skipv.restype = ctypes.c_int
             L.art_decode_attn_q8_skipv.argtypes = [
                 _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, _P]
+            L.art_decode_attn_q8_skipv_path.restype = ctypes.c_int
+            L.art_decode_attn_q8_skipv_path.argtypes = [
+                _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, ctypes.c_int32, _P]
             L.art_read_device_status.restype = ctypes.c_int
             L.art_read_device_status.argtypes = [_P, _P]
             L.art_status_string.restype = ctypes.c_char_p
@@ -188,6 +193,13 @@ def art_decode_attn_q8_skipv(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, 
     return int(lib().art_decode_attn_q8_skipv(
         ctypes.byref(shape), q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, float(tau), _ref(params), o,
         tiles, ws, ws_bytes, stream))
+
+
+def art_decode_attn_q8_skipv_path(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, params, o,
+                                  tiles, ws, ws_bytes, path, stream) -> int:
+    return int(lib().art_decode_attn_q8_skipv_path(
+        ctypes.byref(shape), q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, float(tau), _ref(params), o,
+        tiles, ws, ws_bytes, int(path), stream))
 
 
 def art_read_device_status(ws, stream) -> int:

@@ -247,8 +247,38 @@ EncodeTiledFn encode_fn() {
 
 bool tc_eligible(int kind, int mode, const art_shape* s, const art_paged_kv* pg = nullptr) {
   const int G = s->Hq / s->Hkv;
+  if (kind == artk::KV_Q8)  // q8: 3 or 4 heads per kv head, contiguous cache, natural order
+    return (mode == artk::MODE_SKIP || mode == artk::MODE_SKIP_ART) && s->d == 128 &&
+           (s->tile == 64 || s->tile == 128) && (G == 3 || G == 4) && !pg && s->L_max % 2 == 0;
   return kind == artk::KV_BF16 && (mode == artk::MODE_FULL || mode == artk::MODE_ART) && s->d == 128 &&
          (s->tile == 64 || s->tile == 128) && G >= 1 && G <= 8 && (!pg || pg->page_size % 64 == 0);
+}
+
+// q8 codes [B*Hkv][L_max][128] (bytes) as a 3-D tensor map, box 128 bytes x 128 rows, no swizzle.
+bool make_q8_code_map(CUtensorMap* m, const void* base, const art_shape* s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(s->L_max), static_cast<cuuint64_t>(s->B) * s->Hkv};
+  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(s->L_max) * 128};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q8 scales [B*Hkv][L_max][4] fp16 viewed as [B*Hkv][L_max/2][16 bytes] (two rows per 16 bytes),
+// box 16 bytes x 64: the scales of 128 positions (L_max even).
+bool make_q8_scale_map(CUtensorMap* m, const void* base, const art_shape* s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(s->L_max / 2), static_cast<cuuint64_t>(s->B) * s->Hkv};
+  const cuuint64_t strides[2] = {16, static_cast<cuuint64_t>(s->L_max) * 8};
+  const cuuint32_t box[3] = {16, 64, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // A bf16 page pool [num_pages*Hkv][page_size][128] as a 3-D tensor map; box = 64 d x 64 positions.
@@ -301,10 +331,16 @@ int tc_ncw(int mode, int G, int C, int kt) {
   return (G + hpp - 1) / hpp >= 2 ? 2 : 1;
 }
 
-art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k, const void* v,
-                     const int32_t* seq_lens, const art_params* a, const int32_t* order, float* o,
-                     int32_t* tiles, void* ws, void* stream, const art_paged_kv* pg) {
+// kind KV_BF16, or KV_Q8 (mode MODE_SKIP / MODE_SKIP_ART; ks, vs the scales, tau the V-skip threshold)
+art_status launch_tc(int kind, int mode, const art_shape* s, const void* q, const void* k, const void* v,
+                     const uint16_t* ks, const uint16_t* vs, float tau, const int32_t* seq_lens,
+                     const art_params* a, const int32_t* order, float* o, int32_t* tiles, void* ws, void* stream,
+                     const art_paged_kv* pg) {
   const int G = s->Hq / s->Hkv;
+  const bool q8 = kind == artk::KV_Q8;
+  if (q8) mode = (mode == artk::MODE_SKIP_ART) ? artk::MODE_ART : artk::MODE_FULL;
+  const unsigned nthr = q8 ? artk::tc::Lay<true>::NTHR : artk::tc::Lay<false>::NTHR;
+  const uint32_t smem = q8 ? artk::tc::SMEM_BYTES_Q8 : artk::tc::SMEM_BYTES;
   const bool ord = order != nullptr, paged = pg != nullptr;
   const int n_probe = a ? a->n_probe : 0;
   artk::tc::TcParams p;
@@ -319,7 +355,13 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
     p.n_probe = a->n_probe;
     for (int i = 0; i < a->n_probe; ++i) p.lanes[i] = static_cast<int8_t>(a->probe_lanes[i]);
   }
-  if (pg) {  // the paged path loads 64-position halves from the page pools
+  p.tau = q8 ? tau : 0.f;
+  p.log2tau = (q8 && tau > 0.f) ? static_cast<float>(log2(static_cast<double>(tau))) : -INFINITY;
+  if (q8) {
+    if (!make_q8_code_map(&p.tmK, k, s) || !make_q8_code_map(&p.tmV, v, s) || !make_q8_scale_map(&p.tmK64, ks, s) ||
+        !make_q8_scale_map(&p.tmV64, vs, s))
+      return ART_ERR_CUDA;
+  } else if (pg) {  // the paged path loads 64-position halves from the page pools
     if (!make_pool_map(&p.tmK64, k, s, pg) || !make_pool_map(&p.tmV64, v, s, pg)) return ART_ERR_CUDA;
     p.block_table = pg->block_table;
     p.page_size = pg->page_size;
@@ -333,7 +375,10 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   p.order = order;
   p.n_max = (s->L_max + s->tile - 1) / s->tile;
   int sms = 0;
-  art_status st = prepare(reinterpret_cast<KernelFn>(tc_pick(mode, G, n_probe, ord, paged, 1)), &sms);
+  auto pick = [&](int ncw) -> TcFn {
+    return q8 ? artk::tc::kernel_q8(mode, n_probe <= 16 ? 16 : 32, ncw) : tc_pick(mode, G, n_probe, ord, paged, ncw);
+  };
+  art_status st = prepare(reinterpret_cast<KernelFn>(pick(1)), &sms);
   if (st != ART_OK) return st;
   // one CTA per SM; cluster size C: power of two, units*C <= SMs, C*tiles_per_block <= 32 (one rule lane
   // per tile of a round), no more CTAs than 128-position blocks in a split, and every cluster resident
@@ -351,7 +396,7 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
     while (C_ < artk::CMAX && 1LL * units_ * (2 * C_) <= sms && 2 * C_ * kt <= 32 && 2 * C_ <= max_blocks) C_ *= 2;
     TcFn fn_ = nullptr;
     while (true) {
-      fn_ = tc_pick(mode, G, n_probe, ord, paged, tc_ncw(mode, G, C_, kt));
+      fn_ = pick(tc_ncw(mode, G, C_, kt));
       const art_status st_ = prepare(reinterpret_cast<KernelFn>(fn_), &sms);
       if (st_ != ART_OK) return st_;
       if (C_ == 1) break;
@@ -359,8 +404,8 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
       memset(&lc, 0, sizeof lc);
       cudaLaunchAttribute attr[1];
       lc.gridDim = dim3(static_cast<unsigned>(units_ * C_), 1, 1);
-      lc.blockDim = dim3(artk::tc::NTHR, 1, 1);
-      lc.dynamicSmemBytes = artk::tc::SMEM_BYTES;
+      lc.blockDim = dim3(nthr, 1, 1);
+      lc.dynamicSmemBytes = smem;
       attr[0].id = cudaLaunchAttributeClusterDimension;
       attr[0].val.clusterDim.x = C_;
       attr[0].val.clusterDim.y = 1;
@@ -381,7 +426,8 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   // Full attention with one caller split: split each sequence internally when that puts more CTAs to
   // work at once (the combine kernel merges the parts and reports the caller's counters).
   int S_run = s->num_splits;
-  if (mode == artk::MODE_FULL && s->num_splits == 1) {
+  // (not for q8: the V skip's running maximum is a property of the split)
+  if (mode == artk::MODE_FULL && s->num_splits == 1 && !q8) {
     for (int f = 2; f <= kFullSplitsMax && f <= max_tiles; f *= 2) {
       Pick q2;
       st = choose(f, &q2);
@@ -419,8 +465,8 @@ art_status launch_tc(int mode, const art_shape* s, const void* q, const void* k,
   memset(&lc, 0, sizeof lc);
   cudaLaunchAttribute attr[1];
   lc.gridDim = dim3(static_cast<unsigned>(units * C), 1, 1);
-  lc.blockDim = dim3(artk::tc::NTHR, 1, 1);
-  lc.dynamicSmemBytes = artk::tc::SMEM_BYTES;
+  lc.blockDim = dim3(nthr, 1, 1);
+  lc.dynamicSmemBytes = smem;
   lc.stream = static_cast<cudaStream_t>(stream);
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
@@ -485,13 +531,12 @@ art_status validate_params(const art_params* a, int d, int epc, int* emask) {
   return ART_OK;
 }
 
-art_status launch(int kind, int mode, const art_shape* s, const void* q, const void* k, const void* v,
-                  const uint16_t* ks, const uint16_t* vs, const int32_t* seq_lens, const art_params* a,
-                  float tau, float* o, int32_t* tiles, void* ws, void* stream, const int32_t* order = nullptr,
-                  const art_paged_kv* pg = nullptr) {
+// The one-pass kernel on the CUDA cores (any dtype, d 64 / 128, a thread-block cluster per split).
+art_status launch_cluster(int kind, int mode, const art_shape* s, const void* q, const void* k, const void* v,
+                          const uint16_t* ks, const uint16_t* vs, const int32_t* seq_lens, const art_params* a,
+                          float tau, float* o, int32_t* tiles, void* ws, void* stream,
+                          const int32_t* order = nullptr, const art_paged_kv* pg = nullptr) {
   const int G = s->Hq / s->Hkv;
-  if (tc_eligible(kind, mode, s, pg))
-    return launch_tc(mode, s, q, k, v, seq_lens, a, order, o, tiles, ws, stream, pg);
   KernelInfo ki;
   if (!pick_kernel(kind, mode, s->d, G, &ki)) return ART_ERR_UNSUPPORTED;
   Params p;
@@ -574,6 +619,15 @@ art_status launch(int kind, int mode, const art_shape* s, const void* q, const v
     if (cudaGetLastError() != cudaSuccess) return ART_ERR_CUDA;
   }
   return ART_OK;
+}
+
+art_status launch(int kind, int mode, const art_shape* s, const void* q, const void* k, const void* v,
+                  const uint16_t* ks, const uint16_t* vs, const int32_t* seq_lens, const art_params* a,
+                  float tau, float* o, int32_t* tiles, void* ws, void* stream, const int32_t* order = nullptr,
+                  const art_paged_kv* pg = nullptr) {
+  if (tc_eligible(kind, mode, s, pg))
+    return launch_tc(kind, mode, s, q, k, v, ks, vs, tau, seq_lens, a, order, o, tiles, ws, stream, pg);
+  return launch_cluster(kind, mode, s, q, k, v, ks, vs, seq_lens, a, tau, o, tiles, ws, stream, order, pg);
 }
 
 // Two-pass q8 decode (full attention with the V skip): the kernels, their workspace arrays (after
@@ -689,23 +743,46 @@ art_status art_decode_attn_terminate_noalloc(const art_shape* shape, art_dtype d
                                    kNoAllocScratchBytes, stream);
 }
 
-art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
-                                    const uint16_t* k_scale_f16, const int8_t* v_q, const uint16_t* v_scale_f16,
-                                    const int32_t* seq_lens, float tau, const art_params* params, float* o,
-                                    int32_t* tiles, void* ws, size_t ws_bytes, void* stream) {
+art_status art_decode_attn_q8_skipv_path(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
+                                         const uint16_t* k_scale_f16, const int8_t* v_q,
+                                         const uint16_t* v_scale_f16, const int32_t* seq_lens, float tau,
+                                         const art_params* params, float* o, int32_t* tiles, void* ws,
+                                         size_t ws_bytes, int32_t path, void* stream) {
   art_status st = validate_common(shape, q_bf16, k_q, v_q, seq_lens, o, ws, ws_bytes);
   if (st != ART_OK) return st;
   if (!k_scale_f16 || !v_scale_f16) return ART_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(k_scale_f16) & 15u) || (reinterpret_cast<uintptr_t>(v_scale_f16) & 15u))
     return ART_ERR_INVALID_ARG;
   if (isnan(tau)) return ART_ERR_INVALID_ARG;
+  if (path < ART_Q8_AUTO || path > ART_Q8_CLUSTER) return ART_ERR_INVALID_ARG;
   const long long scale_row_bytes = (shape->d / 32) * 2;
   if ((1LL * shape->L_max * scale_row_bytes) % 16 != 0) return ART_ERR_UNSUPPORTED;
-  if (q8two_eligible(shape, params, ws_bytes))
-    return launch_q8two(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, o, tiles, ws, stream);
   const int mode = params ? artk::MODE_SKIP_ART : artk::MODE_SKIP;
-  return launch(artk::KV_Q8, mode, shape, q_bf16, k_q, v_q, k_scale_f16, v_scale_f16, seq_lens, params, tau, o,
-                tiles, ws, stream);
+  const bool tc = tc_eligible(artk::KV_Q8, mode, shape);
+  const bool two = q8two_eligible(shape, params, ws_bytes);
+  if (path == ART_Q8_TENSOR_CORE && !tc) return ART_ERR_UNSUPPORTED;
+  if (path == ART_Q8_TWO_PASS && !two) return ART_ERR_UNSUPPORTED;
+  // automatic choice: full attention as two streaming passes when the workspace allows (the
+  // fastest q8 full attention), ART (and full attention without the larger workspace) on the tensor
+  // cores, else the cluster kernel
+  if (path == ART_Q8_TWO_PASS || (path == ART_Q8_AUTO && two))
+    return launch_q8two(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, o, tiles, ws, stream);
+  if (path == ART_Q8_TENSOR_CORE || (path == ART_Q8_AUTO && tc))
+    return launch_tc(artk::KV_Q8, mode, shape, q_bf16, k_q, v_q, k_scale_f16, v_scale_f16, tau, seq_lens, params,
+                     nullptr, o, tiles, ws, stream, nullptr);
+  // the one-pass cluster kernel on the CUDA cores
+  KernelInfo ki;
+  if (!pick_kernel(artk::KV_Q8, mode, shape->d, shape->Hq / shape->Hkv, &ki)) return ART_ERR_UNSUPPORTED;
+  return launch_cluster(artk::KV_Q8, mode, shape, q_bf16, k_q, v_q, k_scale_f16, v_scale_f16, seq_lens, params,
+                        tau, o, tiles, ws, stream);
+}
+
+art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, const int8_t* k_q,
+                                    const uint16_t* k_scale_f16, const int8_t* v_q, const uint16_t* v_scale_f16,
+                                    const int32_t* seq_lens, float tau, const art_params* params, float* o,
+                                    int32_t* tiles, void* ws, size_t ws_bytes, void* stream) {
+  return art_decode_attn_q8_skipv_path(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, params, o,
+                                       tiles, ws, ws_bytes, ART_Q8_AUTO, stream);
 }
 
 art_status art_decode_attn_terminate_ordered(const art_shape* shape, art_dtype dtype, const void* q,
@@ -879,10 +956,10 @@ const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_
     kind = dtype == ART_F32 ? artk::KV_F32 : artk::KV_BF16;
     mode = with_art ? artk::MODE_ART : artk::MODE_FULL;
   }
-  if (tc_eligible(kind, mode, shape)) return "art_decode_tc_kernel";
   if (mode == artk::MODE_SKIP && (shape->d == 64 || shape->d == 128) && shape->Hq % shape->Hkv == 0 &&
       shape->Hq / shape->Hkv <= artk::GMAX)
-    return "q8_pv_kernel";
+    return "q8_pv_kernel";  // (two passes, given the q8 workspace)
+  if (tc_eligible(kind, mode, shape)) return "art_decode_tc_kernel";
   KernelInfo ki;
   if (!pick_kernel(kind, mode, shape->d, shape->Hq / shape->Hkv, &ki)) return nullptr;
   return "art_decode_kernel";

@@ -376,3 +376,59 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 }  // namespace artk
+
+#include <cuda_fp16.h>
+namespace artk {
+// Instruction descriptor, kind::f16 with f16 A/B, f32 accumulate.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+  uint32_t r[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr)
+               : "memory");
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Four int8 codes (one 32-bit word) as two f16 pairs, exactly: the byte c + 128 becomes the low
+// mantissa byte of 1024 + (c + 128) (exponent byte 0x64), and 1152 is subtracted.
+__device__ __forceinline__ void codes4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6480u), __ushort_as_half(0x6480u));  // 1152
+  uint32_t a = __byte_perm(u, 0x64646464u, 0x4140u), c = __byte_perm(u, 0x64646464u, 0x4342u);
+  __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
+  __half2 hc = __hsub2(*reinterpret_cast<__half2*>(&c), bias);
+  lo = *reinterpret_cast<uint32_t*>(&ha);
+  hi = *reinterpret_cast<uint32_t*>(&hc);
+}
+
+// Row `row` of a 128 x 128 block of int8 codes (128 bytes per row) into an f16 MMA operand laid
+// out as two 64-column halves of 128-byte rows with the 128-byte swizzle (16-byte chunk index XOR
+// row % 8) -- the layout the TMA gives a bf16 [128 x 128] tile.  Chunks are visited in a
+// row-rotated order so that 8 consecutive rows touch 8 different bank groups.
+__device__ __forceinline__ void convert_code_row(const uint8_t* src, uint8_t* dst, int row) {
+  const uint8_t* srow = src + row * 128;
+  const int r7 = row & 7;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int c = k ^ r7;  // codes 16c .. 16c + 15 of the row
+    const uint4 w = *reinterpret_cast<const uint4*>(srow + c * 16);
+    uint32_t o[8];
+    codes4_to_f16x2(w.x, o[0], o[1]);
+    codes4_to_f16x2(w.y, o[2], o[3]);
+    codes4_to_f16x2(w.z, o[4], o[5]);
+    codes4_to_f16x2(w.w, o[6], o[7]);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int dc = 2 * c + e, h = dc >> 3, cc = dc & 7;  // 8 f16 = one 16-byte operand chunk
+      *reinterpret_cast<uint4*>(dst + h * 16384 + row * 128 + ((cc ^ r7) * 16)) =
+          make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+    }
+  }
+}
+}  // namespace artk

@@ -86,44 +86,83 @@ struct TcParams {
   int32_t* ws_status;
   int B, Hq, Hkv, L_max, T, S, G, C, n_probe, patience;
   float qscale, eps_scale, eps_dir;
+  float tau;      // q8: V-skip threshold (rows with weight below tau leave the numerator); 0 = off
+  float log2tau;  // q8: log2(tau) (scores live in the log2 domain)
   int8_t lanes[PMAX];
 };
 
-// ---- shared-memory map (byte offsets from a 1024-aligned base)
-constexpr uint32_t OFF_STAGE = 0;
-constexpr uint32_t OFF_Q = NSTG * STAGE_BYTES;  // 2 halves x 2 KiB
-constexpr uint32_t OFF_P = OFF_Q + 4096;        // 2 buffers x 4 KiB
-constexpr uint32_t OFF_BAR = OFF_P + 8192;      // mbarriers
+// ---- q8 cache (int8 codes in 32-element blocks along d, one fp16 scale per block)
+// A raw stage holds one 128-position block as loaded: K codes, V codes (128 B per row), then the
+// K and V scales (8 B per row).  The converter warpgroup turns codes into f16 MMA operands.
+constexpr int Q8_NRAW = 2;
+constexpr uint32_t Q8_RAW_K = 0, Q8_RAW_V = 16384, Q8_RAW_KS = 32768, Q8_RAW_VS = 33792, Q8_RAW_BYTES = 34816;
+constexpr uint32_t Q8_SCL_BYTES = 2048;  // a scale-ring entry: K scales [128][4], then V scales [128][4]
+constexpr int Q8_NP = 32;                // P' columns: 4 scale blocks x (4 hi + 4 lo) for up to 4 heads
+// maxima exchange of the V skip, per round: this CTA's caller-tile maxima [KT_MAX][GMAX], then its
+// block maxima [GMAX]
+constexpr uint32_t MXS_FLOATS = KT_MAX * GMAX + GMAX;
+
+// ---- shared-memory map (byte offsets from a 1024-aligned base), per kind of KV cache
+//   bf16: NSTG stages of K and V exactly as TMA loads them (they are the MMA operands themselves);
+//   q8:   Q8_NRAW raw stages, one K operand and two V operands in f16 written by the converter
+//         warpgroup, a two-entry ring of the blocks' scales for the epilogue, and the maxima
+//         exchange areas of the V skip.
+template <bool Q8>
+struct Lay {
+  static constexpr int NWARP = Q8 ? 16 : 12;  // q8: + the converter warpgroup (warps 12..15)
+  static constexpr int NTHR = NWARP * 32;
+  static constexpr uint32_t TMEM_COLS = Q8 ? 256 : 128;
+  static constexpr uint32_t STAGE = 0;
+  static constexpr uint32_t KCV = Q8_NRAW * Q8_RAW_BYTES;
+  static constexpr uint32_t VCV = KCV + 32768;
+  static constexpr uint32_t SCL = VCV + 2 * 32768;
+  static constexpr uint32_t Q = Q8 ? SCL + 2 * Q8_SCL_BYTES : NSTG * STAGE_BYTES;  // 2 halves x 2 KiB
+  static constexpr uint32_t PBUF = Q8 ? 128 * Q8_NP * 2 : 4096;  // one P buffer
+  static constexpr uint32_t P = Q + 4096;
+  static constexpr uint32_t BAR = P + 2 * PBUF;                                 // mbarriers
+  static constexpr uint32_t WRED = BAR + 512;                                   // [2][4][GMAX] per-warp maxima
+  static constexpr uint32_t WSUM = WRED + 4 * 2 * 4 * GMAX;                     // [2][4][GMAX] per-warp sums
+  static constexpr uint32_t TST = WSUM + 4 * 2 * 4 * GMAX;                      // [NSLOT][KT][GMAX][2] tile (m, l)
+  static constexpr uint32_t DEC = TST + 4 * NSLOT * KT_MAX * GMAX * 2;          // [NSLOT][GMAX] int
+  static constexpr uint32_t CTL = DEC + 4 * NSLOT * GMAX;                       // [16] int
+  static constexpr uint32_t RF = CTL + 4 * 16;                                  // [GMAX][RF_SIZE] float
+  static constexpr uint32_t RI = RF + 4 * GMAX * RF_SIZE;                       // [GMAX][RI_SIZE] int
+  static constexpr uint32_t L2P = RI + 4 * GMAX * RI_SIZE;                      // [D] int8
+  static constexpr uint32_t MXS = L2P + D;                                      // q8: [NSLOT][MXS_FLOATS]
+  static constexpr uint32_t MXL = MXS + (Q8 ? 4 * NSLOT * MXS_FLOATS : 0);      // q8: [NWG][2][CMAX][GMAX]
+  static constexpr uint32_t MXP = MXL + (Q8 ? 4 * NWG * 2 * CMAX * GMAX : 0);   // q8: [NWG][GMAX]
+  static constexpr uint32_t PUB = MXP + (Q8 ? 4 * NWG * GMAX : 0);              // [NSLOT] publication slots
+  static_assert(RF % 16 == 0 && PUB % 16 == 0 && TST % 16 == 0 && DEC % 16 == 0, "vector access");
+  static_assert(Q % 1024 == 0 && (!Q8 || (KCV % 1024 == 0 && VCV % 1024 == 0)), "swizzled operands");
+};
+constexpr uint32_t OFF_STAGE = Lay<false>::STAGE;
+constexpr uint32_t OFF_P = Lay<false>::P;
 enum : int {
   B_FULL = 0, B_EMPTY = B_FULL + NSTG, B_SFULL = B_EMPTY + NSTG, B_SFREE = B_SFULL + 2,
   B_OFULL = B_SFREE + 2, B_XFULL = B_OFULL + 2, B_DEC = B_XFULL + NSLOT,
   B_DRAIN = B_DEC + NSLOT,  // [3]: tensor-core ops of the MMA warp, of warpgroup 0's and 1's leaders
-  B_COUNT = B_DRAIN + 3
+  B_COUNT = B_DRAIN + 3,
+  // q8 only: raw stage full / empty, K operand full / empty, V operands full / empty, scale ring
+  // full / empty, maxima exchange of round r (slot r % NSLOT)
+  B_RAWF = B_COUNT, B_RAWE = B_RAWF + Q8_NRAW, B_KCVF = B_RAWE + Q8_NRAW, B_KCVE = B_KCVF + 1,
+  B_VCVF = B_KCVE + 1, B_VCVE = B_VCVF + 2, B_SCLF = B_VCVE + 2, B_SCLE = B_SCLF + 2, B_MXF = B_SCLE + 2,
+  B_COUNT_Q8 = B_MXF + NSLOT
 };
-static_assert(B_COUNT * 8 <= 512, "barrier area");
-constexpr uint32_t OFF_WRED = OFF_BAR + 512;                           // [2][4][GMAX] per-warp maxima
-constexpr uint32_t OFF_WSUM = OFF_WRED + 4 * 2 * 4 * GMAX;             // [2][4][GMAX] per-warp sums
-constexpr uint32_t OFF_TST = OFF_WSUM + 4 * 2 * 4 * GMAX;              // [NSLOT][KT][GMAX][2] tile (m, l)
-constexpr uint32_t OFF_DEC = OFF_TST + 4 * NSLOT * KT_MAX * GMAX * 2;  // [NSLOT][GMAX] int
-constexpr uint32_t OFF_CTL = OFF_DEC + 4 * NSLOT * GMAX;               // [16] int
-constexpr uint32_t OFF_RF = OFF_CTL + 4 * 16;                          // [GMAX][RF_SIZE] float
-constexpr uint32_t OFF_RI = OFF_RF + 4 * GMAX * RF_SIZE;               // [GMAX][RI_SIZE] int
-constexpr uint32_t OFF_L2P = OFF_RI + 4 * GMAX * RI_SIZE;              // [D] int8
-constexpr uint32_t OFF_PUB = OFF_L2P + D;  // [NSLOT] publication slots, sized per kernel (Pub)
-static_assert(OFF_RF % 16 == 0 && OFF_PUB % 16 == 0 && OFF_TST % 16 == 0 && OFF_DEC % 16 == 0, "vector access");
+static_assert(B_COUNT_Q8 * 8 <= 512, "barrier area");
 // Publication slot of a kernel with GP heads per kv head and probe capacity PC, one entry per
 // (tile i of the block, head g), e = i * GP + g:  m_t[KT_MAX * GP], l_t[KT_MAX * GP], then the PC
 // probe lanes of O_t per entry (rows of PC floats, 16-byte aligned for vector loads).
-template <int GP, int PC>
+template <int GP, int PC, bool Q8 = false>
 struct Pub {
   static constexpr uint32_t NE = KT_MAX * GP;
   static constexpr uint32_t OFF_L = NE, OFF_X = 2 * NE;  // float offsets inside a slot
   static constexpr uint32_t SLOT = 4 * NE * (2 + PC);
-  static constexpr uint32_t SMEM_BYTES = OFF_PUB + NSLOT * SLOT + 1024;  // + alignment slack
+  static constexpr uint32_t SMEM_BYTES = Lay<Q8>::PUB + NSLOT * SLOT + 1024;  // + alignment slack
   static_assert((4 * OFF_X) % 16 == 0 && SLOT % 16 == 0, "probe rows 16-byte aligned");
   static_assert(SMEM_BYTES <= 232448, "shared memory per block");
 };
-constexpr uint32_t SMEM_BYTES = Pub<GMAX, PMAX>::SMEM_BYTES;  // the largest instantiation
+constexpr uint32_t SMEM_BYTES = Pub<GMAX, PMAX>::SMEM_BYTES;  // the largest bf16 instantiation
+constexpr uint32_t SMEM_BYTES_Q8 = Pub<4, PMAX, true>::SMEM_BYTES;
 // final reduction (aliases stage 0 after the pipeline has drained):
 // [NWG][GMAX][D] numerators, then [NWG][GMAX] m, [NWG][GMAX] l, [4] ints (slot 0 ends up holding
 // the CTA's combined state)
@@ -138,6 +177,13 @@ enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, 
              CTL_STOPFLAG = 8 };  // [2 rounds][2 controller warps]: all of the warp's heads stopped
 
 __device__ __forceinline__ uint32_t s_col(int b) { return 16u * b; }
+// q8: S buffer b holds 4 accumulators of 16 columns (one per 32-wide scale block of d); O buffer b
+// holds KT_MAX tiles of Q8_NP columns
+__device__ __forceinline__ uint32_t s_col_q8(int b) { return 64u * b; }
+__device__ __forceinline__ uint32_t o_col_q8(int b, int i) { return 128u + 64u * b + 32u * i; }
+constexpr uint32_t idS8 = idesc_f16(128, 16, false, false);
+constexpr uint32_t idO8 = idesc_f16(128, Q8_NP, true, true);
+constexpr int BAR_CNV = 4;  // named barrier of the q8 converter warpgroup
 // instruction descriptors: scores S^T = K . Q^T (both K-major); output O_t^T = V_t^T . P_t^T (both MN-major)
 constexpr uint32_t idS = idesc_bf16(128, 16, false, false);
 constexpr uint32_t idO = idesc_bf16(128, 16, true, true);
@@ -213,10 +259,13 @@ __device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parit
 // code (the ART epilogue and the producer are sensitive to their instruction footprint).
 // NCW: the ART controller: 0 = the sequential controller of a single-CTA cluster, 1 or 2 = the scan
 // controller warps of a cluster (2 when a round's replay needs two or more passes over the heads).
-template <int GP, int MODE, int PC, bool ORD, bool PAGED, int NCW>
-__global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
+template <int GP, int MODE, int PC, bool ORD, bool PAGED, int NCW, bool Q8 = false>
+__global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
-  using PB = Pub<GP, PC>;
+  using LY = Lay<Q8>;
+  using PB = Pub<GP, PC, Q8>;
+  constexpr int NT_ = LY::NTHR;
+  static_assert(!Q8 || (GP == 4 && !ORD && !PAGED), "q8 cache: 3 or 4 query heads per kv head, natural order, contiguous");
   static_assert(GP >= 1 && GP <= 8, "up to 8 query heads per kv head");
   static_assert(PC == 16 || PC == 32, "probe capacity");
   extern __shared__ uint8_t smem_raw[];
@@ -262,17 +311,17 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     return min(KT, t1 - (t0 + j * KT));
   };
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + LY::BAR);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
-  volatile int* ctl = reinterpret_cast<volatile int*>(sm + OFF_CTL);
-  float* wred = reinterpret_cast<float*>(sm + OFF_WRED);
-  float* wsum = reinterpret_cast<float*>(sm + OFF_WSUM);
-  float* tst = reinterpret_cast<float*>(sm + OFF_TST);
-  float* pub = reinterpret_cast<float*>(sm + OFF_PUB);
-  int* dec = reinterpret_cast<int*>(sm + OFF_DEC);
-  float* rf = reinterpret_cast<float*>(sm + OFF_RF);
-  int* ri = reinterpret_cast<int*>(sm + OFF_RI);
-  int8_t* l2p = reinterpret_cast<int8_t*>(sm + OFF_L2P);
+  volatile int* ctl = reinterpret_cast<volatile int*>(sm + LY::CTL);
+  float* wred = reinterpret_cast<float*>(sm + LY::WRED);
+  float* wsum = reinterpret_cast<float*>(sm + LY::WSUM);
+  float* tst = reinterpret_cast<float*>(sm + LY::TST);
+  float* pub = reinterpret_cast<float*>(sm + LY::PUB);
+  int* dec = reinterpret_cast<int*>(sm + LY::DEC);
+  float* rf = reinterpret_cast<float*>(sm + LY::RF);
+  int* ri = reinterpret_cast<int*>(sm + LY::RI);
+  int8_t* l2p = reinterpret_cast<int8_t*>(sm + LY::L2P);
 
   // ---------------------------------------------------------------- setup
   if (tid == 0) {
@@ -290,15 +339,30 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       mbar_init(bar(B_DEC + s), 1);
     }
     for (int s = 0; s < 3; ++s) mbar_init(bar(B_DRAIN + s), 1);
+    if constexpr (Q8) {
+      for (int s = 0; s < Q8_NRAW; ++s) {
+        mbar_init(bar(B_RAWF + s), 1);
+        mbar_init(bar(B_RAWE + s), 1);
+      }
+      mbar_init(bar(B_KCVF), 1);
+      mbar_init(bar(B_KCVE), 1);
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(bar(B_VCVF + s), 1);
+        mbar_init(bar(B_VCVE + s), 1);
+        mbar_init(bar(B_SCLF + s), 1);
+        mbar_init(bar(B_SCLE + s), 128);
+      }
+      for (int s = 0; s < NSLOT; ++s) mbar_init(bar(B_MXF + s), C);
+    }
     fence_mbar_init();
     if (bad_len && rank == 0) atomicOr(p.ws_status, kStatusSeqLen);
   }
   if (tid < 16) ctl[tid] = 0;
-  for (int i = tid; i < D; i += NTHR) l2p[i] = -1;
-  for (int i = tid; i < 8192 / 16; i += NTHR) reinterpret_cast<uint4*>(sm + OFF_P)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < D; i += NT_) l2p[i] = -1;
+  for (int i = tid; i < static_cast<int>(2 * LY::PBUF / 16); i += NT_) reinterpret_cast<uint4*>(sm + LY::P)[i] = make_uint4(0, 0, 0, 0);
   if (ART)
-    for (int i = tid; i < static_cast<int>(NSLOT * PB::SLOT / 16); i += NTHR)
-      reinterpret_cast<uint4*>(sm + OFF_PUB)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = tid; i < static_cast<int>(NSLOT * PB::SLOT / 16); i += NT_)
+      reinterpret_cast<uint4*>(sm + LY::PUB)[i] = make_uint4(0, 0, 0, 0);
   if (tid < GMAX) {
     float* r = rf + tid * RF_SIZE;
     r[RF_M] = -INFINITY;
@@ -311,14 +375,35 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     q[RI_USED] = ns;
     q[RI_STOPREL] = -1;
   }
-  // Q^T as the scores' B operand: K-major, 128-byte swizzle, 16 rows (heads) x 2 halves of 64 d
-  for (int i = tid; i < 16 * 16; i += NTHR) {
+  // Q^T as the scores' B operand: K-major, 128-byte swizzle, 16 rows x 2 halves of 64 d.  bf16: row
+  // n = head n.  q8 (f16 operands on both sides): row n < 8 = f16 of head n, row 8 + n = the f16 of
+  // what that leaves over (bf16 -> f16 hi + lo keeps q to ~22 bits).
+  for (int i = tid; i < 16 * 16; i += NT_) {
     const int n = i >> 4, c = i & 15, h = c >> 3, cc = c & 7;
     uint4 w = make_uint4(0, 0, 0, 0);
-    if (n < G) w = *reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(b) * p.Hq + kvh * G + n) * D + c * 8);
-    *reinterpret_cast<uint4*>(sm + OFF_Q + h * 2048 + n * 128 + ((cc ^ (n & 7)) * 16)) = w;
+    if constexpr (Q8) {
+      const int hn = n & 7;
+      if (hn < G) {
+        const uint4 qv = *reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(b) * p.Hq + kvh * G + hn) * D + c * 8);
+        uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float x0 = __uint_as_float(qw[k] << 16), x1 = __uint_as_float(qw[k] & 0xffff0000u);
+          __half2 hh = __floats2half2_rn(x0, x1);
+          if (n >= 8) {
+            const float2 f = __half22float2(hh);
+            hh = __floats2half2_rn(x0 - f.x, x1 - f.y);
+          }
+          qw[k] = *reinterpret_cast<uint32_t*>(&hh);
+        }
+        w = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+      }
+    } else {
+      if (n < G) w = *reinterpret_cast<const uint4*>(p.q + (static_cast<long long>(b) * p.Hq + kvh * G + n) * D + c * 8);
+    }
+    *reinterpret_cast<uint4*>(sm + LY::Q + h * 2048 + n * 128 + ((cc ^ (n & 7)) * 16)) = w;
   }
-  if (warp == WARP_MMA) tmem_alloc(smem_u32(sm + OFF_CTL + 4 * CTL_TMEM), TMEM_COLS);
+  if (warp == WARP_MMA) tmem_alloc(smem_u32(sm + LY::CTL + 4 * CTL_TMEM), LY::TMEM_COLS);
   __syncthreads();
   if (tid < P) l2p[p.lanes[tid]] = static_cast<int8_t>(tid);
   fence_proxy_async_smem();
@@ -339,7 +424,31 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 
   // ---------------------------------------------------------------- roles
   if (warp == WARP_TMA) {
-    if (lane == 0) {
+    if (Q8 && lane == 0) {
+      // q8: per own block, the K and V codes (tensor maps over [B*Hkv][L_max][128] bytes, box 128 x
+      // 128 rows) and the K and V scales (over [B*Hkv][L_max/2][16 bytes], box 16 x 64: two rows'
+      // scales per 16 bytes) into raw stage jl % Q8_NRAW; positions past L_max are zero-filled
+      int issued = 0, tiles_read = 0;
+      for (int jl = 0; jl < my_blocks; ++jl) {
+        if (ART && ctl[CTL_EXIT]) break;
+        const int rs = jl % Q8_NRAW;
+        if (jl >= Q8_NRAW && !wait_phase(bar(B_RAWE + rs), ((jl / Q8_NRAW) - 1) & 1, ctl, ART, p.ws_status, false))
+          break;
+        const int j = jl * C + rank;
+        const int p0 = pbeg + j * BLK;
+        const uint32_t fb = bar(B_RAWF + rs);
+        const uint32_t st = smem_u32(sm + rs * Q8_RAW_BYTES);
+        mbar_arrive_expect_tx(fb, Q8_RAW_BYTES);
+        tma_load_3d(st + Q8_RAW_K, &p.tmK, fb, 0, p0, zc);
+        tma_load_3d(st + Q8_RAW_V, &p.tmV, fb, 0, p0, zc);
+        tma_load_3d(st + Q8_RAW_KS, &p.tmK64, fb, 0, p0 / 2, zc);
+        tma_load_3d(st + Q8_RAW_VS, &p.tmV64, fb, 0, p0 / 2, zc);
+        ++issued;
+        tiles_read += min(BLK / T, t1 - (t0 + j * (BLK / T)));
+      }
+      ctl[CTL_ISSUED] = issued;
+      ctl[CTL_TREAD] = tiles_read;
+    } else if (lane == 0) {
       int issued = 0, tiles_read = 0;
       // paged cache in natural order: the page ids of a block follow from its position, so those of
       // the next block are loaded while this one's copies are issued and the next stage frees up
@@ -432,7 +541,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
     }
   } else if (warp == WARP_MMA) {
     if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sm + OFF_Q);
+      const uint32_t q_addr = smem_u32(sm + LY::Q);
       // The scores of every own block, in order: K/V landed, S buffer free.  (The PV product of
       // a block is issued by the leader of the epilogue warpgroup that wrote its weights.)
       // Descriptors are built once per operand buffer and stepped by constant offsets: the
@@ -440,7 +549,26 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       // carries into the next field.
       const uint64_t qd0 = smem_desc(q_addr, 16, 1024, 2);
       int consumed = 0;
-      for (int jl = 0; jl < my_blocks; ++jl) {
+      if constexpr (Q8) {
+        // q8: scores from the converted K operand (f16 codes) into 4 accumulators, one per scale
+        // block of 32 d (2 MMAs of 16 d each); the epilogue applies each row's block scales
+        const uint64_t kd0 = smem_desc(smem_u32(sm + LY::KCV), 16, 1024, 2);
+        for (int jl = 0; jl < my_blocks; ++jl) {
+          const int bb = jl & 1;
+          if (!wait_phase(bar(B_KCVF), jl & 1, ctl, ART, p.ws_status, false)) break;
+          if (jl >= 2 && !wait_phase(bar(B_SFREE + bb), ((jl >> 1) - 1) & 1, ctl, ART, p.ws_status, false)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            constexpr uint32_t kq[8] = {0, 2, 4, 6, 1024, 1026, 1028, 1030};
+            constexpr uint32_t qq[8] = {0, 2, 4, 6, 128, 130, 132, 134};
+            umma_bf16(tmem + s_col_q8(bb) + 16u * (kk >> 1), kd0 + kq[kk], qd0 + qq[kk], idS8, kk & 1);
+          }
+          umma_commit(bar(B_SFULL + bb));
+          umma_commit(bar(B_KCVE));  // the K operand may be overwritten once these scores are done
+        }
+      }
+      for (int jl = 0; !Q8 && jl < my_blocks; ++jl) {
         const int stage = jl % NSTG, bb = jl & 1;
         if (!wait_phase(bar(B_FULL + stage), (jl / NSTG) & 1, ctl, ART, p.ws_status, false)) break;
         consumed = jl + 1;
@@ -456,12 +584,54 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
         }
         umma_commit(bar(B_SFULL + bb));
       }
-      ctl[CTL_CONSUMED] = consumed;
+      if (!Q8) ctl[CTL_CONSUMED] = consumed;  // (q8: the converter consumes the raw stages)
       // every tensor-core op this thread issued has completed before the drain barrier fires
       umma_commit(bar(B_DRAIN));
       drain_wait(bar(B_DRAIN), 0, p.ws_status);
     }
     __syncwarp();
+  } else if (Q8 && warp >= WARP_EPI0 + 4 * NWG) {
+    // ------------------------------------------------------------ q8 converter warpgroup
+    // Thread ct owns row ct of each block: its K codes become the f16 K operand (once the previous
+    // block's scores have read it), its scales go to the scale ring (once the epilogue has read
+    // the entry's previous block), its V codes become the f16 V operand (once the PV product two
+    // blocks back has read it); then the raw stage is released.  Waits are taken by thread 0 and
+    // shared through the warpgroup's named barrier.
+    const int ct = tid - 32 * (WARP_EPI0 + 4 * NWG);
+    const bool cl = (ct == 0);
+    auto cv_wait = [&](uint32_t bar_, uint32_t parity) -> bool {
+      bool ok = true;
+      if (cl) ok = wait_phase(bar_, parity, ctl, ART, p.ws_status, false);
+      return named_barrier_and(BAR_CNV, 128, ok);
+    };
+    int consumed = 0;
+    for (int jl = 0; jl < my_blocks; ++jl) {
+      const int rs = jl % Q8_NRAW, vb = jl & 1;
+      const uint8_t* raw = sm + rs * Q8_RAW_BYTES;
+      if (!cv_wait(bar(B_RAWF + rs), (jl / Q8_NRAW) & 1)) break;
+      consumed = jl + 1;
+      if (jl >= 1 && !cv_wait(bar(B_KCVE), (jl - 1) & 1)) break;
+      convert_code_row(raw + Q8_RAW_K, sm + LY::KCV, ct);
+      if (jl >= 2 && !cv_wait(bar(B_SCLE + vb), ((jl >> 1) - 1) & 1)) break;
+      uint8_t* scl = sm + LY::SCL + vb * Q8_SCL_BYTES;
+      *reinterpret_cast<uint2*>(scl + ct * 8) = *reinterpret_cast<const uint2*>(raw + Q8_RAW_KS + ct * 8);
+      *reinterpret_cast<uint2*>(scl + 1024 + ct * 8) = *reinterpret_cast<const uint2*>(raw + Q8_RAW_VS + ct * 8);
+      fence_proxy_async_smem();  // the K operand is read by the tensor cores
+      named_barrier(BAR_CNV, 128);
+      if (cl) {
+        mbar_arrive(bar(B_KCVF));
+        mbar_arrive(bar(B_SCLF + vb));
+      }
+      if (jl >= 2 && !cv_wait(bar(B_VCVE + vb), ((jl >> 1) - 1) & 1)) break;
+      convert_code_row(raw + Q8_RAW_V, sm + LY::VCV + vb * 32768, ct);
+      fence_proxy_async_smem();
+      named_barrier(BAR_CNV, 128);
+      if (cl) {
+        mbar_arrive(bar(B_VCVF + vb));
+        mbar_arrive(bar(B_RAWE + rs));
+      }
+    }
+    if (cl) ctl[CTL_CONSUMED] = consumed;
   } else if (warp >= WARP_EPI0) {
     // ------------------------------------------------------------ epilogue warpgroups
     // Warpgroup wg takes the own blocks jl = wg, wg + NWG, ... (TMEM and smem buffers
@@ -627,6 +797,193 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       }
       return true;
     };
+    // ---- q8: the V skip's threshold.  Row j of caller tile t (T positions) leaves head g's
+    // numerator when its score s_j < m'_t + log2(tau), m'_t the running maximum of the split's
+    // scores after tile t = max(every tile of earlier rounds, every tile of the round's lower-ranked
+    // CTAs, this block's caller tiles up to t).  Each CTA publishes its round's caller-tile and block
+    // maxima and signals every CTA of the cluster (rounds without a block of the CTA too); threads
+    // 0..GP-1 of the warpgroup keep the maximum over all rounds up to two back (mrun2) and take the
+    // round before from the exchange.
+    float mrun2 = -INFINITY;
+    auto mx_publish = [&](int r, int bbx, bool has_block) {
+      float* mo = reinterpret_cast<float*>(sm + LY::MXS) + (r % NSLOT) * MXS_FLOATS;
+      const int ksn = BLK / T, wnt = T / 32;
+      if (er < KT_MAX * GP) {
+        const int i = er / GP, g = er % GP;
+        float mt = -INFINITY;
+        if (has_block && i < ksn && g < G) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            if (w >= i * wnt && w < (i + 1) * wnt) mt = fmaxf(mt, wred[(bbx * 4 + w) * GMAX + g]);
+        }
+        mo[i * GMAX + g] = mt;
+      }
+      if (er < GP) {
+        float mb = -INFINITY;
+        if (has_block && er < G) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) mb = fmaxf(mb, wred[(bbx * 4 + w) * GMAX + er]);
+        }
+        mo[KT_MAX * GMAX + er] = mb;
+      }
+      named_barrier(bar_epi, 128);
+      if (er < C) {
+        if (C > 1) {
+          fence_acq_rel_cluster();
+          mbar_arrive_cluster_relaxed(map_to_rank(bar(B_MXF + r % NSLOT), er));
+        } else {
+          mbar_arrive(bar(B_MXF + r % NSLOT));
+        }
+      }
+    };
+    auto mx_threshold = [&](int r, float (&thr)[GP]) -> bool {
+      bool ok = true;
+      if (leader) {
+        ok = wait_phase(bar(B_MXF + r % NSLOT), (r / NSLOT) & 1, ctl, ART, p.ws_status, C > 1);
+        if (ok && r >= 1)
+          ok = wait_phase(bar(B_MXF + (r - 1) % NSLOT), ((r - 1) / NSLOT) & 1, ctl, ART, p.ws_status, C > 1);
+      }
+      if (!named_barrier_and(bar_epi, 128, ok)) return false;
+      float* mxl = reinterpret_cast<float*>(sm + LY::MXL) + wg * 2 * CMAX * GMAX;
+      const uint32_t mxs = smem_u32(sm + LY::MXS);
+      if (er < C * GP) {  // block maxima of CTA c, this round and the round before
+        const int c = er / GP, g = er % GP;
+        const uint32_t a0 = mxs + 4 * ((r % NSLOT) * MXS_FLOATS + KT_MAX * GMAX + g);
+        mxl[c * GMAX + g] = ld_smem_f32(C > 1 ? map_to_rank(a0, c) : a0, C > 1);
+        float pv = -INFINITY;
+        if (r >= 1) {
+          const uint32_t a1 = mxs + 4 * (((r - 1) % NSLOT) * MXS_FLOATS + KT_MAX * GMAX + g);
+          pv = ld_smem_f32(C > 1 ? map_to_rank(a1, c) : a1, C > 1);
+        }
+        mxl[CMAX * GMAX + c * GMAX + g] = pv;
+      }
+      named_barrier(bar_epi, 128);
+      float* mxp = reinterpret_cast<float*>(sm + LY::MXP) + wg * GMAX;
+      if (er < GP) {
+        float pre = mrun2, nxt = mrun2;
+        for (int c = 0; c < C; ++c) {
+          const float vp = mxl[CMAX * GMAX + c * GMAX + er], vc = mxl[c * GMAX + er];
+          pre = fmaxf(pre, vp);
+          nxt = fmaxf(nxt, fmaxf(vp, vc));
+          if (c < rank) pre = fmaxf(pre, vc);
+        }
+        mxp[er] = pre;
+        mrun2 = nxt;
+      }
+      named_barrier(bar_epi, 128);
+      const float* mo = reinterpret_cast<const float*>(sm + LY::MXS) + (r % NSLOT) * MXS_FLOATS;
+      const int ic = (T == 64) ? (er >> 6) : 0;  // this row's caller tile inside the block
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float m = mxp[g];
+#pragma unroll
+        for (int i = 0; i < KT_MAX; ++i)
+          if (i <= ic) m = fmaxf(m, mo[i * GMAX + g]);
+        thr[g] = m + p.log2tau;
+      }
+      return true;
+    };
+    // q8: scores -> weights -> P'^T in smem -> PV product for own block jl; false if the run ended.
+    // S buffer bb holds, per scale block of 32 d, the products with q's f16 hi part (columns 0..7)
+    // and lo part (8..15); s = sum over blocks of (hi + lo) x the row's K scale of the block.  P'
+    // has, per scale block, f16 hi and lo parts of p x (the row's V scale of the block): columns
+    // 8 * block + {0..3 hi, 4..7 lo} for the 4 heads; a (row, head) below the V-skip threshold
+    // gets 0 there (its weight stays in the denominator).
+    auto s_phase_q8 = [&](int jl) -> bool {
+      const int bb = jl & 1;
+      const int j = jl * C + rank;
+      bool ok = true;
+      if (leader)
+        ok = wait_phase(bar(B_SFULL + bb), (jl >> 1) & 1, ctl, ART, p.ws_status, false) &&
+             wait_phase(bar(B_SCLF + bb), (jl >> 1) & 1, ctl, ART, p.ws_status, false);
+      if (!named_barrier_and(bar_epi, 128, ok)) return false;
+      tc_fence_after();
+      float sh[4][4], sl[4][4];
+#pragma unroll
+      for (int bk = 0; bk < 4; ++bk) {
+        tmem_ld4(tmem + lane_base + s_col_q8(bb) + 16u * bk, sh[bk]);
+        tmem_ld4(tmem + lane_base + s_col_q8(bb) + 16u * bk + 8u, sl[bk]);
+      }
+      const uint8_t* scl = sm + LY::SCL + bb * Q8_SCL_BYTES;
+      const uint2 ksw = *reinterpret_cast<const uint2*>(scl + er * 8);
+      const uint2 vsw = *reinterpret_cast<const uint2*>(scl + 1024 + er * 8);
+      mbar_arrive(bar(B_SCLE + bb));
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar(B_SFREE + bb));
+      auto h2f = [](uint32_t bits) { return __half2float(__ushort_as_half(static_cast<unsigned short>(bits & 0xffffu))); };
+      const float ks[4] = {h2f(ksw.x), h2f(ksw.x >> 16), h2f(ksw.y), h2f(ksw.y >> 16)};
+      const float vs[4] = {h2f(vsw.x), h2f(vsw.x >> 16), h2f(vsw.y), h2f(vsw.y >> 16)};
+      const int pos = pbeg + j * BLK + er;
+      const bool valid = pos < pend;
+      float s2[GP], red[GP], pw[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float sg = 0.f;
+#pragma unroll
+        for (int bk = 0; bk < 4; ++bk) sg = fmaf(ks[bk], sh[bk][g] + sl[bk][g], sg);
+        red[g] = s2[g] = (valid && g < G) ? sg * p.qscale : -INFINITY;
+      }
+      {
+        const float wm = warp_reduce_heads<GP, true>(red, lane);
+        if ((lane & (32 / GP - 1)) == 0) wred[(bb * 4 + wq) * GMAX + lane / (32 / GP)] = wm;
+      }
+      named_barrier(bar_epi, 128);
+      const bool skip_on = p.tau > 0.f;
+      if (skip_on) mx_publish(jl, bb, true);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float mt = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (in_tile(w, w_lo)) mt = fmaxf(mt, wred[(bb * 4 + w) * GMAX + g]);
+        red[g] = pw[g] = (s2[g] == -INFINITY) ? 0.f : ex2_fast(s2[g] - mt);
+      }
+      {
+        const float ws = warp_reduce_heads<GP, false>(red, lane);
+        if ((lane & (32 / GP - 1)) == 0) wsum[(bb * 4 + wq) * GMAX + lane / (32 / GP)] = ws;
+      }
+      float thr[GP];
+#pragma unroll
+      for (int g = 0; g < GP; ++g) thr[g] = -INFINITY;
+      if (skip_on && !mx_threshold(jl, thr)) return false;
+      uint8_t* prow = sm + LY::P + bb * LY::PBUF + (er >> 3) * 512 + (er & 7) * 16;
+#pragma unroll
+      for (int bk = 0; bk < 4; ++bk) {
+        uint32_t hw[2], lw[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int g0 = 2 * h2;
+          const float x0 = (s2[g0] < thr[g0]) ? 0.f : pw[g0] * vs[bk];
+          const float x1 = (s2[g0 + 1] < thr[g0 + 1]) ? 0.f : pw[g0 + 1] * vs[bk];
+          __half2 hh = __floats2half2_rn(x0, x1);
+          const float2 f = __half22float2(hh);
+          __half2 ll = __floats2half2_rn(x0 - f.x, x1 - f.y);
+          hw[h2] = *reinterpret_cast<uint32_t*>(&hh);
+          lw[h2] = *reinterpret_cast<uint32_t*>(&ll);
+        }
+        *reinterpret_cast<uint4*>(prow + bk * 128) = make_uint4(hw[0], hw[1], lw[0], lw[1]);
+      }
+      // every thread's weights are written: the leader issues the PV product once the converter
+      // has written this block's V operand
+      fence_proxy_async_smem();
+      named_barrier(bar_epi, 128);
+      if (leader && wait_phase(bar(B_VCVF + bb), (jl >> 1) & 1, ctl, ART, p.ws_status, false)) {
+        tc_fence_after();
+        const int ntl = block_tiles(jl);
+        const uint64_t vd0 = smem_desc(smem_u32(sm + LY::VCV + bb * 32768), 16384, 1024, 2);
+        const uint64_t pd0 = smem_desc(smem_u32(sm + LY::P + bb * LY::PBUF), 512, 128, 0);
+        const int tsh = (TE == 64) ? 6 : 7;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = (u * 16) >> tsh;
+          if (i < ntl) umma_bf16(tmem + o_col_q8(bb, i), vd0 + (u * 128u), pd0 + (u * 64u), idO8, ((u * 16) & (TE - 1)) != 0);
+        }
+        umma_commit(bar(B_OFULL + bb));
+        umma_commit(bar(B_VCVE + bb));
+      }
+      return true;
+    };
     // O_t readback (thread = d row) for own block jl into ot; tile stats to tst; false if the run ended
     auto o_phase = [&](int jl, int& ntl) -> bool {
       const int bb = jl & 1;
@@ -639,11 +996,20 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
 #pragma unroll
       for (int i = 0; i < KT_MAX; ++i) {
         if (i < ntl) {
-          float ov[16];
-          tmem_ld16(tmem + lane_base + o_col(bb, i), ov);
-          tmem_ld_wait();
+          if constexpr (Q8) {
+            // rows of warp wq are the d rows of scale block wq: its 8 columns (4 hi, 4 lo)
+            float ov[8];
+            tmem_ld8(tmem + lane_base + o_col_q8(bb, i) + 8u * wq, ov);
+            tmem_ld_wait();
 #pragma unroll
-          for (int g = 0; g < GP; ++g) ot[i][g] = ov[g] + ov[8 + g];
+            for (int g = 0; g < GP; ++g) ot[i][g] = ov[g] + ov[4 + g];
+          } else {
+            float ov[16];
+            tmem_ld16(tmem + lane_base + o_col(bb, i), ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int g = 0; g < GP; ++g) ot[i][g] = ov[g] + ov[8 + g];
+          }
         }
       }
       tc_fence_before();  // O of buffer bb is read: the next PV into it comes after a warpgroup barrier
@@ -694,11 +1060,20 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
       return true;
     };
 
-    const int iters = ART ? R : my_blocks;
+    // q8 with the V skip: every round takes part in the maxima exchange, blocks or not
+    const bool mx_on = Q8 && p.tau > 0.f;
+    const int iters = (ART || mx_on) ? R : my_blocks;
     bool streaming = true;
     for (int r = wg; r < iters; r += NWG) {  // own block r of the CTA = ART round r
       int ntl = 0;
-      if (r < my_blocks && streaming) streaming = s_phase(r);
+      if (r < my_blocks && streaming) {
+        if constexpr (Q8)
+          streaming = s_phase_q8(r);
+        else
+          streaming = s_phase(r);
+      } else if (mx_on && streaming && r >= my_blocks) {
+        mx_publish(r, r & 1, false);
+      }
       if (r < my_blocks && streaming) streaming = o_phase(r, ntl);
       if (!ART) {
         if (!streaming) break;  // aborted
@@ -1047,15 +1422,19 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   __syncthreads();  // (1) every role has left its loop
   // drain: copies that were issued but never consumed still land in shared memory
   if (warp == WARP_TMA && lane == 0) {
-    for (int ord = ctl[CTL_CONSUMED]; ord < ctl[CTL_ISSUED]; ++ord)
-      drain_wait(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, p.ws_status);
+    for (int ord = ctl[CTL_CONSUMED]; ord < ctl[CTL_ISSUED]; ++ord) {
+      if (Q8)
+        drain_wait(bar(B_RAWF + ord % Q8_NRAW), (ord / Q8_NRAW) & 1, p.ws_status);
+      else
+        drain_wait(bar(B_FULL + ord % NSTG), (ord / NSTG) & 1, p.ws_status);
+    }
   }
   __syncthreads();  // (2) the ring is quiet: stage 0 can hold the final reduction
   float* red = reinterpret_cast<float*>(sm + OFF_RED);
   int* redi = reinterpret_cast<int*>(sm + OFF_RED + 4 * RED_I);
   // 1. the CTA's two warpgroup states become one (warpgroup 1 hands its state to warpgroup 0)
   const int er_ = 32 * (warp & 3) + lane;
-  if (warp >= WARP_EPI0 + 4) {
+  if (warp >= WARP_EPI0 + 4 && warp < WARP_EPI0 + 4 * NWG) {  // warpgroup 1 (not the q8 converter)
 #pragma unroll
     for (int g = 0; g < GP; ++g)
       if (g < G) red[(GMAX + g) * D + er_] = acc[g];
@@ -1114,7 +1493,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   }
   __syncthreads();
   const int share = (G * D + C - 1) / C;
-  for (int idx = rank * share + tid; idx < min(G * D, (rank + 1) * share); idx += NTHR) {
+  for (int idx = rank * share + tid; idx < min(G * D, (rank + 1) * share); idx += NT_) {
     const int g = idx / D, dd = idx % D;
     float num = 0.f;
 #pragma unroll 4
@@ -1151,7 +1530,7 @@ __global__ void __launch_bounds__(NTHR, 1) art_decode_tc_kernel(const __grid_con
   if (C > 1) cluster_sync_all();
   if (warp == WARP_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, LY::TMEM_COLS);
   }
 }
 

@@ -37,6 +37,8 @@ TcFn kernel_gp1(int mode, int pc, bool ord, bool paged, int ncw);
 TcFn kernel_gp2(int mode, int pc, bool ord, bool paged, int ncw);
 TcFn kernel_gp4(int mode, int pc, bool ord, bool paged, int ncw);
 TcFn kernel_gp8(int mode, int pc, bool ord, bool paged, int ncw);
+// q8 cache, 4 query heads per kv head, natural order, contiguous (defined in art_tc_q8.cu)
+TcFn kernel_q8(int mode, int pc, int ncw);
 
 }  // namespace tc
 }  // namespace artk

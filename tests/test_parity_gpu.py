@@ -20,9 +20,20 @@ from helpers import TOL, check_tiles, oracle_run  # noqa: E402
 pytestmark = pytest.mark.gpu
 
 
-def gpu(w, mode, *, tile=None, S=None, art=None, tau=None, stream=None, two_pass=True):
-    dp = K.upload(w, num_splits=S, tile=tile, q8_two_pass=two_pass)
-    K.decode(dp, mode, art=art, tau=tau, stream=stream)
+def q8_paths(w, mode, tile=None):
+    """The q8 implementations that take this shape and mode (art_decode_attn_q8_skipv_path)."""
+    T = tile or w.tile
+    paths = ["cluster"]
+    if mode == "q8":
+        paths.append("two_pass")
+    if w.d == 128 and w.G in (3, 4) and T in (64, 128) and w.L_max % 2 == 0:
+        paths.append("tensor_core")
+    return paths
+
+
+def gpu(w, mode, *, tile=None, S=None, art=None, tau=None, stream=None, q8_path="auto"):
+    dp = K.upload(w, num_splits=S, tile=tile)
+    K.decode(dp, mode, art=art, tau=tau, stream=stream, q8_path=q8_path)
     st = K.device_status(dp, stream=stream)
     return dict(
         o=dp.o.cpu().numpy(), tiles=dp.tiles.cpu().numpy(), used=dp.split_tiles().cpu().numpy(),
@@ -34,10 +45,10 @@ def n_tiles(w, tile):
     return -(-w.seq_lens.astype(np.int64) // tile)
 
 
-def check_full(w, mode="full", tile=None, S=None, tau=None, two_pass=True):
+def check_full(w, mode="full", tile=None, S=None, tau=None, q8_path="auto"):
     tile = tile or w.tile
     S = S or w.num_splits
-    g = gpu(w, mode, tile=tile, S=S, tau=tau, two_pass=two_pass)
+    g = gpu(w, mode, tile=tile, S=S, tau=tau, q8_path=q8_path)
     assert g["status"] == capi.ART_OK
     r = oracle_run(w, mode, tile=tile, num_splits=S, tau=tau)
     err = np.max(np.abs(g["o"] - r.o))
@@ -49,11 +60,11 @@ def check_full(w, mode="full", tile=None, S=None, tau=None, two_pass=True):
     return g
 
 
-def check_art(w, mode="art", tile=None, S=None, art=None, tau=None):
+def check_art(w, mode="art", tile=None, S=None, art=None, tau=None, q8_path="auto"):
     tile = tile or w.tile
     S = S or w.num_splits
     a = art or w.art
-    g = gpu(w, mode, tile=tile, S=S, art=a, tau=tau)
+    g = gpu(w, mode, tile=tile, S=S, art=a, tau=tau, q8_path=q8_path)
     assert g["status"] == capi.ART_OK
     ref = oracle_run(w, mode, tile=tile, num_splits=S, art=a, tau=tau, metrics=True)
     exact, amb = check_tiles(w, ref.metrics, g["used"], a, tile, S)
@@ -99,9 +110,9 @@ def make_small(kind, d, Hq, Hkv, B, L_max, lens, tile, S, seed=0, **kw):
 def test_full_small(case):
     w = make_small(*case)
     if w.kind == "q8":
-        for two_pass in (True, False):  # two streaming passes / one pass over a cluster
-            check_full(w, "q8", tau=0.0, two_pass=two_pass)
-            check_full(w, "q8", tau=1e-6, two_pass=two_pass)
+        for path in q8_paths(w, "q8"):  # tensor cores / two streaming passes / one pass over a cluster
+            check_full(w, "q8", tau=0.0, q8_path=path)
+            check_full(w, "q8", tau=1e-6, q8_path=path)
     else:
         check_full(w)
 
@@ -122,15 +133,16 @@ def test_art_small(case, setting):
     w = make_small(*case, seed=setting, sink=6.0)
     a = dict(ART_SETTINGS[setting], lanes=I.probe_lanes_strided(w.d, 16 if w.d == 128 else 8))
     mode = "q8_art" if w.kind == "q8" else "art"
-    g, exact, amb = check_art(w, mode, art=a, tau=(1e-6 if w.kind == "q8" else None))
-    n = n_tiles(w, w.tile)
-    S = w.num_splits
-    if a["eps_scale"] == float("inf") and a["eps_dir"] == float("inf"):
-        for b in range(w.B):
-            lens = [((s + 1) * n[b]) // S - (s * n[b]) // S for s in range(S)]
-            assert np.array_equal(g["used"][b], np.tile([min(a["patience"], x) for x in lens], (w.Hq, 1)))
-    if a["eps_scale"] == 0.0:
-        assert np.array_equal(g["tiles"], np.repeat(n[:, None], w.Hq, axis=1))
+    for path in (q8_paths(w, mode) if w.kind == "q8" else ["auto"]):
+        g, exact, amb = check_art(w, mode, art=a, tau=(1e-6 if w.kind == "q8" else None), q8_path=path)
+        n = n_tiles(w, w.tile)
+        S = w.num_splits
+        if a["eps_scale"] == float("inf") and a["eps_dir"] == float("inf"):
+            for b in range(w.B):
+                lens = [((s + 1) * n[b]) // S - (s * n[b]) // S for s in range(S)]
+                assert np.array_equal(g["used"][b], np.tile([min(a["patience"], x) for x in lens], (w.Hq, 1)))
+        if a["eps_scale"] == 0.0:
+            assert np.array_equal(g["tiles"], np.repeat(n[:, None], w.Hq, axis=1))
 
 
 def test_art_stops_somewhere_midway():
@@ -148,8 +160,11 @@ def test_vskip_actually_skips_and_matches():
     w = I.make_workload(kind="q8", B=1, Hq=4, Hkv=1, d=128, L_max=2048, tile=64, seed=5, gumbel_scale=6.0,
                         q_scale=2.0)
     for tau in (1e-3, 1e-6, 0.0, 2.0):
-        for two_pass in (True, False):
-            check_full(w, "q8", tau=tau, two_pass=two_pass)
+        for path in q8_paths(w, "q8"):
+            check_full(w, "q8", tau=tau, q8_path=path)
+        for path in q8_paths(w, "q8_art"):
+            check_art(w, "q8_art", tau=tau, q8_path=path,
+                      art=dict(eps_scale=2e-2, eps_dir=5e-3, patience=2, lanes=I.probe_lanes_strided(128, 16)))
     full = oracle_run(w, "q8", tau=0.0)
     skip = oracle_run(w, "q8", tau=1e-3)
     assert np.max(np.abs(full.o - skip.o)) > 1e-6  # the skip changed something measurable
@@ -174,7 +189,8 @@ def test_q8_two_pass_shapes(case):
     w = I.make_workload(kind="q8", B=B, Hq=Hq, Hkv=Hkv, d=d, L_max=L_max, tile=tile, num_splits=S,
                         seq_lens=lens, seed=77 + tile, gumbel_scale=3.0, q_scale=1.5)
     for tau in (0.0, 1e-4):
-        check_full(w, "q8", tau=tau)
+        for path in q8_paths(w, "q8"):
+            check_full(w, "q8", tau=tau, q8_path=path)
 
 
 def test_q8_two_pass_skips_whole_tiles():
@@ -184,12 +200,34 @@ def test_q8_two_pass_skips_whole_tiles():
     w = I.make_workload(kind="q8", B=2, Hq=8, Hkv=2, d=128, L_max=4096, tile=64, seq_lens=[4096, 3001],
                         seed=11, sink=40.0)
     for tau in (1e-6, 1e-3):
-        g2 = check_full(w, "q8", tau=tau, two_pass=True)
-        g1 = check_full(w, "q8", tau=tau, two_pass=False)
-        assert np.max(np.abs(g1["o"] - g2["o"])) <= TOL["q8"]
+        g2 = check_full(w, "q8", tau=tau, q8_path="two_pass")
+        for path in ("cluster", "tensor_core"):
+            g1 = check_full(w, "q8", tau=tau, q8_path=path)
+            assert np.max(np.abs(g1["o"] - g2["o"])) <= TOL["q8"]
     r = oracle_run(w, "q8", tau=1e-6)
     r0 = oracle_run(w, "q8", tau=0.0)
     assert np.max(np.abs(r.o - r0.o)) > 0.0  # rows were skipped
+
+
+Q8_TC = [
+    # d, Hq, Hkv, B, L_max, lens, tile, S: clusters of up to 8 / 16 CTAs (the running-maximum exchange),
+    # 3 heads per kv head (padded to 4), several splits, ragged tails, length 1
+    (128, 4, 1, 1, 8192, [8192], 64, 1),
+    (128, 8, 2, 2, 6000, [6000, 1234], 128, 1),
+    (128, 12, 4, 2, 4096, [4096, 4000], 64, 3),
+    (128, 4, 1, 3, 3000, [3000, 129, 1], 64, 2),
+]
+
+
+@pytest.mark.parametrize("case", Q8_TC, ids=lambda c: f"g{c[1] // c[2]}-B{c[3]}-L{c[4]}-T{c[6]}-S{c[7]}")
+def test_q8_tensor_core_shapes(case):
+    d, Hq, Hkv, B, L_max, lens, tile, S = case
+    w = I.make_workload(kind="q8", B=B, Hq=Hq, Hkv=Hkv, d=d, L_max=L_max, tile=tile, num_splits=S,
+                        seq_lens=lens, seed=91 + tile, gumbel_scale=4.0, sink=6.0)
+    a = dict(eps_scale=2e-2, eps_dir=5e-3, patience=2, lanes=I.probe_lanes_strided(128, 16))
+    for tau in (0.0, 1e-6, 1e-3):
+        check_full(w, "q8", tau=tau, q8_path="tensor_core")
+        check_art(w, "q8_art", tau=tau, art=a, q8_path="tensor_core")
 
 
 def test_empty_splits_and_tiny_lengths():
