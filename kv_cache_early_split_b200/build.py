@@ -40,30 +40,43 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+# A test build of the same sources in which the tensor-core kernel's bounded waits give up after
+# 1000 SM cycles (instead of about a second): every call aborts early and reports ART_ERR_TIMEOUT,
+# which lets a test drive the timeout path without a hung copy.  The drains keep their long limit.
+SHORT_WAIT_LIB = os.path.join(PKG, "libart_decode_shortwait.so")
+SHORT_WAIT_FLAGS = ["-DART_TC_WAIT_LIMIT_CYCLES=1000LL"]
+
+
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(d) > t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build_short_wait(force: bool = False) -> str:
+    """The short-wait test build (see SHORT_WAIT_FLAGS)."""
+    return build(force=force, lib=SHORT_WAIT_LIB, extra_flags=SHORT_WAIT_FLAGS)
+
+
+def build(force: bool = False, verbose: bool = False, lib: str = LIB, extra_flags=()) -> str:
     """Compile every source to an object (in parallel), then link the shared library."""
     from concurrent.futures import ThreadPoolExecutor
 
-    if not force and not needs_build():
-        return LIB
-    tag = f".tmp{os.getpid()}"
+    if not force and not needs_build(lib):
+        return lib
+    tag = f".{os.path.basename(lib)[:-3]}.tmp{os.getpid()}"
     objs = [os.path.join(PKG, os.path.basename(src)[:-3] + tag + ".o") for src in SOURCES]
-    cmds = [[nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj] for src, obj in zip(SOURCES, objs)]
+    cmds = [[nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+            for src, obj in zip(SOURCES, objs)]
     with ThreadPoolExecutor(len(cmds)) as ex:
         results = list(ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds))
-    tmp = LIB + tag
+    tmp = lib + tag
     link = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", tmp]
     if all(r.returncode == 0 for r in results):
         results.append(subprocess.run(link, capture_output=True, text=True))
         cmds.append(link)
-    log = os.path.join(PKG, "build.log")
+    log = os.path.join(PKG, "build.log" if lib == LIB else os.path.basename(lib)[:-3] + ".build.log")
     with open(log, "w") as f:
         for c, r in zip(cmds, results):
             f.write(" ".join(c) + "\n" + r.stdout + r.stderr)
@@ -74,11 +87,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if bad:
         sys.stderr.write(bad[0].stdout + bad[0].stderr)
         raise RuntimeError(f"nvcc failed (log: {log})")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     if verbose:
         sys.stdout.write("".join(r.stderr for r in results))
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--short-wait" in sys.argv:
+        print(build_short_wait(force="--force" in sys.argv))

@@ -100,57 +100,67 @@ def lib() -> ctypes.CDLL:
                     f"{LIB_PATH} is missing: build it with `python -m kv_cache_early_split_b200.build` "
                     "(there is no fallback implementation)"
                 )
-            L = ctypes.CDLL(LIB_PATH)
-            L.art_workspace_bytes.restype = ctypes.c_size_t
-            L.art_workspace_bytes.argtypes = [_SH]
-            L.art_q8_workspace_bytes.restype = ctypes.c_size_t
-            L.art_q8_workspace_bytes.argtypes = [_SH]
-            L.art_workspace_tiles_read_offset.restype = ctypes.c_size_t
-            L.art_workspace_tiles_read_offset.argtypes = [_SH]
-            L.art_workspace_split_tiles_offset.restype = ctypes.c_size_t
-            L.art_workspace_split_tiles_offset.argtypes = [_SH]
-            L.art_decode_attn_full.restype = ctypes.c_int
-            L.art_decode_attn_full.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
-            L.art_decode_attn_terminate.restype = ctypes.c_int
-            L.art_decode_attn_terminate.argtypes = [
-                _SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, ctypes.c_size_t, _P]
-            L.art_decode_attn_terminate_noalloc.restype = ctypes.c_int
-            L.art_decode_attn_terminate_noalloc.argtypes = [
-                _SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P]
-            L.art_decode_attn_q8_skipv.restype = ctypes.c_int
-            L.art_decode_attn_q8_skipv.argtypes = [
-                _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, _P]
-            L.art_decode_attn_q8_skipv_path.restype = ctypes.c_int
-            L.art_decode_attn_q8_skipv_path.argtypes = [
-                _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, ctypes.c_int32, _P]
-            L.art_read_device_status.restype = ctypes.c_int
-            L.art_read_device_status.argtypes = [_P, _P]
-            L.art_status_string.restype = ctypes.c_char_p
-            L.art_status_string.argtypes = [ctypes.c_int]
-            L.art_tile_order_recency.restype = ctypes.c_int
-            L.art_tile_order_recency.argtypes = [_SH, _P, _P, _P]
-            L.art_tile_key_summary.restype = ctypes.c_int
-            L.art_tile_key_summary.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P]
-            L.art_tile_order_importance.restype = ctypes.c_int
-            L.art_tile_order_importance.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _P]
-            L.art_decode_attn_terminate_ordered.restype = ctypes.c_int
-            L.art_decode_attn_terminate_ordered.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, _P,
-                                                            ctypes.c_size_t, _P]
-            L.art_decode_attn_paged.restype = ctypes.c_int
-            L.art_decode_attn_paged.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _PG, _P, _PA, _P, _P, _P, _P,
-                                                ctypes.c_size_t, _P]
-            L.art_decode_attn_q8_skipv_paged.restype = ctypes.c_int
-            L.art_decode_attn_q8_skipv_paged.argtypes = [_SH, _P, _P, _P, _P, _P, _PG, _P, ctypes.c_float, _PA, _P,
-                                                         _P, _P, ctypes.c_size_t, _P]
-            L.art_evict_random_select.restype = ctypes.c_int
-            L.art_evict_random_select.argtypes = [_SH, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P,
-                                                  _P]
-            L.art_evict_compact.restype = ctypes.c_int
-            L.art_evict_compact.argtypes = [_SH, ctypes.c_int, _P, _P, _P, ctypes.c_int32, _P, _P, _P]
-            L.art_kernel_name.restype = ctypes.c_char_p
-            L.art_kernel_name.argtypes = [_SH, ctypes.c_int, ctypes.c_int32, ctypes.c_int32]
-            _lib = L
+            _lib = _bind(ctypes.CDLL(LIB_PATH))
     return _lib
+
+
+def load_variant(path: str) -> ctypes.CDLL:
+    """A separately built copy of the library (for instance the short-wait test build), with the
+    same signatures bound; its symbols stay local to it."""
+    return _bind(ctypes.CDLL(path))
+
+
+def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the C signatures on a loaded copy of the library."""
+    L.art_workspace_bytes.restype = ctypes.c_size_t
+    L.art_workspace_bytes.argtypes = [_SH]
+    L.art_q8_workspace_bytes.restype = ctypes.c_size_t
+    L.art_q8_workspace_bytes.argtypes = [_SH]
+    L.art_workspace_tiles_read_offset.restype = ctypes.c_size_t
+    L.art_workspace_tiles_read_offset.argtypes = [_SH]
+    L.art_workspace_split_tiles_offset.restype = ctypes.c_size_t
+    L.art_workspace_split_tiles_offset.argtypes = [_SH]
+    L.art_decode_attn_full.restype = ctypes.c_int
+    L.art_decode_attn_full.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+    L.art_decode_attn_terminate.restype = ctypes.c_int
+    L.art_decode_attn_terminate.argtypes = [
+        _SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, ctypes.c_size_t, _P]
+    L.art_decode_attn_terminate_noalloc.restype = ctypes.c_int
+    L.art_decode_attn_terminate_noalloc.argtypes = [
+        _SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P]
+    L.art_decode_attn_q8_skipv.restype = ctypes.c_int
+    L.art_decode_attn_q8_skipv.argtypes = [
+        _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, _P]
+    L.art_decode_attn_q8_skipv_path.restype = ctypes.c_int
+    L.art_decode_attn_q8_skipv_path.argtypes = [
+        _SH, _P, _P, _P, _P, _P, _P, ctypes.c_float, _PA, _P, _P, _P, ctypes.c_size_t, ctypes.c_int32, _P]
+    L.art_read_device_status.restype = ctypes.c_int
+    L.art_read_device_status.argtypes = [_P, _P]
+    L.art_status_string.restype = ctypes.c_char_p
+    L.art_status_string.argtypes = [ctypes.c_int]
+    L.art_tile_order_recency.restype = ctypes.c_int
+    L.art_tile_order_recency.argtypes = [_SH, _P, _P, _P]
+    L.art_tile_key_summary.restype = ctypes.c_int
+    L.art_tile_key_summary.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P]
+    L.art_tile_order_importance.restype = ctypes.c_int
+    L.art_tile_order_importance.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _P]
+    L.art_decode_attn_terminate_ordered.restype = ctypes.c_int
+    L.art_decode_attn_terminate_ordered.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _PA, _P, _P, _P, _P,
+                                                    ctypes.c_size_t, _P]
+    L.art_decode_attn_paged.restype = ctypes.c_int
+    L.art_decode_attn_paged.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _PG, _P, _PA, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]
+    L.art_decode_attn_q8_skipv_paged.restype = ctypes.c_int
+    L.art_decode_attn_q8_skipv_paged.argtypes = [_SH, _P, _P, _P, _P, _P, _PG, _P, ctypes.c_float, _PA, _P,
+                                                 _P, _P, ctypes.c_size_t, _P]
+    L.art_evict_random_select.restype = ctypes.c_int
+    L.art_evict_random_select.argtypes = [_SH, _P, _P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                                          _P]
+    L.art_evict_compact.restype = ctypes.c_int
+    L.art_evict_compact.argtypes = [_SH, ctypes.c_int, _P, _P, _P, ctypes.c_int32, _P, _P, _P]
+    L.art_kernel_name.restype = ctypes.c_char_p
+    L.art_kernel_name.argtypes = [_SH, ctypes.c_int, ctypes.c_int32, ctypes.c_int32]
+    return L
 
 
 def _ref(x):

@@ -189,8 +189,15 @@ constexpr uint32_t idS = idesc_bf16(128, 16, false, false);
 constexpr uint32_t idO = idesc_bf16(128, 16, true, true);
 __device__ __forceinline__ uint32_t o_col(int b, int i) { return 32u + 32u * b + 16u * i; }
 
-// A wait gives up after this many SM clock cycles (about one second at B200 clocks).
-constexpr long long kWaitLimitCycles = 2000000000LL;
+// A wait gives up after this many SM clock cycles (about one second at B200 clocks), sets the
+// timeout bit of the status word and aborts the CTA.  A test build may set a short limit
+// (ART_TC_WAIT_LIMIT_CYCLES) to drive that path; the drains keep their own limit, so a CTA that
+// aborted still waits for the copies and tensor-core ops it issued.
+#ifndef ART_TC_WAIT_LIMIT_CYCLES
+#define ART_TC_WAIT_LIMIT_CYCLES 2000000000LL
+#endif
+constexpr long long kWaitLimitCycles = ART_TC_WAIT_LIMIT_CYCLES;
+constexpr long long kDrainLimitCycles = 2000000000LL;
 // Longest single sleep of a waiting thread between checks of the exit / abort flags.
 constexpr uint32_t kSuspendNs = 2000;
 
@@ -225,7 +232,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, int32_
   if (mbar_try_wait(bar, parity)) return;
   const long long t0 = clock64();
   while (!mbar_try_wait_sleep(bar, parity, kSuspendNs)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > kDrainLimitCycles) {
       atomicOr(status, kStatusTimeout);
       return;
     }
