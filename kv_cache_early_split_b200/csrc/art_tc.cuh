@@ -264,8 +264,8 @@ __device__ __forceinline__ bool wait_decision_phase(uint32_t bar, uint32_t parit
 // PC: probe-lane capacity of the rule replay (16 or 32, lanes beyond n_probe are zero).
 // ORD / PAGED: a traversal sequence / a paged cache; a kernel without them carries none of that
 // code (the ART epilogue and the producer are sensitive to their instruction footprint).
-// NCW: the ART controller: 0 = the sequential controller of a single-CTA cluster, 1 or 2 = the scan
-// controller warps of a cluster (2 when a round's replay needs two or more passes over the heads).
+// NCW: the ART controller: 0 = the sequential controller of a single-CTA cluster; 1 or 2 = the scan
+// controller of a cluster on one warp or two (half of the heads each).
 template <int GP, int MODE, int PC, bool ORD, bool PAGED, int NCW, bool Q8 = false>
 __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const __grid_constant__ TcParams p) {
   constexpr bool ART = (MODE == MODE_ART);
@@ -1141,13 +1141,12 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
       drain_wait(bar(B_DRAIN + 1 + wg), 0, p.ws_status);
     }
   } else if (warp == WARP_CTL || (NCW == 2 && warp == WARP_CTL + 1)) {
-    // NCW = 0: the sequential controller of a single-CTA cluster; 1 or 2: the scan controller(s)
-    // of a cluster (two warps when a round's replay needs two or more passes over the heads)
+    // NCW = 0: the sequential controller of a single-CTA cluster; 1 or 2: the scan controller of a
+    // cluster on one warp (one pass over the heads) or two (half of the heads each)
     // ------------------------------------------------------------ ART controller(s)
     const int TQ = C * KT;    // tiles per round (power of two <= 32)
     const int HPP = 32 / TQ;  // heads per pass
-    constexpr int ncw = NCW > 0 ? NCW : 1;  // the host picks 2 when a round needs two or more passes over the heads
-    const int cw = (NCW == 1) ? 0 : warp - WARP_CTL;
+    const int cw = (NCW == 0) ? 0 : warp - WARP_CTL;  // NCW 2: which half of the heads
     if constexpr (ART && NCW == 0) {
       // Single-CTA cluster: a round is this CTA's KT tiles, replayed one after another.  Head g
       // owns LPH lanes holding CPL probe lanes each; its carried state (m, l, probe accumulators,
@@ -1246,149 +1245,164 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
         __syncwarp();
         if (all) break;
       }
-    } else if (ART && cw < ncw) {
+    } else if constexpr (ART && NCW >= 1) {
+      // Scan controller: lane (hh, q) takes tile q of the round for head g0 + hh.
       const int hh = lane / TQ, q = lane % TQ;
       const int c = q / KT, i = q % KT;
       const int seg0 = hh * TQ;  // first lane of this head's segment
       const unsigned segmask = (TQ == 32) ? 0xffffffffu : ((1u << TQ) - 1u);
       const bool remote = C > 1;  // the tile's publication lives in CTA c of the cluster
       const uint32_t pub_c = remote ? map_to_rank(smem_u32(pub), c) : smem_u32(pub);
-      for (int r = 0; r < R; ++r) {
-        const int sl = r % NSLOT;
-        int okw = 1;
-        if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r / NSLOT) & 1, ctl, false, p.ws_status, true);
-        okw = __shfl_sync(0xffffffffu, okw, 0);
-        if constexpr (NCW == 2) okw = named_barrier_and(BAR_CTL, 64, okw != 0);  // both warps leave together
-        if (!okw) break;
-        const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
-        const uint32_t slot = pub_c + sl * PB::SLOT;
-        for (int g0 = cw * HPP; g0 < G; g0 += ncw * HPP) {
-          const int g = g0 + hh;
-          const bool active = g < G;
-          const int gs = active ? g : 0;
-          float* R_f = rf + gs * RF_SIZE;
-          int* R_i = ri + gs * RI_SIZE;
-          const bool stopped_before = !active || R_i[RI_STOPPED] != 0;
-          const bool valid = !stopped_before && q < nv;
-          float m = -INFINITY, l = 0.f, a[PC];
+      // The part of a round that needs no earlier round: this lane's tile (m, l, probe) from the CTA
+      // that computed it (tiles at or past nv stay empty) ...
+      auto load_tile = [&](uint32_t slot, bool valid, int g, float& m, float& l, float (&a)[PC]) {
+        m = -INFINITY;
+        l = 0.f;
 #pragma unroll
-          for (int k = 0; k < PC; ++k) a[k] = 0.f;
-          if (valid) {  // this tile's (m, l, probe) from the CTA that computed it
-            const uint32_t e = static_cast<uint32_t>(i * GP + g);
-            m = ld_smem_f32(slot + 4 * e, remote);
-            l = ld_smem_f32(slot + 4 * (PB::OFF_L + e), remote);
-            const uint32_t px = slot + 4 * (PB::OFF_X + e * PC);
-#pragma unroll
-            for (int k = 0; k < PC; k += 4) {
-              const float4 v = ld_smem_v4(px + 4 * k, remote);
-              a[k] = v.x, a[k + 1] = v.y, a[k + 2] = v.z, a[k + 3] = v.w;
-            }
-          }
-          // inclusive scan of the merge over the round's tiles (segments of TQ lanes)
-          float cs[5], co[5];
-#pragma unroll
-          for (int lv = 0; lv < 5; ++lv) {
-            const int off = 1 << lv;
-            cs[lv] = 1.f;
-            co[lv] = 0.f;
-            if (off < TQ) {
-              const float mo = __shfl_up_sync(0xffffffffu, m, off, TQ);
-              const float lo = __shfl_up_sync(0xffffffffu, l, off, TQ);
-              if (q >= off) {
-                const float M = fmaxf(m, mo);
-                cs[lv] = rescale_fast(m, M);
-                co[lv] = rescale_fast(mo, M);
-                l = cs[lv] * l + co[lv] * lo;
-                m = M;
-              }
-            }
-          }
-#pragma unroll
-          for (int lv = 0; lv < 5; ++lv) {
-            const int off = 1 << lv;
-            if (off < TQ) {
-#pragma unroll
-              for (int k = 0; k < PC; ++k) {
-                const float ao = __shfl_up_sync(0xffffffffu, a[k], off, TQ);
-                a[k] = cs[lv] * a[k] + co[lv] * ao;
-              }
-            }
-          }
-          // prepend the state carried over from earlier rounds
-          const float4 st = *reinterpret_cast<const float4*>(R_f);  // m, l, |x_prev|, -
-          const float mR = st.x, lR = st.y;
-          const float Mf = fmaxf(mR, m);
-          const float aR = rescale_fast(mR, Mf), aS = rescale_fast(m, Mf);
-          l = aR * lR + aS * l;
-          m = Mf;
-          const float inv_l = __fdividef(1.f, l);
-          float x[PC], sq[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < PC; ++k) a[k] = 0.f;
+        if (valid) {
+          const uint32_t e = static_cast<uint32_t>(i * GP + g);
+          m = ld_smem_f32(slot + 4 * e, remote);
+          l = ld_smem_f32(slot + 4 * (PB::OFF_L + e), remote);
+          const uint32_t px = slot + 4 * (PB::OFF_X + e * PC);
 #pragma unroll
           for (int k = 0; k < PC; k += 4) {
-            const float4 ar = *reinterpret_cast<const float4*>(R_f + RF_A + k);
-            a[k] = aR * ar.x + aS * a[k];
-            a[k + 1] = aR * ar.y + aS * a[k + 1];
-            a[k + 2] = aR * ar.z + aS * a[k + 2];
-            a[k + 3] = aR * ar.w + aS * a[k + 3];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              x[k + u] = a[k + u] * inv_l;
-              sq[u] = fmaf(x[k + u], x[k + u], sq[u]);
-            }
+            const float4 v = ld_smem_v4(px + 4 * k, remote);
+            a[k] = v.x, a[k + 1] = v.y, a[k + 2] = v.z, a[k + 3] = v.w;
           }
-          const float nrm = __fsqrt_rn((sq[0] + sq[1]) + (sq[2] + sq[3]));
-          float nrmp = __shfl_up_sync(0xffffffffu, nrm, 1, TQ);
-          if (q == 0) nrmp = st.z;
-          const bool both = nrm > 0.f && nrmp > 0.f;
-          const float in = both ? __fdividef(1.f, nrm) : 0.f, ip = both ? __fdividef(1.f, nrmp) : 0.f;
-          float dq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int k = 0; k < PC; k += 4) {
-            const float4 xr = *reinterpret_cast<const float4*>(R_f + RF_XP + k);
-            const float xrv[4] = {xr.x, xr.y, xr.z, xr.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float xp = __shfl_up_sync(0xffffffffu, x[k + u], 1, TQ);
-              if (q == 0) xp = xrv[u];
-              const float dl = x[k + u] * in - xp * ip;
-              dq[u] = fmaf(dl, dl, dq[u]);
-            }
-          }
-          const float dd2 = (dq[0] + dq[1]) + (dq[2] + dq[3]);
-          const float d_scale = fabsf(nrm - nrmp);
-          const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd2);
-          const bool hold = valid && (d_scale < p.eps_scale) && (d_dir < p.eps_dir);
-          // patience, for every tile of the round at once: the run ending at tile q is the number
-          // of consecutive holding tiles up to q (plus the carried run when they reach back to the
-          // round's first tile); the head stops at the first tile whose run reaches the patience.
-          const unsigned hbits = (__ballot_sync(0xffffffffu, hold) >> seg0) & segmask;
-          const int run0 = stopped_before ? 0 : R_i[RI_RUN];
-          const unsigned zeros = ~hbits & ((1u << q) - 1u);
-          const int runq = !((hbits >> q) & 1u) ? 0 : (zeros == 0u ? run0 + q + 1 : q - (31 - __clz(zeros)));
-          const bool reach = hold && runq >= p.patience;
-          const unsigned rbits = (__ballot_sync(0xffffffffu, reach) >> seg0) & segmask;
-          const int stop = (!stopped_before && rbits != 0u) ? __ffs(rbits) - 1 : -1;
-          const int srcq = (stop >= 0) ? stop : nv - 1;
-          if (active && !stopped_before && nv > 0 && q == srcq) {
-            *reinterpret_cast<float4*>(R_f) = make_float4(m, l, nrm, 0.f);
-#pragma unroll
-            for (int k = 0; k < PC; k += 4) {
-              *reinterpret_cast<float4*>(R_f + RF_A + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
-              *reinterpret_cast<float4*>(R_f + RF_XP + k) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
-            }
-            R_i[RI_RUN] = runq;
-            if (stop >= 0) {
-              R_i[RI_STOPPED] = 1;
-              R_i[RI_USED] = r * TQ + stop + 1;
-            }
-          }
-          if (active && q == 0) dec[sl * GMAX + g] = stopped_before ? -2 : stop;
-          __syncwarp();
         }
-        if constexpr (NCW == 1) {
+      };
+      // ... merged with the round's earlier tiles of the same head: an inclusive scan over the head's
+      // segment of TQ lanes.
+      auto scan_tiles = [&](float& m, float& l, float (&a)[PC]) {
+        // a loop, not unrolled: the controller's instruction footprint costs more than the loop
+#pragma unroll 1
+        for (int off = 1; off < TQ; off <<= 1) {
+          const float mo = __shfl_up_sync(0xffffffffu, m, off, TQ);
+          const float lo = __shfl_up_sync(0xffffffffu, l, off, TQ);
+          const bool take = q >= off;
+          const float M = fmaxf(m, mo);
+          const float cs = take ? rescale_fast(m, M) : 1.f;
+          const float co = take ? rescale_fast(mo, M) : 0.f;
+          l = cs * l + co * lo;
+          m = take ? M : m;
+#pragma unroll
+          for (int k = 0; k < PC; ++k) {
+            const float ao = __shfl_up_sync(0xffffffffu, a[k], off, TQ);
+            a[k] = cs * a[k] + co * ao;
+          }
+        }
+      };
+      // The part that needs the state carried over from earlier rounds: prepend it, evaluate the rule
+      // at every tile of the round, find the stop, and carry the state of the head's last replayed
+      // tile (the stop, or the round's last tile) into the next round.
+      auto replay_round = [&](int r, int sl, int nv, int g, float m, float l, float (&a)[PC]) {
+        const bool active = g < G;
+        const int gs = active ? g : 0;
+        float* R_f = rf + gs * RF_SIZE;
+        int* R_i = ri + gs * RI_SIZE;
+        const bool stopped_before = !active || R_i[RI_STOPPED] != 0;
+        const bool valid = !stopped_before && q < nv;
+        const float4 st = *reinterpret_cast<const float4*>(R_f);  // m, l, |x_prev|, -
+        const float mR = st.x, lR = st.y;
+        const float Mf = fmaxf(mR, m);
+        const float aR = rescale_fast(mR, Mf), aS = rescale_fast(m, Mf);
+        l = aR * lR + aS * l;
+        m = Mf;
+        const float inv_l = __fdividef(1.f, l);
+        float x[PC], sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < PC; k += 4) {
+          const float4 ar = *reinterpret_cast<const float4*>(R_f + RF_A + k);
+          a[k] = aR * ar.x + aS * a[k];
+          a[k + 1] = aR * ar.y + aS * a[k + 1];
+          a[k + 2] = aR * ar.z + aS * a[k + 2];
+          a[k + 3] = aR * ar.w + aS * a[k + 3];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            x[k + u] = a[k + u] * inv_l;
+            sq[u] = fmaf(x[k + u], x[k + u], sq[u]);
+          }
+        }
+        const float nrm = __fsqrt_rn((sq[0] + sq[1]) + (sq[2] + sq[3]));
+        float nrmp = __shfl_up_sync(0xffffffffu, nrm, 1, TQ);
+        if (q == 0) nrmp = st.z;
+        const bool both = nrm > 0.f && nrmp > 0.f;
+        const float in = both ? __fdividef(1.f, nrm) : 0.f, ip = both ? __fdividef(1.f, nrmp) : 0.f;
+        float dq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < PC; k += 4) {
+          const float4 xr = *reinterpret_cast<const float4*>(R_f + RF_XP + k);
+          const float xrv[4] = {xr.x, xr.y, xr.z, xr.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float xp = __shfl_up_sync(0xffffffffu, x[k + u], 1, TQ);
+            if (q == 0) xp = xrv[u];
+            const float dl = x[k + u] * in - xp * ip;
+            dq[u] = fmaf(dl, dl, dq[u]);
+          }
+        }
+        const float dd2 = (dq[0] + dq[1]) + (dq[2] + dq[3]);
+        const float d_scale = fabsf(nrm - nrmp);
+        const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd2);
+        const bool hold = valid && (d_scale < p.eps_scale) && (d_dir < p.eps_dir);
+        // patience, for every tile of the round at once: the run ending at tile q is the number
+        // of consecutive holding tiles up to q (plus the carried run when they reach back to the
+        // round's first tile); the head stops at the first tile whose run reaches the patience.
+        const unsigned hbits = (__ballot_sync(0xffffffffu, hold) >> seg0) & segmask;
+        const int run0 = stopped_before ? 0 : R_i[RI_RUN];
+        const unsigned zeros = ~hbits & ((1u << q) - 1u);
+        const int runq = !((hbits >> q) & 1u) ? 0 : (zeros == 0u ? run0 + q + 1 : q - (31 - __clz(zeros)));
+        const bool reach = hold && runq >= p.patience;
+        const unsigned rbits = (__ballot_sync(0xffffffffu, reach) >> seg0) & segmask;
+        const int stop = (!stopped_before && rbits != 0u) ? __ffs(rbits) - 1 : -1;
+        const int srcq = (stop >= 0) ? stop : nv - 1;
+        if (active && !stopped_before && nv > 0 && q == srcq) {
+          *reinterpret_cast<float4*>(R_f) = make_float4(m, l, nrm, 0.f);
+#pragma unroll
+          for (int k = 0; k < PC; k += 4) {
+            *reinterpret_cast<float4*>(R_f + RF_A + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
+            *reinterpret_cast<float4*>(R_f + RF_XP + k) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
+          }
+          R_i[RI_RUN] = runq;
+          if (stop >= 0) {
+            R_i[RI_STOPPED] = 1;
+            R_i[RI_USED] = r * TQ + stop + 1;
+          }
+        }
+        if (active && q == 0) dec[sl * GMAX + g] = stopped_before ? -2 : stop;
+        __syncwarp();
+      };
+      if constexpr (NCW == 1) {
+        // One warp, one pass over every head per round.  The loads of round r + 1 are issued before
+        // round r is replayed whenever every CTA has already published it, so that their latency
+        // (distributed shared memory) overlaps the replay.  (Rounds dealt alternately to two warps,
+        // each scanning one round while the other replays the previous one, ran several times slower.)
+        const int g = hh;
+        auto tile_valid = [&](int r) { return g < G && q < t1 - (t0 + r * TQ); };
+        float m, l, a[PC];
+        int okw = 1;
+        if (R > 0) {
+          if (lane == 0) okw = wait_phase(bar(B_XFULL), 0, ctl, false, p.ws_status, true);
+          okw = __shfl_sync(0xffffffffu, okw, 0);
+          if (okw) load_tile(pub_c, tile_valid(0), g, m, l, a);
+        }
+        for (int r = 0; okw && r < R; ++r) {
+          const int sl = r % NSLOT;
+          const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
+          scan_tiles(m, l, a);
+          const int r1 = r + 1, sl1 = r1 % NSLOT;
+          float m1, l1, a1[PC];
+          int pre = 0;
+          if (r1 < R) {
+            if (lane == 0) pre = mbar_test_wait_cluster(bar(B_XFULL + sl1), (r1 / NSLOT) & 1);
+            pre = __shfl_sync(0xffffffffu, pre, 0);
+            if (pre) load_tile(pub_c + sl1 * PB::SLOT, tile_valid(r1), g, m1, l1, a1);
+          }
+          replay_round(r, sl, nv, g, m, l, a);
           if (lane == 0) {
             bool all = true;
-            for (int g = 0; g < G; ++g) all &= (ri[g * RI_SIZE + RI_STOPPED] != 0);
+            for (int gg = 0; gg < G; ++gg) all &= (ri[gg * RI_SIZE + RI_STOPPED] != 0);
             __threadfence_block();
             mbar_arrive(bar(B_DEC + sl));
             if (all) {
@@ -1398,14 +1412,42 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
             }
           }
           __syncwarp();
-          if (ctl[CTL_EXIT]) break;
-        } else {
+          if (ctl[CTL_EXIT] || r1 >= R) break;
+          if (!pre) {
+            if (lane == 0) okw = wait_phase(bar(B_XFULL + sl1), (r1 / NSLOT) & 1, ctl, false, p.ws_status, true);
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            if (!okw) break;
+            load_tile(pub_c + sl1 * PB::SLOT, tile_valid(r1), g, m1, l1, a1);
+          }
+          m = m1;
+          l = l1;
+#pragma unroll
+          for (int k = 0; k < PC; ++k) a[k] = a1[k];
+        }
+      } else {
+        // Two warps, each replaying half of the heads, round after round.
+        for (int r = 0; r < R; ++r) {
+          const int sl = r % NSLOT;
+          int okw = 1;
+          if (lane == 0) okw = wait_phase(bar(B_XFULL + sl), (r / NSLOT) & 1, ctl, false, p.ws_status, true);
+          okw = __shfl_sync(0xffffffffu, okw, 0);
+          okw = named_barrier_and(BAR_CTL, 64, okw != 0);  // both warps leave together
+          if (!okw) break;
+          const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
+          for (int g0 = cw * HPP; g0 < G; g0 += 2 * HPP) {
+            const int g = g0 + hh;
+            const bool sb = g >= G || ri[g * RI_SIZE + RI_STOPPED] != 0;
+            float m, l, a[PC];
+            load_tile(pub_c + sl * PB::SLOT, !sb && q < nv, g, m, l, a);
+            scan_tiles(m, l, a);
+            replay_round(r, sl, nv, g, m, l, a);
+          }
           // this warp's heads all stopped?  (flags double-buffered by round: the named barrier
           // keeps the two warps within one round of each other)
           if (lane == 0) {
             bool mine = true;
-            for (int g0 = cw * HPP; g0 < G; g0 += NCW * HPP)
-              for (int g = g0; g < min(G, g0 + HPP); ++g) mine &= (ri[g * RI_SIZE + RI_STOPPED] != 0);
+            for (int g0 = cw * HPP; g0 < G; g0 += 2 * HPP)
+              for (int gg = g0; gg < min(G, g0 + HPP); ++gg) mine &= (ri[gg * RI_SIZE + RI_STOPPED] != 0);
             ctl[CTL_STOPFLAG + 2 * (r & 1) + cw] = mine ? 1 : 0;
           }
           named_barrier(BAR_CTL, 64);  // both warps' decisions and flags are written
