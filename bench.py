@@ -470,15 +470,29 @@ def scaling_sweep(K, dp, w, mode, steps, stream):
     for k in ks:
         art = dict(w.art, eps_scale=float("inf"), eps_dir=float("inf"), patience=k)
         _, launch = time_mode(K, dp, mode, steps, 2, stream, art=art, flush=flush)
+        check_status(K, dp, w, f"{mode} patience {k}")
         rb = bytes_read(w, dp.tiles_read().cpu().numpy())
         cb = bytes_consumed(w, dp.split_tiles().cpu().numpy())
-        pts.append({"patience": k, "tiles_frac": float(dp.tiles.double().sum().item()) / n_all,
-                    "ms": launch, "kv_bytes_read": rb, "kv_bytes_consumed": cb, "read_over_consumed": rb / cb})
+        pt = {"patience": k, "tiles_frac": float(dp.tiles.double().sum().item()) / n_all,
+              "ms": launch, "kv_bytes_read": rb, "kv_bytes_consumed": cb, "read_over_consumed": rb / cb}
+        # the same call with speculative reads bounded (art_params.max_spec_tiles = 1: a round is read
+        # only if it starts at or before the safe point)
+        _, launch_b = time_mode(K, dp, mode, steps, 2, stream, art=dict(art, max_spec_tiles=1), flush=flush)
+        check_status(K, dp, w, f"{mode} patience {k} bounded")
+        rb_b = bytes_read(w, dp.tiles_read().cpu().numpy())
+        pt["bounded"] = {"max_spec_tiles": 1, "ms": launch_b, "kv_bytes_read": rb_b, "read_over_consumed": rb_b / cb}
+        pts.append(pt)
     x = np.array([p["kv_bytes_read"] for p in pts], dtype=np.float64)
     y = np.array([p["ms"] for p in pts], dtype=np.float64)
     slope, icpt = np.polyfit(x, y, 1) if len(pts) > 1 else (0.0, float(y[0]))
     return {"points": pts, "fit_ms": {"intercept": float(icpt), "per_gb": float(slope) * 1e9},
-            "note": "eps = +inf, patience k: exactly min(k, n) tiles per (head, split)"}
+            "note": "eps = +inf, patience k: exactly min(k, n) tiles per (head, split); 'bounded': the same "
+                    "call with speculative reads bounded to the round at the safe point"}
+
+
+def check_status(K, dp, w, what):
+    if K.device_status(dp) != 0:
+        raise RuntimeError(f"device status not OK after {w.name} {what}")
 
 
 def mode_row(K, dp, w, mode, steps, stream, peak, art=None):

@@ -95,13 +95,26 @@ typedef struct {
 
 /* ART settings (page S2.2, S2.3).  eps_scale is the page's tau (magnitude),
  * eps_dir its phi (direction).  probe_lanes is a HOST array of n_probe lane
- * indices of O; it is copied during the call. */
+ * indices of O; it is copied during the call.
+ *
+ * max_spec_tiles bounds the reading ahead of the stopping rule (it changes which
+ * K/V tiles are read, never the results).  0: no bound -- the kernel reads as far
+ * ahead as its pipeline holds.  n > 0: the tensor-core kernel starts reading a
+ * round of tiles only when that round begins fewer than n tiles past the split's
+ * "safe" point: the number of tiles every head still running must consume before
+ * it can stop (tiles decided so far plus, for the head farthest from stopping,
+ * patience minus its current run of holding tiles).  Tiles before the safe point
+ * are consumed whatever they hold; at most n tiles plus one round past it are read
+ * speculatively.  Negative values are rejected.  The CUDA-core kernel (fp32 / q8
+ * one-pass / d = 64 / other tiles), whose CTAs read one round ahead of the rule
+ * at most, ignores it. */
 typedef struct {
   float eps_scale;
   float eps_dir;
   int32_t patience;
   const int32_t* probe_lanes;
   int32_t n_probe;
+  int32_t max_spec_tiles;
 } art_params;
 
 /* Bytes of workspace a call with this shape needs (0 on an invalid shape).  With one split it

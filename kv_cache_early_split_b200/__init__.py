@@ -148,20 +148,20 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
                                        _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
         name = "art_decode_attn_full"
     elif mode == "art" and order is not None:
-        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"], a.get("max_spec_tiles", 0))
         rc = capi.art_decode_attn_terminate_ordered(
             dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens), params, _ptr(order),
             _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
         name = "art_decode_attn_terminate_ordered"
     elif mode == "art":
-        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"], a.get("max_spec_tiles", 0))
         rc = capi.art_decode_attn_terminate(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), _ptr(dp.seq_lens),
                                             params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes, st)
         name = "art_decode_attn_terminate"
     elif mode in ("q8", "q8_art"):
         params = None
         if mode == "q8_art":
-            params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+            params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"], a.get("max_spec_tiles", 0))
         rc = capi.art_decode_attn_q8_skipv_path(
             dp.shape, _ptr(dp.q), _ptr(dp.k), _ptr(dp.k_scale), _ptr(dp.v), _ptr(dp.v_scale), _ptr(dp.seq_lens),
             dp.tau if tau is None else tau, params, _ptr(dp.o), _ptr(dp.tiles), _ptr(dp.ws), dp.ws_bytes,
@@ -177,7 +177,7 @@ def decode(dp: DeviceProblem, mode: str, *, art: dict | None = None, tau: float 
 def _decode_paged(dp, mode, a, tau, st, check, order):
     params = None
     if mode in ("art", "q8_art"):
-        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"])
+        params = capi.make_params(a["eps_scale"], a["eps_dir"], a["patience"], a["lanes"], a.get("max_spec_tiles", 0))
     if mode in ("full", "art"):
         dtype = capi.ART_F32 if dp.kind == "f32" else capi.ART_BF16
         rc = capi.art_decode_attn_paged(dp.shape, dtype, _ptr(dp.q), _ptr(dp.k), _ptr(dp.v), dp.pages,

@@ -63,6 +63,7 @@ class art_params(ctypes.Structure):
         ("patience", ctypes.c_int32),
         ("probe_lanes", ctypes.POINTER(ctypes.c_int32)),
         ("n_probe", ctypes.c_int32),
+        ("max_spec_tiles", ctypes.c_int32),
     ]
 
 
@@ -268,10 +269,10 @@ def art_kernel_name(shape, dtype, kv_q8, with_art):
     return None if r is None else r.decode()
 
 
-def make_params(eps_scale: float, eps_dir: float, patience: int, lanes) -> art_params:
+def make_params(eps_scale: float, eps_dir: float, patience: int, lanes, max_spec_tiles: int = 0) -> art_params:
     """art_params with its own HOST copy of the lane list (kept alive on the object)."""
     arr = (ctypes.c_int32 * len(lanes))(*[int(x) for x in lanes])
     p = art_params(float(eps_scale), float(eps_dir), int(patience),
-                   ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)), len(lanes))
+                   ctypes.cast(arr, ctypes.POINTER(ctypes.c_int32)), len(lanes), int(max_spec_tiles))
     p._lanes_keepalive = arr
     return p

@@ -353,6 +353,7 @@ art_status launch_tc(int kind, int mode, const art_shape* s, const void* q, cons
     p.eps_dir = a->eps_dir;
     p.patience = a->patience;
     p.n_probe = a->n_probe;
+    p.spec_tiles = a->max_spec_tiles;
     for (int i = 0; i < a->n_probe; ++i) p.lanes[i] = static_cast<int8_t>(a->probe_lanes[i]);
   }
   p.tau = q8 ? tau : 0.f;
@@ -518,7 +519,8 @@ art_status validate_paged(const art_shape* s, const art_paged_kv* pg) {
 
 art_status validate_params(const art_params* a, int d, int epc, int* emask) {
   if (!a || !a->probe_lanes) return ART_ERR_INVALID_ARG;
-  if (a->n_probe < 1 || a->n_probe > artk::PMAX || a->patience < 1) return ART_ERR_INVALID_ARG;
+  if (a->n_probe < 1 || a->n_probe > artk::PMAX || a->patience < 1 || a->max_spec_tiles < 0)
+    return ART_ERR_INVALID_ARG;
   uint64_t seen[2] = {0, 0};
   *emask = 0;
   for (int i = 0; i < a->n_probe; ++i) {

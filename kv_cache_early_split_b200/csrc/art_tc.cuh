@@ -85,6 +85,7 @@ struct TcParams {
   int32_t* ws_tiles_read;
   int32_t* ws_status;
   int B, Hq, Hkv, L_max, T, S, G, C, n_probe, patience;
+  int spec_tiles;  // ART: bound on the tiles read past the safe point (0: none)
   float qscale, eps_scale, eps_dir;
   float tau;      // q8: V-skip threshold (rows with weight below tau leave the numerator); 0 = off
   float log2tau;  // q8: log2(tau) (scores live in the log2 domain)
@@ -174,7 +175,9 @@ constexpr uint32_t RED_W = RED_I + 8, RED_LT = RED_W + CMAX * GMAX, RED_MG = RED
                    RED_DN = RED_MG + GMAX;
 static_assert(4 * (RED_DN + GMAX) <= STAGE_BYTES, "final reduction fits stage 0");
 enum : int { CTL_EXIT = 0, CTL_EXIT_ROUND, CTL_ABORT, CTL_ISSUED, CTL_CONSUMED, CTL_TREAD, CTL_TMEM,
-             CTL_STOPFLAG = 8 };  // [2 rounds][2 controller warps]: all of the warp's heads stopped
+             CTL_STOPFLAG = 8,    // [2 rounds][2 controller warps]: all of the warp's heads stopped
+             CTL_SAFE = 12,      // tiles the split will consume whatever the rest holds (decided so far)
+             CTL_DECIDED = 13 };  // rounds decided so far
 
 __device__ __forceinline__ uint32_t s_col(int b) { return 16u * b; }
 // q8: S buffer b holds 4 accumulators of 16 columns (one per 32-wide scale block of d); O buffer b
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
     fence_mbar_init();
     if (bad_len && rank == 0) atomicOr(p.ws_status, kStatusSeqLen);
   }
-  if (tid < 16) ctl[tid] = 0;
+  if (tid < 16) ctl[tid] = (tid == CTL_SAFE) ? min(ns, p.patience) : 0;  // no head stops before `patience` tiles
   for (int i = tid; i < D; i += NT_) l2p[i] = -1;
   for (int i = tid; i < static_cast<int>(2 * LY::PBUF / 16); i += NT_) reinterpret_cast<uint4*>(sm + LY::P)[i] = make_uint4(0, 0, 0, 0);
   if (ART)
@@ -430,14 +433,40 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
   }
 
   // ---------------------------------------------------------------- roles
+  // (the safe point once every head has stopped: no further round is read)
+  constexpr int kNothingSafe = -(1 << 30);
   if (warp == WARP_TMA) {
+    // ART with a bound on speculative reads: round jl is read only once it begins fewer than
+    // spec_tiles tiles past the safe point.  Until then the thread sleeps on the decision barrier
+    // of the next undecided round and re-reads the safe point and the decision count (so a phase
+    // of the barrier that completed twice meanwhile costs one sleep, never a lost wake-up).  The
+    // decision of round jl - 1 always puts round jl before the safe point unless the run has ended,
+    // so the wait never needs round jl itself.  false: the run ended, or the CTA aborted.
+    auto spec_ok = [&](int jl) -> bool {
+      if (!ART || p.spec_tiles <= 0) return true;
+      long long tw = 0;
+      while (jl * (C * KT) >= ctl[CTL_SAFE] + p.spec_tiles) {
+        if (ctl[CTL_EXIT] || ctl[CTL_ABORT]) return false;
+        const int dn = ctl[CTL_DECIDED];
+        if (!mbar_try_wait_sleep(bar(B_DEC + dn % NSLOT), (dn / NSLOT) & 1, kSuspendNs)) {
+          if (tw == 0) tw = clock64();
+          if (clock64() - tw > kWaitLimitCycles) {
+            atomicOr(p.ws_status, kStatusTimeout);
+            ctl[CTL_ABORT] = 1;
+            return false;
+          }
+        }
+        __threadfence_block();
+      }
+      return true;
+    };
     if (Q8 && lane == 0) {
       // q8: per own block, the K and V codes (tensor maps over [B*Hkv][L_max][128] bytes, box 128 x
       // 128 rows) and the K and V scales (over [B*Hkv][L_max/2][16 bytes], box 16 x 64: two rows'
       // scales per 16 bytes) into raw stage jl % Q8_NRAW; positions past L_max are zero-filled
       int issued = 0, tiles_read = 0;
       for (int jl = 0; jl < my_blocks; ++jl) {
-        if (ART && ctl[CTL_EXIT]) break;
+        if (ART && (ctl[CTL_EXIT] || !spec_ok(jl))) break;
         const int rs = jl % Q8_NRAW;
         if (jl >= Q8_NRAW && !wait_phase(bar(B_RAWE + rs), ((jl / Q8_NRAW) - 1) & 1, ctl, ART, p.ws_status, false))
           break;
@@ -471,7 +500,7 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
       int pg_cur[2] = {0, 0}, pg_next[2] = {0, 0};
       if (pg_ahead) page_ids(0, pg_cur);
       for (int jl = 0; jl < my_blocks; ++jl) {
-        if (ART && ctl[CTL_EXIT]) break;
+        if (ART && (ctl[CTL_EXIT] || !spec_ok(jl))) break;
         const int stage = jl % NSTG;
         if (jl >= NSTG && !wait_phase(bar(B_EMPTY + stage), ((jl / NSTG) - 1) & 1, ctl, ART, p.ws_status, false)) break;
         const int j = jl * C + rank;
@@ -1232,8 +1261,12 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           }
         }
         const bool all = __ballot_sync(0xffffffffu, active && !stopped) == 0u;
+        // the safe point: tiles decided so far plus what the head farthest from stopping still needs
+        const int rem = __reduce_max_sync(0xffffffffu, (active && !stopped) ? p.patience - run : 0);
         __syncwarp();
         if (lane == 0) {
+          ctl[CTL_SAFE] = all ? kNothingSafe : min(ns, (r + 1) * KT + rem);
+          ctl[CTL_DECIDED] = r + 1;
           __threadfence_block();
           mbar_arrive(bar(B_DEC + sl));
           if (all) {
@@ -1402,7 +1435,14 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           replay_round(r, sl, nv, g, m, l, a);
           if (lane == 0) {
             bool all = true;
-            for (int gg = 0; gg < G; ++gg) all &= (ri[gg * RI_SIZE + RI_STOPPED] != 0);
+            int rem = 0;  // the safe point, as in the sequential controller
+            for (int gg = 0; gg < G; ++gg) {
+              const bool sg = ri[gg * RI_SIZE + RI_STOPPED] != 0;
+              all &= sg;
+              if (!sg) rem = max(rem, p.patience - ri[gg * RI_SIZE + RI_RUN]);
+            }
+            ctl[CTL_SAFE] = all ? kNothingSafe : min(ns, (r + 1) * TQ + rem);
+            ctl[CTL_DECIDED] = r + 1;
             __threadfence_block();
             mbar_arrive(bar(B_DEC + sl));
             if (all) {
@@ -1453,6 +1493,11 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           named_barrier(BAR_CTL, 64);  // both warps' decisions and flags are written
           const bool all = ctl[CTL_STOPFLAG + 2 * (r & 1)] && ctl[CTL_STOPFLAG + 2 * (r & 1) + 1];
           if (cw == 0 && lane == 0) {
+            int rem = 0;  // the safe point, as in the sequential controller
+            for (int gg = 0; gg < G; ++gg)
+              if (ri[gg * RI_SIZE + RI_STOPPED] == 0) rem = max(rem, p.patience - ri[gg * RI_SIZE + RI_RUN]);
+            ctl[CTL_SAFE] = all ? kNothingSafe : min(ns, (r + 1) * TQ + rem);
+            ctl[CTL_DECIDED] = r + 1;
             __threadfence_block();
             mbar_arrive(bar(B_DEC + sl));
             if (all) {

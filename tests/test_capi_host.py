@@ -125,6 +125,7 @@ def test_invalid_arguments_terminate(L):
     assert term(s, capi.make_params(1e-3, 1e-4, 1, [0, 128])) == capi.ART_ERR_INVALID_ARG  # lane >= d
     assert term(s, capi.make_params(1e-3, 1e-4, 1, [-1])) == capi.ART_ERR_INVALID_ARG
     assert term(s, capi.make_params(1e-3, 1e-4, 1, [3, 3])) == capi.ART_ERR_INVALID_ARG  # duplicate
+    assert term(s, capi.make_params(1e-3, 1e-4, 1, [0], max_spec_tiles=-1)) == capi.ART_ERR_INVALID_ARG
     assert term(shape(d=64), capi.make_params(1e-3, 1e-4, 1, [64])) == capi.ART_ERR_INVALID_ARG
     assert term(s, ok, ws_bytes=16) == capi.ART_ERR_WORKSPACE
 
