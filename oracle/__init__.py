@@ -84,6 +84,8 @@ def _load():
             lib.oracle_decode_ordered.restype = ctypes.c_int
             lib.oracle_decode_ordered.argtypes = lib.oracle_decode.argtypes[:12] + [ctypes.c_void_p] + \
                 lib.oracle_decode.argtypes[12:]
+            lib.oracle_decode_vskip.restype = ctypes.c_int
+            lib.oracle_decode_vskip.argtypes = lib.oracle_decode_ordered.argtypes + [ctypes.c_void_p]
             lib.oracle_bf16_to_double.restype = ctypes.c_double
             lib.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
             lib.oracle_f16_to_double.restype = ctypes.c_double
@@ -105,10 +107,11 @@ def _ptr(a):
 
 
 class OracleResult:
-    """o [B,Hq,d] float64; tiles [B,Hq]; used [B,Hq,S]; metrics [B,Hq,n,2] or None."""
+    """o [B,Hq,d] float64; tiles [B,Hq]; used [B,Hq,S]; metrics [B,Hq,n,2] or None;
+    vskip [B,Hq,L_max] or None: p / tau of every row weighed with the V skip on (NaN elsewhere)."""
 
-    def __init__(self, o, tiles, used, metrics):
-        self.o, self.tiles, self.used, self.metrics = o, tiles, used, metrics
+    def __init__(self, o, tiles, used, metrics, vskip=None):
+        self.o, self.tiles, self.used, self.metrics, self.vskip = o, tiles, used, metrics, vskip
 
 
 def decode(
@@ -129,6 +132,7 @@ def decode(
     want_metrics: bool = False,
     n_threads: int = 1,
     tile_order: np.ndarray | None = None,
+    want_vskip: bool = False,
 ) -> OracleResult:
     """Run the oracle.
 
@@ -138,6 +142,8 @@ def decode(
     art: None for plain attention, else dict(eps_scale, eps_dir, patience, lanes).
     tile_order: None (natural order) or int32 [B,Hkv,ceil(L_max/tile)]: each (batch, kv head)'s
       traversal sequence; split s walks positions [s*n/S, (s+1)*n/S) of it (see orders.py).
+    want_vskip: also return, for the q8 V skip (tau > 0), p / tau of every row each head weighed
+      (the row left that head's numerator iff the value is below 1).
     """
     lib = _load()
     B, Hq, d = q.shape
@@ -171,11 +177,12 @@ def decode(
     if tile_order is not None:
         order = np.ascontiguousarray(tile_order, dtype=np.int32)
         assert order.shape == (B, Hkv, n_tiles_max), order.shape
-    rc = lib.oracle_decode_ordered(
+    vskip = np.zeros((B, Hq, L_max), np.float64) if want_vskip else None
+    rc = lib.oracle_decode_vskip(
         ctypes.byref(sh), kind, _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale), _ptr(seq),
         ctypes.byref(art_s) if art_s is not None else None, float(tau), _ptr(fu), int(no_break), _ptr(order),
-        _ptr(o), _ptr(used), _ptr(tiles), _ptr(metrics), int(n_threads),
+        _ptr(o), _ptr(used), _ptr(tiles), _ptr(metrics), int(n_threads), _ptr(vskip),
     )
     if rc != 0:
         raise ValueError(f"oracle_decode failed with code {rc}")
-    return OracleResult(o, tiles, used, metrics)
+    return OracleResult(o, tiles, used, metrics, vskip)

@@ -141,13 +141,14 @@ static double l2norm(const double* x, int n) {
  * One (batch, query head).  Returns 0 or a negative error.
  * o: [d]; used: [S]; metrics: NULL or [n_tiles_max][2] (d_scale, d_dir) by position in
  * the traversal sequence; seq: NULL (natural order) or this kv head's [n_tiles_max]
- * traversal sequence.
+ * traversal sequence; vskip: NULL or [L_max], where each row the head weighs with the
+ * V skip on gets p / tau (the row left the numerator iff that is below 1).
  */
 static int decode_one_head(const oracle_shape* sh, int kind, const void* q, const void* k,
                            const void* v, const uint16_t* k_scale, const uint16_t* v_scale,
                            int L, int b, int hq, const oracle_art* art, double tau,
                            const int32_t* forced_used, int no_break, const int32_t* seq,
-                           double* o, int32_t* used, double* metrics, int n_tiles_max) {
+                           double* o, int32_t* used, double* metrics, int n_tiles_max, double* vskip) {
   const int d = sh->d, T = sh->tile, S = sh->num_splits;
   const int G = sh->Hq / sh->Hkv;
   const int kvh = hq / G;
@@ -228,6 +229,7 @@ static int decode_one_head(const oracle_shape* sh, int kind, const void* q, cons
       for (int j = j0; j < j1; ++j) {
         const double p = exp(sc[j - j0] - mnew);
         cur.l += p;
+        if (skip_on && vskip) vskip[j] = p / tau;
         if (skip_on && p < tau) continue;
         decode_row(kind, v, v_scale, row0 + j, d, vr);
         for (int i = 0; i < d; ++i) cur.acc[i] += p * vr[i];
@@ -313,14 +315,17 @@ static int decode_one_head(const oracle_shape* sh, int kind, const void* q, cons
  *   tile_order  NULL (natural order) or [B,Hkv,n_tiles_max]: the traversal sequence
  *            of each (batch, kv head); entries at positions >= ceil(L_b/T) are ignored
  *   n_threads  OpenMP threads over (batch, query head); <= 0: library default
+ *   vskip    NULL or [B,Hq,L_max]: p / tau of every row a head weighed with the q8 V skip
+ *            on (p = exp(s_j - m'), m' the running maximum after the row's tile); the row
+ *            left that head's numerator iff the value is below 1.  NaN elsewhere.
  * A sequence entry outside its split's tiles gives ORACLE_ERR_ARG.
  */
-int oracle_decode_ordered(const oracle_shape* sh, int kind, const void* q, const void* k,
-                          const void* v, const uint16_t* k_scale, const uint16_t* v_scale,
-                          const int32_t* seq_lens, const oracle_art* art, double tau,
-                          const int32_t* forced_used, int no_break, const int32_t* tile_order,
-                          double* o, int32_t* used, int32_t* tiles, double* metrics,
-                          int n_threads) {
+int oracle_decode_vskip(const oracle_shape* sh, int kind, const void* q, const void* k,
+                        const void* v, const uint16_t* k_scale, const uint16_t* v_scale,
+                        const int32_t* seq_lens, const oracle_art* art, double tau,
+                        const int32_t* forced_used, int no_break, const int32_t* tile_order,
+                        double* o, int32_t* used, int32_t* tiles, double* metrics, int n_threads,
+                        double* vskip) {
   if (!sh || !q || !k || !v || !seq_lens || !o || !used || !tiles) return ORACLE_ERR_ARG;
   if (sh->B < 1 || sh->Hq < 1 || sh->Hkv < 1 || sh->d < 1 || sh->L_max < 1 || sh->tile < 1 ||
       sh->num_splits < 1)
@@ -337,6 +342,10 @@ int oracle_decode_ordered(const oracle_shape* sh, int kind, const void* q, const
     if (seq_lens[b] < 1 || seq_lens[b] > sh->L_max) return ORACLE_ERR_SEQLEN;
 
   const int n_tiles_max = (sh->L_max + sh->tile - 1) / sh->tile;
+  if (vskip) {
+    const long nv = (long)sh->B * sh->Hq * sh->L_max;
+    for (long i = 0; i < nv; ++i) vskip[i] = NAN;
+  }
   if (metrics) {
     const long nm = (long)sh->B * sh->Hq * n_tiles_max * 2;
     for (long i = 0; i < nm; ++i) metrics[i] = NAN;
@@ -355,13 +364,25 @@ int oracle_decode_ordered(const oracle_shape* sh, int kind, const void* q, const
     int r = decode_one_head(sh, kind, q, k, v, k_scale, v_scale, seq_lens[b], b, hq, art, tau,
                             forced_used ? forced_used + (long)bh * S : NULL, no_break, seq,
                             o + (long)bh * sh->d, used + (long)bh * S,
-                            metrics ? metrics + (long)bh * n_tiles_max * 2 : NULL, n_tiles_max);
+                            metrics ? metrics + (long)bh * n_tiles_max * 2 : NULL, n_tiles_max,
+                            vskip ? vskip + (long)bh * sh->L_max : NULL);
     if (r < err) err = r;
     int sum = 0;
     for (int s = 0; s < S; ++s) sum += used[(long)bh * S + s];
     tiles[bh] = sum;
   }
   return err;
+}
+
+/* Without the V-skip record. */
+int oracle_decode_ordered(const oracle_shape* sh, int kind, const void* q, const void* k,
+                          const void* v, const uint16_t* k_scale, const uint16_t* v_scale,
+                          const int32_t* seq_lens, const oracle_art* art, double tau,
+                          const int32_t* forced_used, int no_break, const int32_t* tile_order,
+                          double* o, int32_t* used, int32_t* tiles, double* metrics,
+                          int n_threads) {
+  return oracle_decode_vskip(sh, kind, q, k, v, k_scale, v_scale, seq_lens, art, tau, forced_used,
+                             no_break, tile_order, o, used, tiles, metrics, n_threads, NULL);
 }
 
 /* Natural tile order (0, 1, ..., n-1 in every split). */

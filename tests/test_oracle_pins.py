@@ -366,6 +366,43 @@ def test_vskip_error_bound():
     assert nskipped > 0, "the case must actually skip rows"
 
 
+def test_vskip_record_matches_definition():
+    """The oracle's per-row record p / tau (the numerator test of the V skip) against p_j rebuilt
+    from the definition as above; rows past the sequence are NaN."""
+    tau = 1e-3
+    w = I.make_workload(kind="q8", B=1, Hq=4, Hkv=1, d=64, L_max=512, tile=32, seed=4, gumbel_scale=6.0, q_scale=2.0,
+                        seq_lens=[449])
+    r = oracle.decode(kind=oracle.KV_Q8, q=w.q, k=w.k, v=w.v, k_scale=w.k_scale, v_scale=w.v_scale,
+                      seq_lens=w.seq_lens, tile=w.tile, tau=tau, want_vskip=True)
+    q, K, V = _decode_kv(w)
+    T, L, d = w.tile, int(w.seq_lens[0]), w.d
+    for hq in range(w.Hq):
+        s = (K[0, 0, :L] @ q[0, hq]) / math.sqrt(d)
+        run_max = np.maximum.accumulate(np.array([s[t:t + T].max() for t in range(0, L, T)]))
+        p_run = np.exp(s - np.repeat(run_max, T)[:L])
+        assert np.allclose(r.vskip[0, hq, :L], p_run / tau, rtol=1e-9, atol=0.0)
+        assert np.all(np.isnan(r.vskip[0, hq, L:]))
+    assert np.any(r.vskip[0, :, :L] < 1.0) and np.any(r.vskip[0, :, :L] >= 1.0)
+
+
+def test_vskip_record_is_the_skip_set():
+    """With one query head per kv head, leaving a row out of the numerator is the same as zeroing
+    its V row: the output with the skip equals the output without it on V with the recorded rows
+    (p / tau < 1) zeroed, exactly."""
+    tau = 3e-3
+    w = I.make_workload(kind="q8", B=2, Hq=3, Hkv=3, d=64, L_max=384, tile=32, seed=9, gumbel_scale=5.0, q_scale=2.0,
+                        seq_lens=[384, 301], num_splits=2)
+    r = oracle.decode(kind=oracle.KV_Q8, q=w.q, k=w.k, v=w.v, k_scale=w.k_scale, v_scale=w.v_scale,
+                      seq_lens=w.seq_lens, tile=w.tile, num_splits=2, tau=tau, want_vskip=True)
+    v0 = w.v.copy()
+    mask = r.vskip < 1.0  # [B, Hq = Hkv, L_max]; NaN compares False
+    assert mask.sum() > 0
+    v0[mask] = 0
+    r0 = oracle.decode(kind=oracle.KV_Q8, q=w.q, k=w.k, v=v0, k_scale=w.k_scale, v_scale=w.v_scale,
+                       seq_lens=w.seq_lens, tile=w.tile, num_splits=2, tau=0.0)
+    assert np.array_equal(r.o, r0.o)
+
+
 def test_named_workloads_shapes():
     for name in I.WORKLOADS:
         w = I.workload(name, keys_b=[0], keys_h=[0])
