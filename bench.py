@@ -538,9 +538,11 @@ def measure_workload(K, w, dp, args, stream, peak, sweeps=True):
 
 
 def vskip_sweep(K, args, stream, device):
-    """The q8 V-dequant skip threshold tau in {0, 1e-6, 1e-3} on the q8 workload (N(0,1) keys) and on
-    its skewed variant (attention sink, Gumbel key offsets, log-normal V norms): ms per call with and
-    without ART.  tau = 0 skips nothing, so the time differences are the skip's saving."""
+    """The q8 V-dequant skip threshold tau in {0, 1e-6, 1e-3, 1e-2} on the q8 workload (N(0,1) keys)
+    and on its skewed variant (attention sink, Gumbel key offsets, log-normal V norms): ms per call
+    with and without ART.  tau = 0 skips nothing, so the time differences are the skip's saving.
+    For q8 without ART (the two-pass path) also the device's counts: V rows left out of every
+    head's numerator and V tiles not read, as fractions, and the V bytes those tiles saved."""
     import torch
 
     steps = max(3, min(args.steps, 10))
@@ -550,7 +552,7 @@ def vskip_sweep(K, args, stream, device):
         w = I.workload(name)
         dp = K.upload(w, device=device)
         rows = {}
-        for tau in (0.0, 1e-6, 1e-3):
+        for tau in (0.0, 1e-6, 1e-3, 1e-2):
             row = {}
             for mode in ("q8", "q8_art"):
                 for _ in range(2):
@@ -567,12 +569,20 @@ def vskip_sweep(K, args, stream, device):
                              "kv_bytes_read": bytes_read(w, dp.tiles_read().cpu().numpy()),
                              "mean_tiles_frac": float(dp.tiles.float().mean().item())
                              / float((-(-w.seq_lens.astype(np.int64) // w.tile)).mean())}
+                if mode == "q8" and K.kernel_name(dp, mode) == "q8_pv_kernel":
+                    vs = dp.vskip_counts().cpu().numpy().astype(np.int64)
+                    rows_all = float(w.seq_lens.astype(np.int64).sum() * w.Hkv)
+                    tiles_all = float((-(-w.seq_lens.astype(np.int64) // w.tile)).sum() * w.Hkv)
+                    v_row_bytes = w.d + 2 * (w.d // 32)  # codes + fp16 scales
+                    row[mode]["v_rows_skipped_frac"] = float(vs[..., 0].sum()) / rows_all
+                    row[mode]["v_tiles_not_read_frac"] = float(vs[..., 1].sum()) / tiles_all
+                    row[mode]["v_bytes_not_read"] = int(vs[..., 1].sum()) * w.tile * v_row_bytes
             rows[f"tau_{tau:g}"] = row
         if K.device_status(dp) != 0:
             raise RuntimeError("device status not OK after the V-skip sweep")
         for mode in ("q8", "q8_art"):
             base = rows["tau_0"][mode]["ms"]
-            for t in ("tau_1e-06", "tau_0.001"):
+            for t in ("tau_1e-06", "tau_0.001", "tau_0.01"):
                 rows[t][mode]["time_saved_vs_tau0"] = 1.0 - rows[t][mode]["ms"] / base
         out[name] = rows
         del dp

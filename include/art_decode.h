@@ -135,6 +135,15 @@ size_t art_q8_workspace_bytes(const art_shape* shape);
  * last call, speculative prefetch included.  Written by every call. */
 size_t art_workspace_tiles_read_offset(const art_shape* shape);
 
+/* Byte offset inside a workspace of art_q8_workspace_bytes(shape) bytes of the
+ * int32 array vskip[B, Hkv, num_splits][2]: for each (batch, kv head, split),
+ * the V rows left out of every query head's numerator by the V skip (page
+ * "La Elegancia de la Omision": exp(s_j - m') < tau for every head of the group)
+ * and the V tiles not read at all because every row of every head was left out.
+ * Written by the two-pass q8 implementation (art_decode_attn_q8_skipv without
+ * ART, two-pass path) only; other calls leave it untouched. */
+size_t art_workspace_vskip_offset(const art_shape* shape);
+
 /* Byte offset inside ws of the int32 array split_tiles[B, Hq, num_splits]:
  * KV tiles consumed by each (batch, query head, split) in the last call (the
  * per-split terms of `tiles`).  Written by every call. */

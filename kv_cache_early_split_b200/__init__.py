@@ -51,6 +51,16 @@ class DeviceProblem:
         return self.ws[off:off + 4 * n].view(torch.int32).view(s.B, s.Hkv, s.num_splits)
 
 
+    def vskip_counts(self):
+        """int32 [B, Hkv, S, 2]: V rows left out of every head's numerator and V tiles not read,
+        by the last two-pass q8 call (device tensor view; needs the q8 workspace)."""
+        import torch
+
+        off = capi.art_workspace_vskip_offset(self.shape)
+        s = self.shape
+        n = s.B * s.Hkv * s.num_splits * 2
+        return self.ws[off:off + 4 * n].view(torch.int32).view(s.B, s.Hkv, s.num_splits, 2)
+
     def split_tiles(self):
         """int32 [B, Hq, S]: KV tiles consumed per split by the last call (device tensor view)."""
         import torch

@@ -33,6 +33,7 @@ EXPORTS = (
     "art_q8_workspace_bytes",
     "art_workspace_tiles_read_offset",
     "art_workspace_split_tiles_offset",
+    "art_workspace_vskip_offset",
     "art_decode_attn_full",
     "art_decode_attn_terminate",
     "art_decode_attn_terminate_noalloc",
@@ -121,6 +122,8 @@ def _bind(L: ctypes.CDLL) -> ctypes.CDLL:
     L.art_workspace_tiles_read_offset.argtypes = [_SH]
     L.art_workspace_split_tiles_offset.restype = ctypes.c_size_t
     L.art_workspace_split_tiles_offset.argtypes = [_SH]
+    L.art_workspace_vskip_offset.restype = ctypes.c_size_t
+    L.art_workspace_vskip_offset.argtypes = [_SH]
     L.art_decode_attn_full.restype = ctypes.c_int
     L.art_decode_attn_full.argtypes = [_SH, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
     L.art_decode_attn_terminate.restype = ctypes.c_int
@@ -182,6 +185,10 @@ def art_workspace_tiles_read_offset(shape: art_shape) -> int:
 
 def art_workspace_split_tiles_offset(shape: art_shape) -> int:
     return int(lib().art_workspace_split_tiles_offset(ctypes.byref(shape)))
+
+
+def art_workspace_vskip_offset(shape: art_shape) -> int:
+    return int(lib().art_workspace_vskip_offset(ctypes.byref(shape)))
 
 
 def art_decode_attn_full(shape, dtype, q, k, v, seq_lens, o, tiles, ws, ws_bytes, stream) -> int:

@@ -694,6 +694,11 @@ size_t art_q8_workspace_bytes(const art_shape* shape) {
   return q8_ws_total(shape);
 }
 
+size_t art_workspace_vskip_offset(const art_shape* shape) {
+  if (!shape_ok(shape) || shape->Hq % shape->Hkv != 0) return 0;
+  return artk::q8two::layout2(q8_dims(shape), ws_layout(shape).total).vskip;
+}
+
 size_t art_workspace_tiles_read_offset(const art_shape* shape) {
   if (!shape_ok(shape)) return 0;
   return ws_layout(shape).tiles_read;

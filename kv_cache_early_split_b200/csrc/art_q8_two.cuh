@@ -49,6 +49,7 @@ struct Params {
   float* tmax;             // [B*Hkv][n_max][G]  tile maxima
   float* cmax;             // [B*Hkv*S][CPS][G]  chunk maxima
   float* part;             // [B*Hq*S][CPS][2 + D]  chunk states (m, l, acc)
+  int32_t* vskip;          // [B*Hkv*S][2]  rows left out of every head's numerator, V tiles not read
   int B, Hq, Hkv, L_max, T, S, G, GP, CT, CPS, n_max;
   float qscale, tau;
 };
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_kernel(const __grid_constant_
   constexpr int SLOT = Gm::SLOT_CODES + Gm::SLOT_SCALES;  // no scores in this pass's ring
   __shared__ __align__(16) uint8_t s_ring[NW][P][SLOT];
   __shared__ float s_cm[NW][GP];
+  if (blockIdx.x == 0 && threadIdx.x < 2) p.vskip[blockIdx.y * 2 + threadIdx.x] = 0;  // counted by pass 2
   const Range r = cta_range(p);
   if (r.c0 >= r.t1) return;  // empty chunk
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -350,6 +352,8 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Pa
       if (lane == 31) s_ref[g] = mpj;
     }
     if (lane < nct) s_live[lane] = live ? 1 : 0;
+    const unsigned dead = __ballot_sync(0xffffffffu, lane < nct && !live);
+    if (lane == 0 && dead) atomicAdd(&p.vskip[unit * 2 + 1], __popc(dead));
   }
   __syncthreads();
 
@@ -405,6 +409,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Pa
     for (int i = 0; i < EPT / 2; ++i) acc[h][i] = make_float2(0.f, 0.f);
   float l = 0.f, mp = 0.f, fac = 0.f;
   bool live = false;
+  int nskip = 0;  // rows of this lane's row slot left out of every head's numerator
   auto body = [&](int k) {
     if (wc.ik == 0) {
       // a new tile: m'_t of this lane's head; fac = 2^(m'_t - ref) turns a skip-test weight into
@@ -431,6 +436,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Pa
       w[h] = __shfl_sync(0xffffffffu, wk, rsub * GP + h);
       any |= w[h] > 0.f;
     }
+    if (sub == 0 && !any && wc.row0 + rsub < wc.rend) ++nskip;
     if (any) {  // otherwise the row is not dequantised
       uint32_t cw[EPT / 4];
       lds_codes<EPT>(slot + rsub * D + sub * EPT, cw);
@@ -463,6 +469,12 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Pa
     __syncwarp();
   }
   cp_async_wait<0>();
+  {
+    int ns_w = nskip;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ns_w += __shfl_xor_sync(0xffffffffu, ns_w, off);
+    if (lane == 0 && ns_w) atomicAdd(&p.vskip[unit * 2], ns_w);
+  }
 
   // sum over the row groups of the warp, then over the warps
 #pragma unroll
@@ -574,7 +586,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace arrays after the common ones (which end at `base`), sized for the smallest chunk.
 struct Layout2 {
-  size_t scores, tmax, cmax, part, end;
+  size_t scores, tmax, cmax, part, vskip, end;
   int n_max, CT, CPS;
 };
 
@@ -590,7 +602,8 @@ inline Layout2 layout2(const Dims& s, size_t base) {
   q.tmax = align256(q.scores + 4 * bk * size_t(s.L_max) * gp_of(G));
   q.cmax = align256(q.tmax + 4 * bk * size_t(q.n_max) * G);
   q.part = align256(q.cmax + 4 * units * size_t(q.CPS) * G);
-  q.end = align256(q.part + 4 * units * G * size_t(q.CPS) * (size_t(s.d) + 2));
+  q.vskip = align256(q.part + 4 * units * G * size_t(q.CPS) * (size_t(s.d) + 2));
+  q.end = align256(q.vskip + 8 * units);
   return q;
 }
 
@@ -668,6 +681,7 @@ inline cudaError_t launch(const Dims& s, const uint16_t* q, const int8_t* k, con
   p.tmax = reinterpret_cast<float*>(ws + ql.tmax);
   p.cmax = reinterpret_cast<float*>(ws + ql.cmax);
   p.part = reinterpret_cast<float*>(ws + ql.part);
+  p.vskip = reinterpret_cast<int32_t*>(ws + ql.vskip);
   p.B = s.B;
   p.Hq = s.Hq;
   p.Hkv = s.Hkv;
