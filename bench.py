@@ -62,9 +62,14 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweeps", action="store_true",
                     help="time the workload's two modes only (no other workloads, sweeps or extras)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="profiling: the workload's first N sequences only (bit-identical slabs); "
+                         "implies --no-sweeps, and the line is no bench value (config.batch_of says so)")
     a = ap.parse_args(argv)
     if a.mode is None:
         a.mode = "q8_art" if a.workload.startswith("q8") else "art"
+    if a.batch:
+        a.no_sweeps = True
     return a
 
 
@@ -277,7 +282,8 @@ def config_obj(w, mode, args, world):
         "l2": ("L2 flushed (512 MiB write) before every timed launch; step time = the launches' own time"
                if needs_flush(w) else "no flush: KV inputs larger than the 126 MB L2"),
         "parallelism": f"replicas x{world} (weak scaling)" if world > 1 else "single GPU",
-    }
+    } | ({"batch_of": f"first {w.B} sequences of the workload (profiling case, not a bench value)"}
+         if getattr(args, "batch", 0) else {})
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -655,7 +661,7 @@ def run_ours(args):
         torch.cuda.set_device(local)
         init_dist(world, "nccl")
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = I.workload(args.workload)
+    w = I.workload(args.workload, keys_b=list(range(args.batch)) if args.batch else None)
     dp = K.upload(w, device=dev)
     stream = torch.cuda.Stream(device=dev)
     heads = w.B * w.Hq
