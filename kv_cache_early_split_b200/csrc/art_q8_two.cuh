@@ -302,6 +302,220 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_kernel(const __grid_constant_
   }
 }
 
+// ------------------------------------------------------------------ pass 1 on the tensor cores (d = 128, G <= 4)
+// The same outputs as q8_scores_kernel, with the dot products on the tensor cores through warp-level
+// m16n8k16 MMAs (f16 operands, fp32 accumulators): a warp takes 16 rows per group.  A = the rows'
+// K codes, converted exactly to f16 in registers (codes are integers in [-127, 127]); B = the
+// queries as 8 columns, the f16 part of each head's scaled query and the f16 of what that leaves
+// over (≈ 22 bits).  Each 16-wide k-step lies inside one 32-wide scale block and accumulates into
+// that block's accumulator, so each row's four K scales apply in fp32 after the MMAs, exactly as in
+// the CUDA-core pass.  Within a k-step, lane (g, t) supplies positions 4t..4t+3 of the step as MMA
+// k-indices {2t, 2t+1, 2t+8, 2t+9} — one 4-byte word per row — and its B fragment uses the same
+// order (a dot product does not depend on the order of its terms).
+namespace mma16 {
+constexpr int ROWS = 16;                  // rows per group (the MMA's M)
+constexpr int PAD = 144;                  // bytes per staged row: 128 codes + 16 (spreads the banks)
+constexpr int SLOT_CODES = ROWS * PAD;    // 2304
+constexpr int SLOT = SLOT_CODES + ROWS * 8;  // + four fp16 scales per row
+constexpr int PM = 4;                     // ring slots per warp
+constexpr int SMEM = NW * PM * SLOT;      // dynamic shared memory per CTA
+
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Four codes (one word) as two f16 pairs: (code 0, code 1) and (code 2, code 3).  u = c + 128 as a
+// byte, 0x6400 | u is the f16 1024 + u, and subtracting 1152 leaves c exactly.
+__device__ __forceinline__ void word_to_h2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));  // 1152
+  uint32_t x = __byte_perm(u, 0x64646464u, 0x4140u), y = __byte_perm(u, 0x64646464u, 0x4342u);
+  const __half2 a = __hsub2(*reinterpret_cast<const __half2*>(&x), bias);
+  const __half2 b = __hsub2(*reinterpret_cast<const __half2*>(&y), bias);
+  lo = *reinterpret_cast<const uint32_t*>(&a);
+  hi = *reinterpret_cast<const uint32_t*>(&b);
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float x, float y) {
+  __half2 h = __floats2half2_rn(x, y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+}  // namespace mma16
+
+template <int GP>
+__global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_constant__ Params p) {
+  constexpr int D = 128, NB = 4;
+  static_assert(GP <= 4, "4 heads (hi + lo) fill the MMA's 8 columns");
+  extern __shared__ __align__(16) uint8_t s_dyn[];
+  __shared__ float s_cm[NW][4];
+  if (blockIdx.x == 0 && threadIdx.x < 2) p.vskip[blockIdx.y * 2 + threadIdx.x] = 0;  // counted by pass 2
+  const Range r = cta_range(p);
+  if (r.c0 >= r.t1) return;  // empty chunk
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;  // MMA fragment coordinates
+  const int unit = blockIdx.y;
+  const int bk = unit / p.S;
+  const int b = bk / p.Hkv, kvh = bk % p.Hkv;
+  const int T = p.T, G = p.G;
+
+  // B fragments: column n = g is head g's scaled query (hi part) for g < 4, head g - 4's remainder
+  // for g >= 4; step s, lane t holds positions 16 s + 4 t + {0, 1} (b0) and + {2, 3} (b1).
+  uint32_t bq[8][2];
+  {
+    const int hq = g & 3;
+    const bool lo_part = g >= 4;
+    const bool live = hq < G;
+    const long long qrow = static_cast<long long>(b) * p.Hq + kvh * G + (live ? hq : 0);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      float f[4];
+      const uint2 qw = *reinterpret_cast<const uint2*>(p.q + qrow * D + 16 * s + 4 * t);
+      const uint32_t qv[2] = {qw.x, qw.y};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        f[2 * e] = __uint_as_float(qv[e] << 16) * p.qscale;
+        f[2 * e + 1] = __uint_as_float(qv[e] & 0xffff0000u) * p.qscale;
+      }
+      float v[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float h = __half2float(__float2half_rn(f[e]));
+        v[e] = live ? (lo_part ? f[e] - h : h) : 0.f;
+      }
+      bq[s][0] = mma16::pack_h2(v[0], v[1]);
+      bq[s][1] = mma16::pack_h2(v[2], v[3]);
+    }
+  }
+
+  const int8_t* kb = p.k + static_cast<long long>(bk) * p.L_max * D;
+  const uint16_t* ksb = p.ks + static_cast<long long>(bk) * p.L_max * NB;
+  float* scb = p.scores + static_cast<long long>(bk) * p.L_max * GP;
+  const int ipt = T / mma16::ROWS;
+  const int nct = r.c1 - r.c0;
+  const int niter = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ipt;
+  uint8_t* ring = s_dyn + warp * mma16::PM * mma16::SLOT;
+  const uint32_t ring_a = smem_u32(ring);
+  // copies of a group: lane l takes 64 code bytes of row l / 2 (4 x 16 B) and, for l < 16, row l's
+  // scales (8 B); rows past the end are not copied (their stale results are not used)
+  Walk wi, wc;
+  wi.start(r, warp, T);
+  wc = wi;
+  int ki = 0;
+  auto issue = [&]() {
+    if (ki < niter) {
+      const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::SLOT;
+      const int rc = lane >> 1, row = wi.row0 + rc;
+      if (row < wi.rend) {
+        const int8_t* src = kb + static_cast<long long>(row) * D + (lane & 1) * 64;
+        const uint32_t dst = slot + rc * mma16::PAD + (lane & 1) * 64;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cp_async<16>(dst + 16 * j, src + 16 * j);
+      }
+      if (lane < mma16::ROWS && wi.row0 + lane < wi.rend)
+        cp_async<8>(slot + mma16::SLOT_CODES + lane * 8, ksb + static_cast<long long>(wi.row0 + lane) * NB);
+      wi.next(r, T, ipt, mma16::ROWS);
+    }
+    ++ki;
+    cp_async_commit();
+  };
+
+  // per head h in {2t, 2t + 1} (lanes t < 2), rows g and g + 8
+  float cm[2] = {-INFINITY, -INFINITY}, tm[2] = {-INFINITY, -INFINITY};
+  auto body = [&](int k) {
+    const uint8_t* slot = ring + (k % mma16::PM) * mma16::SLOT;
+    float acc[NB][4];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t w0 = *reinterpret_cast<const uint32_t*>(slot + g * mma16::PAD + 16 * s + 4 * t);
+      const uint32_t w1 = *reinterpret_cast<const uint32_t*>(slot + (g + 8) * mma16::PAD + 16 * s + 4 * t);
+      uint32_t a[4];
+      mma16::word_to_h2(w0, a[0], a[2]);
+      mma16::word_to_h2(w1, a[1], a[3]);
+      mma16::mma_f16(acc[s >> 1], a, bq[s][0], bq[s][1]);
+    }
+    // columns 2t, 2t + 1: heads 2t, 2t + 1 (hi part) for t < 2, their remainders for t >= 2
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] += __shfl_xor_sync(0xffffffffu, acc[j][e], 2);
+    const uint2 s0 = *reinterpret_cast<const uint2*>(slot + mma16::SLOT_CODES + g * 8);
+    const uint2 s1 = *reinterpret_cast<const uint2*>(slot + mma16::SLOT_CODES + (g + 8) * 8);
+    const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&s0.x));
+    const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&s0.y));
+    const float2 b0 = __half22float2(*reinterpret_cast<const __half2*>(&s1.x));
+    const float2 b1 = __half22float2(*reinterpret_cast<const __half2*>(&s1.y));
+    const float sc0[NB] = {a0.x, a0.y, a1.x, a1.y}, sc1[NB] = {b0.x, b0.y, b1.x, b1.y};
+    float v[2][2];  // [row g / g + 8][head 2t / 2t + 1]
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      v[0][e] = 0.f;
+      v[1][e] = 0.f;
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        v[0][e] = fmaf(sc0[j], acc[j][e], v[0][e]);
+        v[1][e] = fmaf(sc1[j], acc[j][2 + e], v[1][e]);
+      }
+    }
+    if (t < 2) {
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int row = wc.row0 + g + 8 * rr;
+        if (row < wc.rend) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = 2 * t + e;
+            if (h < G) {
+              scb[static_cast<long long>(row) * GP + h] = v[rr][e];
+              tm[e] = fmaxf(tm[e], v[rr][e]);
+            }
+          }
+        }
+      }
+    }
+    if (wc.ik == ipt - 1) {
+      // last group of tile wc.t: the maximum per head over the rows (lanes of the same t)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) tm[e] = fmaxf(tm[e], __shfl_xor_sync(0xffffffffu, tm[e], off));
+        if (g == 0 && t < 2 && 2 * t + e < G) p.tmax[(static_cast<long long>(bk) * p.n_max + wc.t) * G + 2 * t + e] = tm[e];
+        cm[e] = fmaxf(cm[e], tm[e]);
+        tm[e] = -INFINITY;
+      }
+    }
+    wc.next(r, T, ipt, mma16::ROWS);
+  };
+
+#pragma unroll 1
+  for (int k = 0; k < mma16::PM - 1; ++k) issue();
+#pragma unroll 1
+  for (int k = 0; k < niter; ++k) {
+    issue();
+    cp_async_wait<mma16::PM - 1>();  // group k has landed (this lane's copies) ...
+    __syncwarp();                    // ... and every lane's
+    body(k);
+    __syncwarp();  // every lane is done with the slot before it is refilled
+  }
+  cp_async_wait<0>();
+  if (g == 0 && t < 2) {
+    s_cm[warp][2 * t] = cm[0];
+    s_cm[warp][2 * t + 1] = cm[1];
+  }
+  __syncthreads();
+  if (static_cast<int>(threadIdx.x) < G) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) m = fmaxf(m, s_cm[w][threadIdx.x]);
+    p.cmax[(static_cast<long long>(unit) * p.CPS + blockIdx.x) * G + threadIdx.x] = m;
+  }
+}
+
 // ------------------------------------------------------------------ pass 2: weights, skip, PV
 template <int D, int GP>
 __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Params p) {
@@ -634,7 +848,21 @@ inline int choose_ct(const Dims& s, int sms) {
 template <int D, int GP>
 cudaError_t launch_dg(const Params& p, cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>(p.CPS), static_cast<unsigned>(p.B * p.Hkv * p.S));
-  q8_scores_kernel<D, GP><<<grid, NT, 0, st>>>(p);
+  if constexpr (D == 128 && GP == 4) {  // pass 1 on the tensor cores
+    static bool attr_set[64] = {};  // the dynamic shared-memory limit, raised once per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+      e = cudaFuncSetAttribute(q8_scores_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::SMEM);
+      if (e != cudaSuccess) return e;
+      attr_set[dev] = true;
+    }
+    q8_scores_mma_kernel<GP><<<grid, NT, mma16::SMEM, st>>>(p);
+  } else {
+    q8_scores_kernel<D, GP><<<grid, NT, 0, st>>>(p);
+  }
   q8_pv_kernel<D, GP><<<grid, NT, 0, st>>>(p);
   q8_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p);
   return cudaGetLastError();

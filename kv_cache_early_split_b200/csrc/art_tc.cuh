@@ -1287,12 +1287,13 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
       const bool remote = C > 1;  // the tile's publication lives in CTA c of the cluster
       const uint32_t pub_c = remote ? map_to_rank(smem_u32(pub), c) : smem_u32(pub);
       // The part of a round that needs no earlier round: this lane's tile (m, l, probe) from the CTA
-      // that computed it (tiles at or past nv stay empty) ...
-      auto load_tile = [&](uint32_t slot, bool valid, int g, float& m, float& l, float (&a)[PC]) {
+      // that computed it (tiles at or past nv stay empty) ...  The probe lanes are held as pairs:
+      // the arithmetic below runs on packed f32x2 instructions.
+      auto load_tile = [&](uint32_t slot, bool valid, int g, float& m, float& l, float2 (&a)[PC / 2]) {
         m = -INFINITY;
         l = 0.f;
 #pragma unroll
-        for (int k = 0; k < PC; ++k) a[k] = 0.f;
+        for (int k = 0; k < PC / 2; ++k) a[k] = make_float2(0.f, 0.f);
         if (valid) {
           const uint32_t e = static_cast<uint32_t>(i * GP + g);
           m = ld_smem_f32(slot + 4 * e, remote);
@@ -1301,13 +1302,14 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
 #pragma unroll
           for (int k = 0; k < PC; k += 4) {
             const float4 v = ld_smem_v4(px + 4 * k, remote);
-            a[k] = v.x, a[k + 1] = v.y, a[k + 2] = v.z, a[k + 3] = v.w;
+            a[k / 2] = make_float2(v.x, v.y);
+            a[k / 2 + 1] = make_float2(v.z, v.w);
           }
         }
       };
       // ... merged with the round's earlier tiles of the same head: an inclusive scan over the head's
       // segment of TQ lanes.
-      auto scan_tiles = [&](float& m, float& l, float (&a)[PC]) {
+      auto scan_tiles = [&](float& m, float& l, float2 (&a)[PC / 2]) {
         // a loop, not unrolled: the controller's instruction footprint costs more than the loop
 #pragma unroll 1
         for (int off = 1; off < TQ; off <<= 1) {
@@ -1319,17 +1321,19 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           const float co = take ? rescale_fast(mo, M) : 0.f;
           l = cs * l + co * lo;
           m = take ? M : m;
+          const float2 cs2 = make_float2(cs, cs), co2 = make_float2(co, co);
 #pragma unroll
-          for (int k = 0; k < PC; ++k) {
-            const float ao = __shfl_up_sync(0xffffffffu, a[k], off, TQ);
-            a[k] = cs * a[k] + co * ao;
+          for (int k = 0; k < PC / 2; ++k) {
+            const float2 ao = make_float2(__shfl_up_sync(0xffffffffu, a[k].x, off, TQ),
+                                          __shfl_up_sync(0xffffffffu, a[k].y, off, TQ));
+            a[k] = __ffma2_rn(cs2, a[k], __fmul2_rn(co2, ao));
           }
         }
       };
       // The part that needs the state carried over from earlier rounds: prepend it, evaluate the rule
       // at every tile of the round, find the stop, and carry the state of the head's last replayed
       // tile (the stop, or the round's last tile) into the next round.
-      auto replay_round = [&](int r, int sl, int nv, int g, float m, float l, float (&a)[PC]) {
+      auto replay_round = [&](int r, int sl, int nv, int g, float m, float l, float2 (&a)[PC / 2]) {
         const bool active = g < G;
         const int gs = active ? g : 0;
         float* R_f = rf + gs * RF_SIZE;
@@ -1343,39 +1347,39 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
         l = aR * lR + aS * l;
         m = Mf;
         const float inv_l = __fdividef(1.f, l);
-        float x[PC], sq[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 aR2 = make_float2(aR, aR), aS2 = make_float2(aS, aS), il2 = make_float2(inv_l, inv_l);
+        float2 x[PC / 2], sq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int k = 0; k < PC; k += 4) {
           const float4 ar = *reinterpret_cast<const float4*>(R_f + RF_A + k);
-          a[k] = aR * ar.x + aS * a[k];
-          a[k + 1] = aR * ar.y + aS * a[k + 1];
-          a[k + 2] = aR * ar.z + aS * a[k + 2];
-          a[k + 3] = aR * ar.w + aS * a[k + 3];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            x[k + u] = a[k + u] * inv_l;
-            sq[u] = fmaf(x[k + u], x[k + u], sq[u]);
-          }
+          a[k / 2] = __ffma2_rn(aR2, make_float2(ar.x, ar.y), __fmul2_rn(aS2, a[k / 2]));
+          a[k / 2 + 1] = __ffma2_rn(aR2, make_float2(ar.z, ar.w), __fmul2_rn(aS2, a[k / 2 + 1]));
+          x[k / 2] = __fmul2_rn(a[k / 2], il2);
+          x[k / 2 + 1] = __fmul2_rn(a[k / 2 + 1], il2);
+          sq[0] = __ffma2_rn(x[k / 2], x[k / 2], sq[0]);
+          sq[1] = __ffma2_rn(x[k / 2 + 1], x[k / 2 + 1], sq[1]);
         }
-        const float nrm = __fsqrt_rn((sq[0] + sq[1]) + (sq[2] + sq[3]));
+        const float nrm = __fsqrt_rn((sq[0].x + sq[1].x) + (sq[0].y + sq[1].y));
         float nrmp = __shfl_up_sync(0xffffffffu, nrm, 1, TQ);
         if (q == 0) nrmp = st.z;
         const bool both = nrm > 0.f && nrmp > 0.f;
         const float in = both ? __fdividef(1.f, nrm) : 0.f, ip = both ? __fdividef(1.f, nrmp) : 0.f;
-        float dq[4] = {0.f, 0.f, 0.f, 0.f};
+        const float2 in2 = make_float2(in, in), nip2 = make_float2(-ip, -ip);
+        float2 dq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int k = 0; k < PC; k += 4) {
           const float4 xr = *reinterpret_cast<const float4*>(R_f + RF_XP + k);
-          const float xrv[4] = {xr.x, xr.y, xr.z, xr.w};
+          const float2 xrv[2] = {make_float2(xr.x, xr.y), make_float2(xr.z, xr.w)};
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float xp = __shfl_up_sync(0xffffffffu, x[k + u], 1, TQ);
+          for (int u = 0; u < 2; ++u) {
+            float2 xp = make_float2(__shfl_up_sync(0xffffffffu, x[k / 2 + u].x, 1, TQ),
+                                    __shfl_up_sync(0xffffffffu, x[k / 2 + u].y, 1, TQ));
             if (q == 0) xp = xrv[u];
-            const float dl = x[k + u] * in - xp * ip;
-            dq[u] = fmaf(dl, dl, dq[u]);
+            const float2 dl = __ffma2_rn(x[k / 2 + u], in2, __fmul2_rn(xp, nip2));
+            dq[u] = __ffma2_rn(dl, dl, dq[u]);
           }
         }
-        const float dd2 = (dq[0] + dq[1]) + (dq[2] + dq[3]);
+        const float dd2 = (dq[0].x + dq[1].x) + (dq[0].y + dq[1].y);
         const float d_scale = fabsf(nrm - nrmp);
         const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd2);
         const bool hold = valid && (d_scale < p.eps_scale) && (d_dir < p.eps_dir);
@@ -1394,8 +1398,8 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           *reinterpret_cast<float4*>(R_f) = make_float4(m, l, nrm, 0.f);
 #pragma unroll
           for (int k = 0; k < PC; k += 4) {
-            *reinterpret_cast<float4*>(R_f + RF_A + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
-            *reinterpret_cast<float4*>(R_f + RF_XP + k) = make_float4(x[k], x[k + 1], x[k + 2], x[k + 3]);
+            *reinterpret_cast<float4*>(R_f + RF_A + k) = make_float4(a[k / 2].x, a[k / 2].y, a[k / 2 + 1].x, a[k / 2 + 1].y);
+            *reinterpret_cast<float4*>(R_f + RF_XP + k) = make_float4(x[k / 2].x, x[k / 2].y, x[k / 2 + 1].x, x[k / 2 + 1].y);
           }
           R_i[RI_RUN] = runq;
           if (stop >= 0) {
@@ -1413,7 +1417,8 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
         // each scanning one round while the other replays the previous one, ran several times slower.)
         const int g = hh;
         auto tile_valid = [&](int r) { return g < G && q < t1 - (t0 + r * TQ); };
-        float m, l, a[PC];
+        float m, l;
+        float2 a[PC / 2];
         int okw = 1;
         if (R > 0) {
           if (lane == 0) okw = wait_phase(bar(B_XFULL), 0, ctl, false, p.ws_status, true);
@@ -1425,7 +1430,8 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           const int nv = max(0, min(TQ, t1 - (t0 + r * TQ)));
           scan_tiles(m, l, a);
           const int r1 = r + 1, sl1 = r1 % NSLOT;
-          float m1, l1, a1[PC];
+          float m1, l1;
+          float2 a1[PC / 2];
           int pre = 0;
           if (r1 < R) {
             if (lane == 0) pre = mbar_test_wait_cluster(bar(B_XFULL + sl1), (r1 / NSLOT) & 1);
@@ -1462,7 +1468,7 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           m = m1;
           l = l1;
 #pragma unroll
-          for (int k = 0; k < PC; ++k) a[k] = a1[k];
+          for (int k = 0; k < PC / 2; ++k) a[k] = a1[k];
         }
       } else {
         // Two warps, each replaying half of the heads, round after round.
@@ -1477,7 +1483,8 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           for (int g0 = cw * HPP; g0 < G; g0 += 2 * HPP) {
             const int g = g0 + hh;
             const bool sb = g >= G || ri[g * RI_SIZE + RI_STOPPED] != 0;
-            float m, l, a[PC];
+            float m, l;
+            float2 a[PC / 2];
             load_tile(pub_c + sl * PB::SLOT, !sb && q < nv, g, m, l, a);
             scan_tiles(m, l, a);
             replay_round(r, sl, nv, g, m, l, a);
