@@ -516,6 +516,254 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
   }
 }
 
+// ------------------------------------------------------------------ pass 2 on the tensor cores (d = 128, G <= 4)
+// The same outputs as q8_pv_kernel, with the weighted sum of V rows on the tensor cores: per group of
+// 16 rows and per scale block, O^T += P'^T-shaped A (16 x 16: M = head g's weights times the V scale
+// as f16 hi in row g and lo in row g + 8, K = the 16 rows) times B (16 rows x 8 positions of V, the
+// codes converted exactly to f16).  In n-tile (block b, j) column n is position 32 b + 4 n + j, so a
+// lane's V bytes for a row and block are one 4-byte word.  Weights, the skip test, the denominators
+// and the counters are formed as in q8_pv_kernel: one lane per (row, head) pair, two pairs per lane.
+namespace mma16 {
+constexpr int PV_SLOT = SLOT_CODES + ROWS * 8 + ROWS * 16;  // codes, V scales, scores (4 per row)
+constexpr int PV_RING = NW * PM * PV_SLOT;
+constexpr int PV_ACC = NW * 4 * 128 * 4;
+constexpr int PV_SMEM = PV_RING > PV_ACC ? PV_RING : PV_ACC;
+__device__ __forceinline__ uint32_t pack_hh(__half a, __half b) {
+  __half2 h = __halves2half2(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+}  // namespace mma16
+
+template <int GP>
+__global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant__ Params p) {
+  constexpr int D = 128, NB = 4;
+  static_assert(GP == 4, "one lane per (row, head) pair over 8 rows: four heads");
+  extern __shared__ __align__(16) uint8_t s_dyn[];  // the ring while the rows stream, then the accumulators
+  __shared__ float s_mp[CTMAX][4], s_ref[4];
+  __shared__ int s_live[CTMAX];
+  __shared__ float s_l[NW][4];
+  const Range r = cta_range(p);
+  if (r.c0 >= r.t1) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int unit = blockIdx.y;
+  const int bk = unit / p.S, split = unit % p.S;
+  const int b = bk / p.Hkv, kvh = bk % p.Hkv;
+  const int T = p.T, G = p.G;
+  const float tau = p.tau;
+  const int nct = r.c1 - r.c0;  // <= CTMAX
+
+  // running maxima m'_t, the chunk's reference and the tiles left unread, as in q8_pv_kernel
+  if (warp == 0) {
+    const float* cm = p.cmax + static_cast<long long>(unit) * p.CPS * G;
+    bool live = false;
+    for (int h = 0; h < G; ++h) {
+      float m = -INFINITY;
+      for (int c = lane; c < static_cast<int>(blockIdx.x); c += 32) m = fmaxf(m, cm[c * G + h]);
+      m = warp_max(m);
+      const float own = lane < nct ? p.tmax[(static_cast<long long>(bk) * p.n_max + r.c0 + lane) * G + h]
+                                   : -INFINITY;
+      float x = own;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x = fmaxf(x, y);
+      }
+      const float mpj = fmaxf(m, x);
+      if (lane < nct) {
+        s_mp[lane][h] = mpj;
+        if (!(exp2f(own - mpj) < tau)) live = true;
+      }
+      if (lane == 31) s_ref[h] = mpj;
+    }
+    if (lane < nct) s_live[lane] = live ? 1 : 0;
+    const unsigned dead = __ballot_sync(0xffffffffu, lane < nct && !live);
+    if (lane == 0 && dead) atomicAdd(&p.vskip[unit * 2 + 1], __popc(dead));
+  }
+  __syncthreads();
+
+  const int8_t* vb = p.v + static_cast<long long>(bk) * p.L_max * D;
+  const uint16_t* vsb = p.vs + static_cast<long long>(bk) * p.L_max * NB;
+  const float* scb = p.scores + static_cast<long long>(bk) * p.L_max * GP;
+  const int ipt = T / mma16::ROWS;
+  const int niter = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ipt;
+  uint8_t* ring = s_dyn + warp * mma16::PM * mma16::PV_SLOT;
+  const uint32_t ring_a = smem_u32(ring);
+  constexpr int OFF_VS = mma16::SLOT_CODES, OFF_SC = mma16::SLOT_CODES + mma16::ROWS * 8;
+  // copies of a group: lane l takes 64 code bytes of row l / 2; lanes 0..15 the V scales of row l,
+  // lanes 16..31 the scores of row l - 16.  Rows past the end are not copied; a tile left unread
+  // copies its scores only.
+  Walk wi, wc;
+  wi.start(r, warp, T);
+  wc = wi;
+  int ki = 0;
+  auto issue = [&]() {
+    if (ki < niter) {
+      const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::PV_SLOT;
+      const bool live_t = s_live[wi.t - r.c0] != 0;
+      const int rc = lane >> 1;
+      if (live_t && wi.row0 + rc < wi.rend) {
+        const int8_t* src = vb + static_cast<long long>(wi.row0 + rc) * D + (lane & 1) * 64;
+        const uint32_t dst = slot + rc * mma16::PAD + (lane & 1) * 64;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cp_async<16>(dst + 16 * j, src + 16 * j);
+      }
+      const int rs = lane & 15;
+      if (wi.row0 + rs < wi.rend) {
+        if (lane < 16) {
+          if (live_t) cp_async<8>(slot + OFF_VS + rs * 8, vsb + static_cast<long long>(wi.row0 + rs) * NB);
+        } else {
+          cp_async<16>(slot + OFF_SC + rs * 16, scb + static_cast<long long>(wi.row0 + rs) * GP);
+        }
+      }
+      wi.next(r, T, ipt, mma16::ROWS);
+    }
+    ++ki;
+    cp_async_commit();
+  };
+
+  float acc[16][4];  // n-tile (block b, j) = 4 b + j
+#pragma unroll
+  for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float l = 0.f, mp = 0.f, fac = 0.f;
+  bool live = false;
+  int nskip = 0;
+  const bool head_ok = t < G;
+  auto body = [&](int k) {
+    if (wc.ik == 0) {  // a new tile: m'_t of this lane's head and the factor to the chunk's reference
+      const int j = wc.t - r.c0;
+      mp = head_ok ? s_mp[j][t] : 0.f;
+      fac = head_ok ? exp2f(mp - s_ref[t]) : 0.f;
+      live = s_live[j] != 0;
+    }
+    const uint8_t* slot = ring + (k % mma16::PM) * mma16::PV_SLOT;
+    // weights of rows g and g + 8 for head t
+    float wk[2];
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int row = g + 8 * rr;
+      const bool ok = head_ok && wc.row0 + row < wc.rend;
+      const float sj = ok ? reinterpret_cast<const float*>(slot + OFF_SC + row * 16)[t] : -INFINITY;
+      const float pj = exp2f(sj - mp);  // 0 for rows past the end and padded heads
+      const float wj = pj * fac;
+      l += wj;  // skipped rows stay in the denominator
+      wk[rr] = (live && !(pj < tau) && pj > 0.f) ? wj : 0.f;
+    }
+    const unsigned kb0 = __ballot_sync(0xffffffffu, wk[0] > 0.f), kb1 = __ballot_sync(0xffffffffu, wk[1] > 0.f);
+    if (t == 0) {  // rows g and g + 8 left out of every head's numerator
+      if (wc.row0 + g < wc.rend && ((kb0 >> (4 * g)) & 0xFu) == 0u) ++nskip;
+      if (wc.row0 + g + 8 < wc.rend && ((kb1 >> (4 * g)) & 0xFu) == 0u) ++nskip;
+    }
+    if ((kb0 | kb1) != 0u) {  // otherwise no row of the group is dequantised
+      // A: head g's weights (g < 4) for rows 2t, 2t + 1, 2t + 8, 2t + 9 times each row's V scale
+      const int src = 8 * t + (g & 3);
+      const float w0 = __shfl_sync(0xffffffffu, wk[0], src), w1 = __shfl_sync(0xffffffffu, wk[0], src + 4);
+      const float w2 = __shfl_sync(0xffffffffu, wk[1], src), w3 = __shfl_sync(0xffffffffu, wk[1], src + 4);
+      const uint2 s0 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t) * 8);
+      const uint2 s1 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 1) * 8);
+      const uint2 s2 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 8) * 8);
+      const uint2 s3 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 9) * 8);
+      const uint2 sv[4] = {s0, s1, s2, s3};
+      const float wv[4] = {w0, w1, w2, w3};
+      const int vrow[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
+      uint32_t vw[4][NB];  // [row][block]: this lane's 4 code bytes, positions 32 b + 4 g .. + 3
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb)
+          vw[i][bb] = *reinterpret_cast<const uint32_t*>(slot + vrow[i] * mma16::PAD + 32 * bb + 4 * g) ^ 0x80808080u;
+      const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));  // 1152
+#pragma unroll
+      for (int bb = 0; bb < NB; ++bb) {
+        float x[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t sw = (bb < 2) ? sv[i].x : sv[i].y;
+          const float scale = __half2float(__ushort_as_half(static_cast<unsigned short>((bb & 1) ? (sw >> 16) : (sw & 0xffffu))));
+          x[i] = (wv[i] != 0.f) ? wv[i] * scale : 0.f;  // (the scale of a row not copied may be anything)
+        }
+        uint32_t a[4] = {0u, 0u, 0u, 0u};
+        if (g < 4) {
+          __half hi[4], lo[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            hi[i] = __float2half_rn(x[i]);
+            lo[i] = __float2half_rn(x[i] - __half2float(hi[i]));
+          }
+          a[0] = mma16::pack_hh(hi[0], hi[1]);
+          a[1] = mma16::pack_hh(lo[0], lo[1]);
+          a[2] = mma16::pack_hh(hi[2], hi[3]);
+          a[3] = mma16::pack_hh(lo[2], lo[3]);
+        }
+        // B: rows (2t, 2t + 1) and (2t + 8, 2t + 9) at position 32 b + 4 g + j, for j = 0..3
+        const uint32_t pa0 = __byte_perm(vw[0][bb], vw[1][bb], 0x5140u), pb0 = __byte_perm(vw[0][bb], vw[1][bb], 0x7362u);
+        const uint32_t pa1 = __byte_perm(vw[2][bb], vw[3][bb], 0x5140u), pb1 = __byte_perm(vw[2][bb], vw[3][bb], 0x7362u);
+        const uint32_t p0[2] = {pa0, pb0}, p1[2] = {pa1, pb1};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t x0 = __byte_perm(p0[j >> 1], 0x64646464u, (j & 1) ? 0x4342u : 0x4140u);
+          uint32_t x1 = __byte_perm(p1[j >> 1], 0x64646464u, (j & 1) ? 0x4342u : 0x4140u);
+          const __half2 h0 = __hsub2(*reinterpret_cast<const __half2*>(&x0), bias);
+          const __half2 h1 = __hsub2(*reinterpret_cast<const __half2*>(&x1), bias);
+          mma16::mma_f16(acc[4 * bb + j], a, *reinterpret_cast<const uint32_t*>(&h0),
+                         *reinterpret_cast<const uint32_t*>(&h1));
+        }
+      }
+    }
+    wc.next(r, T, ipt, mma16::ROWS);
+  };
+
+#pragma unroll 1
+  for (int k = 0; k < mma16::PM - 1; ++k) issue();
+#pragma unroll 1
+  for (int k = 0; k < niter; ++k) {
+    issue();
+    cp_async_wait<mma16::PM - 1>();
+    __syncwarp();
+    body(k);
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  {
+    int ns_w = nskip;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ns_w += __shfl_xor_sync(0xffffffffu, ns_w, off);
+    if (lane == 0 && ns_w) atomicAdd(&p.vskip[unit * 2], ns_w);
+  }
+  // the denominators: lanes of the same head t
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+  __syncthreads();  // every warp is done with its ring before the accumulators overwrite it
+  float* s_acc = reinterpret_cast<float*>(s_dyn);  // [NW][4][D]
+  if (g < 4) {  // head g: hi (row g) + lo (row g + 8) at positions 32 b + 4 (2t) + j and 32 b + 4 (2t + 1) + j
+#pragma unroll
+    for (int bb = 0; bb < NB; ++bb)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s_acc[(warp * 4 + g) * D + 32 * bb + 4 * (2 * t) + j] = acc[4 * bb + j][0] + acc[4 * bb + j][2];
+        s_acc[(warp * 4 + g) * D + 32 * bb + 4 * (2 * t + 1) + j] = acc[4 * bb + j][1] + acc[4 * bb + j][3];
+      }
+  }
+  if (lane < 4) s_l[warp][lane] = l;
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * D; idx += NT) {
+    const int h = idx / D, dd = idx % D;
+    float a = 0.f;
+#pragma unroll
+    for (int w2 = 0; w2 < NW; ++w2) a += s_acc[(w2 * 4 + h) * D + dd];
+    const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + h;
+    float* dst = p.part + ((hq * p.S + split) * p.CPS + blockIdx.x) * (2 + D);
+    dst[2 + dd] = a;
+    if (dd == 0) {
+      float lsum = 0.f;
+#pragma unroll
+      for (int w2 = 0; w2 < NW; ++w2) lsum += s_l[w2][h];
+      dst[0] = s_ref[h];
+      dst[1] = lsum;
+    }
+  }
+}
+
 // ------------------------------------------------------------------ pass 2: weights, skip, PV
 template <int D, int GP>
 __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Params p) {
@@ -848,7 +1096,7 @@ inline int choose_ct(const Dims& s, int sms) {
 template <int D, int GP>
 cudaError_t launch_dg(const Params& p, cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>(p.CPS), static_cast<unsigned>(p.B * p.Hkv * p.S));
-  if constexpr (D == 128 && GP == 4) {  // pass 1 on the tensor cores
+  if constexpr (D == 128 && GP == 4) {  // both passes on the tensor cores
     static bool attr_set[64] = {};  // the dynamic shared-memory limit, raised once per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -857,13 +1105,16 @@ cudaError_t launch_dg(const Params& p, cudaStream_t st) {
     if (!attr_set[dev]) {
       e = cudaFuncSetAttribute(q8_scores_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::SMEM);
       if (e != cudaSuccess) return e;
+      e = cudaFuncSetAttribute(q8_pv_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::PV_SMEM);
+      if (e != cudaSuccess) return e;
       attr_set[dev] = true;
     }
     q8_scores_mma_kernel<GP><<<grid, NT, mma16::SMEM, st>>>(p);
+    q8_pv_mma_kernel<GP><<<grid, NT, mma16::PV_SMEM, st>>>(p);
   } else {
     q8_scores_kernel<D, GP><<<grid, NT, 0, st>>>(p);
+    q8_pv_kernel<D, GP><<<grid, NT, 0, st>>>(p);
   }
-  q8_pv_kernel<D, GP><<<grid, NT, 0, st>>>(p);
   q8_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p);
   return cudaGetLastError();
 }
