@@ -307,18 +307,24 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_kernel(const __grid_constant_
 // m16n8k16 MMAs (f16 operands, fp32 accumulators): a warp takes 16 rows per group.  A = the rows'
 // K codes, converted exactly to f16 in registers (codes are integers in [-127, 127]); B = the
 // queries as 8 columns, the f16 part of each head's scaled query and the f16 of what that leaves
-// over (≈ 22 bits).  Each 16-wide k-step lies inside one 32-wide scale block and accumulates into
-// that block's accumulator, so each row's four K scales apply in fp32 after the MMAs, exactly as in
-// the CUDA-core pass.  Within a k-step, lane (g, t) supplies positions 4t..4t+3 of the step as MMA
-// k-indices {2t, 2t+1, 2t+8, 2t+9} — one 4-byte word per row — and its B fragment uses the same
-// order (a dot product does not depend on the order of its terms).
+// over (≈ 22 bits), side by side (column 2h: head h's hi part, 2h + 1: its remainder), so lane
+// (g, t) finds head t's two parts of rows g and g + 8 in its own accumulators.  Each 16-wide k-step
+// lies inside one 32-wide scale block and accumulates into that block's accumulator, so each row's
+// four K scales apply in fp32 after the MMAs, exactly as in the CUDA-core pass.  In block b, lane
+// (g, t) supplies positions 32 b + 8 t .. + 3 to the first k-step and + 4 .. + 7 to the second, as
+// MMA k-indices {2t, 2t+1, 2t+8, 2t+9} — 8 bytes of each row per block — and its B fragment uses
+// the same order (a dot product does not depend on the order of its terms).
 namespace mma16 {
 constexpr int ROWS = 16;                  // rows per group (the MMA's M)
 constexpr int PAD = 144;                  // bytes per staged row: 128 codes + 16 (spreads the banks)
 constexpr int SLOT_CODES = ROWS * PAD;    // 2304
 constexpr int SLOT = SLOT_CODES + ROWS * 8;  // + four fp16 scales per row
 constexpr int PM = 4;                     // ring slots per warp
-constexpr int SMEM = NW * PM * SLOT;      // dynamic shared memory per CTA
+// the scores pass reads 8 bytes per row and block: rows 160 bytes apart keep each half-warp's
+// 8-byte loads on distinct banks
+constexpr int PAD_S = 160;
+constexpr int SLOT_S = ROWS * PAD_S + ROWS * 8;
+constexpr int SMEM = NW * PM * SLOT_S;    // dynamic shared memory per CTA (scores pass)
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -362,18 +368,19 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
   const int b = bk / p.Hkv, kvh = bk % p.Hkv;
   const int T = p.T, G = p.G;
 
-  // B fragments: column n = g is head g's scaled query (hi part) for g < 4, head g - 4's remainder
-  // for g >= 4; step s, lane t holds positions 16 s + 4 t + {0, 1} (b0) and + {2, 3} (b1).
+  // B fragments: column n = g is head g / 2's scaled query, its f16 part for even g, the remainder
+  // for odd g; in step s (block s / 2) lane t holds positions 32 (s / 2) + 8 t + 4 (s % 2) + {0, 1}
+  // (b0) and + {2, 3} (b1).
   uint32_t bq[8][2];
   {
-    const int hq = g & 3;
-    const bool lo_part = g >= 4;
+    const int hq = g >> 1;
+    const bool lo_part = (g & 1) != 0;
     const bool live = hq < G;
     const long long qrow = static_cast<long long>(b) * p.Hq + kvh * G + (live ? hq : 0);
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
       float f[4];
-      const uint2 qw = *reinterpret_cast<const uint2*>(p.q + qrow * D + 16 * s + 4 * t);
+      const uint2 qw = *reinterpret_cast<const uint2*>(p.q + qrow * D + 32 * (s >> 1) + 8 * t + 4 * (s & 1));
       const uint32_t qv[2] = {qw.x, qw.y};
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -397,8 +404,9 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
   const int ipt = T / mma16::ROWS;
   const int nct = r.c1 - r.c0;
   const int niter = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ipt;
-  uint8_t* ring = s_dyn + warp * mma16::PM * mma16::SLOT;
+  uint8_t* ring = s_dyn + warp * mma16::PM * mma16::SLOT_S;
   const uint32_t ring_a = smem_u32(ring);
+  constexpr int OFF_KS = mma16::ROWS * mma16::PAD_S;
   // copies of a group: lane l takes 64 code bytes of row l / 2 (4 x 16 B) and, for l < 16, row l's
   // scales (8 B); rows past the end are not copied (their stale results are not used)
   Walk wi, wc;
@@ -407,87 +415,73 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
   int ki = 0;
   auto issue = [&]() {
     if (ki < niter) {
-      const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::SLOT;
+      const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::SLOT_S;
       const int rc = lane >> 1, row = wi.row0 + rc;
       if (row < wi.rend) {
         const int8_t* src = kb + static_cast<long long>(row) * D + (lane & 1) * 64;
-        const uint32_t dst = slot + rc * mma16::PAD + (lane & 1) * 64;
+        const uint32_t dst = slot + rc * mma16::PAD_S + (lane & 1) * 64;
 #pragma unroll
         for (int j = 0; j < 4; ++j) cp_async<16>(dst + 16 * j, src + 16 * j);
       }
       if (lane < mma16::ROWS && wi.row0 + lane < wi.rend)
-        cp_async<8>(slot + mma16::SLOT_CODES + lane * 8, ksb + static_cast<long long>(wi.row0 + lane) * NB);
+        cp_async<8>(slot + OFF_KS + lane * 8, ksb + static_cast<long long>(wi.row0 + lane) * NB);
       wi.next(r, T, ipt, mma16::ROWS);
     }
     ++ki;
     cp_async_commit();
   };
 
-  // per head h in {2t, 2t + 1} (lanes t < 2), rows g and g + 8
-  float cm[2] = {-INFINITY, -INFINITY}, tm[2] = {-INFINITY, -INFINITY};
+  // head t (lanes with t < G), rows g and g + 8
+  float cm = -INFINITY, tm = -INFINITY;
   auto body = [&](int k) {
-    const uint8_t* slot = ring + (k % mma16::PM) * mma16::SLOT;
+    const uint8_t* slot = ring + (k % mma16::PM) * mma16::SLOT_S;
     float acc[NB][4];
 #pragma unroll
     for (int j = 0; j < NB; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      const uint32_t w0 = *reinterpret_cast<const uint32_t*>(slot + g * mma16::PAD + 16 * s + 4 * t);
-      const uint32_t w1 = *reinterpret_cast<const uint32_t*>(slot + (g + 8) * mma16::PAD + 16 * s + 4 * t);
+    for (int bb = 0; bb < NB; ++bb) {
+      const uint2 w0 = *reinterpret_cast<const uint2*>(slot + g * mma16::PAD_S + 32 * bb + 8 * t);
+      const uint2 w1 = *reinterpret_cast<const uint2*>(slot + (g + 8) * mma16::PAD_S + 32 * bb + 8 * t);
       uint32_t a[4];
-      mma16::word_to_h2(w0, a[0], a[2]);
-      mma16::word_to_h2(w1, a[1], a[3]);
-      mma16::mma_f16(acc[s >> 1], a, bq[s][0], bq[s][1]);
+      mma16::word_to_h2(w0.x, a[0], a[2]);
+      mma16::word_to_h2(w1.x, a[1], a[3]);
+      mma16::mma_f16(acc[bb], a, bq[2 * bb][0], bq[2 * bb][1]);
+      mma16::word_to_h2(w0.y, a[0], a[2]);
+      mma16::word_to_h2(w1.y, a[1], a[3]);
+      mma16::mma_f16(acc[bb], a, bq[2 * bb + 1][0], bq[2 * bb + 1][1]);
     }
-    // columns 2t, 2t + 1: heads 2t, 2t + 1 (hi part) for t < 2, their remainders for t >= 2
-#pragma unroll
-    for (int j = 0; j < NB; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[j][e] += __shfl_xor_sync(0xffffffffu, acc[j][e], 2);
-    const uint2 s0 = *reinterpret_cast<const uint2*>(slot + mma16::SLOT_CODES + g * 8);
-    const uint2 s1 = *reinterpret_cast<const uint2*>(slot + mma16::SLOT_CODES + (g + 8) * 8);
+    // columns 2t (f16 part) and 2t + 1 (remainder) of head t, rows g (0, 1) and g + 8 (2, 3)
+    const uint2 s0 = *reinterpret_cast<const uint2*>(slot + OFF_KS + g * 8);
+    const uint2 s1 = *reinterpret_cast<const uint2*>(slot + OFF_KS + (g + 8) * 8);
     const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&s0.x));
     const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&s0.y));
     const float2 b0 = __half22float2(*reinterpret_cast<const __half2*>(&s1.x));
     const float2 b1 = __half22float2(*reinterpret_cast<const __half2*>(&s1.y));
     const float sc0[NB] = {a0.x, a0.y, a1.x, a1.y}, sc1[NB] = {b0.x, b0.y, b1.x, b1.y};
-    float v[2][2];  // [row g / g + 8][head 2t / 2t + 1]
+    float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      v[0][e] = 0.f;
-      v[1][e] = 0.f;
-#pragma unroll
-      for (int j = 0; j < NB; ++j) {
-        v[0][e] = fmaf(sc0[j], acc[j][e], v[0][e]);
-        v[1][e] = fmaf(sc1[j], acc[j][2 + e], v[1][e]);
-      }
+    for (int j = 0; j < NB; ++j) {
+      v0 = fmaf(sc0[j], acc[j][0] + acc[j][1], v0);
+      v1 = fmaf(sc1[j], acc[j][2] + acc[j][3], v1);
     }
-    if (t < 2) {
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int row = wc.row0 + g + 8 * rr;
-        if (row < wc.rend) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int h = 2 * t + e;
-            if (h < G) {
-              scb[static_cast<long long>(row) * GP + h] = v[rr][e];
-              tm[e] = fmaxf(tm[e], v[rr][e]);
-            }
-          }
-        }
+    if (t < G) {
+      const int row0 = wc.row0 + g;
+      if (row0 < wc.rend) {
+        scb[static_cast<long long>(row0) * GP + t] = v0;
+        tm = fmaxf(tm, v0);
+      }
+      if (row0 + 8 < wc.rend) {
+        scb[static_cast<long long>(row0 + 8) * GP + t] = v1;
+        tm = fmaxf(tm, v1);
       }
     }
     if (wc.ik == ipt - 1) {
-      // last group of tile wc.t: the maximum per head over the rows (lanes of the same t)
+      // last group of tile wc.t: the maximum of head t over the rows (lanes of the same t)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) tm[e] = fmaxf(tm[e], __shfl_xor_sync(0xffffffffu, tm[e], off));
-        if (g == 0 && t < 2 && 2 * t + e < G) p.tmax[(static_cast<long long>(bk) * p.n_max + wc.t) * G + 2 * t + e] = tm[e];
-        cm[e] = fmaxf(cm[e], tm[e]);
-        tm[e] = -INFINITY;
-      }
+      for (int off = 4; off < 32; off <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, off));
+      if (g == 0 && t < G) p.tmax[(static_cast<long long>(bk) * p.n_max + wc.t) * G + t] = tm;
+      cm = fmaxf(cm, tm);
+      tm = -INFINITY;
     }
     wc.next(r, T, ipt, mma16::ROWS);
   };
@@ -503,10 +497,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
     __syncwarp();  // every lane is done with the slot before it is refilled
   }
   cp_async_wait<0>();
-  if (g == 0 && t < 2) {
-    s_cm[warp][2 * t] = cm[0];
-    s_cm[warp][2 * t + 1] = cm[1];
-  }
+  if (g == 0) s_cm[warp][t] = cm;
   __syncthreads();
   if (static_cast<int>(threadIdx.x) < G) {
     float m = -INFINITY;
