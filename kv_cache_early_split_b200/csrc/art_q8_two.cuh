@@ -588,6 +588,11 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   wi.start(r, warp, T);
   wc = wi;
   int ki = 0;
+  // the V-scale areas of this warp's ring start as zeros: a row never copied then scales to a finite
+  // value, and its weight (zero) keeps it out of the sum
+  for (int i = lane; i < mma16::PM * mma16::ROWS * 2; i += 32)
+    reinterpret_cast<uint32_t*>(ring + (i / (mma16::ROWS * 2)) * mma16::PV_SLOT + OFF_VS)[i % (mma16::ROWS * 2)] = 0u;
+  __syncwarp();
   auto issue = [&]() {
     if (ki < niter) {
       const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::PV_SLOT;
@@ -654,41 +659,38 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       const uint2 s1 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 1) * 8);
       const uint2 s2 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 8) * 8);
       const uint2 s3 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 9) * 8);
-      const uint2 sv[4] = {s0, s1, s2, s3};
-      const float wv[4] = {w0, w1, w2, w3};
+      // (V scales of a row not copied: an earlier row's, or zero)
+      const uint32_t sv[4][2] = {{s0.x, s0.y}, {s1.x, s1.y}, {s2.x, s2.y}, {s3.x, s3.y}};
       const int vrow[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
-      uint32_t vw[4][NB];  // [row][block]: this lane's 4 code bytes, positions 32 b + 4 g .. + 3
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int bb = 0; bb < NB; ++bb)
-          vw[i][bb] = *reinterpret_cast<const uint32_t*>(slot + vrow[i] * mma16::PAD + 32 * bb + 4 * g) ^ 0x80808080u;
       const __half2 bias = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6480)));  // 1152
 #pragma unroll
       for (int bb = 0; bb < NB; ++bb) {
-        float x[4];
+        uint32_t vw[4];  // this lane's 4 code bytes of each row, positions 32 b + 4 g .. + 3
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          vw[i] = *reinterpret_cast<const uint32_t*>(slot + vrow[i] * mma16::PAD + 32 * bb + 4 * g) ^ 0x80808080u;
+        float sc[4];  // the four rows' scales of block bb
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint32_t sw = (bb < 2) ? sv[i].x : sv[i].y;
-          const float scale = __half2float(__ushort_as_half(static_cast<unsigned short>((bb & 1) ? (sw >> 16) : (sw & 0xffffu))));
-          x[i] = (wv[i] != 0.f) ? wv[i] * scale : 0.f;  // (the scale of a row not copied may be anything)
+          const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sv[i][bb >> 1]));
+          sc[i] = (bb & 1) ? s2.y : s2.x;
         }
         uint32_t a[4] = {0u, 0u, 0u, 0u};
-        if (g < 4) {
-          __half hi[4], lo[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            hi[i] = __float2half_rn(x[i]);
-            lo[i] = __float2half_rn(x[i] - __half2float(hi[i]));
-          }
-          a[0] = mma16::pack_hh(hi[0], hi[1]);
-          a[1] = mma16::pack_hh(lo[0], lo[1]);
-          a[2] = mma16::pack_hh(hi[2], hi[3]);
-          a[3] = mma16::pack_hh(lo[2], lo[3]);
+        if (g < 4) {  // weight x scale of rows (2t, 2t + 1) and (2t + 8, 2t + 9): f16 part and remainder
+          const float2 x01 = __fmul2_rn(make_float2(w0, w1), make_float2(sc[0], sc[1]));
+          const float2 x23 = __fmul2_rn(make_float2(w2, w3), make_float2(sc[2], sc[3]));
+          const __half2 h01 = __float22half2_rn(x01), h23 = __float22half2_rn(x23);
+          const float2 m1 = make_float2(-1.f, -1.f);
+          const __half2 l01 = __float22half2_rn(__ffma2_rn(__half22float2(h01), m1, x01));
+          const __half2 l23 = __float22half2_rn(__ffma2_rn(__half22float2(h23), m1, x23));
+          a[0] = *reinterpret_cast<const uint32_t*>(&h01);
+          a[1] = *reinterpret_cast<const uint32_t*>(&l01);
+          a[2] = *reinterpret_cast<const uint32_t*>(&h23);
+          a[3] = *reinterpret_cast<const uint32_t*>(&l23);
         }
         // B: rows (2t, 2t + 1) and (2t + 8, 2t + 9) at position 32 b + 4 g + j, for j = 0..3
-        const uint32_t pa0 = __byte_perm(vw[0][bb], vw[1][bb], 0x5140u), pb0 = __byte_perm(vw[0][bb], vw[1][bb], 0x7362u);
-        const uint32_t pa1 = __byte_perm(vw[2][bb], vw[3][bb], 0x5140u), pb1 = __byte_perm(vw[2][bb], vw[3][bb], 0x7362u);
+        const uint32_t pa0 = __byte_perm(vw[0], vw[1], 0x5140u), pb0 = __byte_perm(vw[0], vw[1], 0x7362u);
+        const uint32_t pa1 = __byte_perm(vw[2], vw[3], 0x5140u), pb1 = __byte_perm(vw[2], vw[3], 0x7362u);
         const uint32_t p0[2] = {pa0, pb0}, p1[2] = {pa1, pb1};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
