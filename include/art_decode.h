@@ -81,7 +81,9 @@ typedef enum {
   ART_ERR_TIMEOUT = -5,     /* device: a bounded wait gave up (status word) */
   ART_ERR_SEQLEN = -6,      /* device: a seq_len outside [1, L_max] (status word) */
   ART_ERR_ORDER = -7,       /* device: a tile_order entry outside its split (status word) */
-  ART_ERR_PAGE = -8         /* device: a block_table entry outside [0, num_pages) (status word) */
+  ART_ERR_PAGE = -8,        /* device: a block_table entry outside [0, num_pages) (status word) */
+  ART_ERR_INDEX = -9        /* device, debug build (-DART_DEBUG) only: an index check of a kernel
+                               failed (status word); regular builds never report it */
 } art_status;
 
 typedef enum { ART_F32 = 0, ART_BF16 = 1 } art_dtype;

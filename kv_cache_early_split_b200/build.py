@@ -47,6 +47,12 @@ SHORT_WAIT_LIB = os.path.join(PKG, "libart_decode_shortwait.so")
 SHORT_WAIT_FLAGS = ["-DART_TC_WAIT_LIMIT_CYCLES=1000LL"]
 
 
+# The debug build: the same sources with the device index checks compiled in (ART_DCHECK): a failed
+# check sets the status word's index bit and the call reports ART_ERR_INDEX -- no trap, no fault.
+DEBUG_LIB = os.path.join(PKG, "libart_decode_debug.so")
+DEBUG_FLAGS = ["-DART_DEBUG"]
+
+
 def needs_build(lib: str = LIB) -> bool:
     if not os.path.exists(lib):
         return True
@@ -57,6 +63,11 @@ def needs_build(lib: str = LIB) -> bool:
 def build_short_wait(force: bool = False) -> str:
     """The short-wait test build (see SHORT_WAIT_FLAGS)."""
     return build(force=force, lib=SHORT_WAIT_LIB, extra_flags=SHORT_WAIT_FLAGS)
+
+
+def build_debug(force: bool = False) -> str:
+    """The debug build with device index checks (see DEBUG_FLAGS)."""
+    return build(force=force, lib=DEBUG_LIB, extra_flags=DEBUG_FLAGS)
 
 
 def build(force: bool = False, verbose: bool = False, lib: str = LIB, extra_flags=()) -> str:
@@ -97,3 +108,5 @@ if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
     if "--short-wait" in sys.argv:
         print(build_short_wait(force="--force" in sys.argv))
+    if "--debug" in sys.argv:
+        print(build_debug(force="--force" in sys.argv))

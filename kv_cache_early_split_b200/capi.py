@@ -22,6 +22,7 @@ ART_ERR_TIMEOUT = -5
 ART_ERR_SEQLEN = -6
 ART_ERR_ORDER = -7
 ART_ERR_PAGE = -8
+ART_ERR_INDEX = -9  # debug build (-DART_DEBUG) only
 ART_F32 = 0
 ART_BF16 = 1
 ART_KV_F32, ART_KV_BF16, ART_KV_Q8 = 0, 1, 2

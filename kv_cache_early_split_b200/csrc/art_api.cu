@@ -949,6 +949,7 @@ art_status art_read_device_status(void* ws, void* stream) {
   if (h & artk::kStatusTimeout) return ART_ERR_TIMEOUT;
   if (h & artk::kStatusOrder) return ART_ERR_ORDER;
   if (h & artk::kStatusPage) return ART_ERR_PAGE;
+  if (h & artk::kStatusIndex) return ART_ERR_INDEX;
   return ART_OK;
 }
 
@@ -983,6 +984,7 @@ const char* art_status_string(art_status status) {
     case ART_ERR_SEQLEN: return "ART_ERR_SEQLEN";
     case ART_ERR_ORDER: return "ART_ERR_ORDER";
     case ART_ERR_PAGE: return "ART_ERR_PAGE";
+    case ART_ERR_INDEX: return "ART_ERR_INDEX";
   }
   return "ART_ERR_UNKNOWN";
 }

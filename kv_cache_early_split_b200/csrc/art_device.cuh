@@ -13,6 +13,21 @@ constexpr int kStatusSeqLen = 1;
 constexpr int kStatusTimeout = 2;
 constexpr int kStatusOrder = 4;  // a traversal-sequence entry outside its split
 constexpr int kStatusPage = 8;   // a block-table entry outside the page pool
+constexpr int kStatusIndex = 16;  // a device index check of a debug build failed
+
+// Device index checks of the debug build (-DART_DEBUG): a failed check sets the status word's
+// index bit (the call then reports ART_ERR_INDEX) and execution goes on -- no trap, so the check
+// can sit in front of any access.  Regular builds compile the checks away.
+#ifdef ART_DEBUG
+#define ART_DCHECK(cond, status)                             \
+  do {                                                       \
+    if (!(cond)) atomicOr((status), ::artk::kStatusIndex);   \
+  } while (0)
+#else
+#define ART_DCHECK(cond, status) \
+  do {                           \
+  } while (0)
+#endif
 
 // A wait gives up after this many nanoseconds of %globaltimer time.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;

@@ -358,6 +358,9 @@ __global__ void __launch_bounds__(NT, 1) art_decode_kernel(const __grid_constant
       }
       row = (static_cast<long long>(pg) * p.Hkv + kvh) * p.page_size + pos0 % p.page_size;
     }
+    ART_DCHECK(t >= t0 && t < t1 && rows >= 1 && rows <= T, p.ws_status);
+    ART_DCHECK(p.block_table || t * T + rows <= p.L_max, p.ws_status);
+    ART_DCHECK(stage < p.nstage, p.ws_status);
     uint32_t bytes = 2u * rows * ROWB;
     uint32_t sbytes = 0;
     if constexpr (KIND == KV_Q8) {

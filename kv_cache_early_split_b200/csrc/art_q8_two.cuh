@@ -479,6 +479,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
       // last group of tile wc.t: the maximum of head t over the rows (lanes of the same t)
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, off));
+      ART_DCHECK(wc.t >= r.c0 && wc.t < r.c1 && wc.t < p.n_max, p.ws_status);
       if (g == 0 && t < G) p.tmax[(static_cast<long long>(bk) * p.n_max + wc.t) * G + t] = tm;
       cm = fmaxf(cm, tm);
       tm = -INFINITY;
@@ -596,6 +597,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   auto issue = [&]() {
     if (ki < niter) {
       const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::PV_SLOT;
+      ART_DCHECK(wi.t >= r.c0 && wi.t < r.c1 && wi.t - r.c0 < CTMAX && wi.row0 >= wi.t * T && wi.row0 < (wi.t + 1) * T, p.ws_status);
       const bool live_t = s_live[wi.t - r.c0] != 0;
       const int rc = lane >> 1;
       if (live_t && wi.row0 + rc < wi.rend) {

@@ -472,6 +472,7 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
           break;
         const int j = jl * C + rank;
         const int p0 = pbeg + j * BLK;
+        ART_DCHECK(j < nblk && p0 >= 0 && p0 < p.L_max && (p0 & 1) == 0, p.ws_status);  // (scales: row pairs)
         const uint32_t fb = bar(B_RAWF + rs);
         const uint32_t st = smem_u32(sm + rs * Q8_RAW_BYTES);
         mbar_arrive_expect_tx(fb, Q8_RAW_BYTES);
@@ -514,6 +515,7 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
             if (ph != __ldg(ord_seq + t0 + j)) atomicOr(p.ws_status, kStatusOrder);
             p0 = ph * BLK;
           }
+          ART_DCHECK(j < nblk && p0 >= 0 && p0 < L, p.ws_status);
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           tma_load_3d(st, &p.tmK, fb, 0, p0, zc);
           tma_load_3d(st + 16384, &p.tmK, fb, 64, p0, zc);
@@ -1286,6 +1288,7 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
       const unsigned segmask = (TQ == 32) ? 0xffffffffu : ((1u << TQ) - 1u);
       const bool remote = C > 1;  // the tile's publication lives in CTA c of the cluster
       const uint32_t pub_c = remote ? map_to_rank(smem_u32(pub), c) : smem_u32(pub);
+      ART_DCHECK(c < C && TQ <= 32 && (32 % TQ) == 0, p.ws_status);
       // The part of a round that needs no earlier round: this lane's tile (m, l, probe) from the CTA
       // that computed it (tiles at or past nv stay empty) ...  The probe lanes are held as pairs:
       // the arithmetic below runs on packed f32x2 instructions.
@@ -1618,6 +1621,7 @@ __global__ void __launch_bounds__(Lay<Q8>::NTHR, 1) art_decode_tc_kernel(const _
     if (tid < G) {
       const long long hq = static_cast<long long>(b) * p.Hq + kvh * G + tid;
       const int used = bad_len ? 0 : (ART ? ri[tid * RI_SIZE + RI_USED] : ns);
+      ART_DCHECK(used >= 0 && used <= ns && hq < static_cast<long long>(p.B) * p.Hq, p.ws_status);
       p.ws_used[hq * p.S + split] = used;
       if (p.S == 1 && p.tiles) p.tiles[hq] = used;
     }

@@ -178,6 +178,7 @@ def test_kernel_name_query(L):
 def test_status_strings_new_codes(L):
     assert capi.art_status_string(capi.ART_ERR_ORDER) == "ART_ERR_ORDER"
     assert capi.art_status_string(capi.ART_ERR_PAGE) == "ART_ERR_PAGE"
+    assert capi.art_status_string(capi.ART_ERR_INDEX) == "ART_ERR_INDEX"
 
 
 def test_invalid_arguments_orders(L):
