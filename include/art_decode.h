@@ -72,6 +72,13 @@
 extern "C" {
 #endif
 
+/* The library is compiled with hidden visibility; only the declarations below are exported.
+ * That also keeps two builds of it (the regular and a test build) loaded in one process from
+ * sharing internal state, such as a once-per-device flag inside an inline function. */
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+
 typedef enum {
   ART_OK = 0,
   ART_ERR_INVALID_ARG = -1, /* a NULL pointer, a negative size, bad lanes ... */
@@ -374,6 +381,10 @@ const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_
 
 /* Static, human-readable name of a status code. */
 const char* art_status_string(art_status status);
+
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
 
 #ifdef __cplusplus
 }

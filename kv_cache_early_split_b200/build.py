@@ -28,6 +28,8 @@ NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC",
+    "-Xcompiler", "-fvisibility=hidden",
+    "-Xcompiler", "-fvisibility-inlines-hidden",
     "-Xptxas", "-v",
     "--expt-relaxed-constexpr",
 ]
