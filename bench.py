@@ -575,7 +575,7 @@ def vskip_sweep(K, args, stream, device):
                              "kv_bytes_read": bytes_read(w, dp.tiles_read().cpu().numpy()),
                              "mean_tiles_frac": float(dp.tiles.float().mean().item())
                              / float((-(-w.seq_lens.astype(np.int64) // w.tile)).mean())}
-                if mode == "q8" and K.kernel_name(dp, mode) == "q8_pv_kernel":
+                if mode == "q8" and K.kernel_name(dp, mode).startswith("q8_pv"):
                     vs = dp.vskip_counts().cpu().numpy().astype(np.int64)
                     rows_all = float(w.seq_lens.astype(np.int64).sum() * w.Hkv)
                     tiles_all = float((-(-w.seq_lens.astype(np.int64) // w.tile)).sum() * w.Hkv)
@@ -776,7 +776,8 @@ def run_ours(args):
     kernel = K.kernel_name(dp, args.mode)
     traffic = measured_traffic(w.name, args.mode, kernel)
     if launches_per_call(K, dp, w, args.mode) == 3:
-        kernel = "q8_scores_kernel + q8_pv_kernel + q8_combine_kernel (timed as one call)"
+        mma = "_mma" if kernel == "q8_pv_mma_kernel" else ""
+        kernel = f"q8_scores{mma}_kernel + q8_pv{mma}_kernel + q8_combine_kernel (timed as one call)"
     elif w.num_splits > 1:
         kernel += " (timed with its split combine kernel)"
     line = {

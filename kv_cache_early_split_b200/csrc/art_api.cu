@@ -965,8 +965,8 @@ const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_
     mode = with_art ? artk::MODE_ART : artk::MODE_FULL;
   }
   if (mode == artk::MODE_SKIP && (shape->d == 64 || shape->d == 128) && shape->Hq % shape->Hkv == 0 &&
-      shape->Hq / shape->Hkv <= artk::GMAX)
-    return "q8_pv_kernel";  // (two passes, given the q8 workspace)
+      shape->Hq / shape->Hkv <= artk::GMAX)  // two passes, given the q8 workspace
+    return (shape->d == 128 && artk::q8two::gp_of(shape->Hq / shape->Hkv) == 4) ? "q8_pv_mma_kernel" : "q8_pv_kernel";
   if (tc_eligible(kind, mode, shape)) return "art_decode_tc_kernel";
   KernelInfo ki;
   if (!pick_kernel(kind, mode, shape->d, shape->Hq / shape->Hkv, &ki)) return nullptr;

@@ -161,7 +161,8 @@ def test_kernel_name_query(L):
     # q8 ART with 3 or 4 heads per kv head, d = 128, tile 64 / 128, even L_max: the tensor cores;
     # q8 full attention: two streaming passes (the second named) given the q8 workspace
     assert capi.art_kernel_name(tc, capi.ART_BF16, True, True) == "art_decode_tc_kernel"
-    assert capi.art_kernel_name(tc, capi.ART_BF16, True, False) == "q8_pv_kernel"
+    assert capi.art_kernel_name(tc, capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
+    assert capi.art_kernel_name(shape(Hq=24, Hkv=8, d=128, tile=64), capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
     assert capi.art_kernel_name(shape(Hq=24, Hkv=8, d=128, tile=128), capi.ART_BF16, 1, 1) == "art_decode_tc_kernel"
     # other q8 shapes: full attention as two streaming passes (the second named), ART one pass
     q8o = shape(Hq=16, Hkv=8, d=128, tile=64)

@@ -54,7 +54,7 @@ def test_vskip_counts_match_oracle(tau, S):
     w = I.make_workload(kind="q8", B=2, Hq=8, Hkv=2, d=128, L_max=4096, tile=64, num_splits=S,
                         seq_lens=[4096, 2777], seed=61, sink=8.0, gumbel_scale=2.0, lognormal_v=True, tau=tau)
     dp = K.upload(w)
-    assert K.kernel_name(dp, "q8") == "q8_pv_kernel"
+    assert K.kernel_name(dp, "q8") == "q8_pv_mma_kernel"
     K.decode(dp, "q8", tau=tau, q8_path="two_pass")
     assert K.device_status(dp) == capi.ART_OK
     got = dp.vskip_counts().cpu().numpy().astype(np.int64)
