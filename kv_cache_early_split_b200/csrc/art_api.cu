@@ -267,6 +267,20 @@ bool make_q8_code_map(CUtensorMap* m, const void* base, const art_shape* s) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// q8 codes [B*Hkv][L_max][128] for the two-pass tensor-core path: box 128 bytes x 32 rows, 128-byte
+// swizzle (two row groups of the MMA per copy).
+bool make_q8_group_map(CUtensorMap* m, const void* base, const art_shape* s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(s->L_max), static_cast<cuuint64_t>(s->B) * s->Hkv};
+  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(s->L_max) * 128};
+  const cuuint32_t box[3] = {128, artk::q8two::mma16::STEP, 1};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // q8 scales [B*Hkv][L_max][4] fp16 viewed as [B*Hkv][L_max/2][16 bytes] (two rows per 16 bytes),
 // box 16 bytes x 64: the scales of 128 positions (L_max even).
 bool make_q8_scale_map(CUtensorMap* m, const void* base, const art_shape* s) {
@@ -648,8 +662,12 @@ art_status launch_q8two(const art_shape* s, const void* q, const int8_t* k, cons
                         const uint16_t* vs, const int32_t* seq_lens, float tau, float* o, int32_t* tiles, void* ws,
                         void* stream) {
   const WsLayout w = ws_layout(s);
+  CUtensorMap tmk, tmv;
+  const bool maps = artk::q8two::uses_maps(q8_dims(s));
+  if (maps && (!make_q8_group_map(&tmk, k, s) || !make_q8_group_map(&tmv, v, s))) return ART_ERR_CUDA;
   const cudaError_t e = artk::q8two::launch(q8_dims(s), static_cast<const uint16_t*>(q), k, ks, v, vs, seq_lens,
                                             tau, o, tiles, static_cast<uint8_t*>(ws), w.tiles_read, w.used, w.total,
+                                            maps ? &tmk : nullptr, maps ? &tmv : nullptr,
                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ART_OK : ART_ERR_CUDA;
 }
@@ -966,7 +984,7 @@ const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_
   }
   if (mode == artk::MODE_SKIP && (shape->d == 64 || shape->d == 128) && shape->Hq % shape->Hkv == 0 &&
       shape->Hq / shape->Hkv <= artk::GMAX)  // two passes, given the q8 workspace
-    return (shape->d == 128 && artk::q8two::gp_of(shape->Hq / shape->Hkv) == 4) ? "q8_pv_mma_kernel" : "q8_pv_kernel";
+    return artk::q8two::uses_maps(q8_dims(shape)) ? "q8_pv_mma_kernel" : "q8_pv_kernel";
   if (tc_eligible(kind, mode, shape)) return "art_decode_tc_kernel";
   KernelInfo ki;
   if (!pick_kernel(kind, mode, shape->d, shape->Hq / shape->Hkv, &ki)) return nullptr;

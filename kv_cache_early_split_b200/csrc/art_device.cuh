@@ -391,6 +391,13 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // The same check with acquire semantics at cluster scope (arrivals that come from other CTAs).
+// Programmatic dependent launch: a grid launched with programmatic stream serialisation may start
+// while the grid before it on the stream is still running; grid_dep_wait() returns once that grid has
+// completed and its memory operations are visible (at once when there is no such grid), and
+// grid_dep_launch() lets the next grid of the stream be scheduled before this one ends.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -20,6 +20,7 @@
 // scores per row.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -34,6 +35,7 @@ constexpr int P = 8;       // ring slots per warp (row groups in flight)
 constexpr int CTMAX = 32;  // tiles per chunk at most (one lane per tile in the in-chunk prefix)
 
 struct Params {
+  CUtensorMap tmK, tmV;  // tensor-core passes: K / V codes, boxes of 16 rows x 128 bytes, 128-byte swizzle
   const uint16_t* q;   // [B, Hq, D] bf16 bits
   const int8_t* k;     // [B, Hkv, L_max, D] codes
   const uint16_t* ks;  // [B, Hkv, L_max, D/32] fp16 bits
@@ -52,6 +54,7 @@ struct Params {
   int32_t* vskip;          // [B*Hkv*S][2]  rows left out of every head's numerator, V tiles not read
   int B, Hq, Hkv, L_max, T, S, G, GP, CT, CPS, n_max;
   float qscale, tau;
+  bool has_maps;  // tmK / tmV set
 };
 
 // Smallest chunk: at least 128 rows per warp where that stays within CTMAX tiles.
@@ -185,6 +188,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_kernel(const __grid_constant_
   constexpr int SLOT = Gm::SLOT_CODES + Gm::SLOT_SCALES;  // no scores in this pass's ring
   __shared__ __align__(16) uint8_t s_ring[NW][P][SLOT];
   __shared__ float s_cm[NW][GP];
+  grid_dep_launch();  // pass 2's CTAs may take the SMs this grid leaves (they wait for its results)
   if (blockIdx.x == 0 && threadIdx.x < 2) p.vskip[blockIdx.y * 2 + threadIdx.x] = 0;  // counted by pass 2
   const Range r = cta_range(p);
   if (r.c0 >= r.t1) return;  // empty chunk
@@ -315,16 +319,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_kernel(const __grid_constant_
 // MMA k-indices {2t, 2t+1, 2t+8, 2t+9} — 8 bytes of each row per block — and its B fragment uses
 // the same order (a dot product does not depend on the order of its terms).
 namespace mma16 {
-constexpr int ROWS = 16;                  // rows per group (the MMA's M)
-constexpr int PAD = 144;                  // bytes per staged row: 128 codes + 16 (spreads the banks)
-constexpr int SLOT_CODES = ROWS * PAD;    // 2304
-constexpr int SLOT = SLOT_CODES + ROWS * 8;  // + four fp16 scales per row
-constexpr int PM = 4;                     // ring slots per warp
-// the scores pass reads 8 bytes per row and block: rows 160 bytes apart keep each half-warp's
-// 8-byte loads on distinct banks
-constexpr int PAD_S = 160;
-constexpr int SLOT_S = ROWS * PAD_S + ROWS * 8;
-constexpr int SMEM = NW * PM * SLOT_S;    // dynamic shared memory per CTA (scores pass)
+constexpr int ROWS = 16;  // rows per group (the MMA's M)
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -350,6 +345,30 @@ __device__ __forceinline__ uint32_t pack_h2(float x, float y) {
   __half2 h = __floats2half2_rn(x, y);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+
+// The codes of a step (two groups, 32 rows of one tile) arrive as one TMA box of 32 rows x 128 bytes
+// with the 128-byte swizzle: the 16-byte chunk c of row R lands at chunk c ^ (R % 8), so a lane's
+// reads of rows g and g + 8 (and the PV pass's of rows 2t .. 2t + 9) fall on distinct banks with no
+// padding.  One copy instruction per 4 KiB: per-lane 16-byte copies, and then 2 KiB boxes, were
+// what bounded the passes (measured with the arithmetic taken out).
+constexpr int STEP = 32;
+constexpr int BOX = STEP * 128;
+constexpr int PB = 3;   // boxes per warp in flight, scores pass
+constexpr int PBV = 2;  // PV pass (its scores and scales take the rest of the shared memory)
+__device__ __forceinline__ uint32_t swz(int row, int byte) {
+  return static_cast<uint32_t>(row * 128 + ((((byte >> 4) ^ row) & 7) << 4) + (byte & 15));
+}
+// dynamic shared memory of the scores pass: 1 KiB of alignment slack (the swizzle wants 1 KiB
+// aligned boxes), then per warp PB boxes, PB x 32 rows of scales and PB barriers
+constexpr int TSM_SCALES = NW * PB * BOX;
+constexpr int TSM_BARS = TSM_SCALES + NW * PB * STEP * 8;
+constexpr int TSMEM = 1024 + TSM_BARS + NW * PB * 8;
+// the PV pass: per warp PBV boxes, PBV x 32 rows of V scales, PBV x 32 rows of scores (16 bytes each)
+// and PBV barriers; after the rows, the same memory holds the warps' accumulators
+constexpr int PSM_VS = NW * PBV * BOX;
+constexpr int PSM_SC = PSM_VS + NW * PBV * STEP * 8;
+constexpr int PSM_BARS = PSM_SC + NW * PBV * STEP * 16;
+constexpr int PSMEM_RING = 1024 + PSM_BARS + NW * PBV * 8;
 }  // namespace mma16
 
 template <int GP>
@@ -358,6 +377,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
   static_assert(GP <= 4, "4 heads (hi + lo) fill the MMA's 8 columns");
   extern __shared__ __align__(16) uint8_t s_dyn[];
   __shared__ float s_cm[NW][4];
+  grid_dep_launch();  // pass 2's CTAs may take the SMs this grid leaves (they wait for its results)
   if (blockIdx.x == 0 && threadIdx.x < 2) p.vskip[blockIdx.y * 2 + threadIdx.x] = 0;  // counted by pass 2
   const Range r = cta_range(p);
   if (r.c0 >= r.t1) return;  // empty chunk
@@ -398,50 +418,59 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
     }
   }
 
-  const int8_t* kb = p.k + static_cast<long long>(bk) * p.L_max * D;
   const uint16_t* ksb = p.ks + static_cast<long long>(bk) * p.L_max * NB;
   float* scb = p.scores + static_cast<long long>(bk) * p.L_max * GP;
-  const int ipt = T / mma16::ROWS;
+  const int ipt = T / mma16::ROWS, ips = T / mma16::STEP;  // groups and steps per tile (T >= 32)
   const int nct = r.c1 - r.c0;
-  const int niter = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ipt;
-  uint8_t* ring = s_dyn + warp * mma16::PM * mma16::SLOT_S;
-  const uint32_t ring_a = smem_u32(ring);
-  constexpr int OFF_KS = mma16::ROWS * mma16::PAD_S;
-  // copies of a group: lane l takes 64 code bytes of row l / 2 (4 x 16 B) and, for l < 16, row l's
-  // scales (8 B); rows past the end are not copied (their stale results are not used)
+  const int nsteps = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ips;
+  const uint32_t dyn = smem_u32(s_dyn), base = (dyn + 1023u) & ~1023u;
+  uint8_t* const codes = s_dyn + (base - dyn) + warp * mma16::PB * mma16::BOX;
+  uint8_t* const scales = s_dyn + (base - dyn) + mma16::TSM_SCALES + warp * mma16::PB * mma16::STEP * 8;
+  const uint32_t bars = base + mma16::TSM_BARS + warp * mma16::PB * 8;
+  if (lane == 0) {
+    for (int i = 0; i < mma16::PB; ++i) mbar_init(bars + 8 * i, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // copies of a step: one TMA box of 32 code rows (rows past the tensor's end read as zeros; rows
+  // past the sequence are copied and their results dropped; a step wholly past it copies nothing)
+  // and, lane l, row l's scales (8 B)
   Walk wi, wc;
   wi.start(r, warp, T);
   wc = wi;
-  int ki = 0;
+  int ks = 0;
+  uint32_t pend = 0u, phase = 0u;  // bit s: slot s has a box in flight / the parity it completes
   auto issue = [&]() {
-    if (ki < niter) {
-      const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::SLOT_S;
-      const int rc = lane >> 1, row = wi.row0 + rc;
-      if (row < wi.rend) {
-        const int8_t* src = kb + static_cast<long long>(row) * D + (lane & 1) * 64;
-        const uint32_t dst = slot + rc * mma16::PAD_S + (lane & 1) * 64;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) cp_async<16>(dst + 16 * j, src + 16 * j);
+    if (ks < nsteps) {
+      const int sl = ks % mma16::PB;
+      if (wi.row0 < wi.rend) {
+        ART_DCHECK(wi.row0 >= 0 && wi.row0 < p.L_max, p.ws_status);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bars + 8 * sl, mma16::BOX);
+          tma_load_3d(smem_u32(codes + sl * mma16::BOX), &p.tmK, bars + 8 * sl, 0, wi.row0, bk);
+        }
+        pend |= 1u << sl;
       }
-      if (lane < mma16::ROWS && wi.row0 + lane < wi.rend)
-        cp_async<8>(slot + OFF_KS + lane * 8, ksb + static_cast<long long>(wi.row0 + lane) * NB);
-      wi.next(r, T, ipt, mma16::ROWS);
+      if (wi.row0 + lane < wi.rend)
+        cp_async<8>(smem_u32(scales + sl * mma16::STEP * 8) + lane * 8, ksb + static_cast<long long>(wi.row0 + lane) * NB);
+      wi.next(r, T, ips, mma16::STEP);
     }
-    ++ki;
+    ++ks;
     cp_async_commit();
   };
 
-  // head t (lanes with t < G), rows g and g + 8
+  // head t (lanes with t < G), rows g and g + 8: the scores of a group ...
   float cm = -INFINITY, tm = -INFINITY;
-  auto body = [&](int k) {
-    const uint8_t* slot = ring + (k % mma16::PM) * mma16::SLOT_S;
+  auto scores = [&](int sl, int half, float& v0, float& v1) {
+    const uint8_t* box = codes + sl * mma16::BOX + half * mma16::ROWS * 128;  // rows 16 half .. (same swizzle phase)
+    const uint8_t* ksl = scales + (sl * mma16::STEP + half * mma16::ROWS) * 8;
     float acc[NB][4];
 #pragma unroll
     for (int j = 0; j < NB; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 #pragma unroll
     for (int bb = 0; bb < NB; ++bb) {
-      const uint2 w0 = *reinterpret_cast<const uint2*>(slot + g * mma16::PAD_S + 32 * bb + 8 * t);
-      const uint2 w1 = *reinterpret_cast<const uint2*>(slot + (g + 8) * mma16::PAD_S + 32 * bb + 8 * t);
+      const uint2 w0 = *reinterpret_cast<const uint2*>(box + mma16::swz(g, 32 * bb + 8 * t));
+      const uint2 w1 = *reinterpret_cast<const uint2*>(box + mma16::swz(g + 8, 32 * bb + 8 * t));
       uint32_t a[4];
       mma16::word_to_h2(w0.x, a[0], a[2]);
       mma16::word_to_h2(w1.x, a[1], a[3]);
@@ -451,19 +480,23 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
       mma16::mma_f16(acc[bb], a, bq[2 * bb + 1][0], bq[2 * bb + 1][1]);
     }
     // columns 2t (f16 part) and 2t + 1 (remainder) of head t, rows g (0, 1) and g + 8 (2, 3)
-    const uint2 s0 = *reinterpret_cast<const uint2*>(slot + OFF_KS + g * 8);
-    const uint2 s1 = *reinterpret_cast<const uint2*>(slot + OFF_KS + (g + 8) * 8);
+    const uint2 s0 = *reinterpret_cast<const uint2*>(ksl + g * 8);
+    const uint2 s1 = *reinterpret_cast<const uint2*>(ksl + (g + 8) * 8);
     const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&s0.x));
     const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&s0.y));
     const float2 b0 = __half22float2(*reinterpret_cast<const __half2*>(&s1.x));
     const float2 b1 = __half22float2(*reinterpret_cast<const __half2*>(&s1.y));
     const float sc0[NB] = {a0.x, a0.y, a1.x, a1.y}, sc1[NB] = {b0.x, b0.y, b1.x, b1.y};
-    float v0 = 0.f, v1 = 0.f;
+    v0 = 0.f;
+    v1 = 0.f;
 #pragma unroll
     for (int j = 0; j < NB; ++j) {
       v0 = fmaf(sc0[j], acc[j][0] + acc[j][1], v0);
       v1 = fmaf(sc1[j], acc[j][2] + acc[j][3], v1);
     }
+  };
+  // ... then stored, with the tile maxima, in walk order
+  auto finish = [&](float v0, float v1) {
     if (t < G) {
       const int row0 = wc.row0 + g;
       if (row0 < wc.rend) {
@@ -487,15 +520,26 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
     wc.next(r, T, ipt, mma16::ROWS);
   };
 
+  // the two groups of a step together, so that their loads, conversions and MMAs interleave
 #pragma unroll 1
-  for (int k = 0; k < mma16::PM - 1; ++k) issue();
+  for (int i = 0; i < mma16::PB; ++i) issue();
 #pragma unroll 1
-  for (int k = 0; k < niter; ++k) {
-    issue();
-    cp_async_wait<mma16::PM - 1>();  // group k has landed (this lane's copies) ...
-    __syncwarp();                    // ... and every lane's
-    body(k);
+  for (int k = 0; k < nsteps; ++k) {
+    const int sl = k % mma16::PB;
+    cp_async_wait<mma16::PB - 1>();  // the scales of step k have landed (this lane's) ...
+    if ((pend >> sl) & 1u) {         // ... its codes
+      mbar_wait_bounded(bars + 8 * sl, (phase >> sl) & 1u, p.ws_status);
+      phase ^= 1u << sl;
+      pend &= ~(1u << sl);
+    }
+    __syncwarp();  // ... and every lane's scales
+    float x0, x1, y0, y1;
+    scores(sl, 0, x0, x1);
+    scores(sl, 1, y0, y1);
+    finish(x0, x1);
+    finish(y0, y1);
     __syncwarp();  // every lane is done with the slot before it is refilled
+    issue();
   }
   cp_async_wait<0>();
   if (g == 0) s_cm[warp][t] = cm;
@@ -516,10 +560,8 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
 // lane's V bytes for a row and block are one 4-byte word.  Weights, the skip test, the denominators
 // and the counters are formed as in q8_pv_kernel: one lane per (row, head) pair, two pairs per lane.
 namespace mma16 {
-constexpr int PV_SLOT = SLOT_CODES + ROWS * 8 + ROWS * 16;  // codes, V scales, scores (4 per row)
-constexpr int PV_RING = NW * PM * PV_SLOT;
 constexpr int PV_ACC = NW * 4 * 128 * 4;
-constexpr int PV_SMEM = PV_RING > PV_ACC ? PV_RING : PV_ACC;
+constexpr int PV_SMEM = PSMEM_RING > PV_ACC ? PSMEM_RING : PV_ACC;
 __device__ __forceinline__ uint32_t pack_hh(__half a, __half b) {
   __half2 h = __halves2half2(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -534,6 +576,8 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   __shared__ float s_mp[CTMAX][4], s_ref[4];
   __shared__ int s_live[CTMAX];
   __shared__ float s_l[NW][4];
+  grid_dep_wait();  // pass 1's scores and maxima
+  grid_dep_launch();
   const Range r = cta_range(p);
   if (r.c0 >= r.t1) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -574,49 +618,53 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   }
   __syncthreads();
 
-  const int8_t* vb = p.v + static_cast<long long>(bk) * p.L_max * D;
   const uint16_t* vsb = p.vs + static_cast<long long>(bk) * p.L_max * NB;
   const float* scb = p.scores + static_cast<long long>(bk) * p.L_max * GP;
-  const int ipt = T / mma16::ROWS;
-  const int niter = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ipt;
-  uint8_t* ring = s_dyn + warp * mma16::PM * mma16::PV_SLOT;
-  const uint32_t ring_a = smem_u32(ring);
-  constexpr int OFF_VS = mma16::SLOT_CODES, OFF_SC = mma16::SLOT_CODES + mma16::ROWS * 8;
-  // copies of a group: lane l takes 64 code bytes of row l / 2; lanes 0..15 the V scales of row l,
-  // lanes 16..31 the scores of row l - 16.  Rows past the end are not copied; a tile left unread
-  // copies its scores only.
+  const int ipt = T / mma16::ROWS, ips = T / mma16::STEP;  // groups and steps per tile (T >= 32)
+  const int nsteps = (warp < nct ? (nct - warp + NW - 1) / NW : 0) * ips;
+  const uint32_t dyn = smem_u32(s_dyn), base = (dyn + 1023u) & ~1023u;
+  uint8_t* const codes = s_dyn + (base - dyn) + warp * mma16::PBV * mma16::BOX;
+  uint8_t* const vscales = s_dyn + (base - dyn) + mma16::PSM_VS + warp * mma16::PBV * mma16::STEP * 8;
+  uint8_t* const srows = s_dyn + (base - dyn) + mma16::PSM_SC + warp * mma16::PBV * mma16::STEP * 16;
+  const uint32_t bars = base + mma16::PSM_BARS + warp * mma16::PBV * 8;
+  if (lane == 0) {
+    for (int i = 0; i < mma16::PBV; ++i) mbar_init(bars + 8 * i, 1);
+    fence_mbar_init();
+  }
+  // copies of a step (32 rows of a tile): one TMA box of V code rows (skipped for a tile left unread
+  // and for a step wholly past the sequence), and per lane l the V scales (not for a tile left unread)
+  // and the scores of row l; rows past the sequence are copied (codes) or not copied (scales, scores)
+  // and weigh zero
+  uint32_t pend = 0u, phase = 0u;  // bit s: slot s has a box in flight / the parity it completes
   Walk wi, wc;
   wi.start(r, warp, T);
   wc = wi;
-  int ki = 0;
+  int ks = 0;
   // the V-scale areas of this warp's ring start as zeros: a row never copied then scales to a finite
   // value, and its weight (zero) keeps it out of the sum
-  for (int i = lane; i < mma16::PM * mma16::ROWS * 2; i += 32)
-    reinterpret_cast<uint32_t*>(ring + (i / (mma16::ROWS * 2)) * mma16::PV_SLOT + OFF_VS)[i % (mma16::ROWS * 2)] = 0u;
+  for (int i = lane; i < mma16::PBV * mma16::STEP * 2; i += 32) reinterpret_cast<uint32_t*>(vscales)[i] = 0u;
   __syncwarp();
   auto issue = [&]() {
-    if (ki < niter) {
-      const uint32_t slot = ring_a + (ki % mma16::PM) * mma16::PV_SLOT;
+    if (ks < nsteps) {
+      const int sl = ks % mma16::PBV;
       ART_DCHECK(wi.t >= r.c0 && wi.t < r.c1 && wi.t - r.c0 < CTMAX && wi.row0 >= wi.t * T && wi.row0 < (wi.t + 1) * T, p.ws_status);
+      ART_DCHECK(wi.row0 >= 0 && (wi.row0 < p.L_max || wi.row0 >= wi.rend), p.ws_status);
       const bool live_t = s_live[wi.t - r.c0] != 0;
-      const int rc = lane >> 1;
-      if (live_t && wi.row0 + rc < wi.rend) {
-        const int8_t* src = vb + static_cast<long long>(wi.row0 + rc) * D + (lane & 1) * 64;
-        const uint32_t dst = slot + rc * mma16::PAD + (lane & 1) * 64;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) cp_async<16>(dst + 16 * j, src + 16 * j);
-      }
-      const int rs = lane & 15;
-      if (wi.row0 + rs < wi.rend) {
-        if (lane < 16) {
-          if (live_t) cp_async<8>(slot + OFF_VS + rs * 8, vsb + static_cast<long long>(wi.row0 + rs) * NB);
-        } else {
-          cp_async<16>(slot + OFF_SC + rs * 16, scb + static_cast<long long>(wi.row0 + rs) * GP);
+      if (live_t && wi.row0 < wi.rend) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bars + 8 * sl, mma16::BOX);
+          tma_load_3d(smem_u32(codes + sl * mma16::BOX), &p.tmV, bars + 8 * sl, 0, wi.row0, bk);
         }
+        pend |= 1u << sl;
       }
-      wi.next(r, T, ipt, mma16::ROWS);
+      if (wi.row0 + lane < wi.rend) {
+        if (live_t)
+          cp_async<8>(smem_u32(vscales + sl * mma16::STEP * 8) + lane * 8, vsb + static_cast<long long>(wi.row0 + lane) * NB);
+        cp_async<16>(smem_u32(srows + sl * mma16::STEP * 16) + lane * 16, scb + static_cast<long long>(wi.row0 + lane) * GP);
+      }
+      wi.next(r, T, ips, mma16::STEP);
     }
-    ++ki;
+    ++ks;
     cp_async_commit();
   };
 
@@ -627,21 +675,23 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   bool live = false;
   int nskip = 0;
   const bool head_ok = t < G;
-  auto body = [&](int k) {
+  auto body = [&](int sl, int half) {
     if (wc.ik == 0) {  // a new tile: m'_t of this lane's head and the factor to the chunk's reference
       const int j = wc.t - r.c0;
       mp = head_ok ? s_mp[j][t] : 0.f;
       fac = head_ok ? exp2f(mp - s_ref[t]) : 0.f;
       live = s_live[j] != 0;
     }
-    const uint8_t* slot = ring + (k % mma16::PM) * mma16::PV_SLOT;
+    const uint8_t* box = codes + sl * mma16::BOX + half * mma16::ROWS * 128;  // rows 16 half .. (same swizzle phase)
+    const uint8_t* vsl = vscales + (sl * mma16::STEP + half * mma16::ROWS) * 8;
+    const uint8_t* ssl = srows + (sl * mma16::STEP + half * mma16::ROWS) * 16;
     // weights of rows g and g + 8 for head t
     float wk[2];
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
       const int row = g + 8 * rr;
       const bool ok = head_ok && wc.row0 + row < wc.rend;
-      const float sj = ok ? reinterpret_cast<const float*>(slot + OFF_SC + row * 16)[t] : -INFINITY;
+      const float sj = ok ? reinterpret_cast<const float*>(ssl + row * 16)[t] : -INFINITY;
       const float pj = exp2f(sj - mp);  // 0 for rows past the end and padded heads
       const float wj = pj * fac;
       l += wj;  // skipped rows stay in the denominator
@@ -657,10 +707,10 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       const int src = 8 * t + (g & 3);
       const float w0 = __shfl_sync(0xffffffffu, wk[0], src), w1 = __shfl_sync(0xffffffffu, wk[0], src + 4);
       const float w2 = __shfl_sync(0xffffffffu, wk[1], src), w3 = __shfl_sync(0xffffffffu, wk[1], src + 4);
-      const uint2 s0 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t) * 8);
-      const uint2 s1 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 1) * 8);
-      const uint2 s2 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 8) * 8);
-      const uint2 s3 = *reinterpret_cast<const uint2*>(slot + OFF_VS + (2 * t + 9) * 8);
+      const uint2 s0 = *reinterpret_cast<const uint2*>(vsl + (2 * t) * 8);
+      const uint2 s1 = *reinterpret_cast<const uint2*>(vsl + (2 * t + 1) * 8);
+      const uint2 s2 = *reinterpret_cast<const uint2*>(vsl + (2 * t + 8) * 8);
+      const uint2 s3 = *reinterpret_cast<const uint2*>(vsl + (2 * t + 9) * 8);
       // (V scales of a row not copied: an earlier row's, or zero)
       const uint32_t sv[4][2] = {{s0.x, s0.y}, {s1.x, s1.y}, {s2.x, s2.y}, {s3.x, s3.y}};
       const int vrow[4] = {2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9};
@@ -670,7 +720,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
         uint32_t vw[4];  // this lane's 4 code bytes of each row, positions 32 b + 4 g .. + 3
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          vw[i] = *reinterpret_cast<const uint32_t*>(slot + vrow[i] * mma16::PAD + 32 * bb + 4 * g) ^ 0x80808080u;
+          vw[i] = *reinterpret_cast<const uint32_t*>(box + mma16::swz(vrow[i], 32 * bb + 4 * g)) ^ 0x80808080u;
         float sc[4];  // the four rows' scales of block bb
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -709,13 +759,20 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   };
 
 #pragma unroll 1
-  for (int k = 0; k < mma16::PM - 1; ++k) issue();
+  for (int k = 0; k < mma16::PBV - 1; ++k) issue();
 #pragma unroll 1
-  for (int k = 0; k < niter; ++k) {
-    issue();
-    cp_async_wait<mma16::PM - 1>();
+  for (int k = 0; k < nsteps; ++k) {
+    issue();                          // step k + PBV - 1, into the slot step k - 1 left
+    cp_async_wait<mma16::PBV - 1>();  // step k's scales and scores (this lane's copies)
+    const int sl = k % mma16::PBV;
+    if ((pend >> sl) & 1u) {  // its V codes, when they were copied
+      mbar_wait_bounded(bars + 8 * sl, (phase >> sl) & 1u, p.ws_status);
+      phase ^= 1u << sl;
+      pend &= ~(1u << sl);
+    }
     __syncwarp();
-    body(k);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) body(sl, half);
     __syncwarp();
   }
   cp_async_wait<0>();
@@ -770,6 +827,8 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Pa
   __shared__ float s_mp[CTMAX][GP], s_ref[GP];
   __shared__ int s_live[CTMAX];
   __shared__ float s_l[NW][GP];
+  grid_dep_wait();  // pass 1's scores and maxima
+  grid_dep_launch();
   const Range r = cta_range(p);
   if (r.c0 >= r.t1) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -984,6 +1043,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Pa
 template <int D>
 __global__ void __launch_bounds__(D) q8_combine_kernel(const __grid_constant__ Params p) {
   constexpr int CU = 8;
+  grid_dep_wait();  // pass 2's chunk states
   const int hq = blockIdx.x;
   const int dd = threadIdx.x;
   const int b = hq / p.Hq, h = hq % p.Hq;
@@ -1088,29 +1148,54 @@ inline int choose_ct(const Dims& s, int sms) {
   return best;
 }
 
+// Launch a pass that reads the previous pass's results with programmatic stream serialisation: its
+// CTAs may be scheduled while the previous grid finishes and wait in grid_dep_wait() for its results.
+template <typename Kernel>
+cudaError_t launch_after(Kernel kernel, dim3 grid, int threads, size_t smem, cudaStream_t st, const Params& p) {
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
+  lc.gridDim = grid;
+  lc.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelEx(&lc, kernel, p);
+}
+
 template <int D, int GP>
 cudaError_t launch_dg(const Params& p, cudaStream_t st) {
   const dim3 grid(static_cast<unsigned>(p.CPS), static_cast<unsigned>(p.B * p.Hkv * p.S));
-  if constexpr (D == 128 && GP == 4) {  // both passes on the tensor cores
-    static bool attr_set[64] = {};  // the dynamic shared-memory limit, raised once per device
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-      e = cudaFuncSetAttribute(q8_scores_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::SMEM);
+  bool mma = false;
+  if constexpr (D == 128 && GP == 4) mma = p.T >= mma16::STEP;
+  if (mma) {  // both passes on the tensor cores, fed by TMA
+    if constexpr (D == 128 && GP == 4) {
+      if (!p.has_maps) return cudaErrorInvalidValue;
+      static bool attr_set[64] = {};  // the dynamic shared-memory limit, raised once per device
+      int dev = 0;
+      cudaError_t e = cudaGetDevice(&dev);
       if (e != cudaSuccess) return e;
-      e = cudaFuncSetAttribute(q8_pv_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::PV_SMEM);
-      if (e != cudaSuccess) return e;
-      attr_set[dev] = true;
+      if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+      if (!attr_set[dev]) {
+        e = cudaFuncSetAttribute(q8_scores_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::TSMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(q8_pv_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::PV_SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+      }
+      q8_scores_mma_kernel<GP><<<grid, NT, mma16::TSMEM, st>>>(p);
+      cudaError_t e2 = launch_after(q8_pv_mma_kernel<GP>, grid, NT, mma16::PV_SMEM, st, p);
+      if (e2 != cudaSuccess) return e2;
     }
-    q8_scores_mma_kernel<GP><<<grid, NT, mma16::SMEM, st>>>(p);
-    q8_pv_mma_kernel<GP><<<grid, NT, mma16::PV_SMEM, st>>>(p);
   } else {
     q8_scores_kernel<D, GP><<<grid, NT, 0, st>>>(p);
-    q8_pv_kernel<D, GP><<<grid, NT, 0, st>>>(p);
+    cudaError_t e2 = launch_after(q8_pv_kernel<D, GP>, grid, NT, 0, st, p);
+    if (e2 != cudaSuccess) return e2;
   }
-  q8_combine_kernel<D><<<p.B * p.Hq, D, 0, st>>>(p);
+  cudaError_t e3 = launch_after(q8_combine_kernel<D>, dim3(static_cast<unsigned>(p.B * p.Hq)), D, 0, st, p);
+  if (e3 != cudaSuccess) return e3;
   return cudaGetLastError();
 }
 
@@ -1122,11 +1207,17 @@ cudaError_t launch_d(const Params& p, cudaStream_t st) {
   return launch_dg<D, 8>(p, st);
 }
 
+// The passes on the tensor cores (d = 128, 3 or 4 heads per kv head) take K and V codes through
+// tensor maps (tma_box_maps); the others do not.
+inline bool uses_maps(const Dims& s) { return s.d == 128 && gp_of(s.Hq / s.Hkv) == 4 && s.T >= mma16::STEP; }
+
 // Enqueue the three kernels.  ws: the caller's workspace; tiles_read_off / used_off: the common
-// per-split counters inside it; base: where the common arrays end.
+// per-split counters inside it; base: where the common arrays end; tmk / tmv: the code maps when
+// uses_maps(s), else NULL.
 inline cudaError_t launch(const Dims& s, const uint16_t* q, const int8_t* k, const uint16_t* ks, const int8_t* v,
                           const uint16_t* vs, const int32_t* seq_lens, float tau, float* o, int32_t* tiles,
-                          uint8_t* ws, size_t tiles_read_off, size_t used_off, size_t base, cudaStream_t st) {
+                          uint8_t* ws, size_t tiles_read_off, size_t used_off, size_t base, const CUtensorMap* tmk,
+                          const CUtensorMap* tmv, cudaStream_t st) {
   static int sms_of[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1140,6 +1231,11 @@ inline cudaError_t launch(const Dims& s, const uint16_t* q, const int8_t* k, con
   }
   const Layout2 ql = layout2(s, base);
   Params p;
+  p.has_maps = tmk != nullptr && tmv != nullptr;
+  if (p.has_maps) {
+    p.tmK = *tmk;
+    p.tmV = *tmv;
+  }
   p.q = q;
   p.k = k;
   p.ks = ks;
