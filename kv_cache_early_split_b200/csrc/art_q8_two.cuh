@@ -589,16 +589,27 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   const float tau = p.tau;
   const int nct = r.c1 - r.c0;  // <= CTMAX
 
-  // running maxima m'_t, the chunk's reference and the tiles left unread, as in q8_pv_kernel
+  // running maxima m'_t, the chunk's reference and the tiles left unread, as in q8_pv_kernel; the
+  // maxima of every head are loaded together (one round trip to memory, not one per head)
   if (warp == 0) {
     const float* cm = p.cmax + static_cast<long long>(unit) * p.CPS * G;
+    const float* tmx = p.tmax + (static_cast<long long>(bk) * p.n_max + r.c0 + lane) * G;
+    float mc[4], own4[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      own4[h] = (h < G && lane < nct) ? tmx[h] : -INFINITY;
+      mc[h] = -INFINITY;
+    }
+    for (int c = lane; c < static_cast<int>(blockIdx.x); c += 32)
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        if (h < G) mc[h] = fmaxf(mc[h], cm[c * G + h]);
     bool live = false;
-    for (int h = 0; h < G; ++h) {
-      float m = -INFINITY;
-      for (int c = lane; c < static_cast<int>(blockIdx.x); c += 32) m = fmaxf(m, cm[c * G + h]);
-      m = warp_max(m);
-      const float own = lane < nct ? p.tmax[(static_cast<long long>(bk) * p.n_max + r.c0 + lane) * G + h]
-                                   : -INFINITY;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      if (h >= G) break;
+      const float m = warp_max(mc[h]);
+      const float own = own4[h];
       float x = own;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {

@@ -163,6 +163,9 @@ def test_kernel_name_query(L):
     assert capi.art_kernel_name(tc, capi.ART_BF16, True, True) == "art_decode_tc_kernel"
     assert capi.art_kernel_name(tc, capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
     assert capi.art_kernel_name(shape(Hq=24, Hkv=8, d=128, tile=64), capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
+    # (the tensor-core passes move 32-row steps: tiles of 16 take the CUDA-core passes)
+    assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=128, tile=16), capi.ART_BF16, True, False) == "q8_pv_kernel"
+    assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=128, tile=32), capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
     assert capi.art_kernel_name(shape(Hq=24, Hkv=8, d=128, tile=128), capi.ART_BF16, 1, 1) == "art_decode_tc_kernel"
     # other q8 shapes: full attention as two streaming passes (the second named), ART one pass
     q8o = shape(Hq=16, Hkv=8, d=128, tile=64)

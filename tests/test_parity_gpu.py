@@ -180,6 +180,12 @@ Q8_TWO_PASS = [
     (64, 16, 2, 3, 2500, [2500, 777, 3], 128, 4),
     (128, 8, 1, 1, 4096, [4096], 256, 1),
     (128, 32, 8, 1, 2048, [2000], 64, 8),
+    # the tensor-core passes (d = 128, 3 or 4 heads, tile >= 32): 32-row steps at tile 32 with a
+    # length that ends inside a step and a tensor end inside a box (L_max = 3002), tiles of 128 and
+    # 256, a sequence shorter than one step
+    (128, 8, 2, 2, 3002, [2999, 20], 32, 3),
+    (128, 12, 3, 1, 6000, [5999], 128, 2),
+    (128, 4, 1, 2, 4096, [4096, 300], 256, 1),
 ]
 
 
