@@ -203,10 +203,14 @@ def measured_traffic(workload, mode, kernel_name):
 
 
 def launches_per_call(K, dp, w, mode) -> int:
-    """Kernels one decode call launches: q8 full attention over a two-pass workspace runs scores,
-    weights + PV and combine; every other call one kernel, plus the split combine with S > 1."""
-    if mode == "q8" and dp.ws_bytes >= K.capi.art_q8_workspace_bytes(dp.shape):
-        return 3
+    """Kernels one decode call launches: q8 over a two-pass workspace runs scores, weights + PV and
+    combine (with ART: scores, probe pass, rule, limited pass, combine); every other call one
+    kernel, plus the split combine with S > 1."""
+    if mode in ("q8", "q8_art") and dp.ws_bytes >= K.capi.art_q8_workspace_bytes(dp.shape):
+        if mode == "q8":
+            return 3
+        if K.kernel_name(dp, mode) == "q8_pv_mma_kernel":
+            return 5
     return 1 + (1 if w.num_splits > 1 else 0)
 
 
@@ -778,6 +782,9 @@ def run_ours(args):
     if launches_per_call(K, dp, w, args.mode) == 3:
         mma = "_mma" if kernel == "q8_pv_mma_kernel" else ""
         kernel = f"q8_scores{mma}_kernel + q8_pv{mma}_kernel + q8_combine_kernel (timed as one call)"
+    elif launches_per_call(K, dp, w, args.mode) == 5:
+        kernel = ("q8_scores_mma_kernel + q8_pv_mma_kernel (probe pass) + q8_rule_kernel + q8_pv_mma_kernel "
+                  "(limited pass) + q8_combine_kernel (timed as one call)")
     elif w.num_splits > 1:
         kernel += " (timed with its split combine kernel)"
     line = {

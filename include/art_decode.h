@@ -375,7 +375,9 @@ art_status art_read_device_status(void* ws, void* stream);
  * asks about art_decode_attn_q8_skipv (dtype is then ignored); with_art != 0
  * about the ART variant.  q8 without ART names the second of the two passes
  * that run when the workspace holds art_q8_workspace_bytes: "q8_pv_mma_kernel"
- * (tensor cores; d = 128, tile >= 32, 3 or 4 heads per kv head) or "q8_pv_kernel".  A query only: no CUDA call, nothing enqueued.  The
+ * (tensor cores; d = 128, tile >= 32, 3 or 4 heads per kv head) or "q8_pv_kernel";
+ * q8 with ART on such a shape names "q8_pv_mma_kernel" too (the passes that run
+ * with that workspace: scores, probe pass, rule, limited pass, combine).  A query only: no CUDA call, nothing enqueued.  The
  * pages have no counterpart; it names the kernel for profiling and reports.
  * With num_splits > 1 a second, small kernel (art_combine_kernel) follows. */
 const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_q8, int32_t with_art);

@@ -654,20 +654,26 @@ artk::q8two::Dims q8_dims(const art_shape* s) {
 
 size_t q8_ws_total(const art_shape* s) { return artk::q8two::workspace_end(q8_dims(s), ws_layout(s).total); }
 
+// Full attention on any shape; ART (the rule over per-tile probe records) on the tensor-core passes.
 bool q8two_eligible(const art_shape* s, const art_params* params, size_t ws_bytes) {
-  return !params && ws_bytes >= q8_ws_total(s) && artk::q8two::grid_ok(q8_dims(s));
+  if (params && !artk::q8two::uses_maps(q8_dims(s))) return false;
+  return ws_bytes >= q8_ws_total(s) && artk::q8two::grid_ok(q8_dims(s));
 }
 
 art_status launch_q8two(const art_shape* s, const void* q, const int8_t* k, const uint16_t* ks, const int8_t* v,
-                        const uint16_t* vs, const int32_t* seq_lens, float tau, float* o, int32_t* tiles, void* ws,
-                        void* stream) {
+                        const uint16_t* vs, const int32_t* seq_lens, float tau, const art_params* params, float* o,
+                        int32_t* tiles, void* ws, void* stream) {
   const WsLayout w = ws_layout(s);
   CUtensorMap tmk, tmv;
   const bool maps = artk::q8two::uses_maps(q8_dims(s));
   if (maps && (!make_q8_group_map(&tmk, k, s) || !make_q8_group_map(&tmv, v, s))) return ART_ERR_CUDA;
+  artk::q8two::Rule rule{};
+  if (params)
+    rule = artk::q8two::Rule{params->n_probe, params->patience, params->eps_scale, params->eps_dir,
+                             params->probe_lanes};
   const cudaError_t e = artk::q8two::launch(q8_dims(s), static_cast<const uint16_t*>(q), k, ks, v, vs, seq_lens,
                                             tau, o, tiles, static_cast<uint8_t*>(ws), w.tiles_read, w.used, w.total,
-                                            maps ? &tmk : nullptr, maps ? &tmv : nullptr,
+                                            maps ? &tmk : nullptr, maps ? &tmv : nullptr, params ? &rule : nullptr,
                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? ART_OK : ART_ERR_CUDA;
 }
@@ -783,15 +789,21 @@ art_status art_decode_attn_q8_skipv_path(const art_shape* shape, const void* q_b
   const long long scale_row_bytes = (shape->d / 32) * 2;
   if ((1LL * shape->L_max * scale_row_bytes) % 16 != 0) return ART_ERR_UNSUPPORTED;
   const int mode = params ? artk::MODE_SKIP_ART : artk::MODE_SKIP;
+  if (params) {
+    int emask = 0;
+    st = validate_params(params, shape->d, 8, &emask);
+    if (st != ART_OK) return st;
+  }
   const bool tc = tc_eligible(artk::KV_Q8, mode, shape);
   const bool two = q8two_eligible(shape, params, ws_bytes);
   if (path == ART_Q8_TENSOR_CORE && !tc) return ART_ERR_UNSUPPORTED;
   if (path == ART_Q8_TWO_PASS && !two) return ART_ERR_UNSUPPORTED;
-  // automatic choice: full attention as two streaming passes when the workspace allows (the
-  // fastest q8 full attention), ART (and full attention without the larger workspace) on the tensor
-  // cores, else the cluster kernel
+  // automatic choice: two streaming passes when the workspace allows (full attention on every
+  // shape, ART on the tensor-core passes: the fastest q8 paths), else the tensor-core decode kernel,
+  // else the cluster kernel
   if (path == ART_Q8_TWO_PASS || (path == ART_Q8_AUTO && two))
-    return launch_q8two(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, o, tiles, ws, stream);
+    return launch_q8two(shape, q_bf16, k_q, k_scale_f16, v_q, v_scale_f16, seq_lens, tau, params, o, tiles, ws,
+                        stream);
   if (path == ART_Q8_TENSOR_CORE || (path == ART_Q8_AUTO && tc))
     return launch_tc(artk::KV_Q8, mode, shape, q_bf16, k_q, v_q, k_scale_f16, v_scale_f16, tau, seq_lens, params,
                      nullptr, o, tiles, ws, stream, nullptr);
@@ -985,6 +997,8 @@ const char* art_kernel_name(const art_shape* shape, art_dtype dtype, int32_t kv_
   if (mode == artk::MODE_SKIP && (shape->d == 64 || shape->d == 128) && shape->Hq % shape->Hkv == 0 &&
       shape->Hq / shape->Hkv <= artk::GMAX)  // two passes, given the q8 workspace
     return artk::q8two::uses_maps(q8_dims(shape)) ? "q8_pv_mma_kernel" : "q8_pv_kernel";
+  if (mode == artk::MODE_SKIP_ART && shape->Hq % shape->Hkv == 0 && artk::q8two::uses_maps(q8_dims(shape)))
+    return "q8_pv_mma_kernel";  // the probe and limited passes, given the q8 workspace
   if (tc_eligible(kind, mode, shape)) return "art_decode_tc_kernel";
   KernelInfo ki;
   if (!pick_kernel(kind, mode, shape->d, shape->Hq / shape->Hkv, &ki)) return nullptr;

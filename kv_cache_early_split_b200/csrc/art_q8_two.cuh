@@ -52,10 +52,19 @@ struct Params {
   float* cmax;             // [B*Hkv*S][CPS][G]  chunk maxima
   float* part;             // [B*Hq*S][CPS][2 + D]  chunk states (m, l, acc)
   int32_t* vskip;          // [B*Hkv*S][2]  rows left out of every head's numerator, V tiles not read
+  // ART on the two passes: per-tile probe records, the rule's stop tiles, the rule's settings
+  float* probe;            // [B*Hq][n_max][REC]  m'_t, l_t, the tile's probe lanes of acc_t (own reference)
+  int32_t* stop;           // [B*Hq*S]  absolute index of the last consumed tile of each split
   int B, Hq, Hkv, L_max, T, S, G, GP, CT, CPS, n_max;
   float qscale, tau;
   bool has_maps;  // tmK / tmV set
+  bool art;       // the ART rule decides the tiles consumed (probe pass, rule, limited pass)
+  int n_probe, patience;
+  float eps_scale, eps_dir;
+  int lanes[32];
 };
+
+constexpr int REC = 34;  // floats per probe record: m'_t, l_t, up to 32 probe lanes
 
 // Smallest chunk: at least 128 rows per warp where that stays within CTMAX tiles.
 __host__ __device__ inline int chunk_tiles_min(int T) {
@@ -568,14 +577,21 @@ __device__ __forceinline__ uint32_t pack_hh(__half a, __half b) {
 }
 }  // namespace mma16
 
-template <int GP>
+// PASS 0: full attention (chunk states).  With the ART rule: PASS 1, the probe pass -- per tile and
+// head the record (m'_t, l_t, the probe lanes of acc_t), each tile on its own reference m'_t, no chunk
+// states -- and PASS 2, the limited pass -- chunk states over the tiles each head consumes (up to its
+// stop tile from the rule), on a reference no later than its last consumed tile.
+template <int GP, int PASS>
 __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant__ Params p) {
   constexpr int D = 128, NB = 4;
   static_assert(GP == 4, "one lane per (row, head) pair over 8 rows: four heads");
+  static_assert(PASS >= 0 && PASS <= 2, "pass");
   extern __shared__ __align__(16) uint8_t s_dyn[];  // the ring while the rows stream, then the accumulators
   __shared__ float s_mp[CTMAX][4], s_ref[4];
   __shared__ int s_live[CTMAX];
   __shared__ float s_l[NW][4];
+  __shared__ int s_pidx[PASS == 1 ? 128 : 1];  // probe index of each position, or -1
+  __shared__ int s_stop[4];
   grid_dep_wait();  // pass 1's scores and maxima
   grid_dep_launch();
   const Range r = cta_range(p);
@@ -604,6 +620,12 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
 #pragma unroll
       for (int h = 0; h < 4; ++h)
         if (h < G) mc[h] = fmaxf(mc[h], cm[c * G + h]);
+    // the limited pass: each head's last consumed tile and their maximum (tiles past it are not read)
+    const int my_stop = (PASS == 2 && lane < G) ? p.stop[(static_cast<long long>(b) * p.Hq + kvh * G + lane) * p.S + split] : -1;
+    int smax = my_stop;
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) smax = max(smax, __shfl_xor_sync(0xffffffffu, smax, off));
+    smax = __shfl_sync(0xffffffffu, smax, 0);  // (lanes 0..3 hold the heads' stops)
     bool live = false;
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
@@ -623,9 +645,23 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       }
       if (lane == 31) s_ref[h] = mpj;
     }
+    if (PASS == 2) live = live && r.c0 + lane <= smax;
     if (lane < nct) s_live[lane] = live ? 1 : 0;
     const unsigned dead = __ballot_sync(0xffffffffu, lane < nct && !live);
-    if (lane == 0 && dead) atomicAdd(&p.vskip[unit * 2 + 1], __popc(dead));
+    if (PASS != 2 && lane == 0 && dead) atomicAdd(&p.vskip[unit * 2 + 1], __popc(dead));
+    if constexpr (PASS == 2) {  // the reference: m' at the last tile of the chunk the head consumes
+      __syncwarp();
+      if (lane < G) {
+        const int last = min(r.c1 - 1, my_stop);
+        s_ref[lane] = last >= r.c0 ? s_mp[last - r.c0][lane] : -INFINITY;
+        s_stop[lane] = my_stop;
+      }
+    }
+    if constexpr (PASS == 1) {
+      for (int i = lane; i < 128; i += 32) s_pidx[i] = -1;
+      __syncwarp();
+      if (lane < p.n_probe) s_pidx[p.lanes[lane]] = lane;
+    }
   }
   __syncthreads();
 
@@ -690,7 +726,9 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
     if (wc.ik == 0) {  // a new tile: m'_t of this lane's head and the factor to the chunk's reference
       const int j = wc.t - r.c0;
       mp = head_ok ? s_mp[j][t] : 0.f;
-      fac = head_ok ? exp2f(mp - s_ref[t]) : 0.f;
+      if constexpr (PASS == 0) fac = head_ok ? exp2f(mp - s_ref[t]) : 0.f;
+      if constexpr (PASS == 1) fac = head_ok ? 1.f : 0.f;  // the tile's own reference
+      if constexpr (PASS == 2) fac = (head_ok && wc.t <= s_stop[t]) ? exp2f(mp - s_ref[t]) : 0.f;
       live = s_live[j] != 0;
     }
     const uint8_t* box = codes + sl * mma16::BOX + half * mma16::ROWS * 128;  // rows 16 half .. (same swizzle phase)
@@ -709,7 +747,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       wk[rr] = (live && !(pj < tau) && pj > 0.f) ? wj : 0.f;
     }
     const unsigned kb0 = __ballot_sync(0xffffffffu, wk[0] > 0.f), kb1 = __ballot_sync(0xffffffffu, wk[1] > 0.f);
-    if (t == 0) {  // rows g and g + 8 left out of every head's numerator
+    if (PASS != 2 && t == 0) {  // rows g and g + 8 left out of every head's numerator
       if (wc.row0 + g < wc.rend && ((kb0 >> (4 * g)) & 0xFu) == 0u) ++nskip;
       if (wc.row0 + g + 8 < wc.rend && ((kb1 >> (4 * g)) & 0xFu) == 0u) ++nskip;
     }
@@ -768,6 +806,33 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
     }
     wc.next(r, T, ipt, mma16::ROWS);
   };
+  // the probe pass, at the end of a tile: its records (head t's m'_t and denominator, head g's probe
+  // lanes of the accumulators: f16 part in row g + remainder in row g + 8), then fresh sums
+  auto flush = [&](int tile) {
+    float lt = l;  // head t's denominator over the tile (lanes of the same t)
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, off);
+    const long long rec0 = (static_cast<long long>(b) * p.Hq + kvh * G) * p.n_max + tile;  // head 0's
+    ART_DCHECK(tile >= 0 && tile < p.n_max, p.ws_status);
+    if (g == 0 && head_ok) {
+      float* rc = p.probe + (rec0 + static_cast<long long>(t) * p.n_max) * REC;
+      rc[0] = mp;
+      rc[1] = lt;
+    }
+    if (g < G) {
+      float* rc = p.probe + (rec0 + static_cast<long long>(g) * p.n_max) * REC;
+#pragma unroll
+      for (int idx = 0; idx < 16; ++idx)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int pi = s_pidx[32 * (idx >> 2) + 4 * (2 * t + c) + (idx & 3)];
+          if (pi >= 0) rc[2 + pi] = acc[idx][c] + acc[idx][c + 2];
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+    l = 0.f;
+  };
 
 #pragma unroll 1
   for (int k = 0; k < mma16::PBV - 1; ++k) issue();
@@ -782,8 +847,11 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       pend &= ~(1u << sl);
     }
     __syncwarp();
+    const int t_step = wc.t;  // (a step never straddles two tiles)
 #pragma unroll
     for (int half = 0; half < 2; ++half) body(sl, half);
+    if constexpr (PASS == 1)
+      if (wc.ik == 0) flush(t_step);  // the step ended its tile
     __syncwarp();
   }
   cp_async_wait<0>();
@@ -793,6 +861,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
     for (int off = 16; off >= 1; off >>= 1) ns_w += __shfl_xor_sync(0xffffffffu, ns_w, off);
     if (lane == 0 && ns_w) atomicAdd(&p.vskip[unit * 2], ns_w);
   }
+  if constexpr (PASS == 1) return;  // the records are the pass's output
   // the denominators: lanes of the same head t
 #pragma unroll
   for (int off = 4; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
@@ -824,6 +893,175 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       dst[0] = s_ref[h];
       dst[1] = lsum;
     }
+  }
+}
+
+// ------------------------------------------------------------------ the ART rule over the probe records
+// One CTA of RW warps per (query head, split), 32 * RW tiles of the split per round, thread = tile:
+// the records' running merge (an inclusive scan of the online-softmax merge within each warp, the
+// warps' totals and the state carried from earlier rounds prepended) gives every tile's probe
+// x^(t) = acc^(t)[lanes] / l^(t); with the previous tile's probe (zeros before the first tile) the
+// magnitude change | |x^(t)| - |x^(t-1)| | and the direction change 1 - cos =
+// |x^(t)/|x^(t)| - x^(t-1)/|x^(t-1)||^2 / 2 (0 when both probes are zero, 1 when one is); a tile holds
+// when both are below their thresholds, and the split stops at the first tile whose run of holding
+// tiles reaches the patience ("Resumen Tecnico: ART", S2.2-S2.3).  Output: the stop tile (absolute
+// index; the split's last tile when the rule never fires) and the tiles consumed.
+constexpr int RW = 8;
+constexpr int kNoStop = 0x7fffffff;
+template <int PC>
+struct RuleState {
+  float m, l, a[PC];
+};
+
+template <int PC>
+__global__ void __launch_bounds__(RW * 32) q8_rule_kernel(const __grid_constant__ Params p) {
+  grid_dep_wait();  // the probe pass's records
+  grid_dep_launch();
+  __shared__ RuleState<PC> s_tot[RW];             // each warp's merged records
+  __shared__ float s_lx[RW][PC], s_ln[RW];        // each warp's last probe and its norm
+  __shared__ int s_allh[RW], s_trail[RW], s_first[RW];
+  __shared__ RuleState<PC> s_carry;               // the state carried from earlier rounds ...
+  __shared__ float s_cx[PC], s_cn;                // ... its probe and norm
+  __shared__ int s_crun, s_stop;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int hq = static_cast<int>(blockIdx.x / p.S), split = static_cast<int>(blockIdx.x % p.S);
+  int L = p.seq_lens[hq / p.Hq];
+  if (L < 1 || L > p.L_max) L = 0;
+  const int n = (L + p.T - 1) / p.T;
+  const int ta = static_cast<int>((static_cast<long long>(split) * n) / p.S);
+  const int tb = static_cast<int>((static_cast<long long>(split + 1) * n) / p.S);
+  auto rescale = [](float x, float M) { return x == -INFINITY ? 0.f : exp2f(x - M); };
+  // (m, l, a) <- earlier (mo, lo, ao) merged with (m, l, a)
+  auto merge = [&](float& m, float& l, float (&a)[PC], float mo, float lo, const float* ao) {
+    const float M = fmaxf(m, mo);
+    const float cs = rescale(m, M), co = rescale(mo, M);
+    l = cs * l + co * lo;
+    m = M;
+#pragma unroll
+    for (int i = 0; i < PC; ++i) a[i] = cs * a[i] + co * ao[i];
+  };
+  if (threadIdx.x == 0) {
+    s_carry.m = -INFINITY;
+    s_carry.l = 0.f;
+    s_cn = 0.f;
+    s_crun = 0;
+    s_stop = -1;
+  }
+  if (threadIdx.x < PC) s_carry.a[threadIdx.x] = s_cx[threadIdx.x] = 0.f;
+  __syncthreads();
+  for (int base = ta; base < tb; base += RW * 32) {
+    const int tt = base + warp * 32 + lane;
+    const bool valid = tt < tb;
+    float m = -INFINITY, l = 0.f, a[PC];
+#pragma unroll
+    for (int i = 0; i < PC; ++i) a[i] = 0.f;
+    if (valid) {
+      const float* rc = p.probe + (static_cast<long long>(hq) * p.n_max + tt) * REC;
+      m = rc[0];
+      l = rc[1];
+#pragma unroll
+      for (int i = 0; i < PC; ++i) a[i] = i < p.n_probe ? rc[2 + i] : 0.f;
+    }
+#pragma unroll 1
+    for (int off = 1; off < 32; off <<= 1) {  // the warp's inclusive scan
+      const float mo = __shfl_up_sync(0xffffffffu, m, off), lo = __shfl_up_sync(0xffffffffu, l, off);
+      float ao[PC];
+#pragma unroll
+      for (int i = 0; i < PC; ++i) ao[i] = __shfl_up_sync(0xffffffffu, a[i], off);
+      if (lane >= off) merge(m, l, a, mo, lo, ao);
+    }
+    if (lane == 31) {
+      s_tot[warp].m = m;
+      s_tot[warp].l = l;
+#pragma unroll
+      for (int i = 0; i < PC; ++i) s_tot[warp].a[i] = a[i];
+    }
+    __syncthreads();
+    {  // prepend the earlier warps' totals and the carried state
+      float cm = s_carry.m, cl = s_carry.l, ca[PC];
+#pragma unroll
+      for (int i = 0; i < PC; ++i) ca[i] = s_carry.a[i];
+      for (int u = 0; u < warp; ++u) {
+        float tm = s_tot[u].m, tl = s_tot[u].l, tv[PC];
+#pragma unroll
+        for (int i = 0; i < PC; ++i) tv[i] = s_tot[u].a[i];
+        merge(tm, tl, tv, cm, cl, ca);
+        cm = tm;
+        cl = tl;
+#pragma unroll
+        for (int i = 0; i < PC; ++i) ca[i] = tv[i];
+      }
+      merge(m, l, a, cm, cl, ca);
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float x[PC], sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < PC; ++i) {
+      x[i] = a[i] * inv;
+      sq = fmaf(x[i], x[i], sq);
+    }
+    const float nrm = sqrtf(sq);
+    if (lane == 31) {
+#pragma unroll
+      for (int i = 0; i < PC; ++i) s_lx[warp][i] = x[i];
+      s_ln[warp] = nrm;
+    }
+    __syncthreads();
+    float nrmp = __shfl_up_sync(0xffffffffu, nrm, 1);
+    if (lane == 0) nrmp = warp == 0 ? s_cn : s_ln[warp - 1];
+    const bool both = nrm > 0.f && nrmp > 0.f;
+    const float in = both ? 1.f / nrm : 0.f, ip = both ? 1.f / nrmp : 0.f;
+    float dd = 0.f;
+#pragma unroll
+    for (int i = 0; i < PC; ++i) {
+      float xp = __shfl_up_sync(0xffffffffu, x[i], 1);
+      if (lane == 0) xp = warp == 0 ? s_cx[i] : s_lx[warp - 1][i];
+      const float dl = x[i] * in - xp * ip;
+      dd = fmaf(dl, dl, dd);
+    }
+    const float d_scale = fabsf(nrm - nrmp);
+    const float d_dir = (nrm == 0.f && nrmp == 0.f) ? 0.f : ((nrm == 0.f || nrmp == 0.f) ? 1.f : 0.5f * dd);
+    const bool hold = valid && d_scale < p.eps_scale && d_dir < p.eps_dir;
+    const unsigned hbits = __ballot_sync(0xffffffffu, hold);
+    if (lane == 0) {
+      s_allh[warp] = hbits == 0xffffffffu;
+      s_trail[warp] = __clz(~hbits);  // holding tiles at the warp's end
+    }
+    __syncthreads();
+    int crun = s_crun;  // the run of holding tiles entering this warp
+    for (int u = 0; u < warp; ++u) crun = s_allh[u] ? crun + 32 : s_trail[u];
+    const unsigned zeros = ~hbits & ((1u << lane) - 1u);
+    const int run = !hold ? 0 : (zeros == 0u ? crun + lane + 1 : lane - (31 - __clz(zeros)));
+    const unsigned rbits = __ballot_sync(0xffffffffu, hold && run >= p.patience);
+    if (lane == 0) s_first[warp] = rbits ? tt + __ffs(rbits) - 1 : kNoStop;
+    // the round's last tile carries its state into the next round
+    const int last = min(base + RW * 32, tb) - 1;
+    __syncthreads();
+    int first = kNoStop;
+#pragma unroll
+    for (int u = 0; u < RW; ++u) first = min(first, s_first[u]);
+    if (first != kNoStop) {
+      if (threadIdx.x == 0) s_stop = first;
+      break;  // (uniform: every thread saw the same minimum)
+    }
+    if (tt == last) {
+      s_carry.m = m;
+      s_carry.l = l;
+#pragma unroll
+      for (int i = 0; i < PC; ++i) {
+        s_carry.a[i] = a[i];
+        s_cx[i] = x[i];
+      }
+      s_cn = nrm;
+      s_crun = run;
+    }
+    __syncthreads();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int stop = s_stop >= 0 ? s_stop : tb - 1;  // every tile (an empty split: none)
+    p.stop[static_cast<long long>(hq) * p.S + split] = stop;
+    p.ws_used[static_cast<long long>(hq) * p.S + split] = stop - ta + 1;
   }
 }
 
@@ -1094,13 +1332,18 @@ __global__ void __launch_bounds__(D) q8_combine_kernel(const __grid_constant__ P
       }
     }
     if (dd == 0) {
-      p.ws_used[static_cast<long long>(hq) * p.S + s] = ns;
-      if (h % p.G == 0) p.ws_tiles_read[static_cast<long long>(bk) * p.S + s] = ns;
+      if (!p.art) p.ws_used[static_cast<long long>(hq) * p.S + s] = ns;  // (with ART: the rule's count)
+      if (h % p.G == 0) p.ws_tiles_read[static_cast<long long>(bk) * p.S + s] = ns;  // every K tile is read
     }
   }
   p.o[static_cast<long long>(hq) * D + dd] = bad ? __int_as_float(0x7fc00000) : num / den;
   if (dd == 0) {
-    if (p.tiles) p.tiles[hq] = n_tiles;
+    int consumed = n_tiles;
+    if (p.art) {
+      consumed = 0;
+      for (int s = 0; s < p.S; ++s) consumed += p.ws_used[static_cast<long long>(hq) * p.S + s];
+    }
+    if (p.tiles) p.tiles[hq] = consumed;
     if (bad && h == 0) atomicOr(p.ws_status, kStatusSeqLen);
   }
 }
@@ -1114,7 +1357,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace arrays after the common ones (which end at `base`), sized for the smallest chunk.
 struct Layout2 {
-  size_t scores, tmax, cmax, part, vskip, end;
+  size_t scores, tmax, cmax, part, vskip, probe, stop, end;
   int n_max, CT, CPS;
 };
 
@@ -1131,7 +1374,9 @@ inline Layout2 layout2(const Dims& s, size_t base) {
   q.cmax = align256(q.tmax + 4 * bk * size_t(q.n_max) * G);
   q.part = align256(q.cmax + 4 * units * size_t(q.CPS) * G);
   q.vskip = align256(q.part + 4 * units * G * size_t(q.CPS) * (size_t(s.d) + 2));
-  q.end = align256(q.vskip + 8 * units);
+  q.probe = align256(q.vskip + 8 * units);
+  q.stop = align256(q.probe + 4 * size_t(s.B) * s.Hq * size_t(q.n_max) * REC);
+  q.end = align256(q.stop + 4 * units * G);
   return q;
 }
 
@@ -1162,7 +1407,8 @@ inline int choose_ct(const Dims& s, int sms) {
 // Launch a pass that reads the previous pass's results with programmatic stream serialisation: its
 // CTAs may be scheduled while the previous grid finishes and wait in grid_dep_wait() for its results.
 template <typename Kernel>
-cudaError_t launch_after(Kernel kernel, dim3 grid, int threads, size_t smem, cudaStream_t st, const Params& p) {
+cudaError_t launch_after(Kernel kernel, dim3 grid, int threads, size_t smem, cudaStream_t st, const Params& p,
+                         bool overlap = true) {
   cudaLaunchConfig_t lc = {};
   cudaLaunchAttribute attr[1];
   lc.gridDim = grid;
@@ -1170,7 +1416,7 @@ cudaError_t launch_after(Kernel kernel, dim3 grid, int threads, size_t smem, cud
   lc.dynamicSmemBytes = smem;
   lc.stream = st;
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
   lc.attrs = attr;
   lc.numAttrs = 1;
   return cudaLaunchKernelEx(&lc, kernel, p);
@@ -1192,20 +1438,38 @@ cudaError_t launch_dg(const Params& p, cudaStream_t st) {
       if (!attr_set[dev]) {
         e = cudaFuncSetAttribute(q8_scores_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::TSMEM);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(q8_pv_mma_kernel<GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::PV_SMEM);
+        e = cudaFuncSetAttribute(q8_pv_mma_kernel<GP, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::PV_SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(q8_pv_mma_kernel<GP, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::PV_SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(q8_pv_mma_kernel<GP, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, mma16::PV_SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
       }
       q8_scores_mma_kernel<GP><<<grid, NT, mma16::TSMEM, st>>>(p);
-      cudaError_t e2 = launch_after(q8_pv_mma_kernel<GP>, grid, NT, mma16::PV_SMEM, st, p);
-      if (e2 != cudaSuccess) return e2;
+      if (p.art) {  // probe pass, the rule, the limited pass, in plain stream order (measured: letting
+                    // these launches overlap made the chain 20% slower)
+        cudaError_t e2 = launch_after(q8_pv_mma_kernel<GP, 1>, grid, NT, mma16::PV_SMEM, st, p, false);
+        if (e2 != cudaSuccess) return e2;
+        const dim3 rule_grid(static_cast<unsigned>(p.B * p.Hq * p.S));
+        e2 = p.n_probe <= 16 ? launch_after(q8_rule_kernel<16>, rule_grid, RW * 32, 0, st, p, false)
+                             : launch_after(q8_rule_kernel<32>, rule_grid, RW * 32, 0, st, p, false);
+        if (e2 != cudaSuccess) return e2;
+        e2 = launch_after(q8_pv_mma_kernel<GP, 2>, grid, NT, mma16::PV_SMEM, st, p, false);
+        if (e2 != cudaSuccess) return e2;
+      } else {
+        cudaError_t e2 = launch_after(q8_pv_mma_kernel<GP, 0>, grid, NT, mma16::PV_SMEM, st, p);
+        if (e2 != cudaSuccess) return e2;
+      }
     }
   } else {
+    if (p.art) return cudaErrorInvalidValue;  // the rule runs on the tensor-core passes only
     q8_scores_kernel<D, GP><<<grid, NT, 0, st>>>(p);
     cudaError_t e2 = launch_after(q8_pv_kernel<D, GP>, grid, NT, 0, st, p);
     if (e2 != cudaSuccess) return e2;
   }
-  cudaError_t e3 = launch_after(q8_combine_kernel<D>, dim3(static_cast<unsigned>(p.B * p.Hq)), D, 0, st, p);
+  cudaError_t e3 = launch_after(q8_combine_kernel<D>, dim3(static_cast<unsigned>(p.B * p.Hq)), D, 0, st, p,
+                                !p.art);
   if (e3 != cudaSuccess) return e3;
   return cudaGetLastError();
 }
@@ -1225,10 +1489,17 @@ inline bool uses_maps(const Dims& s) { return s.d == 128 && gp_of(s.Hq / s.Hkv) 
 // Enqueue the three kernels.  ws: the caller's workspace; tiles_read_off / used_off: the common
 // per-split counters inside it; base: where the common arrays end; tmk / tmv: the code maps when
 // uses_maps(s), else NULL.
+// The rule's settings, for ART on the two passes (n_probe lanes in [0, 128), n_probe <= 32).
+struct Rule {
+  int n_probe, patience;
+  float eps_scale, eps_dir;
+  const int32_t* lanes;  // host
+};
+
 inline cudaError_t launch(const Dims& s, const uint16_t* q, const int8_t* k, const uint16_t* ks, const int8_t* v,
                           const uint16_t* vs, const int32_t* seq_lens, float tau, float* o, int32_t* tiles,
                           uint8_t* ws, size_t tiles_read_off, size_t used_off, size_t base, const CUtensorMap* tmk,
-                          const CUtensorMap* tmv, cudaStream_t st) {
+                          const CUtensorMap* tmv, const Rule* rule, cudaStream_t st) {
   static int sms_of[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1263,6 +1534,14 @@ inline cudaError_t launch(const Dims& s, const uint16_t* q, const int8_t* k, con
   p.cmax = reinterpret_cast<float*>(ws + ql.cmax);
   p.part = reinterpret_cast<float*>(ws + ql.part);
   p.vskip = reinterpret_cast<int32_t*>(ws + ql.vskip);
+  p.probe = reinterpret_cast<float*>(ws + ql.probe);
+  p.stop = reinterpret_cast<int32_t*>(ws + ql.stop);
+  p.art = rule != nullptr;
+  p.n_probe = rule ? rule->n_probe : 0;
+  p.patience = rule ? rule->patience : 1;
+  p.eps_scale = rule ? rule->eps_scale : 0.f;
+  p.eps_dir = rule ? rule->eps_dir : 0.f;
+  for (int i = 0; i < 32; ++i) p.lanes[i] = (rule && i < rule->n_probe) ? rule->lanes[i] : 0;
   p.B = s.B;
   p.Hq = s.Hq;
   p.Hkv = s.Hkv;

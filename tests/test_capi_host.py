@@ -61,7 +61,8 @@ def test_workspace_sizes(L):
 
 def test_q8_workspace_sizes(L):
     """The two-pass q8 workspace extends the common one: scores [B, Hkv, L_max, G] fp32, tile and
-    chunk maxima, and a (2 + d)-float state per query head and chunk of every split."""
+    chunk maxima, a (2 + d)-float state per query head and chunk of every split, and for ART a
+    34-float probe record per query head and tile plus a stop tile per query head and split."""
     for kw in (dict(), dict(num_splits=3), dict(d=64, tile=16), dict(Hq=8, Hkv=8, tile=256), dict(B=1, L_max=1)):
         s = shape(**kw)
         base, q8 = capi.art_workspace_bytes(s), capi.art_q8_workspace_bytes(s)
@@ -70,10 +71,12 @@ def test_q8_workspace_sizes(L):
         chunks = -(-n_max // s.num_splits)  # chunks of at least one tile per split
         ct = min(32, 8 * max(1, 128 // s.tile))
         assert q8 >= base + 4 * s.B * s.Hq * s.num_splits * -(-chunks // ct) * (s.d + 2)
+        assert q8 >= base + 4 * s.B * s.Hq * n_max * 34 + 4 * s.B * s.Hq * s.num_splits
     assert capi.art_q8_workspace_bytes(shape(B=0)) == 0
-    # the default q8 workload: 2 x 8 kv heads x 32768 positions x 4 heads of scores = 8 MiB and change
+    # the default q8 workload: 2 x 8 kv heads x 32768 positions x 4 heads of scores = 8 MiB, and
+    # 2 x 32 heads x 512 tiles of 136-byte probe records = 4.25 MiB, and change
     s = shape(B=2)
-    assert capi.art_q8_workspace_bytes(s) - capi.art_workspace_bytes(s) < 12 << 20
+    assert capi.art_q8_workspace_bytes(s) - capi.art_workspace_bytes(s) < 15 << 20
 
 
 A = 0x100000  # fake 16-byte aligned device addresses (never dereferenced)
@@ -160,13 +163,13 @@ def test_kernel_name_query(L):
     assert capi.art_kernel_name(tc, capi.ART_F32, False, True) == "art_decode_kernel"
     # q8 ART with 3 or 4 heads per kv head, d = 128, tile 64 / 128, even L_max: the tensor cores;
     # q8 full attention: two streaming passes (the second named) given the q8 workspace
-    assert capi.art_kernel_name(tc, capi.ART_BF16, True, True) == "art_decode_tc_kernel"
+    assert capi.art_kernel_name(tc, capi.ART_BF16, True, True) == "q8_pv_mma_kernel"  # (given the q8 workspace)
     assert capi.art_kernel_name(tc, capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
     assert capi.art_kernel_name(shape(Hq=24, Hkv=8, d=128, tile=64), capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
     # (the tensor-core passes move 32-row steps: tiles of 16 take the CUDA-core passes)
     assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=128, tile=16), capi.ART_BF16, True, False) == "q8_pv_kernel"
     assert capi.art_kernel_name(shape(Hq=32, Hkv=8, d=128, tile=32), capi.ART_BF16, True, False) == "q8_pv_mma_kernel"
-    assert capi.art_kernel_name(shape(Hq=24, Hkv=8, d=128, tile=128), capi.ART_BF16, 1, 1) == "art_decode_tc_kernel"
+    assert capi.art_kernel_name(shape(Hq=24, Hkv=8, d=128, tile=128), capi.ART_BF16, 1, 1) == "q8_pv_mma_kernel"
     # other q8 shapes: full attention as two streaming passes (the second named), ART one pass
     q8o = shape(Hq=16, Hkv=8, d=128, tile=64)
     assert capi.art_kernel_name(q8o, capi.ART_BF16, True, False) == "q8_pv_kernel"

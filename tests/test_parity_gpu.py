@@ -24,8 +24,8 @@ def q8_paths(w, mode, tile=None):
     """The q8 implementations that take this shape and mode (art_decode_attn_q8_skipv_path)."""
     T = tile or w.tile
     paths = ["cluster"]
-    if mode == "q8":
-        paths.append("two_pass")
+    if mode == "q8" or (w.d == 128 and w.G in (3, 4) and T >= 32):
+        paths.append("two_pass")  # (ART: the rule over probe records, on the tensor-core passes)
     if w.d == 128 and w.G in (3, 4) and T in (64, 128) and w.L_max % 2 == 0:
         paths.append("tensor_core")
     return paths
