@@ -469,7 +469,7 @@ def paged_sweep(K, w, steps, stream):
     return out
 
 
-def scaling_sweep(K, dp, w, mode, steps, stream):
+def scaling_sweep(K, dp, w, mode, steps, stream, q8_path="auto"):
     """Thresholds +inf and patience k stop every (head, split) after exactly min(k, n) tiles, so the
     time per call against KV bytes read should be a line with a small intercept."""
     n = int(-(-int(w.seq_lens.max()) // w.tile)) // max(1, w.num_splits)
@@ -479,7 +479,7 @@ def scaling_sweep(K, dp, w, mode, steps, stream):
     pts = []
     for k in ks:
         art = dict(w.art, eps_scale=float("inf"), eps_dir=float("inf"), patience=k)
-        _, launch = time_mode(K, dp, mode, steps, 2, stream, art=art, flush=flush)
+        _, launch = time_mode(K, dp, mode, steps, 2, stream, art=art, flush=flush, q8_path=q8_path)
         check_status(K, dp, w, f"{mode} patience {k}")
         rb = bytes_read(w, dp.tiles_read().cpu().numpy())
         cb = bytes_consumed(w, dp.split_tiles().cpu().numpy())
@@ -487,7 +487,8 @@ def scaling_sweep(K, dp, w, mode, steps, stream):
               "ms": launch, "kv_bytes_read": rb, "kv_bytes_consumed": cb, "read_over_consumed": rb / cb}
         # the same call with speculative reads bounded (art_params.max_spec_tiles = 1: a round is read
         # only if it starts at or before the safe point)
-        _, launch_b = time_mode(K, dp, mode, steps, 2, stream, art=dict(art, max_spec_tiles=1), flush=flush)
+        _, launch_b = time_mode(K, dp, mode, steps, 2, stream, art=dict(art, max_spec_tiles=1), flush=flush,
+                                q8_path=q8_path)
         check_status(K, dp, w, f"{mode} patience {k} bounded")
         rb_b = bytes_read(w, dp.tiles_read().cpu().numpy())
         pt["bounded"] = {"max_spec_tiles": 1, "ms": launch_b, "kv_bytes_read": rb_b, "read_over_consumed": rb_b / cb}
@@ -505,11 +506,11 @@ def check_status(K, dp, w, what):
         raise RuntimeError(f"device status not OK after {w.name} {what}")
 
 
-def mode_row(K, dp, w, mode, steps, stream, peak, art=None):
+def mode_row(K, dp, w, mode, steps, stream, peak, art=None, q8_path="auto"):
     """Time one mode on a workload's buffers; throughput, KV bytes read (device counters) and
     consumed (the slowest head of each kv head), and tile counts of the last call."""
     flush = needs_flush(w)
-    _, launch = time_mode(K, dp, mode, steps, 2, stream, art=art, flush=flush)
+    _, launch = time_mode(K, dp, mode, steps, 2, stream, art=art, flush=flush, q8_path=q8_path)
     if K.device_status(dp) != 0:
         raise RuntimeError(f"device status not OK after {w.name} {mode}")
     n_full = -(-w.seq_lens.astype(np.int64) // w.tile)
@@ -538,12 +539,20 @@ def measure_workload(K, w, dp, args, stream, peak, sweeps=True):
     out["art_over_full_time"] = a["ms"] / f["ms"]
     # time per consumed byte, ART over full (1.0: ART time follows what it consumed exactly)
     out["art_per_consumed_byte_over_full"] = (a["ms"] / a["kv_bytes_consumed"]) / (f["ms"] / f["kv_bytes_read"])
+    # q8 with ART: the default (the rule over the two passes' probe records, which reads every K and
+    # V tile once and the consumed V tiles again) and the tensor-core decode kernel (reads follow the
+    # rule, a few rounds ahead), whose scaling sweep below shows time against bytes read
+    scaling_path = "auto"
+    if w.kind == "q8" and K.kernel_name(dp, art_mode) == "q8_pv_mma_kernel":
+        out["q8_art_tensor_core"] = mode_row(K, dp, w, art_mode, steps, stream, peak, q8_path="tensor_core")
+        scaling_path = "tensor_core"
     if sweeps:
         eps0 = dict(w.art, eps_scale=0.0, eps_dir=0.0)
         e = mode_row(K, dp, w, art_mode, steps, stream, peak, art=eps0)
         out["overhead_eps0"] = {"ms": e["ms"], "ratio_to_full": e["ms"] / f["ms"],
                                 "note": "eps = 0: ART never stops and reads every tile"}
-        out["scaling"] = scaling_sweep(K, dp, w, art_mode, steps, stream)
+        out["scaling"] = scaling_sweep(K, dp, w, art_mode, steps, stream, q8_path=scaling_path)
+        out["scaling"]["q8_path"] = scaling_path
     return out
 
 
@@ -564,15 +573,16 @@ def vskip_sweep(K, args, stream, device):
         rows = {}
         for tau in (0.0, 1e-6, 1e-3, 1e-2):
             row = {}
-            for mode in ("q8", "q8_art"):
+            for mode, path in (("q8", "auto"), ("q8_art", "auto"), ("q8_art_tensor_core", "tensor_core")):
+                call = mode[:6] if mode.startswith("q8_art") else mode
                 for _ in range(2):
-                    K.decode(dp, mode, tau=tau, stream=stream.cuda_stream)
+                    K.decode(dp, call, tau=tau, stream=stream.cuda_stream, q8_path=path)
                 torch.cuda.synchronize()
                 ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
                 for e0, e1 in ev:
                     l2_flush(stream)
                     e0.record(stream)
-                    K.decode(dp, mode, tau=tau, stream=stream.cuda_stream)
+                    K.decode(dp, call, tau=tau, stream=stream.cuda_stream, q8_path=path)
                     e1.record(stream)
                 torch.cuda.synchronize()
                 row[mode] = {"ms": sum(a.elapsed_time(b) for a, b in ev) / steps,
@@ -590,7 +600,7 @@ def vskip_sweep(K, args, stream, device):
             rows[f"tau_{tau:g}"] = row
         if K.device_status(dp) != 0:
             raise RuntimeError("device status not OK after the V-skip sweep")
-        for mode in ("q8", "q8_art"):
+        for mode in ("q8", "q8_art", "q8_art_tensor_core"):
             base = rows["tau_0"][mode]["ms"]
             for t in ("tau_1e-06", "tau_0.001", "tau_0.01"):
                 rows[t][mode]["time_saved_vs_tau0"] = 1.0 - rows[t][mode]["ms"] / base
@@ -626,14 +636,14 @@ def l2_flush(stream):
         _flush_buf.fill_(1)
 
 
-def time_mode(K, dp, mode, steps, warmup, stream, art=None, flush=False):
+def time_mode(K, dp, mode, steps, warmup, stream, art=None, flush=False, q8_path="auto"):
     """Device time of `steps` calls: (total ms, mean per-launch ms from per-launch events).  With
     flush, L2 is overwritten before every launch and the total is the sum of the launches' own
     times (the flushes are not counted)."""
     import torch
 
     for _ in range(warmup):
-        K.decode(dp, mode, art=art, stream=stream.cuda_stream)
+        K.decode(dp, mode, art=art, stream=stream.cuda_stream, q8_path=q8_path)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -644,7 +654,7 @@ def time_mode(K, dp, mode, steps, warmup, stream, art=None, flush=False):
         if flush:
             l2_flush(stream)
         ev[i][0].record(stream)
-        K.decode(dp, mode, art=art, stream=stream.cuda_stream)
+        K.decode(dp, mode, art=art, stream=stream.cuda_stream, q8_path=q8_path)
         ev[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()

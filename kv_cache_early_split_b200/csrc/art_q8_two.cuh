@@ -590,7 +590,8 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   __shared__ float s_mp[CTMAX][4], s_ref[4];
   __shared__ int s_live[CTMAX];
   __shared__ float s_l[NW][4];
-  __shared__ int s_pidx[PASS == 1 ? 128 : 1];  // probe index of each position, or -1
+  __shared__ int s_plane[PASS == 1 ? 32 : 1];                   // the probe lanes (d positions)
+  __shared__ __align__(16) float s_wg[PASS == 1 ? NW : 1][16][4];  // a group's weights, row x head
   __shared__ int s_stop[4];
   grid_dep_wait();  // pass 1's scores and maxima
   grid_dep_launch();
@@ -657,11 +658,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
         s_stop[lane] = my_stop;
       }
     }
-    if constexpr (PASS == 1) {
-      for (int i = lane; i < 128; i += 32) s_pidx[i] = -1;
-      __syncwarp();
-      if (lane < p.n_probe) s_pidx[p.lanes[lane]] = lane;
-    }
+    if constexpr (PASS == 1) s_plane[lane] = lane < p.n_probe ? p.lanes[lane] : 0;
   }
   __syncthreads();
 
@@ -718,6 +715,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   float acc[16][4];  // n-tile (block b, j) = 4 b + j
 #pragma unroll
   for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  float pacc[4] = {0.f, 0.f, 0.f, 0.f};  // the probe pass: probe `lane` of each head over the tile
   float l = 0.f, mp = 0.f, fac = 0.f;
   bool live = false;
   int nskip = 0;
@@ -751,7 +749,32 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       if (wc.row0 + g < wc.rend && ((kb0 >> (4 * g)) & 0xFu) == 0u) ++nskip;
       if (wc.row0 + g + 8 < wc.rend && ((kb1 >> (4 * g)) & 0xFu) == 0u) ++nskip;
     }
-    if ((kb0 | kb1) != 0u) {  // otherwise no row of the group is dequantised
+    if constexpr (PASS == 1) {
+      // the probe pass needs the probe lanes of the sums only: lane i < n_probe takes probe i over the
+      // group's 16 rows and the heads (weights through shared memory), on the CUDA cores
+      if (head_ok) {
+        s_wg[warp][g][t] = wk[0];
+        s_wg[warp][g + 8][t] = wk[1];
+      } else if (t < 4) {
+        s_wg[warp][g][t] = 0.f;
+        s_wg[warp][g + 8][t] = 0.f;
+      }
+      __syncwarp();
+      if ((kb0 | kb1) != 0u && lane < p.n_probe) {
+        const int pos = s_plane[lane], blk = pos >> 5;
+#pragma unroll 4
+        for (int row = 0; row < mma16::ROWS; ++row) {
+          const float code = static_cast<float>(static_cast<int8_t>(box[mma16::swz(row, pos)]));
+          const float vv = code * __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(vsl + row * 8)[blk]));
+          const float4 w4 = *reinterpret_cast<const float4*>(&s_wg[warp][row][0]);
+          pacc[0] = fmaf(w4.x, vv, pacc[0]);
+          pacc[1] = fmaf(w4.y, vv, pacc[1]);
+          pacc[2] = fmaf(w4.z, vv, pacc[2]);
+          pacc[3] = fmaf(w4.w, vv, pacc[3]);
+        }
+      }
+      __syncwarp();
+    } else if ((kb0 | kb1) != 0u) {  // otherwise no row of the group is dequantised
       // A: head g's weights (g < 4) for rows 2t, 2t + 1, 2t + 8, 2t + 9 times each row's V scale
       const int src = 8 * t + (g & 3);
       const float w0 = __shfl_sync(0xffffffffu, wk[0], src), w1 = __shfl_sync(0xffffffffu, wk[0], src + 4);
@@ -808,7 +831,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   };
   // the probe pass, at the end of a tile: its records (head t's m'_t and denominator, head g's probe
   // lanes of the accumulators: f16 part in row g + remainder in row g + 8), then fresh sums
-  auto flush = [&](int tile) {
+  auto flush = [&](int tile) {  // (the probe pass)
     float lt = l;  // head t's denominator over the tile (lanes of the same t)
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, off);
@@ -819,18 +842,13 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       rc[0] = mp;
       rc[1] = lt;
     }
-    if (g < G) {
-      float* rc = p.probe + (rec0 + static_cast<long long>(g) * p.n_max) * REC;
+    if (lane < p.n_probe) {  // probe `lane` of every head
 #pragma unroll
-      for (int idx = 0; idx < 16; ++idx)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int pi = s_pidx[32 * (idx >> 2) + 4 * (2 * t + c) + (idx & 3)];
-          if (pi >= 0) rc[2 + pi] = acc[idx][c] + acc[idx][c + 2];
-        }
+      for (int h = 0; h < 4; ++h) {
+        if (h < G) p.probe[(rec0 + static_cast<long long>(h) * p.n_max) * REC + 2 + lane] = pacc[h];
+        pacc[h] = 0.f;
+      }
     }
-#pragma unroll
-    for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
     l = 0.f;
   };
 
