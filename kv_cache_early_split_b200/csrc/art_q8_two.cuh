@@ -924,7 +924,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
 // when both are below their thresholds, and the split stops at the first tile whose run of holding
 // tiles reaches the patience ("Resumen Tecnico: ART", S2.2-S2.3).  Output: the stop tile (absolute
 // index; the split's last tile when the rule never fires) and the tiles consumed.
-constexpr int RW = 8;
+constexpr int RW = 16;
 constexpr int kNoStop = 0x7fffffff;
 template <int PC>
 struct RuleState {
