@@ -116,7 +116,8 @@ typedef struct {
  * are consumed whatever they hold; at most n tiles plus one round past it are read
  * speculatively.  Negative values are rejected.  The CUDA-core kernel (fp32 / q8
  * one-pass / d = 64 / other tiles), whose CTAs read one round ahead of the rule
- * at most, ignores it. */
+ * at most, ignores it, and so does q8 ART on the two streaming passes (which
+ * reads every tile; ART_Q8_TENSOR_CORE keeps the bound). */
 typedef struct {
   float eps_scale;
   float eps_dir;
@@ -214,10 +215,14 @@ art_status art_decode_attn_terminate_noalloc(const art_shape* shape, art_dtype d
  * ART; otherwise ART as in art_decode_attn_terminate.
  * The library picks one of three implementations (same rule, same outputs within rounding,
  * same counters; a tile counts as read when it was fetched):
- *   - without ART and with ws_bytes >= art_q8_workspace_bytes(shape) (and B*Hkv*num_splits
- *     <= 65535), two streaming passes over the whole GPU: scores and tile maxima from K, then
- *     the running maxima m', the skip test and the V products (a tile whose rows all fail the
- *     test for every head is not read), then a combine;
+ *   - with ws_bytes >= art_q8_workspace_bytes(shape) (and B*Hkv*num_splits <= 65535), two
+ *     streaming passes over the whole GPU: scores and tile maxima from K, then the running
+ *     maxima m', the skip test and the V products (a tile whose rows all fail the test for
+ *     every head is not read), then a combine.  With ART (d = 128, tile >= 32, 3 or 4 query
+ *     heads per kv head) the V pass runs twice around the rule: a probe pass records per tile
+ *     and head (m'_t, l_t, the probe lanes of the tile's sum), a rule kernel finds each head's
+ *     stop tile from those records, and the second pass sums the consumed tiles only.  Every
+ *     K tile is read (tiles read = all tiles) and max_spec_tiles does not apply;
  *   - otherwise on the tensor cores when d = 128, 3 or 4 query heads per kv head, tile 64 or
  *     128 and L_max even: int8 codes become f16 MMA operands exactly, the scores take the K
  *     scales per 32-element block in fp32, the V scales are folded into the weights, and the
@@ -234,7 +239,7 @@ art_status art_decode_attn_q8_skipv(const art_shape* shape, const void* q_bf16, 
 typedef enum {
   ART_Q8_AUTO = 0,         /* the library's choice (as art_decode_attn_q8_skipv) */
   ART_Q8_TENSOR_CORE = 1,  /* tcgen05 tensor cores */
-  ART_Q8_TWO_PASS = 2,     /* two streaming passes + combine (no ART; q8 workspace) */
+  ART_Q8_TWO_PASS = 2,     /* two streaming passes + combine (q8 workspace; ART: + probe pass and rule) */
   ART_Q8_CLUSTER = 3       /* one pass on the CUDA cores over a thread-block cluster */
 } art_q8_path;
 

@@ -364,6 +364,24 @@ constexpr int STEP = 32;
 constexpr int BOX = STEP * 128;
 constexpr int PB = 3;   // boxes per warp in flight, scores pass
 constexpr int PBV = 2;  // PV pass (its scores and scales take the rest of the shared memory)
+// Wait for slot sl's box (bounded; the warp agrees on the outcome).  On success the slot's pending bit
+// clears and its parity flips; after a timeout (the status word has ART_ERR_TIMEOUT) the bit stays
+// set, so that the caller stops issuing and drains the slots still pending before it leaves.
+__device__ __forceinline__ bool wait_box(uint32_t bars, int sl, uint32_t& pend, uint32_t& phase, int32_t* status) {
+  if (!((pend >> sl) & 1u)) return true;
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bars + 8 * sl, (phase >> sl) & 1u, status));
+  if (ok) {
+    phase ^= 1u << sl;
+    pend &= ~(1u << sl);
+  }
+  return ok;
+}
+// ... the drain: one more bounded wait on every slot still pending
+__device__ __forceinline__ void drain_boxes(uint32_t bars, int slots, uint32_t pend, uint32_t phase, int32_t* status) {
+  for (int sl = 0; sl < slots; ++sl)
+    if ((pend >> sl) & 1u) mbar_wait_bounded(bars + 8 * sl, (phase >> sl) & 1u, status);
+}
+
 __device__ __forceinline__ uint32_t swz(int row, int byte) {
   return static_cast<uint32_t>(row * 128 + ((((byte >> 4) ^ row) & 7) << 4) + (byte & 15));
 }
@@ -536,11 +554,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
   for (int k = 0; k < nsteps; ++k) {
     const int sl = k % mma16::PB;
     cp_async_wait<mma16::PB - 1>();  // the scales of step k have landed (this lane's) ...
-    if ((pend >> sl) & 1u) {         // ... its codes
-      mbar_wait_bounded(bars + 8 * sl, (phase >> sl) & 1u, p.ws_status);
-      phase ^= 1u << sl;
-      pend &= ~(1u << sl);
-    }
+    if (!mma16::wait_box(bars, sl, pend, phase, p.ws_status)) break;  // ... its codes
     __syncwarp();  // ... and every lane's scales
     float x0, x1, y0, y1;
     scores(sl, 0, x0, x1);
@@ -550,6 +564,7 @@ __global__ void __launch_bounds__(NT, 2) q8_scores_mma_kernel(const __grid_const
     __syncwarp();  // every lane is done with the slot before it is refilled
     issue();
   }
+  mma16::drain_boxes(bars, mma16::PB, pend, phase, p.ws_status);  // (only after a timeout)
   cp_async_wait<0>();
   if (g == 0) s_cm[warp][t] = cm;
   __syncthreads();
@@ -859,11 +874,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
     issue();                          // step k + PBV - 1, into the slot step k - 1 left
     cp_async_wait<mma16::PBV - 1>();  // step k's scales and scores (this lane's copies)
     const int sl = k % mma16::PBV;
-    if ((pend >> sl) & 1u) {  // its V codes, when they were copied
-      mbar_wait_bounded(bars + 8 * sl, (phase >> sl) & 1u, p.ws_status);
-      phase ^= 1u << sl;
-      pend &= ~(1u << sl);
-    }
+    if (!mma16::wait_box(bars, sl, pend, phase, p.ws_status)) break;  // its V codes, when they were copied
     __syncwarp();
     const int t_step = wc.t;  // (a step never straddles two tiles)
 #pragma unroll
@@ -872,6 +883,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       if (wc.ik == 0) flush(t_step);  // the step ended its tile
     __syncwarp();
   }
+  mma16::drain_boxes(bars, mma16::PBV, pend, phase, p.ws_status);  // (only after a timeout)
   cp_async_wait<0>();
   {
     int ns_w = nskip;

@@ -56,7 +56,8 @@ def run(dp, mode, art, cap):
 def test_bounded_speculation_same_results_fewer_reads(name, kw, mode, caps, tq_max):
     w = I.make_workload(d=128, tile=64, seed=47, **kw)
     dp = K.upload(w)
-    assert K.kernel_name(dp, mode) == "art_decode_tc_kernel", name
+    # (q8: the decode kernel is pinned by path; the query names the default, the two-pass rule)
+    assert K.kernel_name(dp, mode) == ("q8_pv_mma_kernel" if mode == "q8_art" else "art_decode_tc_kernel"), name
     o0, t0, r0, s0 = run(dp, mode, w.art, 0)
     # the oracle, run to the GPU's own stop tiles
     ref = oracle_run(w, "q8" if mode == "q8_art" else "full", forced_used=s0)
