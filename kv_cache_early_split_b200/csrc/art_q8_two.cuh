@@ -65,6 +65,7 @@ struct Params {
 };
 
 constexpr int REC = 34;  // floats per probe record: m'_t, l_t, up to 32 probe lanes
+static_assert(REC % 2 == 0, "records start on 8-byte boundaries");
 
 // Smallest chunk: at least 128 rows per warp where that stays within CTMAX tiles.
 __host__ __device__ inline int chunk_tiles_min(int T) {
@@ -730,7 +731,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
   float acc[16][4];  // n-tile (block b, j) = 4 b + j
 #pragma unroll
   for (int n = 0; n < 16; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-  float pacc[4] = {0.f, 0.f, 0.f, 0.f};  // the probe pass: probe `lane` of each head over the tile
+  float pacc[4] = {0.f, 0.f, 0.f, 0.f};  // the probe pass: this lane's probe lane of each head, over the tile
   float l = 0.f, mp = 0.f, fac = 0.f;
   bool live = false;
   int nskip = 0;
@@ -775,10 +776,13 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
         s_wg[warp][g + 8][t] = 0.f;
       }
       __syncwarp();
-      if ((kb0 | kb1) != 0u && lane < p.n_probe) {
-        const int pos = s_plane[lane], blk = pos >> 5;
+      // up to 16 probe lanes: two lanes per probe lane, 8 rows each (the halves add at the flush)
+      const bool halves = p.n_probe <= 16;
+      const int pi = halves ? (lane & 15) : lane, r0 = halves ? (lane >> 4) * 8 : 0;
+      if ((kb0 | kb1) != 0u && pi < p.n_probe) {
+        const int pos = s_plane[pi], blk = pos >> 5;
 #pragma unroll 4
-        for (int row = 0; row < mma16::ROWS; ++row) {
+        for (int row = r0; row < r0 + (halves ? 8 : mma16::ROWS); ++row) {
           const float code = static_cast<float>(static_cast<int8_t>(box[mma16::swz(row, pos)]));
           const float vv = code * __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(vsl + row * 8)[blk]));
           const float4 w4 = *reinterpret_cast<const float4*>(&s_wg[warp][row][0]);
@@ -857,13 +861,17 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_mma_kernel(const __grid_constant_
       rc[0] = mp;
       rc[1] = lt;
     }
+    if (p.n_probe <= 16) {  // the two halves of each probe lane
+#pragma unroll
+      for (int h = 0; h < 4; ++h) pacc[h] += __shfl_xor_sync(0xffffffffu, pacc[h], 16);
+    }
     if (lane < p.n_probe) {  // probe `lane` of every head
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
+      for (int h = 0; h < 4; ++h)
         if (h < G) p.probe[(rec0 + static_cast<long long>(h) * p.n_max) * REC + 2 + lane] = pacc[h];
-        pacc[h] = 0.f;
-      }
     }
+#pragma unroll
+    for (int h = 0; h < 4; ++h) pacc[h] = 0.f;
     l = 0.f;
   };
 
@@ -985,12 +993,17 @@ __global__ void __launch_bounds__(RW * 32) q8_rule_kernel(const __grid_constant_
     float m = -INFINITY, l = 0.f, a[PC];
 #pragma unroll
     for (int i = 0; i < PC; ++i) a[i] = 0.f;
-    if (valid) {
-      const float* rc = p.probe + (static_cast<long long>(hq) * p.n_max + tt) * REC;
-      m = rc[0];
-      l = rc[1];
+    if (valid) {  // (records are 136 bytes apart: 8-byte loads)
+      const float2* rc = reinterpret_cast<const float2*>(p.probe + (static_cast<long long>(hq) * p.n_max + tt) * REC);
+      const float2 ml = rc[0];
+      m = ml.x;
+      l = ml.y;
 #pragma unroll
-      for (int i = 0; i < PC; ++i) a[i] = i < p.n_probe ? rc[2 + i] : 0.f;
+      for (int i = 0; i < PC; i += 2) {
+        const float2 v = rc[1 + i / 2];
+        a[i] = i < p.n_probe ? v.x : 0.f;
+        a[i + 1] = i + 1 < p.n_probe ? v.y : 0.f;
+      }
     }
 #pragma unroll 1
     for (int off = 1; off < 32; off <<= 1) {  // the warp's inclusive scan
