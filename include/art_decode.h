@@ -133,11 +133,11 @@ typedef struct {
  * keep the caller's split layout either way. */
 size_t art_workspace_bytes(const art_shape* shape);
 
-/* Bytes of workspace art_decode_attn_q8_skipv needs to run full attention (params == NULL) as
- * two streaming passes: art_workspace_bytes(shape) plus scores [B, Hkv, L_max, GP] fp32 (GP the
- * next power of two >= Hq/Hkv), tile and chunk maxima and per-chunk partial states (0 on an
- * invalid shape).  The offsets below
- * hold for this larger workspace too. */
+/* Bytes of workspace art_decode_attn_q8_skipv needs to run as two streaming passes:
+ * art_workspace_bytes(shape) plus scores [B, Hkv, L_max, GP] fp32 (GP the next power of two
+ * >= Hq/Hkv), tile and chunk maxima, per-chunk partial states and, for ART, a 136-byte probe
+ * record per query head and tile and a stop tile per query head and split (0 on an invalid
+ * shape).  The offsets below hold for this larger workspace too. */
 size_t art_q8_workspace_bytes(const art_shape* shape);
 
 /* Byte offset inside ws of the int32 array tiles_read[B, Hkv, num_splits]:
@@ -150,8 +150,9 @@ size_t art_workspace_tiles_read_offset(const art_shape* shape);
  * the V rows left out of every query head's numerator by the V skip (page
  * "La Elegancia de la Omision": exp(s_j - m') < tau for every head of the group)
  * and the V tiles not read at all because every row of every head was left out.
- * Written by the two-pass q8 implementation (art_decode_attn_q8_skipv without
- * ART, two-pass path) only; other calls leave it untouched. */
+ * Written by the two-pass q8 implementation (art_decode_attn_q8_skipv on the
+ * two-pass path; with ART, by its probe pass, over every tile) only; other calls
+ * leave it untouched. */
 size_t art_workspace_vskip_offset(const art_shape* shape);
 
 /* Byte offset inside ws of the int32 array split_tiles[B, Hq, num_splits]:
