@@ -59,6 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=I.WORKLOADS)
     ap.add_argument("--mode", default=None, choices=("art", "full", "q8", "q8_art"))
+    ap.add_argument("--q8-path", default="auto", choices=("auto", "tensor_core", "two_pass", "cluster"),
+                    help="q8 implementation of the timed mode (art_decode_attn_q8_skipv_path); default the library's")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweeps", action="store_true",
                     help="time the workload's two modes only (no other workloads, sweeps or extras)")
@@ -202,11 +204,12 @@ def measured_traffic(workload, mode, kernel_name):
         return None
 
 
-def launches_per_call(K, dp, w, mode) -> int:
+def launches_per_call(K, dp, w, mode, q8_path="auto") -> int:
     """Kernels one decode call launches: q8 over a two-pass workspace runs scores, weights + PV and
     combine (with ART: scores, probe pass, rule, limited pass, combine); every other call one
     kernel, plus the split combine with S > 1."""
-    if mode in ("q8", "q8_art") and dp.ws_bytes >= K.capi.art_q8_workspace_bytes(dp.shape):
+    if (mode in ("q8", "q8_art") and q8_path in ("auto", "two_pass")
+            and dp.ws_bytes >= K.capi.art_q8_workspace_bytes(dp.shape)):
         if mode == "q8":
             return 3
         if K.kernel_name(dp, mode) == "q8_pv_mma_kernel":
@@ -684,19 +687,20 @@ def run_ours(args):
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     sampler = ClockSampler(f"GPU-{uuid}" if uuid is not None else str(torch.cuda.current_device()))
+    q8_path = args.q8_path if w.kind == "q8" else "auto"
     for _ in range(args.warmup):
-        K.decode(dp, args.mode, stream=stream.cuda_stream)
+        K.decode(dp, args.mode, stream=stream.cuda_stream, q8_path=q8_path)
     torch.cuda.synchronize()
     sampler.start()
     flush = needs_flush(w)
-    total_ms, launch_ms = time_mode(K, dp, args.mode, args.steps, 0, stream, flush=flush)
+    total_ms, launch_ms = time_mode(K, dp, args.mode, args.steps, 0, stream, flush=flush, q8_path=q8_path)
     clocks = sampler.stop()
     if K.device_status(dp) != 0:
         raise RuntimeError("device status not OK after the timed region")
     tiles_read = dp.tiles_read().cpu().numpy()
     used = dp.split_tiles().cpu().numpy()
     tiles = dp.tiles.cpu().numpy()
-    gpu_launches = args.steps * launches_per_call(K, dp, w, args.mode)
+    gpu_launches = args.steps * launches_per_call(K, dp, w, args.mode, q8_path)
 
     max_ms, all_heads = aggregate(total_ms, heads * args.steps)
     value = all_heads / (max_ms / 1e3)
@@ -755,7 +759,7 @@ def run_ours(args):
     t_host = torch.empty_like(dp.tiles, device="cpu").pin_memory()
     for _ in range(args.warmup):
         dp.q.copy_(q_host, non_blocking=True)
-        K.decode(dp, args.mode)
+        K.decode(dp, args.mode, q8_path=q8_path)
         o_host.copy_(dp.o, non_blocking=True)
         t_host.copy_(dp.tiles, non_blocking=True)
     torch.cuda.synchronize()
@@ -765,7 +769,7 @@ def run_ours(args):
     e0.record(cur)
     for _ in range(args.steps):
         dp.q.copy_(q_host, non_blocking=True)
-        K.decode(dp, args.mode)
+        K.decode(dp, args.mode, q8_path=q8_path)
         o_host.copy_(dp.o, non_blocking=True)
         t_host.copy_(dp.tiles, non_blocking=True)
     e1.record(cur)
@@ -788,11 +792,16 @@ def run_ours(args):
                "sample": f"{passes} whole passes of the workload ({h_done} query heads, {secs:.1f} s)"}
 
     kernel = K.kernel_name(dp, args.mode)
-    traffic = measured_traffic(w.name, args.mode, kernel)
-    if launches_per_call(K, dp, w, args.mode) == 3:
+    if q8_path == "tensor_core":
+        kernel = "art_decode_tc_kernel"
+    elif q8_path == "cluster":
+        kernel = "art_decode_kernel"
+    # (the committed DRAM figures are for the library's default path of each mode)
+    traffic = measured_traffic(w.name, args.mode, kernel) if q8_path == "auto" else None
+    if launches_per_call(K, dp, w, args.mode, q8_path) == 3:
         mma = "_mma" if kernel == "q8_pv_mma_kernel" else ""
         kernel = f"q8_scores{mma}_kernel + q8_pv{mma}_kernel + q8_combine_kernel (timed as one call)"
-    elif launches_per_call(K, dp, w, args.mode) == 5:
+    elif launches_per_call(K, dp, w, args.mode, q8_path) == 5:
         kernel = ("q8_scores_mma_kernel + q8_pv_mma_kernel (probe pass) + q8_rule_kernel + q8_pv_mma_kernel "
                   "(limited pass) + q8_combine_kernel (timed as one call)")
     elif w.num_splits > 1:
