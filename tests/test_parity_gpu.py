@@ -277,3 +277,27 @@ def test_unsupported_tile_returns_error():
     dp = K.upload(w)
     rc = K.decode(dp, "full", check=False)
     assert rc == capi.ART_ERR_UNSUPPORTED
+
+
+Q8_ART_TWO_PASS = [
+    # d, Hq, Hkv, B, L_max, lens, tile, S, n_probe, patience: the rule over per-tile records with more
+    # than one round of its CTA (over 512 tiles in a split), 32 probe lanes (one lane per probe lane in
+    # the probe pass, the wider rule kernel), 20 lanes, 3 heads per kv head, tile 32, splits
+    (128, 4, 1, 1, 40960, [40960], 64, 1, 16, 1),
+    (128, 8, 2, 2, 12288, [12288, 5001], 32, 2, 32, 2),
+    (128, 6, 2, 1, 9000, [8999], 64, 3, 20, 3),
+]
+
+
+@pytest.mark.parametrize("case", Q8_ART_TWO_PASS, ids=lambda c: f"L{c[4]}-T{c[6]}-S{c[7]}-P{c[8]}-p{c[9]}")
+def test_q8_art_two_pass_rounds_and_probe_widths(case):
+    d, Hq, Hkv, B, L_max, lens, tile, S, n_probe, patience = case
+    lanes = I.probe_lanes_strided(d, n_probe) if 128 % n_probe == 0 else [(7 * i) % d for i in range(n_probe)]
+    w = I.make_workload(kind="q8", B=B, Hq=Hq, Hkv=Hkv, d=d, L_max=L_max, tile=tile, num_splits=S,
+                        seq_lens=lens, seed=91 + n_probe, sink=6.0, gumbel_scale=2.0)
+    # the workloads' thresholds (late stops), and thresholds that always hold with a patience of 600
+    # (a split of more than 600 tiles stops at its 600th, in the rule kernel's second round)
+    for art in (dict(eps_scale=1e-3, eps_dir=1e-4, patience=patience, lanes=lanes),
+                dict(eps_scale=1e9, eps_dir=1e9, patience=600, lanes=lanes)):
+        for tau in (1e-6, 1e-3):
+            check_art(w, "q8_art", art=art, tau=tau, q8_path="two_pass")
