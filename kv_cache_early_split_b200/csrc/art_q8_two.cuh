@@ -1334,7 +1334,7 @@ __global__ void __launch_bounds__(NT, 2) q8_pv_kernel(const __grid_constant__ Pa
 // then the per-split counters of the caller's split layout.
 template <int D>
 __global__ void __launch_bounds__(D) q8_combine_kernel(const __grid_constant__ Params p) {
-  constexpr int CU = 8;
+  constexpr int CU = 32;  // chunk states loaded per batch (a split of up to 32 chunks in one round trip)
   grid_dep_wait();  // pass 2's chunk states
   const int hq = blockIdx.x;
   const int dd = threadIdx.x;
