@@ -797,7 +797,7 @@ def run_ours(args):
     elif q8_path == "cluster":
         kernel = "art_decode_kernel"
     # (the committed DRAM figures are for the library's default path of each mode)
-    traffic = measured_traffic(w.name, args.mode, kernel) if q8_path == "auto" else None
+    traffic = measured_traffic(w.name, args.mode, kernel) if q8_path == "auto" and not args.batch else None
     if launches_per_call(K, dp, w, args.mode, q8_path) == 3:
         mma = "_mma" if kernel == "q8_pv_mma_kernel" else ""
         kernel = f"q8_scores{mma}_kernel + q8_pv{mma}_kernel + q8_combine_kernel (timed as one call)"
