@@ -148,6 +148,18 @@ def test_invalid_arguments_q8(L):
     s2 = shape(L_max=32767)
     assert q8(s2, ws_bytes=capi.art_q8_workspace_bytes(s2)) == capi.ART_ERR_UNSUPPORTED
     assert q8(s, ws_bytes=capi.art_workspace_bytes(s) - 16) == capi.ART_ERR_WORKSPACE
+    # ART on the two passes: the rule's settings are checked before any launch, and shapes outside the
+    # tensor-core passes (d = 64, tile 16, 8 heads per kv head) are refused on that path
+    art = capi.make_params(1e-3, 1e-4, 2, [0, 8, 16])
+    assert q8(s, params=capi.make_params(1e-3, 1e-4, 1, [200]), ws_bytes=big) == capi.ART_ERR_INVALID_ARG
+    assert q8(s, params=capi.make_params(1e-3, 1e-4, 0, [0]), ws_bytes=big) == capi.ART_ERR_INVALID_ARG
+
+    def two_pass(sh):
+        return capi.art_decode_attn_q8_skipv_path(sh, A, A * 2, A * 8, A * 3, A * 9, A * 4, 1e-6, art, A * 5, A * 6,
+                                                  A * 7, capi.art_q8_workspace_bytes(sh), capi.ART_Q8_TWO_PASS, None)
+    assert two_pass(shape(d=64)) == capi.ART_ERR_UNSUPPORTED
+    assert two_pass(shape(tile=16)) == capi.ART_ERR_UNSUPPORTED
+    assert two_pass(shape(Hq=64, Hkv=8)) == capi.ART_ERR_UNSUPPORTED
 
 
 def test_read_status_rejects_null(L):
